@@ -1,0 +1,455 @@
+"""Benchmark of the IndexCache sparse-attention layer stack on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload prefill_8k] [--pattern P] [--no-cpu-baseline]
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+the layer loop with the F-layer indexer + top-k and every layer's sparse
+attention (ic_layer_stack_forward), inputs resident in HBM.  The default
+workload is the 8K-token prefill: B=1, L=8192, 8 layers FSSSFSSS, indexer
+32 heads x 128, k=2048, attention 16 query heads / 1 KV head x 128.
+
+Prints ONE JSON line (rank 0).  `value` is prefill tokens/s over the stack
+(B*L*N / max-over-ranks step time).  `kernels` breaks the step down per
+kernel from CUDA events recorded on the launching stream inside the timed
+steps; `roofline` is for the kernel with the largest share of the step.
+With N > 1 (torchrun) every rank runs an independent replica of the workload
+(the query rows of different sequences never interact), so scaling is weak
+and no collective is on the data path; the barrier and the max-over-ranks
+reduction of the step time are the only collectives.
+
+--impl reference times the CPU oracle (the plain fp64 restatement used by the
+tests) on the host cores, on a bounded sample of query rows of the same
+workload, and prints the same line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import ctypes
+import io
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from lightning_indexer_top_relu_b200 import synth  # noqa: E402
+
+METRIC = "prefill tokens/s over F/S layer stack; indexer TFLOP/s & top-k/attn HBM GB/s"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ---------------------------------------------------------------- algorithmic work
+
+def work_per_layer(wl):
+    """Algorithmic flops / bytes of each step of one layer (causal)."""
+    B, Lq, Lk, q0, k = wl.B, wl.Lq, wl.Lk, wl.q_offset, wl.k
+    t = np.arange(Lq, dtype=np.float64) + q0
+    vis = np.minimum(t + 1, Lk)
+    sum_vis = B * vis.sum()                       # sum over rows of visible positions
+    sel = B * np.minimum(vis, k).sum()            # sum over rows of selected positions
+    rows = B * Lq
+    w = {}
+    w["indexer_flops"] = 2.0 * wl.H_I * wl.d_I * sum_vis
+    # q_I + w read once, k_I once per batch element, causal scores written
+    w["indexer_bytes"] = (rows * wl.H_I * wl.d_I * 2 + rows * wl.H_I * 4 + B * Lk * wl.d_I * 2
+                          + 4 * sum_vis)
+    w["topk_bytes"] = 4 * sum_vis + 4.0 * rows * k
+    w["attn_flops"] = 4.0 * wl.Hq * wl.d * sel
+    # gathered K and V rows + q + out + index rows
+    w["attn_bytes"] = 4.0 * wl.d * sel + 2 * 2.0 * rows * wl.Hq * wl.d + 4.0 * rows * k
+    return w
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"ic_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for row in csv.reader(f):
+                if len(row) < 9:
+                    continue
+                try:
+                    sm.append(float(row[1]))
+                    mx = float(row[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, row[5:9]):
+                    if v.strip().lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU oracle leg
+
+def oracle_rows_per_s(wl, pattern, layers_cpu, budget_s=15.0, seed=5):
+    """Times the oracle on a bounded sample of query rows; returns (rows/s, sample desc)."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    total = wl.B * wl.Lq
+    n = 8
+    elapsed, done = 0.0, 0
+    while True:
+        rows = np.sort(rng.choice(total, size=min(n, total), replace=False))
+        t0 = time.perf_counter()
+        oracle.layer_stack(pattern, layers_cpu, wl.k, wl.q_offset, rows=rows)
+        dt = time.perf_counter() - t0
+        elapsed += dt
+        done += len(rows)
+        if elapsed >= budget_s or n >= total:
+            break
+        # grow toward the budget
+        n = int(min(total, max(2 * n, n * (budget_s - elapsed) / max(dt, 1e-3))))
+    return done / elapsed, f"{done} uniformly drawn query rows of {total}, all {len(pattern)} layers, {elapsed:.1f} s"
+
+
+def run_reference(args, wl, pattern):
+    """The CPU oracle as the reference arm (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    layers = synth.make_layers(wl, indexer_for_all=False) if pattern == wl.pattern else \
+        synth.make_layers(wl)
+    total = wl.B * wl.Lq
+    rng = np.random.default_rng(11)
+    n_rows = max(1, min(total, args.ref_rows))
+    for _ in range(args.warmup if args.warmup > 0 else 0):
+        pass  # the oracle has no warm-up state; warm-up steps are not repeated
+    times = []
+    for s in range(args.steps):
+        rows = np.sort(rng.choice(total, size=n_rows, replace=False))
+        t0 = time.perf_counter()
+        oracle.layer_stack(pattern, layers, wl.k, wl.q_offset, rows=rows)
+        times.append(time.perf_counter() - t0)
+    sec = float(np.sum(times))
+    value = n_rows * args.steps / sec
+    sample = f"{n_rows} uniformly drawn query rows of {total} per step, all {len(pattern)} layers"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * sec / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(wl, pattern, args),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(wl, pattern, args):
+    return {"workload": wl.name, "B": wl.B, "L": wl.Lq, "Lk": wl.Lk, "q_offset": wl.q_offset,
+            "layers": wl.n_layers, "pattern": pattern, "H_I": wl.H_I, "d_I": wl.d_I,
+            "k": wl.k, "Hq": wl.Hq, "Hkv": 1, "d": wl.d,
+            "parallelism": "replicas" if args.gpus > 1 else "single",
+            "l2": "flushed (256 MiB write) before every timed step"}
+
+
+# ---------------------------------------------------------------- GPU leg
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="prefill_8k", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--pattern", default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-all-f", action="store_true")
+    ap.add_argument("--ref-rows", type=int, default=64)
+    ap.add_argument("--cpu-budget-s", type=float, default=15.0)
+    args = ap.parse_args()
+    wl = synth.WORKLOADS[args.workload]
+    pattern = args.pattern or wl.pattern
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        return run_reference(args, wl, pattern)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+
+    from lightning_indexer_top_relu_b200 import indexcache as ic
+
+    peaks = load_peaks()
+    need_all = (not args.no_all_f) and any(c in "S0" for c in pattern)
+    layers_cpu = synth.make_layers(wl, indexer_for_all=need_all)
+    pinned = [{k: v.pin_memory() for k, v in L.items()} for L in layers_cpu]
+    layers = [{k: v.to(dev, non_blocking=True) for k, v in L.items()} for L in pinned]
+    torch.cuda.synchronize()
+    dims = ic.make_dims(wl.B, wl.Lq, wl.Lk, wl.q_offset, wl.H_I, wl.d_I, wl.Hq, wl.d, wl.k)
+    stack = ic.LayerStack(pattern, layers, dims)
+    stream = torch.cuda.current_stream()
+    n = wl.n_layers
+    flush = torch.empty(256 * 1024 * 1024 // 4, device=dev, dtype=torch.float32)
+
+    # per-kernel marks: 4 events per layer per step
+    def new_marks():
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(4 * n)]
+        arr = (ctypes.c_void_p * (4 * n))(*[e.cuda_event for e in evs])
+        for e in evs:  # make sure the events exist before their handles are used
+            e.record(stream)
+        return evs, arr
+
+    lib = ic.lib()
+    lib.ic_layer_stack_forward_events.restype = ctypes.c_int
+    lib.ic_layer_stack_forward_events.argtypes = [ctypes.c_char_p, ctypes.c_int,
+                                                  ctypes.POINTER(ic.ICLayer),
+                                                  ctypes.POINTER(ic.ICDims), ctypes.c_void_p,
+                                                  ctypes.c_void_p, ctypes.c_size_t,
+                                                  ctypes.c_void_p, ctypes.c_void_p]
+
+    def step(marks=None):
+        if marks is None:
+            stack.forward(stream)
+        else:
+            rc = lib.ic_layer_stack_forward_events(
+                stack._pattern_b, n, stack.table, ctypes.byref(stack.dims),
+                stack.idx_cache.data_ptr(), stack.ws.data_ptr(), stack.ws.numel(),
+                stream.cuda_stream, ctypes.cast(marks, ctypes.c_void_p))
+            if rc != 0:
+                raise ic.IndexCacheError(rc, "ic_layer_stack_forward_events")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if ic.get_last_device_error() != 0:
+        raise RuntimeError("device error during warm-up")
+
+    marks = [new_marks() for _ in range(args.steps)]
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    if pg is not None:
+        pg.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    wall0 = time.perf_counter()
+    for s in range(args.steps):
+        flush.fill_(float(s))                    # L2 flush outside the step's events
+        starts[s].record(stream)
+        step(marks[s][1])
+        ends[s].record(stream)
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    if pg is not None:
+        pg.barrier()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if ic.get_last_device_error() != 0:
+        raise RuntimeError("device error during the timed steps")
+
+    step_ms = [starts[s].elapsed_time(ends[s]) for s in range(args.steps)]
+    total_ms = float(np.sum(step_ms))
+    if pg is not None:
+        t = torch.tensor([total_ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    tokens = wl.B * wl.Lq * world
+    value = tokens / (ms_per_step / 1e3)
+
+    # ---- per-kernel breakdown from the marks
+    ki = {"indexer": [], "topk": [], "attn": []}
+    for evs, _ in marks:
+        for l, c in enumerate(pattern):
+            if c in "F1":
+                ki["indexer"].append(evs[4 * l].elapsed_time(evs[4 * l + 1]))
+                ki["topk"].append(evs[4 * l + 1].elapsed_time(evs[4 * l + 2]))
+            ki["attn"].append(evs[4 * l + 2].elapsed_time(evs[4 * l + 3]))
+    w = work_per_layer(wl)
+    n_f = sum(c in "F1" for c in pattern)
+    kernels = {}
+    per_step = {}
+    for name, vals in ki.items():
+        if not vals:
+            continue
+        avg = float(np.mean(vals))
+        per_step[name] = float(np.sum(vals)) / args.steps
+        ent = {"launches_per_step": len(vals) // args.steps, "ms_per_launch": avg,
+               "share": per_step[name] / ms_per_step}
+        if name == "indexer":
+            ent["tflops"] = w["indexer_flops"] / (avg * 1e-3) / 1e12
+            ent["frac_of_bf16_peak"] = ent["tflops"] / peaks["bf16_tflops"]
+            ent["gbs"] = w["indexer_bytes"] / (avg * 1e-3) / 1e9
+        elif name == "topk":
+            ent["gbs"] = w["topk_bytes"] / (avg * 1e-3) / 1e9
+            ent["frac_of_hbm"] = ent["gbs"] / peaks["hbm_gbs"]
+        else:
+            ent["tflops"] = w["attn_flops"] / (avg * 1e-3) / 1e12
+            ent["logical_gbs"] = w["attn_bytes"] / (avg * 1e-3) / 1e9
+            ent["frac_of_hbm"] = ent["logical_gbs"] / peaks["hbm_gbs"]
+        kernels[name] = ent
+    dom = max(kernels, key=lambda k: kernels[k]["share"])
+    if dom == "indexer":
+        ach = kernels[dom]["tflops"]
+        roof = {"kernel": "indexer_scores", "bound": "tensor", "achieved": ach,
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"],
+                "traffic": None,
+                "algorithmic_per_launch": w["indexer_flops"]}
+    elif dom == "topk":
+        ach = kernels[dom]["gbs"]
+        roof = {"kernel": "topk_select", "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": ach / peaks["hbm_gbs"], "traffic": None,
+                "algorithmic_per_launch": w["topk_bytes"]}
+    else:
+        ach = kernels[dom]["logical_gbs"]
+        roof = {"kernel": "sparse_attn", "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": ach / peaks["hbm_gbs"], "traffic": None,
+                "algorithmic_per_launch": w["attn_bytes"]}
+    roof["peak_source"] = peaks["source"]
+
+    launches_per_step = 0
+    for c in pattern:
+        launches_per_step += (2 if c in "F1" else 0) + 1   # indexer + top-k, attention
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded Gaussian, correlated layers)",
+            "config": config_of(wl, pattern, args), "gpu_launches": launches_per_step * args.steps,
+            "kernels": kernels, "roofline": roof,
+            "indexer_share": (per_step.get("indexer", 0) + per_step.get("topk", 0)) / ms_per_step,
+            "wall_s_timed": wall}
+    if clk is not None:
+        line["clocks"] = clk
+
+    # ---- the same stack with every layer Full, for the F/S speed-up
+    if need_all:
+        stack_f = ic.LayerStack("F" * n, layers, dims)
+        for _ in range(2):
+            stack_f.forward(stream)
+        ts = []
+        for s in range(max(3, args.steps // 2)):
+            flush.fill_(float(s))
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            stack_f.forward(stream)
+            b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        msf = float(np.mean(ts))
+        line["all_f"] = {"pattern": "F" * n, "ms_per_step": msf,
+                         "value": wl.B * wl.Lq * world / (msf / 1e3),
+                         "speedup_of_pattern": msf / ms_per_step}
+        del stack_f
+
+    # ---- end to end through the public API with host buffers
+    if not args.no_e2e:
+        outs_host = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in stack.outs]
+        h2d = sum(v.numel() * v.element_size() for i, L in enumerate(pinned) for k, v in L.items()
+                  if k in ("q", "k", "v") or pattern[i] in "F1")
+        d2h = sum(o.numel() * o.element_size() for o in stack.outs)
+
+        def e2e_step():
+            for i, L in enumerate(pinned):
+                for k, v in L.items():
+                    if k in ("q", "k", "v") or pattern[i] in "F1":
+                        layers[i][k].copy_(v, non_blocking=True)
+            stack.forward(stream)
+            for o, h in zip(stack.outs, outs_host):
+                h.copy_(o, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if pg is not None:
+            pg.barrier()
+        a.record(stream)
+        k_e2e = max(3, args.steps // 2)
+        for _ in range(k_e2e):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b) / k_e2e
+        if pg is not None:
+            t = torch.tensor([e_ms], device=dev)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            e_ms = float(t.item())
+        line["e2e"] = {"value": wl.B * wl.Lq * world / (e_ms / 1e3), "unit": "tokens/s",
+                       "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                       "ms_per_step": e_ms}
+
+    # ---- CPU oracle baseline (rank 0, N=1 only)
+    if not args.no_cpu_baseline and world == 1:
+        import oracle
+        rps, sample = oracle_rows_per_s(wl, pattern, layers_cpu, budget_s=args.cpu_budget_s)
+        line["cpu_baseline"] = {"value": rps, "unit": "tokens/s", "cores": oracle.num_threads(),
+                                "kind": "oracle", "sample": sample}
+
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,189 @@
+/*
+ * indexcache.h — C ABI of libindexcache.so: a DSA-style sparse-attention
+ * layer stack with IndexCache cross-layer index reuse, for NVIDIA B200
+ * (sm_100a).
+ *
+ * Sources.  "IndexCache: Accelerating Sparse Attention via Cross-Layer Index
+ * Reuse" (arXiv 2603.12201), as described by:
+ *   - the fugumt digest, Abstract: a lightning indexer selects the top-k most
+ *     relevant tokens per query, reducing core attention from O(L^2) to
+ *     O(Lk); Full layers run their own indexers, Shared layers reuse the
+ *     nearest Full layer's top-k indices;
+ *   - the kualia.ai review, "The Redundancy That Was Sitting There": the
+ *     index cache is a temporary buffer holding only the current index tensor,
+ *     overwritten at each F layer;
+ *   - the skill page, Step 3 (IndexCacheManager.get_indices_for_layer): an S
+ *     layer with nothing cached is an error;
+ *   - the knowledge note "Cross-Layer Index Reuse", How It Works: the anchor
+ *     layer scores the visible positions; following layers run their own
+ *     sparse attention over the stored positions.
+ * The pages print no indexer formula; this library computes the standard
+ * lightning-indexer score s[t,s] = sum_j w[t,j] * max(0, q_I[t,j] . k_I[s]).
+ *
+ * Conventions for every entry point:
+ *   - Pointers are DEVICE pointers to caller-owned, contiguous, row-major
+ *     buffers (shapes below).  bf16 tensors are passed as uint16_t bit
+ *     patterns.  The library allocates nothing and keeps no state from one
+ *     call to the next (so no index cache can leak between sequences).
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and runs asynchronously.  Argument errors are detected on the
+ *     host and returned before anything is launched.
+ *   - Query row i of batch b sits at absolute position t = q_offset + i and
+ *     sees key positions s <= t.  Requirement: q_offset + Lq <= Lk.
+ *     Prefill: q_offset = 0, Lq = Lk.  Decode: Lq = 1, q_offset = Lk - 1.
+ *   - Supported shapes: d_I in {64, 128}; H_I a power of two in [4, 128];
+ *     d in {64, 128}; Hq in {8, 16}; Hkv == 1 (MQA); 1 <= k <= Lk.  Other
+ *     shapes return IC_ERR_UNSUPPORTED.  bf16 buffers must be 16-byte
+ *     aligned (IC_ERR_UNSUPPORTED otherwise).
+ *   - Device-side faults are never raised on purpose: kernels report an
+ *     out-of-range attention index or a timed-out wait into a device error
+ *     word that ic_get_last_device_error() reads.
+ */
+#ifndef INDEXCACHE_H
+#define INDEXCACHE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *ic_stream_t;
+
+typedef enum {
+    IC_OK = 0,
+    IC_ERR_INVALID_ARG = 1,        /* null pointer, negative size, bad pattern character */
+    IC_ERR_UNSUPPORTED = 2,        /* shape outside the supported set, misaligned pointer */
+    IC_ERR_NO_CACHED_INDICES = 3,  /* an S layer precedes every F layer */
+    IC_ERR_WORKSPACE_TOO_SMALL = 4,
+    IC_ERR_CUDA = 5,               /* a CUDA runtime/driver call or launch failed */
+    IC_ERR_TIMEOUT = 6             /* a kernel's bounded wait gave up (device error word) */
+} ic_status;
+
+/* Static text for a status code. */
+const char *ic_status_string(int status);
+
+/* Detail text of the last failing call on this host thread ("" if none). */
+const char *ic_last_error_message(void);
+
+/* Synchronises `stream`, reads and clears the current device's error word.
+ * Returns IC_OK, IC_ERR_TIMEOUT (a bounded wait expired) or
+ * IC_ERR_INVALID_ARG (an attention index outside [0, t] was skipped), or
+ * IC_ERR_CUDA if the synchronisation itself failed. */
+int ic_get_last_device_error(ic_stream_t stream);
+
+/*
+ * Step a1 — lightning indexer scores (digest Abstract; review Introduction:
+ * the indexer scores all preceding tokens).
+ *   q_idx  [B, Lq, H_I, d_I] bf16     k_idx [B, Lk, d_I] bf16
+ *   w      [B, Lq, H_I]      fp32     scores [B, Lq, Lk] fp32 (written)
+ * scores[b,i,s] = sum_j w[b,i,j] * max(0, q_idx[b,i,j,:] . k_idx[b,s,:]) for
+ * s <= t = q_offset + i, and -INFINITY for t < s < Lk.  bf16 products,
+ * fp32 accumulation (tcgen05 tensor cores).
+ */
+int ic_indexer_scores(const uint16_t *q_idx, const uint16_t *k_idx, const float *w, int B,
+                      int Lq, int Lk, int H_I, int d_I, int q_offset, float *scores,
+                      ic_stream_t stream);
+
+/*
+ * Step a2 — per-row top-k (digest Abstract: the indexer selects the top-k
+ * tokens per query).
+ *   scores [B, Lq, Lk] fp32 (only s <= t is read)   idx [B, Lq, k] int32 (written)
+ * Row (b, i) keeps the min(k, t+1) visible positions first in the order
+ * (score descending, position ascending), written in ascending position
+ * order; the remaining slots are -1.  Scores compare as IEEE floats (-0 ==
+ * +0); NaN scores are outside the contract.  Exact (bit-for-bit
+ * deterministic).
+ */
+int ic_topk_select(const float *scores, int B, int Lq, int Lk, int q_offset, int k,
+                   int32_t *idx, ic_stream_t stream);
+
+/*
+ * Step a4 — sparse attention over the cached positions (digest Abstract:
+ * core attention over k tokens; knowledge note: each layer runs its own
+ * sparse attention over the stored positions).  MQA: Hkv must be 1.
+ *   q [B, Lq, Hq, d] bf16   k, v [B, Lk, Hkv, d] bf16   idx [B, Lq, k] int32
+ *   out [B, Lq, Hq, d] bf16 (written)   lse [B, Lq, Hq] fp32 (written; may be NULL)
+ * For each (b, i, h) over the slots whose index lies in [0, t]:
+ *   z = scale * q . K[idx], out = sum softmax(z) * V[idx], lse = ln sum e^z.
+ * Slots holding -1 are empty.  A slot outside [0, t] is skipped and flags
+ * IC_ERR_INVALID_ARG in the device error word.  A row with no valid slot
+ * gives out = 0, lse = -INFINITY.  scale <= 0 selects 1/sqrt(d).
+ * ws/ws_bytes: optional device workspace; with at least
+ * ic_sparse_attn_workspace_bytes(...) bytes, rows with few of them (decode)
+ * split their slots over several CTAs.  ws may be NULL (ws_bytes 0).
+ */
+int ic_sparse_attn(const uint16_t *q, const uint16_t *k, const uint16_t *v, const int32_t *idx,
+                   int B, int Lq, int Lk, int Hq, int Hkv, int d, int k_slots, int q_offset,
+                   float scale, uint16_t *out, float *lse, void *ws, size_t ws_bytes,
+                   ic_stream_t stream);
+
+/* Workspace that lets ic_sparse_attn use its preferred slot split. */
+size_t ic_sparse_attn_workspace_bytes(int B, int Lq, int Hq, int d, int k_slots);
+
+/* One layer of the stack.  S layers may leave q_idx, k_idx and w NULL. */
+typedef struct {
+    const uint16_t *q;      /* [B, Lq, Hq, d] bf16 */
+    const uint16_t *k;      /* [B, Lk, Hkv, d] bf16 */
+    const uint16_t *v;      /* [B, Lk, Hkv, d] bf16 */
+    const uint16_t *q_idx;  /* [B, Lq, H_I, d_I] bf16 (F layers) */
+    const uint16_t *k_idx;  /* [B, Lk, d_I] bf16 (F layers) */
+    const float *w;         /* [B, Lq, H_I] fp32 (F layers) */
+    uint16_t *out;          /* [B, Lq, Hq, d] bf16, written */
+    float *lse;             /* [B, Lq, Hq] fp32, written; may be NULL */
+    int32_t *idx_dump;      /* [B, Lq, k] int32: copy of the indices this layer used; may be NULL */
+} ic_layer;
+
+typedef struct {
+    int B, Lq, Lk, q_offset;
+    int H_I, d_I;
+    int Hq, Hkv, d;
+    int k;
+    float scale;            /* <= 0 -> 1/sqrt(d) */
+} ic_dims;
+
+/*
+ * Workspace for ic_layer_stack_forward.  rows_per_chunk <= 0 asks for the
+ * size that scores every query row of an F layer in one pass; a positive
+ * value asks for the size of chunks of that many rows (rounded up to the
+ * indexer's query block).  Returns 0 for invalid dims.
+ */
+size_t ic_layer_stack_workspace_bytes(const ic_dims *dims, int n_layers, long long rows_per_chunk);
+
+/*
+ * Steps a1-a5 — the IndexCache layer loop (skill page Step 3; technical
+ * summary, Methodologie; review: "a single conditional branch").
+ * pattern: n_layers characters, 'F' or '1' = Full layer, 'S' or '0' = Shared.
+ * For layer l: if F, the indexer scores and the top-k overwrite idx_cache
+ * ([B, Lq, k] int32, caller-owned, the one index cache); then every layer
+ * attends over idx_cache.  An S layer therefore uses exactly the indices of
+ * the nearest preceding F layer.  pattern[0] must be F
+ * (IC_ERR_NO_CACHED_INDICES otherwise, before any launch).
+ * ws: device workspace of ws_bytes; F-layer scores are produced in row
+ * chunks that fit in it; fewer than one query block of rows returns
+ * IC_ERR_WORKSPACE_TOO_SMALL.  No host synchronisation happens inside, so
+ * the whole call can be captured into a CUDA graph.
+ */
+int ic_layer_stack_forward(const char *pattern, int n_layers, const ic_layer *layers,
+                           const ic_dims *dims, int32_t *idx_cache, void *ws, size_t ws_bytes,
+                           ic_stream_t stream);
+
+/*
+ * ic_layer_stack_forward with per-layer timing marks: the same launches,
+ * plus cudaEventRecord on `stream` of events[4*l + j] (each a cudaEvent_t;
+ * NULL entries are skipped) at j=0 layer start, j=1 after the indexer
+ * (when the layer's scores take one chunk; otherwise after indexer + top-k),
+ * j=2 before the attention, j=3 after the attention.  For S layers j=0..2
+ * coincide.  events holds 4*n_layers entries.
+ */
+int ic_layer_stack_forward_events(const char *pattern, int n_layers, const ic_layer *layers,
+                                  const ic_dims *dims, int32_t *idx_cache, void *ws,
+                                  size_t ws_bytes, ic_stream_t stream, void *const *events);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* INDEXCACHE_H */

@@ -1,0 +1,560 @@
+// libindexcache.so: the C ABI declared in include/indexcache.h.
+//
+// Host side only validates arguments, builds TMA descriptors, sizes grids and
+// enqueues the sm_100a kernels on the caller's stream; every step of the
+// computation runs in the kernels below.  Nothing is allocated and nothing is
+// cached between calls except per-device launch attributes.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/indexcache.h"
+#include "common.cuh"
+#include "indexer_scores.cuh"
+#include "sparse_attn.cuh"
+#include "topk_select.cuh"
+
+namespace {
+
+thread_local char g_msg[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof g_msg, fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+    return fail(IC_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+// ---------------------------------------------------------------- device facts
+
+constexpr int MAX_DEV = 64;
+std::mutex g_mu;
+int g_sms[MAX_DEV];
+bool g_attr_done[MAX_DEV];
+
+int device_setup(int* dev_out, int* sms_out);
+
+// ---------------------------------------------------------------- TMA descriptors
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+int get_encode() {
+    if (g_encode) return IC_OK;
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
+        return fail(IC_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+    g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    return IC_OK;
+}
+
+// 3-D bf16 tensor {d0 (contiguous), d1, d2}, 128-byte swizzled boxes {64, box1, 1}.
+int make_tmap_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                 uint32_t box1) {
+    int rc = get_encode();
+    if (rc) return rc;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+    cuuint32_t box[3] = {64, box1, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(IC_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return IC_OK;
+}
+
+// ---------------------------------------------------------------- indexer
+
+struct IndexerGeom {
+    int QB, N, nqb;
+};
+
+IndexerGeom indexer_geom(int Lq, int H) {
+    IndexerGeom g;
+    g.QB = std::min(ic::IDX_NMAX / H, Lq);
+    g.N = ((g.QB * H + 15) / 16) * 16;
+    g.nqb = (Lq + g.QB - 1) / g.QB;
+    return g;
+}
+
+long long block_row_start(const IndexerGeom& g, int Lq, long long gb) {
+    return (gb / g.nqb) * (long long)Lq + (gb % g.nqb) * (long long)g.QB;
+}
+
+template <int H, int DI>
+void set_indexer_attr() {
+    cudaFuncSetAttribute(ic::indexer_scores_kernel<H, DI>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         ic::IndexerSmem<DI>::ALLOC);
+}
+
+template <int H, int DI>
+cudaError_t launch_indexer_t(const CUtensorMap& tq, const CUtensorMap& tk,
+                             const ic::IndexerArgs& a, int grid, cudaStream_t st) {
+    ic::indexer_scores_kernel<H, DI>
+        <<<grid, ic::IDX_THREADS, ic::IndexerSmem<DI>::ALLOC, st>>>(tq, tk, a);
+    return cudaGetLastError();
+}
+
+template <int DI>
+cudaError_t launch_indexer_h(int H, const CUtensorMap& tq, const CUtensorMap& tk,
+                             const ic::IndexerArgs& a, int grid, cudaStream_t st) {
+    switch (H) {
+        case 4: return launch_indexer_t<4, DI>(tq, tk, a, grid, st);
+        case 8: return launch_indexer_t<8, DI>(tq, tk, a, grid, st);
+        case 16: return launch_indexer_t<16, DI>(tq, tk, a, grid, st);
+        case 32: return launch_indexer_t<32, DI>(tq, tk, a, grid, st);
+        case 64: return launch_indexer_t<64, DI>(tq, tk, a, grid, st);
+        case 128: return launch_indexer_t<128, DI>(tq, tk, a, grid, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+// Scores query blocks [g0, g1) into `scores` (row = flattened row - row of g0).
+int launch_indexer(const uint16_t* q_idx, const uint16_t* k_idx, const float* w, int B, int Lq,
+                   int Lk, int H, int dI, int q_offset, long long g0, long long g1, float* scores,
+                   long long ld, bool fill_masked, int sms, cudaStream_t st) {
+    const IndexerGeom geo = indexer_geom(Lq, H);
+    CUtensorMap tq, tk;
+    int rc = make_tmap_3d(&tq, q_idx, (uint64_t)dI, (uint64_t)Lq * H, (uint64_t)B, (uint32_t)geo.N);
+    if (rc) return rc;
+    rc = make_tmap_3d(&tk, k_idx, (uint64_t)dI, (uint64_t)Lk, (uint64_t)B, (uint32_t)ic::IDX_BM);
+    if (rc) return rc;
+
+    // Total key tiles of the range, to size work units.
+    long long total = 0;
+    int max_nt = 0;
+    for (long long gb = g0; gb < g1; ++gb) {
+        const int i0 = (int)(gb % geo.nqb) * geo.QB;
+        const int nq = std::min(geo.QB, Lq - i0);
+        const int n_vis = std::min(q_offset + i0 + nq, Lk);
+        const int nt = (n_vis + ic::IDX_BM - 1) / ic::IDX_BM;
+        total += nt;
+        max_nt = std::max(max_nt, nt);
+    }
+    int tpu = (int)std::min<long long>(64, std::max<long long>(4, total / (6LL * sms)));
+    tpu = std::min(tpu, std::max(1, max_nt));
+    const int max_splits = (max_nt + tpu - 1) / tpu;
+
+    ic::IndexerArgs a;
+    a.w = w;
+    a.scores = scores;
+    a.ld = ld;
+    a.B = B;
+    a.Lq = Lq;
+    a.Lk = Lk;
+    a.q_offset = q_offset;
+    a.QB = geo.QB;
+    a.N = geo.N;
+    a.nqb = geo.nqb;
+    a.g0 = (int)g0;
+    a.g1 = (int)g1;
+    a.row_base = block_row_start(geo, Lq, g0);
+    a.tpu = tpu;
+    a.max_splits = max_splits;
+    const long long n_units = (g1 - g0) * (long long)max_splits;
+    const int grid = (int)std::min<long long>(n_units, sms);
+    if (grid <= 0) return IC_OK;
+    cudaError_t e = dI == 64 ? launch_indexer_h<64>(H, tq, tk, a, grid, st)
+                             : launch_indexer_h<128>(H, tq, tk, a, grid, st);
+    if (e != cudaSuccess) return cuda_fail(e, "indexer_scores launch");
+    if (fill_masked) {
+        const long long n_rows = block_row_start(geo, Lq, g1) - a.row_base;
+        const int fg = (int)std::min<long long>(n_rows, 65535);
+        ic::indexer_fill_masked_kernel<<<fg, 256, 0, st>>>(scores, ld, Lq, Lk, q_offset, geo.QB,
+                                                           a.row_base, n_rows);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "indexer fill launch");
+    }
+    return IC_OK;
+}
+
+// ---------------------------------------------------------------- top-k
+
+int launch_topk(const float* scores, long long ld, long long row_base, long long n_rows, int Lq,
+                int Lk, int q_offset, int k, int32_t* idx, cudaStream_t st) {
+    if (n_rows <= 0) return IC_OK;
+    const int n_max = std::min(Lk, q_offset + Lq);
+    cudaError_t e;
+    if (n_max <= ic::TK_CACHE_MAX) {
+        const int smem = ic::TK_SMEM_FIXED + n_max * 4;
+        ic::topk_select_kernel<true><<<(unsigned)n_rows, ic::TK_THREADS, smem, st>>>(
+            scores, ld, row_base, n_rows, Lq, Lk, q_offset, k, idx);
+    } else {
+        ic::topk_select_kernel<false><<<(unsigned)n_rows, ic::TK_THREADS, ic::TK_SMEM_FIXED, st>>>(
+            scores, ld, row_base, n_rows, Lq, Lk, q_offset, k, idx);
+    }
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "topk_select launch");
+    return IC_OK;
+}
+
+// ---------------------------------------------------------------- sparse attention
+
+int attn_splits(long long n_rows, int k_slots, int sms) {
+    if (n_rows >= 2LL * sms) return 1;
+    long long s = (2LL * sms + n_rows - 1) / n_rows;
+    s = std::min<long long>(s, (k_slots + ic::SA_CHUNK - 1) / ic::SA_CHUNK);
+    s = std::min<long long>(s, 64);
+    return (int)std::max<long long>(1, s);
+}
+
+size_t attn_ws_bytes(long long n_rows, int splits, int Hq, int d) {
+    if (splits <= 1) return 0;
+    return (size_t)n_rows * splits * (size_t)Hq * (d + 1) * sizeof(float);
+}
+
+int launch_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* idx,
+                int B, int Lq, int Lk, int Hq, int d, int k_slots, int q_offset, float scale,
+                uint16_t* out, float* lse, void* ws, size_t ws_bytes, bool trim, int sms,
+                cudaStream_t st) {
+    const long long n_rows = (long long)B * Lq;
+    if (n_rows <= 0) return IC_OK;
+    int splits = attn_splits(n_rows, k_slots, sms);
+    while (splits > 1 && (ws == nullptr || attn_ws_bytes(n_rows, splits, Hq, d) > ws_bytes))
+        splits = splits / 2;
+    ic::SparseAttnArgs a;
+    a.q = reinterpret_cast<const __nv_bfloat16*>(q);
+    a.k = reinterpret_cast<const __nv_bfloat16*>(k);
+    a.v = reinterpret_cast<const __nv_bfloat16*>(v);
+    a.idx = idx;
+    a.out = reinterpret_cast<__nv_bfloat16*>(out);
+    a.lse = lse;
+    a.part_o = splits > 1 ? reinterpret_cast<float*>(ws) : nullptr;
+    a.part_lse = splits > 1 ? reinterpret_cast<float*>(ws) + n_rows * splits * (long long)Hq * d
+                            : nullptr;
+    a.Lq = Lq;
+    a.Lk = Lk;
+    a.Hq = Hq;
+    a.kslots = k_slots;
+    a.q_offset = q_offset;
+    a.splits = splits;
+    a.slots_per_split = (k_slots + splits - 1) / splits;
+    a.trim = trim ? 1 : 0;
+    const float sc = scale > 0.0f ? scale : 1.0f / std::sqrt((float)d);
+    a.scale_log2 = sc * ic::LOG2E;
+    a.n_rows = n_rows;
+    dim3 grid((unsigned)n_rows, (unsigned)splits);
+    if (d == 64) {
+        ic::sparse_attn_kernel<64><<<grid, ic::SA_THREADS, ic::SaSmem<64>::BYTES, st>>>(a);
+    } else {
+        ic::sparse_attn_kernel<128><<<grid, ic::SA_THREADS, ic::SaSmem<128>::BYTES, st>>>(a);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "sparse_attn launch");
+    if (splits > 1) {
+        if (d == 64)
+            ic::sparse_attn_combine_kernel<64><<<(unsigned)n_rows, 256, 0, st>>>(a);
+        else
+            ic::sparse_attn_combine_kernel<128><<<(unsigned)n_rows, 256, 0, st>>>(a);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "sparse_attn combine launch");
+    }
+    return IC_OK;
+}
+
+// ---------------------------------------------------------------- per-device setup
+
+int device_setup(int* dev_out, int* sms_out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= MAX_DEV) return fail(IC_ERR_UNSUPPORTED, "device ordinal %d", dev);
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_attr_done[dev]) {
+        int major = 0, minor = 0, sms = 0;
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+        if (major != 10 || minor != 0)
+            return fail(IC_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a",
+                        dev, major, minor);
+        set_indexer_attr<4, 64>();   set_indexer_attr<4, 128>();
+        set_indexer_attr<8, 64>();   set_indexer_attr<8, 128>();
+        set_indexer_attr<16, 64>();  set_indexer_attr<16, 128>();
+        set_indexer_attr<32, 64>();  set_indexer_attr<32, 128>();
+        set_indexer_attr<64, 64>();  set_indexer_attr<64, 128>();
+        set_indexer_attr<128, 64>(); set_indexer_attr<128, 128>();
+        cudaFuncSetAttribute(ic::topk_select_kernel<true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             ic::TK_SMEM_FIXED + ic::TK_CACHE_MAX * 4);
+        cudaFuncSetAttribute(ic::sparse_attn_kernel<64>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, ic::SaSmem<64>::BYTES);
+        cudaFuncSetAttribute(ic::sparse_attn_kernel<128>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, ic::SaSmem<128>::BYTES);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+        g_sms[dev] = sms;
+        g_attr_done[dev] = true;
+    }
+    *dev_out = dev;
+    *sms_out = g_sms[dev];
+    return IC_OK;
+}
+
+// ---------------------------------------------------------------- validation
+
+int check_indexer_shape(int H, int dI) {
+    if (dI != 64 && dI != 128) return fail(IC_ERR_UNSUPPORTED, "d_I=%d (supported: 64, 128)", dI);
+    if (!pow2(H) || H < 4 || H > 128)
+        return fail(IC_ERR_UNSUPPORTED, "H_I=%d (supported: powers of two in [4, 128])", H);
+    return IC_OK;
+}
+
+int check_attn_shape(int Hq, int Hkv, int d) {
+    if (Hkv != 1) return fail(IC_ERR_UNSUPPORTED, "Hkv=%d (only MQA, Hkv=1)", Hkv);
+    if (d != 64 && d != 128) return fail(IC_ERR_UNSUPPORTED, "d=%d (supported: 64, 128)", d);
+    if (Hq != 8 && Hq != 16) return fail(IC_ERR_UNSUPPORTED, "Hq=%d (supported: 8, 16)", Hq);
+    return IC_OK;
+}
+
+int check_positions(int B, int Lq, int Lk, int q_offset) {
+    if (B < 0 || Lq < 0 || Lk < 0 || q_offset < 0)
+        return fail(IC_ERR_INVALID_ARG, "negative size (B=%d Lq=%d Lk=%d q_offset=%d)", B, Lq, Lk,
+                    q_offset);
+    if ((long long)q_offset + Lq > Lk)
+        return fail(IC_ERR_INVALID_ARG, "q_offset + Lq = %lld exceeds Lk = %d",
+                    (long long)q_offset + Lq, Lk);
+    return IC_OK;
+}
+
+}  // namespace
+
+// ======================================================================= C ABI
+
+extern "C" {
+
+const char* ic_status_string(int status) {
+    switch (status) {
+        case IC_OK: return "IC_OK";
+        case IC_ERR_INVALID_ARG: return "IC_ERR_INVALID_ARG";
+        case IC_ERR_UNSUPPORTED: return "IC_ERR_UNSUPPORTED";
+        case IC_ERR_NO_CACHED_INDICES: return "IC_ERR_NO_CACHED_INDICES";
+        case IC_ERR_WORKSPACE_TOO_SMALL: return "IC_ERR_WORKSPACE_TOO_SMALL";
+        case IC_ERR_CUDA: return "IC_ERR_CUDA";
+        case IC_ERR_TIMEOUT: return "IC_ERR_TIMEOUT";
+        default: return "IC_ERR_UNKNOWN";
+    }
+}
+
+const char* ic_last_error_message(void) { return g_msg; }
+
+int ic_get_last_device_error(ic_stream_t stream) {
+    cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    unsigned int v = 0;
+    e = cudaMemcpyFromSymbol(&v, ic::g_dev_error, sizeof v);
+    if (e != cudaSuccess) return cuda_fail(e, "read device error word");
+    if (v) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(ic::g_dev_error, &zero, sizeof zero);
+        if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
+    }
+    if (v & ic::DEV_ERR_TIMEOUT) return fail(IC_ERR_TIMEOUT, "a kernel wait timed out");
+    if (v & ic::DEV_ERR_BAD_INDEX)
+        return fail(IC_ERR_INVALID_ARG, "an attention index outside [0, t] was skipped");
+    return IC_OK;
+}
+
+int ic_indexer_scores(const uint16_t* q_idx, const uint16_t* k_idx, const float* w, int B,
+                      int Lq, int Lk, int H_I, int d_I, int q_offset, float* scores,
+                      ic_stream_t stream) {
+    int rc = check_positions(B, Lq, Lk, q_offset);
+    if (rc) return rc;
+    if ((rc = check_indexer_shape(H_I, d_I))) return rc;
+    if (B == 0 || Lq == 0) return IC_OK;
+    if (!q_idx || !k_idx || !w || !scores) return fail(IC_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(q_idx) || !aligned16(k_idx))
+        return fail(IC_ERR_UNSUPPORTED, "q_idx and k_idx must be 16-byte aligned");
+    if ((long long)Lq * H_I > (1LL << 31)) return fail(IC_ERR_UNSUPPORTED, "Lq*H_I too large");
+    int dev, sms;
+    if ((rc = device_setup(&dev, &sms))) return rc;
+    const IndexerGeom geo = indexer_geom(Lq, H_I);
+    return launch_indexer(q_idx, k_idx, w, B, Lq, Lk, H_I, d_I, q_offset, 0,
+                          (long long)B * geo.nqb, scores, Lk, true, sms,
+                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+int ic_topk_select(const float* scores, int B, int Lq, int Lk, int q_offset, int k, int32_t* idx,
+                   ic_stream_t stream) {
+    int rc = check_positions(B, Lq, Lk, q_offset);
+    if (rc) return rc;
+    if (k < 1) return fail(IC_ERR_INVALID_ARG, "k=%d", k);
+    if (B == 0 || Lq == 0) return IC_OK;
+    if (!scores || !idx) return fail(IC_ERR_INVALID_ARG, "null pointer");
+    int dev, sms;
+    if ((rc = device_setup(&dev, &sms))) return rc;
+    return launch_topk(scores, Lk, 0, (long long)B * Lq, Lq, Lk, q_offset, k, idx,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t ic_sparse_attn_workspace_bytes(int B, int Lq, int Hq, int d, int k_slots) {
+    if (B <= 0 || Lq <= 0 || Hq <= 0 || d <= 0 || k_slots <= 0) return 0;
+    int dev, sms;
+    if (device_setup(&dev, &sms)) sms = 148;
+    const long long n_rows = (long long)B * Lq;
+    return attn_ws_bytes(n_rows, attn_splits(n_rows, k_slots, sms), Hq, d);
+}
+
+int ic_sparse_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* idx,
+                   int B, int Lq, int Lk, int Hq, int Hkv, int d, int k_slots, int q_offset,
+                   float scale, uint16_t* out, float* lse, void* ws, size_t ws_bytes,
+                   ic_stream_t stream) {
+    int rc = check_positions(B, Lq, Lk, q_offset);
+    if (rc) return rc;
+    if ((rc = check_attn_shape(Hq, Hkv, d))) return rc;
+    if (k_slots < 1) return fail(IC_ERR_INVALID_ARG, "k=%d", k_slots);
+    if (B == 0 || Lq == 0) return IC_OK;
+    if (!q || !k || !v || !idx || !out) return fail(IC_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v))
+        return fail(IC_ERR_UNSUPPORTED, "q, k and v must be 16-byte aligned");
+    if (!std::isfinite(scale)) return fail(IC_ERR_INVALID_ARG, "scale is not finite");
+    int dev, sms;
+    if ((rc = device_setup(&dev, &sms))) return rc;
+    return launch_attn(q, k, v, idx, B, Lq, Lk, Hq, d, k_slots, q_offset, scale, out, lse, ws,
+                       ws_bytes, false, sms, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t ic_layer_stack_workspace_bytes(const ic_dims* dims, int n_layers, long long rows_per_chunk) {
+    if (!dims || n_layers < 1) return 0;
+    if (check_positions(dims->B, dims->Lq, dims->Lk, dims->q_offset) ||
+        check_indexer_shape(dims->H_I, dims->d_I) || dims->k < 1)
+        return 0;
+    const IndexerGeom geo = indexer_geom(std::max(dims->Lq, 1), dims->H_I);
+    const long long n_rows = (long long)dims->B * dims->Lq;
+    long long blocks = (long long)dims->B * geo.nqb;
+    if (rows_per_chunk > 0)
+        blocks = std::min(blocks, std::max(1LL, (rows_per_chunk + geo.QB - 1) / geo.QB));
+    const size_t scores = (size_t)blocks * geo.QB * (size_t)dims->Lk * sizeof(float);
+    const size_t attn = ic_sparse_attn_workspace_bytes(dims->B, dims->Lq, dims->Hq, dims->d, dims->k);
+    (void)n_rows;
+    return std::max(scores, attn);
+}
+
+static int stack_forward(const char* pattern, int n_layers, const ic_layer* layers,
+                         const ic_dims* dims, int32_t* idx_cache, void* ws, size_t ws_bytes,
+                         ic_stream_t stream, void* const* events) {
+    if (!pattern || !layers || !dims || !idx_cache || n_layers < 1)
+        return fail(IC_ERR_INVALID_ARG, "null argument or n_layers < 1");
+    if ((int)strnlen(pattern, (size_t)n_layers + 1) != n_layers)
+        return fail(IC_ERR_INVALID_ARG, "pattern length differs from n_layers=%d", n_layers);
+    for (int l = 0; l < n_layers; ++l) {
+        const char c = pattern[l];
+        if (c != 'F' && c != '1' && c != 'S' && c != '0')
+            return fail(IC_ERR_INVALID_ARG, "pattern[%d]='%c' is neither F/1 nor S/0", l, c);
+    }
+    if (pattern[0] == 'S' || pattern[0] == '0')
+        return fail(IC_ERR_NO_CACHED_INDICES,
+                    "layer 0 is Shared: no cached indices available before the first F layer");
+    const ic_dims& D = *dims;
+    int rc = check_positions(D.B, D.Lq, D.Lk, D.q_offset);
+    if (rc) return rc;
+    if ((rc = check_indexer_shape(D.H_I, D.d_I))) return rc;
+    if ((rc = check_attn_shape(D.Hq, D.Hkv, D.d))) return rc;
+    if (D.k < 1 || D.k > D.Lk) return fail(IC_ERR_INVALID_ARG, "k=%d outside [1, Lk]", D.k);
+    if (!std::isfinite(D.scale)) return fail(IC_ERR_INVALID_ARG, "scale is not finite");
+    for (int l = 0; l < n_layers; ++l) {
+        const ic_layer& L = layers[l];
+        const bool full = pattern[l] == 'F' || pattern[l] == '1';
+        if (!L.q || !L.k || !L.v || !L.out)
+            return fail(IC_ERR_INVALID_ARG, "layer %d: null q/k/v/out", l);
+        if (!aligned16(L.q) || !aligned16(L.k) || !aligned16(L.v))
+            return fail(IC_ERR_UNSUPPORTED, "layer %d: q, k, v must be 16-byte aligned", l);
+        if (full) {
+            if (!L.q_idx || !L.k_idx || !L.w)
+                return fail(IC_ERR_INVALID_ARG, "layer %d is F but q_idx/k_idx/w is null", l);
+            if (!aligned16(L.q_idx) || !aligned16(L.k_idx))
+                return fail(IC_ERR_UNSUPPORTED, "layer %d: q_idx, k_idx must be 16-byte aligned", l);
+        }
+    }
+    if (D.B == 0 || D.Lq == 0) return IC_OK;
+    if ((long long)D.Lq * D.H_I > (1LL << 31)) return fail(IC_ERR_UNSUPPORTED, "Lq*H_I too large");
+    int dev, sms;
+    if ((rc = device_setup(&dev, &sms))) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+    const IndexerGeom geo = indexer_geom(D.Lq, D.H_I);
+    const long long n_blocks = (long long)D.B * geo.nqb;
+    const long long n_rows = (long long)D.B * D.Lq;
+    const size_t block_bytes = (size_t)geo.QB * (size_t)D.Lk * sizeof(float);
+    if (!ws || ws_bytes < block_bytes)
+        return fail(IC_ERR_WORKSPACE_TOO_SMALL,
+                    "workspace of %zu bytes is below one query block of scores (%zu bytes)",
+                    ws_bytes, block_bytes);
+    const long long blocks_per_chunk = std::min<long long>(n_blocks, (long long)(ws_bytes / block_bytes));
+    float* sc = reinterpret_cast<float*>(ws);
+
+    auto mark = [&](int l, int slot) -> int {
+        if (!events || !events[4 * l + slot]) return IC_OK;
+        cudaError_t e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(events[4 * l + slot]), st);
+        return e == cudaSuccess ? IC_OK : cuda_fail(e, "cudaEventRecord");
+    };
+    const bool one_chunk = blocks_per_chunk >= n_blocks;
+    for (int l = 0; l < n_layers; ++l) {
+        const ic_layer& L = layers[l];
+        const bool full = pattern[l] == 'F' || pattern[l] == '1';
+        if ((rc = mark(l, 0))) return rc;
+        if (full) {
+            for (long long g0 = 0; g0 < n_blocks; g0 += blocks_per_chunk) {
+                const long long g1 = std::min(n_blocks, g0 + blocks_per_chunk);
+                rc = launch_indexer(L.q_idx, L.k_idx, L.w, D.B, D.Lq, D.Lk, D.H_I, D.d_I,
+                                    D.q_offset, g0, g1, sc, D.Lk, false, sms, st);
+                if (rc) return rc;
+                if (one_chunk && (rc = mark(l, 1))) return rc;
+                const long long r0 = block_row_start(geo, D.Lq, g0);
+                const long long r1 = block_row_start(geo, D.Lq, g1);
+                rc = launch_topk(sc, D.Lk, r0, r1 - r0, D.Lq, D.Lk, D.q_offset, D.k, idx_cache, st);
+                if (rc) return rc;
+            }
+        }
+        if (!(full && one_chunk) && (rc = mark(l, 1))) return rc;
+        if ((rc = mark(l, 2))) return rc;
+        rc = launch_attn(L.q, L.k, L.v, idx_cache, D.B, D.Lq, D.Lk, D.Hq, D.d, D.k, D.q_offset,
+                         D.scale, L.out, L.lse, ws, ws_bytes, true, sms, st);
+        if (rc) return rc;
+        if ((rc = mark(l, 3))) return rc;
+        if (L.idx_dump) {
+            cudaError_t e = cudaMemcpyAsync(L.idx_dump, idx_cache,
+                                            (size_t)n_rows * D.k * sizeof(int32_t),
+                                            cudaMemcpyDeviceToDevice, st);
+            if (e != cudaSuccess) return cuda_fail(e, "idx_dump copy");
+        }
+    }
+    return IC_OK;
+}
+
+int ic_layer_stack_forward(const char* pattern, int n_layers, const ic_layer* layers,
+                           const ic_dims* dims, int32_t* idx_cache, void* ws, size_t ws_bytes,
+                           ic_stream_t stream) {
+    return stack_forward(pattern, n_layers, layers, dims, idx_cache, ws, ws_bytes, stream, nullptr);
+}
+
+int ic_layer_stack_forward_events(const char* pattern, int n_layers, const ic_layer* layers,
+                                  const ic_dims* dims, int32_t* idx_cache, void* ws,
+                                  size_t ws_bytes, ic_stream_t stream, void* const* events) {
+    return stack_forward(pattern, n_layers, layers, dims, idx_cache, ws, ws_bytes, stream, events);
+}
+
+}  // extern "C"

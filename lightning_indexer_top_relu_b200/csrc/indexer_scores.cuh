@@ -1,0 +1,302 @@
+// Lightning indexer scores on the 5th-generation tensor cores (sm_100a).
+//
+// Computes, for query rows t and visible keys s <= t,
+//     score[t, s] = sum_j w[t, j] * max(0, q_I[t, j] . k_I[s])
+// (the IndexCache papers describe the indexer as scoring every preceding
+// token of the query; the score form is the standard lightning-indexer one,
+// which the pages do not print).
+//
+// Tile mapping.  Keys sit on the MMA M axis (128 TMEM lanes) and
+// (query, head) pairs on N: one tcgen05.mma of M=128, N=QB*H_I (<= 256),
+// K=d_I computes q_I[t,j] . k_I[s] for 128 keys x QB queries x H_I heads.
+// The epilogue thread that owns TMEM lane s then holds every head of every
+// query of the block for key s, so the ReLU and the w-weighted head sum are
+// a per-thread register reduction, and the score stores run along s
+// (coalesced).
+//
+// Pipeline (one persistent CTA per SM, warp-specialised):
+//   warp 0      TMA producer: the query block (B operand, once per work
+//               unit, double-buffered) and k_I tiles (A operand, 3-stage ring)
+//   warp 1      TMEM allocator + single-thread MMA issuer
+//   warps 2..5  epilogue: tcgen05.ld -> ReLU -> w-weighted head sum -> causal
+//               mask -> fp32 score stores; two TMEM accumulators (2 x 256
+//               columns) let the epilogue of tile j overlap the MMA of j+1.
+// A work unit is (query block, run of up to `tpu` key tiles); units are
+// walked longest-causal-row first and dealt round-robin to the CTAs.
+#pragma once
+
+#include "common.cuh"
+
+namespace ic {
+
+constexpr int IDX_BM = 128;          // keys per tile = TMEM lanes
+constexpr int IDX_NMAX = 256;        // max (query, head) columns per MMA
+constexpr int IDX_STAGES = 3;        // k_I tile ring depth
+constexpr int IDX_EPI_WARPS = 4;
+constexpr int IDX_THREADS = 64 + 32 * IDX_EPI_WARPS;
+
+struct IndexerArgs {
+    const float* w;        // [B, Lq, H]
+    float* scores;         // row (flattened query row - row_base), stride ld
+    long long ld;
+    int B, Lq, Lk, q_offset;
+    int QB;                // queries per block
+    int N;                 // MMA N (QB*H rounded up to 16)
+    int nqb;               // query blocks per batch element
+    int g0, g1;            // flattened query-block range of this launch
+    long long row_base;    // flattened row of the first row of block g0
+    int tpu;               // key tiles per work unit
+    int max_splits;        // work units per query block (some may be empty)
+};
+
+template <int DI>
+struct IndexerSmem {
+    static constexpr int Q_BYTES = IDX_NMAX * DI * 2;     // one query block
+    static constexpr int A_BYTES = IDX_BM * DI * 2;       // one k_I tile
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_A = OFF_Q + 2 * Q_BYTES;
+    static constexpr int OFF_BAR = OFF_A + IDX_STAGES * A_BYTES;
+    static constexpr int N_BARS = 2 + 2 + IDX_STAGES + IDX_STAGES + 2 + 2;
+    static constexpr int OFF_SLOT = OFF_BAR + N_BARS * 8;
+    static constexpr int BYTES = OFF_SLOT + 16;
+    // 1024 B of slack for the 1024-B alignment of the swizzled tiles; never
+    // less than 120 KB so that two CTAs (each holding all 512 TMEM columns)
+    // can never share an SM and wait on each other's allocation.
+    static constexpr int ALLOC = (BYTES + 1024) > 120 * 1024 ? (BYTES + 1024) : 120 * 1024;
+};
+
+struct UnitInfo {
+    int b, i0, nq, j0, j1;
+};
+
+__device__ __forceinline__ UnitInfo unit_info(const IndexerArgs& a, long long u) {
+    UnitInfo r;
+    int g = a.g1 - 1 - (int)(u / a.max_splits);
+    int split = (int)(u % a.max_splits);
+    r.b = g / a.nqb;
+    r.i0 = (g % a.nqb) * a.QB;
+    r.nq = min(a.QB, a.Lq - r.i0);
+    int t_last = a.q_offset + r.i0 + r.nq - 1;
+    int n_vis = min(t_last + 1, a.Lk);
+    int nt = (n_vis + IDX_BM - 1) / IDX_BM;
+    r.j0 = split * a.tpu;
+    r.j1 = min(r.j0 + a.tpu, nt);
+    return r;
+}
+
+template <int H, int DI>
+__global__ void __launch_bounds__(IDX_THREADS, 1)
+indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                      const __grid_constant__ CUtensorMap tmap_k, const IndexerArgs args) {
+    using S = IndexerSmem<DI>;
+    constexpr int KBOX = DI / 64;                 // 64-element (128-byte) swizzle boxes along d_I
+    constexpr int QBMAX = IDX_NMAX / H;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    uint8_t* q_s = smem + S::OFF_Q;
+    uint8_t* a_s = smem + S::OFF_A;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
+    uint64_t* q_full = bars;
+    uint64_t* q_empty = bars + 2;
+    uint64_t* a_full = bars + 4;
+    uint64_t* a_empty = a_full + IDX_STAGES;
+    uint64_t* acc_full = a_empty + IDX_STAGES;
+    uint64_t* acc_empty = acc_full + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::OFF_SLOT);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const long long n_units = (long long)(args.g1 - args.g0) * args.max_splits;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&q_full[i], 1);
+            mbar_init(&q_empty[i], 1);
+            mbar_init(&acc_full[i], 1);
+            mbar_init(&acc_empty[i], 32 * IDX_EPI_WARPS);
+        }
+        for (int i = 0; i < IDX_STAGES; ++i) {
+            mbar_init(&a_full[i], 1);
+            mbar_init(&a_empty[i], 1);
+        }
+        fence_barrier_init();
+        tma_prefetch_desc(&tmap_q);
+        tma_prefetch_desc(&tmap_k);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer
+            const uint32_t q_bytes = (uint32_t)args.N * 128u * KBOX;
+            const uint32_t a_bytes = (uint32_t)S::A_BYTES;
+            uint32_t uq = 0, ta = 0;
+            bool ok = true;
+            for (long long u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+                UnitInfo ui = unit_info(args, u);
+                if (ui.j0 >= ui.j1) continue;
+                const int qb = uq & 1;
+                if (!mbar_wait(&q_empty[qb], ((uq >> 1) & 1) ^ 1)) { ok = false; break; }
+                mbar_arrive_expect_tx(&q_full[qb], q_bytes);
+                uint8_t* qdst = q_s + qb * S::Q_BYTES;
+                for (int kb = 0; kb < KBOX; ++kb)
+                    tma_load_3d(qdst + kb * args.N * 128, &tmap_q, &q_full[qb], kb * 64, ui.i0 * H,
+                                ui.b);
+                ++uq;
+                for (int j = ui.j0; j < ui.j1; ++j, ++ta) {
+                    const int st = ta % IDX_STAGES;
+                    if (!mbar_wait(&a_empty[st], ((ta / IDX_STAGES) & 1) ^ 1)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&a_full[st], a_bytes);
+                    uint8_t* adst = a_s + st * S::A_BYTES;
+                    for (int kb = 0; kb < KBOX; ++kb)
+                        tma_load_3d(adst + kb * IDX_BM * 128, &tmap_k, &a_full[st], kb * 64,
+                                    j * IDX_BM, ui.b);
+                }
+            }
+            // Drain: every load issued has landed before the CTA may retire.
+            for (uint32_t i = (uq > 2 ? uq - 2 : 0); i < uq; ++i)
+                mbar_wait(&q_full[i & 1], (i >> 1) & 1);
+            for (uint32_t i = (ta > IDX_STAGES ? ta - IDX_STAGES : 0); i < ta; ++i)
+                mbar_wait(&a_full[i % IDX_STAGES], (i / IDX_STAGES) & 1);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------- MMA issuer
+            const uint32_t idesc = idesc_bf16_f32(IDX_BM, args.N);
+            uint32_t uq = 0, ta = 0;
+            bool ok = true;
+            for (long long u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+                UnitInfo ui = unit_info(args, u);
+                if (ui.j0 >= ui.j1) continue;
+                const int qb = uq & 1;
+                if (!mbar_wait(&q_full[qb], (uq >> 1) & 1)) { ok = false; break; }
+                const uint32_t q_addr = smem_u32(q_s + qb * S::Q_BYTES);
+                for (int j = ui.j0; j < ui.j1; ++j, ++ta) {
+                    const int st = ta % IDX_STAGES;
+                    const int ab = ta & 1;
+                    if (!mbar_wait(&a_full[st], (ta / IDX_STAGES) & 1)) { ok = false; break; }
+                    if (!mbar_wait(&acc_empty[ab], ((ta >> 1) & 1) ^ 1)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(a_s + st * S::A_BYTES);
+                    const uint32_t d_tmem = tmem_base + (uint32_t)(ab * IDX_NMAX);
+#pragma unroll
+                    for (int kk = 0; kk < DI / 16; ++kk) {
+                        const uint32_t koff = (uint32_t)((kk & 3) * 32);
+                        const uint64_t ad =
+                            sw128_kmajor_desc(a_addr + (kk >> 2) * IDX_BM * 128 + koff);
+                        const uint64_t bd =
+                            sw128_kmajor_desc(q_addr + (kk >> 2) * args.N * 128 + koff);
+                        tc_mma_f16(d_tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
+                    }
+                    tc_commit(&a_empty[st]);
+                    tc_commit(&acc_full[ab]);
+                }
+                if (!ok) break;
+                tc_commit(&q_empty[qb]);
+                ++uq;
+            }
+        }
+    } else {
+        // ---------------- epilogue (warps 2..5)
+        const int wq = warp & 3;                  // TMEM lane quarter this warp may read
+        const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
+        uint32_t ta = 0;
+        bool ok = true;
+        for (long long u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+            UnitInfo ui = unit_info(args, u);
+            if (ui.j0 >= ui.j1) continue;
+            // Head weights of this query block (the same for every key).  Read
+            // through L1 by all threads (broadcast); no block barrier here, so a
+            // thread whose bounded wait gives up can never strand the others.
+            const float* wsrc = args.w + ((long long)ui.b * args.Lq + ui.i0) * H;
+            const int wvalid = ui.nq * H;
+
+            const long long row0 = (long long)ui.b * args.Lq + ui.i0 - args.row_base;
+            const int t0 = args.q_offset + ui.i0;
+            for (int j = ui.j0; j < ui.j1; ++j, ++ta) {
+                const int ab = ta & 1;
+                if (!mbar_wait(&acc_full[ab], (ta >> 1) & 1)) { ok = false; break; }
+                tc_fence_after();
+                float acc[QBMAX];
+#pragma unroll
+                for (int q = 0; q < QBMAX; ++q) acc[q] = 0.0f;
+                const uint32_t taddr = tmem_base + lane_base + (uint32_t)(ab * IDX_NMAX);
+#pragma unroll
+                for (int cc = 0; cc < IDX_NMAX / 32; ++cc) {
+                    if (cc * 32 < args.N) {
+                        float wc[32];
+#pragma unroll
+                        for (int jj = 0; jj < 32; jj += 4) {
+                            const int c = cc * 32 + jj;
+                            const float4 wv = c < wvalid
+                                ? __ldg(reinterpret_cast<const float4*>(wsrc + c))
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+                            wc[jj] = wv.x; wc[jj + 1] = wv.y; wc[jj + 2] = wv.z; wc[jj + 3] = wv.w;
+                        }
+                        uint32_t v[32];
+                        tmem_ld_32x32b_x32(taddr + cc * 32, v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int jj = 0; jj < 32; jj += 4) {
+                            const float wj[4] = {wc[jj], wc[jj + 1], wc[jj + 2], wc[jj + 3]};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int q = (cc * 32 + jj + e) / H;
+                                acc[q] = fmaf(wj[e], fmaxf(__uint_as_float(v[jj + e]), 0.0f), acc[q]);
+                            }
+                        }
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&acc_empty[ab]);
+                const int s = j * IDX_BM + wq * 32 + lane;
+                if (s < args.Lk) {
+                    float* dst = args.scores + row0 * args.ld + s;
+#pragma unroll
+                    for (int q = 0; q < QBMAX; ++q) {
+                        if (q < ui.nq) {
+                            const float val = (s <= t0 + q) ? acc[q] : -INFINITY;
+                            dst[(long long)q * args.ld] = val;
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, 512);
+    }
+}
+
+// Writes -inf into score columns [ntiles*128, Lk) of each row: the part of a
+// row beyond the key tiles the indexer visited, all of it invisible.
+__global__ void indexer_fill_masked_kernel(float* scores, long long ld, int Lq, int Lk,
+                                           int q_offset, int QB, long long row_base,
+                                           long long n_rows) {
+    for (long long row = blockIdx.x; row < n_rows; row += gridDim.x) {
+        long long fr = row_base + row;
+        int i = (int)(fr % Lq);
+        int i0 = (i / QB) * QB;
+        int nq = min(QB, Lq - i0);
+        int t_last = q_offset + i0 + nq - 1;
+        int n_vis = min(t_last + 1, Lk);
+        int start = ((n_vis + IDX_BM - 1) / IDX_BM) * IDX_BM;
+        float* dst = scores + row * ld;
+        for (int s = start + threadIdx.x; s < Lk; s += blockDim.x) dst[s] = -INFINITY;
+    }
+}
+
+}  // namespace ic

@@ -1,0 +1,227 @@
+"""ctypes binding of libindexcache.so (argument marshalling only).
+
+Every function here takes torch CUDA tensors, checks dtype/shape/contiguity,
+and passes raw device pointers to the C ABI of the same name
+(include/indexcache.h).  No step of the computation happens in Python, and
+there is no fallback: importing this module fails loudly when the CUDA
+library has not been built, and each call raises IndexCacheError on a
+non-zero status.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libindexcache.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m lightning_indexer_top_relu_b200.build` "
+        "(there is no CPU fallback)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+IC_OK = 0
+STATUS = {0: "IC_OK", 1: "IC_ERR_INVALID_ARG", 2: "IC_ERR_UNSUPPORTED",
+          3: "IC_ERR_NO_CACHED_INDICES", 4: "IC_ERR_WORKSPACE_TOO_SMALL", 5: "IC_ERR_CUDA",
+          6: "IC_ERR_TIMEOUT"}
+EXPORTS = ("ic_status_string", "ic_last_error_message", "ic_get_last_device_error",
+           "ic_indexer_scores", "ic_topk_select", "ic_sparse_attn",
+           "ic_sparse_attn_workspace_bytes", "ic_layer_stack_workspace_bytes",
+           "ic_layer_stack_forward")
+
+
+class IndexCacheError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _lib.ic_last_error_message().decode(errors="replace")
+        super().__init__(f"{where}: {STATUS.get(status, status)}: {msg}")
+
+
+class NoCachedIndices(IndexCacheError):
+    pass
+
+
+class ICLayer(ctypes.Structure):
+    _fields_ = [("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+                ("q_idx", ctypes.c_void_p), ("k_idx", ctypes.c_void_p), ("w", ctypes.c_void_p),
+                ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p), ("idx_dump", ctypes.c_void_p)]
+
+
+class ICDims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Lq", ctypes.c_int), ("Lk", ctypes.c_int),
+                ("q_offset", ctypes.c_int), ("H_I", ctypes.c_int), ("d_I", ctypes.c_int),
+                ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int), ("d", ctypes.c_int),
+                ("k", ctypes.c_int), ("scale", ctypes.c_float)]
+
+
+_P, _I, _F, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+_lib.ic_status_string.restype = ctypes.c_char_p
+_lib.ic_status_string.argtypes = [_I]
+_lib.ic_last_error_message.restype = ctypes.c_char_p
+_lib.ic_last_error_message.argtypes = []
+_lib.ic_get_last_device_error.restype = _I
+_lib.ic_get_last_device_error.argtypes = [_P]
+_lib.ic_indexer_scores.restype = _I
+_lib.ic_indexer_scores.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P]
+_lib.ic_topk_select.restype = _I
+_lib.ic_topk_select.argtypes = [_P, _I, _I, _I, _I, _I, _P, _P]
+_lib.ic_sparse_attn.restype = _I
+_lib.ic_sparse_attn.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P,
+                                _Z, _P]
+_lib.ic_sparse_attn_workspace_bytes.restype = _Z
+_lib.ic_sparse_attn_workspace_bytes.argtypes = [_I, _I, _I, _I, _I]
+_lib.ic_layer_stack_workspace_bytes.restype = _Z
+_lib.ic_layer_stack_workspace_bytes.argtypes = [ctypes.POINTER(ICDims), _I, ctypes.c_longlong]
+_lib.ic_layer_stack_forward.restype = _I
+_lib.ic_layer_stack_forward.argtypes = [ctypes.c_char_p, _I, ctypes.POINTER(ICLayer),
+                                        ctypes.POINTER(ICDims), _P, _P, _Z, _P]
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+def _check(rc: int, where: str):
+    if rc != IC_OK:
+        if rc == 3:
+            raise NoCachedIndices(rc, where)
+        raise IndexCacheError(rc, where)
+
+
+def _ptr(t: Optional[torch.Tensor], dtype=None, name="tensor") -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def get_last_device_error(stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the device error status."""
+    return int(_lib.ic_get_last_device_error(_stream(stream)))
+
+
+def indexer_scores(q_idx, k_idx, w, q_offset: int = 0, out=None, stream=None) -> torch.Tensor:
+    """scores [B,Lq,Lk] fp32 from q_idx [B,Lq,H_I,d_I] bf16, k_idx [B,Lk,d_I] bf16, w [B,Lq,H_I] fp32."""
+    B, Lq, H, dI = q_idx.shape
+    Lk = k_idx.shape[1]
+    if out is None:
+        out = torch.empty(B, Lq, Lk, device=q_idx.device, dtype=torch.float32)
+    rc = _lib.ic_indexer_scores(_ptr(q_idx, torch.bfloat16, "q_idx"), _ptr(k_idx, torch.bfloat16, "k_idx"),
+                                _ptr(w, torch.float32, "w"), B, Lq, Lk, H, dI, q_offset,
+                                _ptr(out, torch.float32, "scores"), _stream(stream))
+    _check(rc, "ic_indexer_scores")
+    return out
+
+
+def topk_select(scores, k: int, q_offset: int = 0, out=None, stream=None) -> torch.Tensor:
+    """idx [B,Lq,k] int32 (ascending positions, -1 padded) from scores [B,Lq,Lk] fp32."""
+    B, Lq, Lk = scores.shape
+    if out is None:
+        out = torch.empty(B, Lq, k, device=scores.device, dtype=torch.int32)
+    rc = _lib.ic_topk_select(_ptr(scores, torch.float32, "scores"), B, Lq, Lk, q_offset, k,
+                             _ptr(out, torch.int32, "idx"), _stream(stream))
+    _check(rc, "ic_topk_select")
+    return out
+
+
+def sparse_attn_workspace_bytes(B: int, Lq: int, Hq: int, d: int, k: int) -> int:
+    return int(_lib.ic_sparse_attn_workspace_bytes(B, Lq, Hq, d, k))
+
+
+def sparse_attn(q, k, v, idx, q_offset: int = 0, scale: float = 0.0, out=None, lse=None,
+                want_lse: bool = True, ws=None, stream=None):
+    """(out [B,Lq,Hq,d] bf16, lse [B,Lq,Hq] fp32) over the positions in idx [B,Lq,k] int32."""
+    B, Lq, Hq, d = q.shape
+    Lk = k.shape[1]
+    Hkv = k.shape[2] if k.dim() == 4 else 1
+    kslots = idx.shape[-1]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(B, Lq, Hq, device=q.device, dtype=torch.float32)
+    if ws is None:
+        nbytes = sparse_attn_workspace_bytes(B, Lq, Hq, d, kslots)
+        ws = torch.empty(max(nbytes, 1), device=q.device, dtype=torch.uint8) if nbytes else None
+    rc = _lib.ic_sparse_attn(_ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
+                             _ptr(v, torch.bfloat16, "v"), _ptr(idx, torch.int32, "idx"), B, Lq,
+                             Lk, Hq, Hkv, d, kslots, q_offset, float(scale),
+                             _ptr(out, torch.bfloat16, "out"), _ptr(lse, torch.float32, "lse"),
+                             _ptr(ws, None, "ws"), 0 if ws is None else ws.numel() * ws.element_size(),
+                             _stream(stream))
+    _check(rc, "ic_sparse_attn")
+    return out, lse
+
+
+def make_dims(B, Lq, Lk, q_offset, H_I, d_I, Hq, d, k, scale=0.0, Hkv=1) -> ICDims:
+    return ICDims(B, Lq, Lk, q_offset, H_I, d_I, Hq, Hkv, d, k, float(scale))
+
+
+def layer_stack_workspace_bytes(dims: ICDims, n_layers: int, rows_per_chunk: int = 0) -> int:
+    return int(_lib.ic_layer_stack_workspace_bytes(ctypes.byref(dims), n_layers, rows_per_chunk))
+
+
+class LayerStack:
+    """Holds the C layer table for repeated ic_layer_stack_forward calls.
+
+    layers: per layer a dict with 'q','k','v' (and 'q_idx','k_idx','w' for F
+    layers) CUDA tensors; outputs are allocated once here.
+    """
+
+    def __init__(self, pattern: str, layers: Sequence[dict], dims: ICDims, *, want_lse=False,
+                 dump_idx=False, ws_bytes: Optional[int] = None, rows_per_chunk: int = 0):
+        self.pattern = pattern
+        self.dims = dims
+        n = len(layers)
+        dev = layers[0]["q"].device
+        self.layers = list(layers)
+        self.outs = [torch.empty_like(L["q"]) for L in layers]
+        self.lses = [torch.empty(dims.B, dims.Lq, dims.Hq, device=dev, dtype=torch.float32)
+                     if want_lse else None for _ in layers]
+        self.dumps = [torch.empty(dims.B, dims.Lq, dims.k, device=dev, dtype=torch.int32)
+                      if dump_idx else None for _ in layers]
+        self.idx_cache = torch.empty(dims.B, dims.Lq, dims.k, device=dev, dtype=torch.int32)
+        if ws_bytes is None:
+            ws_bytes = layer_stack_workspace_bytes(dims, n, rows_per_chunk)
+        self.ws = torch.empty(max(int(ws_bytes), 16), device=dev, dtype=torch.uint8)
+        self.table = (ICLayer * n)()
+        for i, L in enumerate(layers):
+            full = pattern[i] in "F1" if i < len(pattern) else False
+            self.table[i] = ICLayer(
+                _ptr(L["q"], torch.bfloat16, "q"), _ptr(L["k"], torch.bfloat16, "k"),
+                _ptr(L["v"], torch.bfloat16, "v"),
+                _ptr(L.get("q_idx"), torch.bfloat16, "q_idx") if full else None,
+                _ptr(L.get("k_idx"), torch.bfloat16, "k_idx") if full else None,
+                _ptr(L.get("w"), torch.float32, "w") if full else None,
+                _ptr(self.outs[i], torch.bfloat16, "out"),
+                _ptr(self.lses[i], torch.float32, "lse"), _ptr(self.dumps[i], torch.int32, "dump"))
+        self._pattern_b = pattern.encode()
+
+    def forward(self, stream=None):
+        rc = _lib.ic_layer_stack_forward(self._pattern_b, len(self.layers), self.table,
+                                         ctypes.byref(self.dims), _ptr(self.idx_cache),
+                                         _ptr(self.ws), self.ws.numel(), _stream(stream))
+        _check(rc, "ic_layer_stack_forward")
+        return self.outs
+
+
+def layer_stack_forward(pattern: str, layers: Sequence[dict], dims: ICDims, **kw):
+    """One-shot helper: builds a LayerStack and runs it once."""
+    st = LayerStack(pattern, layers, dims, **kw)
+    st.forward()
+    return st

@@ -1,0 +1,120 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every function include/indexcache.h declares, and rejects bad arguments
+before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from lightning_indexer_top_relu_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "indexcache.h")
+
+
+@pytest.fixture(scope="module")
+def ic():
+    build.build()
+    from lightning_indexer_top_relu_b200 import indexcache
+    return indexcache
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b(ic_[a-z0-9_]+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_header_declares_the_four_steps():
+    names = declared_functions()
+    for n in ("ic_indexer_scores", "ic_topk_select", "ic_sparse_attn", "ic_layer_stack_forward"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(ic):
+    lib = ctypes.CDLL(ic.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+    assert set(ic.EXPORTS) <= set(declared_functions())
+
+
+def test_status_strings(ic):
+    lib = ic.lib()
+    for code, name in ic.STATUS.items():
+        assert lib.ic_status_string(code).decode() == name
+
+
+def _dims(ic, **kw):
+    base = dict(B=1, Lq=64, Lk=64, q_offset=0, H_I=4, d_I=64, Hq=8, d=64, k=8)
+    base.update(kw)
+    return ic.make_dims(**base)
+
+
+def _stack_call(ic, pattern, dims, n_layers=None, table=None):
+    n = len(pattern) if n_layers is None else n_layers
+    if table is None:
+        table = (ic.ICLayer * max(n, 1))()
+        for i in range(max(n, 1)):
+            # fake, 16-byte aligned non-null device addresses: validation must
+            # reject the call before anything dereferences them
+            table[i] = ic.ICLayer(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, 0x7000, None, None)
+    return ic.lib().ic_layer_stack_forward(pattern.encode(), n, table, ctypes.byref(dims), 0x8000,
+                                           0x9000, 1 << 20, None)
+
+
+def test_leading_shared_layer_is_rejected_before_launch(ic):
+    d = _dims(ic)
+    assert _stack_call(ic, "SFSS", d) == 3          # IC_ERR_NO_CACHED_INDICES
+    assert _stack_call(ic, "0111", d) == 3
+    assert b"Shared" in ic.lib().ic_last_error_message()
+
+
+def test_bad_pattern_and_lengths(ic):
+    d = _dims(ic)
+    assert _stack_call(ic, "FXSS", d) == 1
+    assert _stack_call(ic, "FSS", d, n_layers=4) == 1   # strlen != n_layers
+    assert _stack_call(ic, "F", d, n_layers=0) == 1
+
+
+def test_unsupported_shapes(ic):
+    assert _stack_call(ic, "FS", _dims(ic, d_I=96)) == 2
+    assert _stack_call(ic, "FS", _dims(ic, H_I=6)) == 2
+    assert _stack_call(ic, "FS", _dims(ic, d=80)) == 2
+    assert _stack_call(ic, "FS", _dims(ic, Hq=12)) == 2
+    d = _dims(ic)
+    d.Hkv = 2
+    assert _stack_call(ic, "FS", d) == 2
+
+
+def test_bad_sizes(ic):
+    assert _stack_call(ic, "FS", _dims(ic, k=0)) == 1
+    assert _stack_call(ic, "FS", _dims(ic, k=65)) == 1          # k > Lk
+    assert _stack_call(ic, "FS", _dims(ic, Lq=64, Lk=32)) == 1   # q_offset + Lq > Lk
+    assert _stack_call(ic, "FS", _dims(ic, q_offset=-1)) == 1
+    lib = ic.lib()
+    assert lib.ic_topk_select(0x1000, 1, 4, 4, 0, 0, 0x2000, None) == 1       # k = 0
+    assert lib.ic_indexer_scores(None, 0x1000, 0x2000, 1, 4, 4, 4, 64, 0, 0x3000, None) == 1
+    assert lib.ic_indexer_scores(0x1008, 0x1000, 0x2000, 1, 4, 4, 4, 64, 0, 0x3000, None) == 2
+    assert lib.ic_sparse_attn(0x1000, 0x1000, 0x1000, 0x1000, 1, 4, 4, 8, 1, 64, 0, 0, 0.0,
+                              0x1000, None, None, 0, None) == 1             # k = 0
+
+
+def test_null_layer_tensors(ic):
+    table = (ic.ICLayer * 2)()
+    table[0] = ic.ICLayer(0x1000, 0x2000, 0x3000, None, 0x5000, 0x6000, 0x7000, None, None)
+    table[1] = ic.ICLayer(0x1000, 0x2000, 0x3000, None, None, None, 0x7000, None, None)
+    assert _stack_call(ic, "FS", _dims(ic), table=table) == 1   # F layer without q_idx
+    table[0] = ic.ICLayer(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, 0x7000, None, None)
+    table[1] = ic.ICLayer(0x1000, None, 0x3000, None, None, None, 0x7000, None, None)
+    assert _stack_call(ic, "FS", _dims(ic), table=table) == 1   # missing k
+
+
+def test_workspace_query(ic):
+    d = _dims(ic, Lq=512, Lk=512, H_I=4)
+    full = ic.layer_stack_workspace_bytes(d, 4)
+    assert full >= 512 * 512 * 4
+    one_block = ic.layer_stack_workspace_bytes(d, 4, rows_per_chunk=1)
+    assert 0 < one_block < full
+    assert ic.layer_stack_workspace_bytes(_dims(ic, d_I=96), 4) == 0
