@@ -148,10 +148,11 @@ def oracle_rows_per_s(wl, pattern, layers_cpu, budget_s=15.0, seed=5):
         dt = time.perf_counter() - t0
         elapsed += dt
         done += len(rows)
-        if elapsed >= budget_s or n >= total:
+        if elapsed >= 0.8 * budget_s or done >= total:
             break
-        # grow toward the budget
-        n = int(min(total, max(2 * n, n * (budget_s - elapsed) / max(dt, 1e-3))))
+        # next sample sized to land near the budget
+        rate = done / elapsed
+        n = int(min(total, max(8, rate * (budget_s - elapsed))))
     return done / elapsed, f"{done} uniformly drawn query rows of {total}, all {len(pattern)} layers, {elapsed:.1f} s"
 
 
@@ -203,8 +204,8 @@ def config_of(wl, pattern, args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
-    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="prefill_8k", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--pattern", default=None)
@@ -251,9 +252,10 @@ def main():
     # per-kernel marks: 4 events per layer per step
     def new_marks():
         evs = [torch.cuda.Event(enable_timing=True) for _ in range(4 * n)]
-        arr = (ctypes.c_void_p * (4 * n))(*[e.cuda_event for e in evs])
-        for e in evs:  # make sure the events exist before their handles are used
+        for e in evs:  # torch creates the CUDA event on first record
             e.record(stream)
+        arr = (ctypes.c_void_p * (4 * n))(*[e.cuda_event for e in evs])
+        assert all(arr), "CUDA event handles must exist before they are handed to the library"
         return evs, arr
 
     lib = ic.lib()

@@ -10,14 +10,33 @@
 
 namespace ic {
 
+// One error word per device, read and cleared by ic_get_last_device_error.
+static __device__ unsigned int g_dev_error;
+
 // Error bits a kernel ORs into the device error word (never a trap).
 enum : unsigned int {
     DEV_ERR_TIMEOUT = 1u,     // a bounded wait gave up
     DEV_ERR_BAD_INDEX = 2u,   // an attention index outside [0, t] (skipped)
+    DEV_ERR_SMEM = 4u,        // the 1024-aligned shared-memory layout did not fit (kernel skipped)
 };
 
-// One error word per device, read and cleared by ic_get_last_device_error.
-static __device__ unsigned int g_dev_error;
+constexpr int MAX_DYN_SMEM = 232448;          // 227 KB opt-in per CTA on sm_100
+
+// Aligns the dynamic shared memory base to 1024 bytes (128-byte swizzle
+// atoms).  Returns nullptr -- and reports DEV_ERR_SMEM -- when `bytes` from
+// the aligned base would run past the launch's dynamic allocation; callers
+// then return before touching shared memory.
+__device__ __forceinline__ uint8_t* align_smem_1024(uint8_t* raw, uint32_t bytes) {
+    uint32_t dyn;
+    asm volatile("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn));
+    const uintptr_t p = reinterpret_cast<uintptr_t>(raw);
+    const uintptr_t q = (p + 1023) & ~uintptr_t(1023);
+    if ((uint32_t)(q - p) + bytes > dyn) {
+        if (threadIdx.x == 0) atomicOr(&g_dev_error, DEV_ERR_SMEM);
+        return nullptr;
+    }
+    return reinterpret_cast<uint8_t*>(q);
+}
 
 // Every spin-wait gives up after this many nanoseconds of %globaltimer.
 constexpr unsigned long long WAIT_LIMIT_NS = 2000000000ull;
@@ -94,6 +113,16 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
         "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// 1-D bulk copy global -> this CTA's shared memory (16-byte aligned, size a
+// multiple of 16), completing on an mbarrier's transaction count.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
 }
 

@@ -15,12 +15,16 @@
 // (coalesced).
 //
 // Pipeline (one persistent CTA per SM, warp-specialised):
-//   warp 0      TMA producer: the query block (B operand, once per work
-//               unit, double-buffered) and k_I tiles (A operand, 3-stage ring)
+//   warp 0      TMA producer: the query block (B operand) and its head
+//               weights w (bulk copy), once per work unit, double-buffered;
+//               k_I tiles (A operand) through a 3-stage ring
 //   warp 1      TMEM allocator + single-thread MMA issuer
-//   warps 2..5  epilogue: tcgen05.ld -> ReLU -> w-weighted head sum -> causal
-//               mask -> fp32 score stores; two TMEM accumulators (2 x 256
-//               columns) let the epilogue of tile j overlap the MMA of j+1.
+//   warps 2..9  epilogue: tcgen05.ld -> ReLU -> w-weighted head sum -> causal
+//               mask -> fp32 score stores.  Warp w reads TMEM lane quarter
+//               w % 4 and the half of the block's queries given by (w-2) / 4,
+//               so two warps share each SM sub-partition.  Two TMEM
+//               accumulators (2 x 256 columns) let the epilogue of tile j
+//               overlap the MMA of tile j+1.
 // A work unit is (query block, run of up to `tpu` key tiles); units are
 // walked longest-causal-row first and dealt round-robin to the CTAs.
 #pragma once
@@ -32,7 +36,7 @@ namespace ic {
 constexpr int IDX_BM = 128;          // keys per tile = TMEM lanes
 constexpr int IDX_NMAX = 256;        // max (query, head) columns per MMA
 constexpr int IDX_STAGES = 3;        // k_I tile ring depth
-constexpr int IDX_EPI_WARPS = 4;
+constexpr int IDX_EPI_WARPS = 8;
 constexpr int IDX_THREADS = 64 + 32 * IDX_EPI_WARPS;
 
 struct IndexerArgs {
@@ -55,14 +59,18 @@ struct IndexerSmem {
     static constexpr int A_BYTES = IDX_BM * DI * 2;       // one k_I tile
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_A = OFF_Q + 2 * Q_BYTES;
-    static constexpr int OFF_BAR = OFF_A + IDX_STAGES * A_BYTES;
+    static constexpr int OFF_W = OFF_A + IDX_STAGES * A_BYTES;   // 2 x 256 fp32 head weights
+    static constexpr int OFF_BAR = OFF_W + 2 * IDX_NMAX * 4;
     static constexpr int N_BARS = 2 + 2 + IDX_STAGES + IDX_STAGES + 2 + 2;
     static constexpr int OFF_SLOT = OFF_BAR + N_BARS * 8;
     static constexpr int BYTES = OFF_SLOT + 16;
-    // 1024 B of slack for the 1024-B alignment of the swizzled tiles; never
-    // less than 120 KB so that two CTAs (each holding all 512 TMEM columns)
-    // can never share an SM and wait on each other's allocation.
-    static constexpr int ALLOC = (BYTES + 1024) > 120 * 1024 ? (BYTES + 1024) : 120 * 1024;
+    // Up to 1024 B of slack for the 1024-B alignment of the swizzled tiles
+    // (capped at the 227 KB limit; the kernel checks the aligned layout
+    // fits); never less than 120 KB so that two CTAs, each holding all 512
+    // TMEM columns, can never share an SM and wait on each other's allocation.
+    static constexpr int ALLOC_RAW = (BYTES + 1024) < MAX_DYN_SMEM ? (BYTES + 1024) : MAX_DYN_SMEM;
+    static constexpr int ALLOC = ALLOC_RAW > 120 * 1024 ? ALLOC_RAW : 120 * 1024;
+    static_assert(BYTES <= MAX_DYN_SMEM, "indexer shared-memory layout too large");
 };
 
 struct UnitInfo {
@@ -93,10 +101,11 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
     constexpr int QBMAX = IDX_NMAX / H;
 
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                               ~uintptr_t(1023));
+    uint8_t* smem = align_smem_1024(smem_raw, S::BYTES);
+    if (smem == nullptr) return;                  // uniform: every thread sees the same sizes
     uint8_t* q_s = smem + S::OFF_Q;
     uint8_t* a_s = smem + S::OFF_A;
+    float* w_s = reinterpret_cast<float*>(smem + S::OFF_W);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
     uint64_t* q_full = bars;
     uint64_t* q_empty = bars + 2;
@@ -113,7 +122,9 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
             mbar_init(&q_full[i], 1);
-            mbar_init(&q_empty[i], 1);
+            // freed by the MMA commit of the unit's last tile and by every
+            // epilogue warp once it has read the unit's head weights
+            mbar_init(&q_empty[i], 1 + IDX_EPI_WARPS);
             mbar_init(&acc_full[i], 1);
             mbar_init(&acc_empty[i], 32 * IDX_EPI_WARPS);
         }
@@ -146,11 +157,14 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 if (ui.j0 >= ui.j1) continue;
                 const int qb = uq & 1;
                 if (!mbar_wait(&q_empty[qb], ((uq >> 1) & 1) ^ 1)) { ok = false; break; }
-                mbar_arrive_expect_tx(&q_full[qb], q_bytes);
+                const uint32_t w_bytes = (uint32_t)(ui.nq * H * 4);
+                mbar_arrive_expect_tx(&q_full[qb], q_bytes + w_bytes);
                 uint8_t* qdst = q_s + qb * S::Q_BYTES;
                 for (int kb = 0; kb < KBOX; ++kb)
                     tma_load_3d(qdst + kb * args.N * 128, &tmap_q, &q_full[qb], kb * 64, ui.i0 * H,
                                 ui.b);
+                bulk_load(w_s + qb * IDX_NMAX, args.w + ((long long)ui.b * args.Lq + ui.i0) * H,
+                          w_bytes, &q_full[qb]);
                 ++uq;
                 for (int j = ui.j0; j < ui.j1; ++j, ++ta) {
                     const int st = ta % IDX_STAGES;
@@ -206,52 +220,58 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
             }
         }
     } else {
-        // ---------------- epilogue (warps 2..5)
+        // ---------------- epilogue (warps 2..9)
         const int wq = warp & 3;                  // TMEM lane quarter this warp may read
+        const int cg = (warp - 2) >> 2;           // which half of the block's queries
         const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
-        uint32_t ta = 0;
+        constexpr int QH = (QBMAX + 1) / 2;       // queries per half at most
+        uint32_t ta = 0, uq = 0;
         bool ok = true;
         for (long long u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
             UnitInfo ui = unit_info(args, u);
             if (ui.j0 >= ui.j1) continue;
-            // Head weights of this query block (the same for every key).  Read
-            // through L1 by all threads (broadcast); no block barrier here, so a
-            // thread whose bounded wait gives up can never strand the others.
-            const float* wsrc = args.w + ((long long)ui.b * args.Lq + ui.i0) * H;
-            const int wvalid = ui.nq * H;
-
-            const long long row0 = (long long)ui.b * args.Lq + ui.i0 - args.row_base;
-            const int t0 = args.q_offset + ui.i0;
+            const int qb = uq & 1;
+            // queries [qlo, qhi) of this block belong to this warp
+            const int qhalf = (args.QB + 1) / 2;
+            const int qlo = cg * qhalf;
+            const int qhi = min(ui.nq, qlo + qhalf);
+            const int ncol = (qhi > qlo ? qhi - qlo : 0) * H;        // multiple of 4
+            const int nchunk = (ncol + 31) / 32;
+            // the unit's head weights are in w_s[qb] once q_full[qb] completed
+            if (!mbar_wait(&q_full[qb], (uq >> 1) & 1)) { ok = false; break; }
+            const float* wsm = w_s + qb * IDX_NMAX + qlo * H;
+            const long long row0 = (long long)ui.b * args.Lq + ui.i0 + qlo - args.row_base;
+            const int t0 = args.q_offset + ui.i0 + qlo;
             for (int j = ui.j0; j < ui.j1; ++j, ++ta) {
                 const int ab = ta & 1;
                 if (!mbar_wait(&acc_full[ab], (ta >> 1) & 1)) { ok = false; break; }
                 tc_fence_after();
-                float acc[QBMAX];
+                float acc[QH];
 #pragma unroll
-                for (int q = 0; q < QBMAX; ++q) acc[q] = 0.0f;
-                const uint32_t taddr = tmem_base + lane_base + (uint32_t)(ab * IDX_NMAX);
+                for (int q = 0; q < QH; ++q) acc[q] = 0.0f;
+                const uint32_t taddr =
+                    tmem_base + lane_base + (uint32_t)(ab * IDX_NMAX + qlo * H);
+                // 64 columns per batch: two 32-column TMEM loads, one wait, reduce.
 #pragma unroll
-                for (int cc = 0; cc < IDX_NMAX / 32; ++cc) {
-                    if (cc * 32 < args.N) {
-                        float wc[32];
-#pragma unroll
-                        for (int jj = 0; jj < 32; jj += 4) {
-                            const int c = cc * 32 + jj;
-                            const float4 wv = c < wvalid
-                                ? __ldg(reinterpret_cast<const float4*>(wsrc + c))
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-                            wc[jj] = wv.x; wc[jj + 1] = wv.y; wc[jj + 2] = wv.z; wc[jj + 3] = wv.w;
-                        }
-                        uint32_t v[32];
-                        tmem_ld_32x32b_x32(taddr + cc * 32, v);
+                for (int bt = 0; bt < (QH * H + 63) / 64; ++bt) {
+                    if (bt * 2 < nchunk) {
+                        uint32_t v[64];
+                        tmem_ld_32x32b_x32(taddr + bt * 64, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+                        if (bt * 2 + 1 < nchunk)
+                            tmem_ld_32x32b_x32(taddr + bt * 64 + 32,
+                                               *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
                         tmem_ld_wait();
 #pragma unroll
-                        for (int jj = 0; jj < 32; jj += 4) {
-                            const float wj[4] = {wc[jj], wc[jj + 1], wc[jj + 2], wc[jj + 3]};
+                        for (int jj = 0; jj < 64; jj += 4) {
+                            const int c = bt * 64 + jj;
+                            if (c < ncol) {
+                                const float4 wv = *reinterpret_cast<const float4*>(wsm + c);
+                                const float wj[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int q = (cc * 32 + jj + e) / H;
-                                acc[q] = fmaf(wj[e], fmaxf(__uint_as_float(v[jj + e]), 0.0f), acc[q]);
+                                for (int e = 0; e < 4; ++e) {
+                                    const int q = (bt * 64 + jj + e) / H;
+                                    acc[q] = fmaf(wj[e], fmaxf(__uint_as_float(v[jj + e]), 0.0f), acc[q]);
+                                }
                             }
                         }
                     }
@@ -262,14 +282,18 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 if (s < args.Lk) {
                     float* dst = args.scores + row0 * args.ld + s;
 #pragma unroll
-                    for (int q = 0; q < QBMAX; ++q) {
-                        if (q < ui.nq) {
+                    for (int q = 0; q < QH; ++q) {
+                        if (q < qhi - qlo) {
                             const float val = (s <= t0 + q) ? acc[q] : -INFINITY;
                             dst[(long long)q * args.ld] = val;
                         }
                     }
                 }
             }
+            if (!ok) break;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&q_empty[qb]);
+            ++uq;
         }
     }
 

@@ -5,24 +5,31 @@
 // (IndexCache: every layer, F or S, runs its own sparse attention over the k
 // positions held in the index cache; all query heads share the one K/V head).
 //
-// One CTA handles one query row (all heads) and one split of its slots.  Per
-// 64-slot chunk the CTA gathers the 64 K rows and 64 V rows with 16-byte
-// cp.async copies (a 128-bit, fully coalesced load per thread per piece, rows
-// XOR-swizzled in shared memory so ldmatrix is bank-conflict free), double
-// buffered.  Each of the 4 warps then takes 16 of the slots: S = Q K^T and
-// O += P V run on the tensor cores (m16n8k16, bf16 in, fp32 accumulate), the
-// softmax is online in fp32 (exp2 with the scale pre-multiplied by log2 e).
-// The warps' partial (max, sum, O) merge through shared memory at the end.
-// With several splits per row each split writes (O / l, log2-sum-exp) to the
-// caller's workspace and a combine kernel merges them.
+// One CTA handles one query row (all heads) and one split of its slots.  The
+// CTA first stages up to 2048 of the row's indices in shared memory in one
+// coalesced burst (validating them), so no copy ever waits on an index load.
+// Its 4 warps then work independently on interleaved blocks of 16 slots (warp
+// w takes blocks w, w+4, ...).  Each warp runs its own 3-stage cp.async pipeline: 16
+// lanes copy one 256-byte K row (or V row) per instruction, so every request
+// is a full, coalesced 128-byte line pair; rows land XOR-swizzled in shared
+// memory so the ldmatrix reads are bank-conflict free.  S = Q K^T and
+// O += P V run on the tensor cores (m16n8k16, bf16 in, fp32 accumulate); the
+// softmax is online in fp32 (exp2 with the scale pre-multiplied by log2 e)
+// and the O rescale is skipped while the running max does not move.  The
+// warps' partial (max, sum, O) merge through shared memory at the end; with
+// several splits per row each split writes (O / l, log2-sum-exp) to the
+// caller's workspace and a combine kernel merges the splits.
 #pragma once
 
 #include "common.cuh"
 
 namespace ic {
 
-constexpr int SA_THREADS = 128;
-constexpr int SA_CHUNK = 64;
+constexpr int SA_BLOCK = 16;                 // slots per warp iteration
+constexpr int SA_WARPS = 4;
+constexpr int SA_THREADS = 32 * SA_WARPS;
+constexpr int SA_STAGES = 3;
+constexpr int SA_IDX_TILE = 2048;            // indices staged in shared memory at a time
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 
@@ -44,20 +51,25 @@ struct SparseAttnArgs {
 
 template <int D>
 struct SaSmem {
-    static constexpr int ROW = D * 2;                     // bytes per K/V/Q row
+    static constexpr int ROW = D * 2;                          // bytes per K/V/Q row
+    static constexpr int BLK = SA_BLOCK * ROW;                 // one block of K (or V) rows
+    static constexpr int STAGE = 2 * BLK;                      // K then V
     static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = OFF_Q + 16 * ROW;
-    static constexpr int OFF_V = OFF_K + 2 * SA_CHUNK * ROW;
-    static constexpr int OFF_IDX = OFF_V + 2 * SA_CHUNK * ROW;
-    static constexpr int BYTES = OFF_IDX + 2 * SA_CHUNK * 4;
-    // merge buffers (reuse the K/V region after the main loop)
-    static constexpr int MERGE_O = OFF_K;                                  // [4][16][D] f32
-    static constexpr int MERGE_ML = OFF_K + 4 * 16 * D * 4;                // [4][16][2] f32
-    static_assert(MERGE_ML + 4 * 16 * 2 * 4 <= OFF_IDX, "merge buffer overflow");
+    static constexpr int OFF_KV = 16 * ROW;
+    static constexpr int WARP_KV = SA_STAGES * STAGE;
+    static constexpr int OFF_IDX = OFF_KV + SA_WARPS * WARP_KV;
+    static constexpr int BYTES = OFF_IDX + SA_IDX_TILE * 4;
+    // merge buffers reuse the K/V rings once every warp has finished
+    static constexpr int MERGE_O = OFF_KV;                                  // [4][16][D] f32
+    static constexpr int MERGE_ML = OFF_KV + SA_WARPS * 16 * D * 4;         // [4][16][2] f32
+    static_assert(MERGE_ML + SA_WARPS * 16 * 2 * 4 <= OFF_IDX, "merge buffer overflow");
 };
 
-__device__ __forceinline__ uint32_t swz(int row, int chunk, int row_bytes) {
-    return (uint32_t)(row * row_bytes + ((chunk ^ (row & 7)) << 4));
+// Byte offset of 16-byte chunk c of row r in a [rows][D] bf16 tile whose
+// chunks are XOR-swizzled by (r mod 8).
+template <int D>
+__device__ __forceinline__ uint32_t swz(int r, int c) {
+    return (uint32_t)(r * (D * 2) + ((c ^ (r & 7)) << 4));
 }
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
@@ -99,13 +111,13 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(SA_THREADS)
+__global__ void __launch_bounds__(SA_THREADS, 2)
 sparse_attn_kernel(const SparseAttnArgs a) {
     using S = SaSmem<D>;
-    constexpr int CPR = D / 8;                 // 16-byte pieces per row
+    constexpr int CPR = D / 8;                 // 16-byte chunks per row (16 or 8)
+    constexpr int RPI = 32 / CPR;              // rows copied per warp instruction (2 or 4)
     extern __shared__ __align__(128) uint8_t sa_smem[];
     const uint32_t sbase = smem_u32(sa_smem);
-    int32_t* idx_s = reinterpret_cast<int32_t*>(sa_smem + S::OFF_IDX);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const long long row = a.n_rows - 1 - (long long)blockIdx.x;     // longest rows first
@@ -116,11 +128,12 @@ sparse_attn_kernel(const SparseAttnArgs a) {
     const int kend = a.trim ? min(a.kslots, t + 1) : a.kslots;
     const int s0 = split * a.slots_per_split;
     const int s1 = min(s0 + a.slots_per_split, kend);
-    const int nchunks = s1 > s0 ? (s1 - s0 + SA_CHUNK - 1) / SA_CHUNK : 0;
 
     const __nv_bfloat16* kb = a.k + (long long)b * a.Lk * D;
     const __nv_bfloat16* vb = a.v + (long long)b * a.Lk * D;
     const int32_t* irow = a.idx + row * a.kslots;
+    const uint32_t kv_base = sbase + S::OFF_KV + warp * S::WARP_KV;
+    int32_t* idx_s = reinterpret_cast<int32_t*>(sa_smem + S::OFF_IDX);
 
     // Q rows (heads) -> shared memory, rows >= Hq zero.
     {
@@ -129,139 +142,150 @@ sparse_attn_kernel(const SparseAttnArgs a) {
             const int h = p / CPR, c = p % CPR;
             uint4 val = make_uint4(0, 0, 0, 0);
             if (h < a.Hq) val = qsrc[h * CPR + c];
-            *reinterpret_cast<uint4*>(sa_smem + S::OFF_Q + swz(h, c, S::ROW)) = val;
+            *reinterpret_cast<uint4*>(sa_smem + S::OFF_Q + swz<D>(h, c)) = val;
         }
-    }
-
-    auto issue = [&](int chunk, int st) {
-        const int base = s0 + chunk * SA_CHUNK;
-        if (tid < SA_CHUNK) {
-            const int slot = base + tid;
-            int id = -1;
-            if (slot < s1) {
-                id = __ldg(irow + slot);
-                if (id != -1 && (id < 0 || id > tmax)) {
-                    report(DEV_ERR_BAD_INDEX);
-                    id = -1;
-                }
-            }
-            idx_s[st * SA_CHUNK + tid] = id;
-        }
-        for (int p = tid; p < SA_CHUNK * CPR; p += SA_THREADS) {
-            const int r = p / CPR, c = p % CPR;
-            const int slot = base + r;
-            int id = slot < s1 ? __ldg(irow + slot) : -1;
-            const bool ok = id >= 0 && id <= tmax;
-            const long long off = (long long)(ok ? id : 0) * D + c * 8;
-            const uint32_t dk = sbase + S::OFF_K + st * SA_CHUNK * S::ROW + swz(r, c, S::ROW);
-            const uint32_t dv = sbase + S::OFF_V + st * SA_CHUNK * S::ROW + swz(r, c, S::ROW);
-            cp_async16(dk, kb + off, ok);
-            cp_async16(dv, vb + off, ok);
-        }
-        cp_async_commit();
-    };
-
-    if (nchunks > 0) issue(0, 0);
-    __syncthreads();
-
-    // Q fragments (A operand, m16 x k16 per k-step) stay in registers.
-    uint32_t qf[D / 16][4];
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-        const int r = (lane & 7) + ((lane >> 3) & 1) * 8;
-        const int c = 2 * kk + (lane >> 4);
-        ldsm_x4(sbase + S::OFF_Q + swz(r, c, S::ROW), qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3]);
     }
 
     float o[D / 8][4];
 #pragma unroll
     for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f;
+    uint32_t qf[D / 16][4];
 
-    for (int ch = 0; ch < nchunks; ++ch) {
-        const int st = ch & 1;
-        if (ch + 1 < nchunks) {
-            issue(ch + 1, st ^ 1);
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
+    // Slots [s0, s1) are processed in tiles of SA_IDX_TILE staged indices.
+    for (int tile0 = s0; tile0 < s1 || (tile0 == s0 && s1 <= s0); tile0 += SA_IDX_TILE) {
+        const int tile1 = min(tile0 + SA_IDX_TILE, s1);
+        const int ntile = max(tile1 - tile0, 0);
+        __syncthreads();                  // previous tile fully consumed
+        for (int i = tid; i < SA_IDX_TILE; i += SA_THREADS) {
+            int id = -1;
+            if (i < ntile) {
+                id = __ldg(irow + tile0 + i);
+                if (id != -1 && (id < 0 || id > tmax)) {
+                    report(DEV_ERR_BAD_INDEX);
+                    id = -1;
+                }
+            }
+            idx_s[i] = id;
         }
         __syncthreads();
-
-        const uint32_t kbase = sbase + S::OFF_K + st * SA_CHUNK * S::ROW;
-        const uint32_t vbase = sbase + S::OFF_V + st * SA_CHUNK * S::ROW;
-        const int key0 = warp * 16;
-        float sc[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
+        if (tile0 == s0) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-            const int r = key0 + (lane & 7) + (lane >> 4) * 8;
-            const int c = 2 * kk + ((lane >> 3) & 1);
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4(kbase + swz(r, c, S::ROW), b0, b1, b2, b3);
-            mma_bf16(sc[0], qf[kk], b0, b1);
-            mma_bf16(sc[1], qf[kk], b2, b3);
-        }
-        // mask + scale (log2 domain)
-        const int* ids = idx_s + st * SA_CHUNK + key0;
-        float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int col = nt * 8 + (lane & 3) * 2 + e;
-                const bool ok = ids[col] >= 0;
-                sc[nt][e] = ok ? sc[nt][e] * a.scale_log2 : -INFINITY;
-                sc[nt][2 + e] = ok ? sc[nt][2 + e] * a.scale_log2 : -INFINITY;
-                mx0 = fmaxf(mx0, sc[nt][e]);
-                mx1 = fmaxf(mx1, sc[nt][2 + e]);
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const int r = (lane & 7) + ((lane >> 3) & 1) * 8;
+                const int c = 2 * kk + (lane >> 4);
+                ldsm_x4(sbase + S::OFF_Q + swz<D>(r, c), qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3]);
             }
         }
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-        const float base0 = mn0 == -INFINITY ? 0.0f : mn0;
-        const float base1 = mn1 == -INFINITY ? 0.0f : mn1;
-        const float al0 = exp2f(m0 - base0), al1 = exp2f(m1 - base1);
-        m0 = mn0;
-        m1 = mn1;
-        float p[2][4];
-        float rs0 = 0.0f, rs1 = 0.0f;
+        const int nblk = (ntile + SA_BLOCK - 1) / SA_BLOCK;
+        const int niter = nblk > warp ? (nblk - warp + SA_WARPS - 1) / SA_WARPS : 0;
+
+        // Copies block (warp + SA_WARPS * it) of this tile into stage `st`.
+        auto issue = [&](int it, int st) {
+            const int* ids = idx_s + (warp + SA_WARPS * it) * SA_BLOCK;
+            const uint32_t kdst = kv_base + st * S::STAGE;
+            const uint32_t vdst = kdst + S::BLK;
+            const int c = lane % CPR;
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            p[nt][0] = exp2f(sc[nt][0] - base0);
-            p[nt][1] = exp2f(sc[nt][1] - base0);
-            p[nt][2] = exp2f(sc[nt][2] - base1);
-            p[nt][3] = exp2f(sc[nt][3] - base1);
-            rs0 += p[nt][0] + p[nt][1];
-            rs1 += p[nt][2] + p[nt][3];
-        }
-        l0 = l0 * al0 + rs0;
-        l1 = l1 * al1 + rs1;
+            for (int i = 0; i < SA_BLOCK / RPI; ++i) {
+                const int r = i * RPI + lane / CPR;
+                const int rid = ids[r];
+                const bool ok = rid >= 0;
+                const long long off = (long long)(ok ? rid : 0) * D + c * 8;
+                cp_async16(kdst + swz<D>(r, c), kb + off, ok);
+                cp_async16(vdst + swz<D>(r, c), vb + off, ok);
+            }
+        };
 #pragma unroll
-        for (int i = 0; i < D / 8; ++i) {
-            o[i][0] *= al0;
-            o[i][1] *= al0;
-            o[i][2] *= al1;
-            o[i][3] *= al1;
+        for (int p = 0; p < SA_STAGES - 1; ++p) {
+            if (p < niter) issue(p, p);
+            cp_async_commit();
         }
-        uint32_t pa[4];
-        pa[0] = pack_bf16(p[0][0], p[0][1]);
-        pa[1] = pack_bf16(p[0][2], p[0][3]);
-        pa[2] = pack_bf16(p[1][0], p[1][1]);
-        pa[3] = pack_bf16(p[1][2], p[1][3]);
+
+        for (int it = 0; it < niter; ++it) {
+            const int nx = it + SA_STAGES - 1;
+            if (nx < niter) issue(nx, nx % SA_STAGES);
+            cp_async_commit();
+            cp_async_wait<SA_STAGES - 1>();
+            __syncwarp();
+            const int st = it % SA_STAGES;
+            const uint32_t kbase = kv_base + st * S::STAGE;
+            const uint32_t vbase = kbase + S::BLK;
+            float sc[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
 #pragma unroll
-        for (int dn = 0; dn < D / 16; ++dn) {
-            const int r = key0 + (lane & 7) + ((lane >> 3) & 1) * 8;
-            const int c = 2 * dn + (lane >> 4);
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4_t(vbase + swz(r, c, S::ROW), b0, b1, b2, b3);
-            mma_bf16(o[2 * dn], pa, b0, b1);
-            mma_bf16(o[2 * dn + 1], pa, b2, b3);
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const int r = (lane & 7) + (lane >> 4) * 8;
+                const int c = 2 * kk + ((lane >> 3) & 1);
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4(kbase + swz<D>(r, c), b0, b1, b2, b3);
+                mma_bf16(sc[0], qf[kk], b0, b1);
+                mma_bf16(sc[1], qf[kk], b2, b3);
+            }
+            const int* ids = idx_s + (warp + SA_WARPS * it) * SA_BLOCK;
+            float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const bool valid = ids[nt * 8 + (lane & 3) * 2 + e] >= 0;
+                    sc[nt][e] = valid ? sc[nt][e] * a.scale_log2 : -INFINITY;
+                    sc[nt][2 + e] = valid ? sc[nt][2 + e] * a.scale_log2 : -INFINITY;
+                    mx0 = fmaxf(mx0, sc[nt][e]);
+                    mx1 = fmaxf(mx1, sc[nt][2 + e]);
+                }
+            }
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+            const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+            const float base0 = mn0 == -INFINITY ? 0.0f : mn0;
+            const float base1 = mn1 == -INFINITY ? 0.0f : mn1;
+            const float al0 = exp2f(m0 - base0), al1 = exp2f(m1 - base1);
+            m0 = mn0;
+            m1 = mn1;
+            float p[2][4];
+            float rs0 = 0.0f, rs1 = 0.0f;
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                p[nt][0] = exp2f(sc[nt][0] - base0);
+                p[nt][1] = exp2f(sc[nt][1] - base0);
+                p[nt][2] = exp2f(sc[nt][2] - base1);
+                p[nt][3] = exp2f(sc[nt][3] - base1);
+                rs0 += p[nt][0] + p[nt][1];
+                rs1 += p[nt][2] + p[nt][3];
+            }
+            l0 = l0 * al0 + rs0;
+            l1 = l1 * al1 + rs1;
+            if (__any_sync(0xffffffffu, al0 != 1.0f || al1 != 1.0f)) {
+#pragma unroll
+                for (int i = 0; i < D / 8; ++i) {
+                    o[i][0] *= al0;
+                    o[i][1] *= al0;
+                    o[i][2] *= al1;
+                    o[i][3] *= al1;
+                }
+            }
+            uint32_t pa[4];
+            pa[0] = pack_bf16(p[0][0], p[0][1]);
+            pa[1] = pack_bf16(p[0][2], p[0][3]);
+            pa[2] = pack_bf16(p[1][0], p[1][1]);
+            pa[3] = pack_bf16(p[1][2], p[1][3]);
+#pragma unroll
+            for (int dn = 0; dn < D / 16; ++dn) {
+                const int r = (lane & 7) + ((lane >> 3) & 1) * 8;
+                const int c = 2 * dn + (lane >> 4);
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_t(vbase + swz<D>(r, c), b0, b1, b2, b3);
+                mma_bf16(o[2 * dn], pa, b0, b1);
+                mma_bf16(o[2 * dn + 1], pa, b2, b3);
+            }
+            __syncwarp();      // every lane is done with this stage before it is refilled
         }
-        __syncthreads();
+        cp_async_wait<0>();
+        if (tile1 >= s1) break;
     }
+    cp_async_wait<0>();
 
     // Row sums were kept per thread; reduce over the quad.
     l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
@@ -269,7 +293,7 @@ sparse_attn_kernel(const SparseAttnArgs a) {
     l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
     l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
 
-    // Merge the 4 warps through shared memory.
+    __syncthreads();       // all warps are past their rings: reuse them for the merge
     float* mo = reinterpret_cast<float*>(sa_smem + S::MERGE_O);
     float* ml = reinterpret_cast<float*>(sa_smem + S::MERGE_ML);
     const int g = lane >> 2, cq = (lane & 3) * 2;
@@ -294,11 +318,11 @@ sparse_attn_kernel(const SparseAttnArgs a) {
         const int h = e / D, dcol = e % D;
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < 4; ++w) M = fmaxf(M, ml[(w * 16 + h) * 2]);
+        for (int w = 0; w < SA_WARPS; ++w) M = fmaxf(M, ml[(w * 16 + h) * 2]);
         float L = 0.0f, acc = 0.0f;
         if (M != -INFINITY) {
 #pragma unroll
-            for (int w = 0; w < 4; ++w) {
+            for (int w = 0; w < SA_WARPS; ++w) {
                 const float f = exp2f(ml[(w * 16 + h) * 2] - M);
                 L += f * ml[(w * 16 + h) * 2 + 1];
                 acc += f * mo[(w * 16 + h) * D + dcol];
