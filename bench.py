@@ -80,6 +80,36 @@ def work_per_layer(wl):
     return w
 
 
+# ---------------------------------------------------------------- ncu traffic
+
+_KERNEL_SRC = {"sparse_attn": ("sparse_attn_kernel", "sparse_attn.cuh"),
+               "indexer_scores": ("indexer_scores_kernel", "indexer_scores.cuh"),
+               "topk_select": ("topk_select_kernel", "topk_select.cuh")}
+
+
+def profile_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary of this kernel and
+    workload, or None when there is none or the kernel source changed since
+    the counters were taken (the summary records a hash of the source)."""
+    import hashlib
+    name, src = _KERNEL_SRC[kernel]
+    path = os.path.join(ROOT, "profiles", f"{name}_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    h = hashlib.sha256()
+    for f in (src, "common.cuh"):
+        with open(os.path.join(ROOT, "lightning_indexer_top_relu_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    want, traffic = None, None
+    with open(path) as fh:
+        for line in fh:
+            if line.startswith("source_hash:"):
+                want = line.split(":", 1)[1].strip()
+            elif line.startswith("dram_bytes_per_launch:"):
+                traffic = int(line.split(":", 1)[1].strip())
+    return traffic if want == h.hexdigest()[:16] else None
+
+
 # ---------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -191,6 +221,22 @@ def run_reference(args, wl, pattern):
     return 0
 
 
+def aggregate_over_ranks(ms_per_step: float, tokens_per_step: float, dist_mod=None, device=None):
+    """Whole-job throughput: step time = max over ranks, tokens = sum over ranks.
+
+    Returns (max ms per step, total tokens per step, tokens/s).  With no process
+    group (N = 1) the local numbers are returned unchanged.
+    """
+    if dist_mod is None:
+        return ms_per_step, tokens_per_step, tokens_per_step / (ms_per_step / 1e3)
+    t = torch.tensor([ms_per_step], dtype=torch.float64, device=device)
+    n = torch.tensor([tokens_per_step], dtype=torch.float64, device=device)
+    dist_mod.all_reduce(t, op=dist_mod.ReduceOp.MAX)
+    dist_mod.all_reduce(n, op=dist_mod.ReduceOp.SUM)
+    ms, tok = float(t.item()), float(n.item())
+    return ms, tok, tok / (ms / 1e3)
+
+
 def config_of(wl, pattern, args):
     return {"workload": wl.name, "B": wl.B, "L": wl.Lq, "Lk": wl.Lk, "q_offset": wl.q_offset,
             "layers": wl.n_layers, "pattern": pattern, "H_I": wl.H_I, "d_I": wl.d_I,
@@ -258,24 +304,8 @@ def main():
         assert all(arr), "CUDA event handles must exist before they are handed to the library"
         return evs, arr
 
-    lib = ic.lib()
-    lib.ic_layer_stack_forward_events.restype = ctypes.c_int
-    lib.ic_layer_stack_forward_events.argtypes = [ctypes.c_char_p, ctypes.c_int,
-                                                  ctypes.POINTER(ic.ICLayer),
-                                                  ctypes.POINTER(ic.ICDims), ctypes.c_void_p,
-                                                  ctypes.c_void_p, ctypes.c_size_t,
-                                                  ctypes.c_void_p, ctypes.c_void_p]
-
     def step(marks=None):
-        if marks is None:
-            stack.forward(stream)
-        else:
-            rc = lib.ic_layer_stack_forward_events(
-                stack._pattern_b, n, stack.table, ctypes.byref(stack.dims),
-                stack.idx_cache.data_ptr(), stack.ws.data_ptr(), stack.ws.numel(),
-                stream.cuda_stream, ctypes.cast(marks, ctypes.c_void_p))
-            if rc != 0:
-                raise ic.IndexCacheError(rc, "ic_layer_stack_forward_events")
+        stack.forward(stream, events=marks)
 
     for _ in range(args.warmup):
         step()
@@ -308,14 +338,8 @@ def main():
         raise RuntimeError("device error during the timed steps")
 
     step_ms = [starts[s].elapsed_time(ends[s]) for s in range(args.steps)]
-    total_ms = float(np.sum(step_ms))
-    if pg is not None:
-        t = torch.tensor([total_ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        total_ms = float(t.item())
-    ms_per_step = total_ms / args.steps
-    tokens = wl.B * wl.Lq * world
-    value = tokens / (ms_per_step / 1e3)
+    local_ms = float(np.sum(step_ms)) / args.steps
+    ms_per_step, tokens, value = aggregate_over_ranks(local_ms, float(wl.B * wl.Lq), pg, dev)
 
     # ---- per-kernel breakdown from the marks
     ki = {"indexer": [], "topk": [], "attn": []}
@@ -366,6 +390,10 @@ def main():
                 "unit": "GB/s", "frac": ach / peaks["hbm_gbs"], "traffic": None,
                 "algorithmic_per_launch": w["attn_bytes"]}
     roof["peak_source"] = peaks["source"]
+    roof["traffic"] = profile_traffic(roof["kernel"], wl.name)
+    if roof["kernel"] == "sparse_attn":
+        roof["note"] = ("achieved counts the logical K/V gather bytes; at this size a layer's K/V "
+                        "stay L2-resident, so DRAM traffic (`traffic`) is far below them")
 
     launches_per_step = 0
     for c in pattern:
@@ -397,8 +425,9 @@ def main():
             torch.cuda.synchronize()
             ts.append(a.elapsed_time(b))
         msf = float(np.mean(ts))
+        msf, _, vf = aggregate_over_ranks(msf, float(wl.B * wl.Lq), pg, dev)
         line["all_f"] = {"pattern": "F" * n, "ms_per_step": msf,
-                         "value": wl.B * wl.Lq * world / (msf / 1e3),
+                         "value": vf,
                          "speedup_of_pattern": msf / ms_per_step}
         del stack_f
 
@@ -429,12 +458,9 @@ def main():
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize()
-        e_ms = a.elapsed_time(b) / k_e2e
-        if pg is not None:
-            t = torch.tensor([e_ms], device=dev)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            e_ms = float(t.item())
-        line["e2e"] = {"value": wl.B * wl.Lq * world / (e_ms / 1e3), "unit": "tokens/s",
+        e_ms, e_tok, e_val = aggregate_over_ranks(a.elapsed_time(b) / k_e2e, float(wl.B * wl.Lq),
+                                                  pg, dev)
+        line["e2e"] = {"value": e_val, "unit": "tokens/s",
                        "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                        "ms_per_step": e_ms}
 

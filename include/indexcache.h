@@ -75,6 +75,16 @@ const char *ic_last_error_message(void);
 int ic_get_last_device_error(ic_stream_t stream);
 
 /*
+ * Failure-detection self test.  Launches one CTA whose thread waits on an
+ * mbarrier that nothing ever arrives on, for at most timeout_us microseconds
+ * (clamped to [1, 2000000]).  The bounded wait gives up, the kernel records a
+ * timeout in the device error word and returns, so the next
+ * ic_get_last_device_error() returns IC_ERR_TIMEOUT and the CUDA context stays
+ * usable.  It exercises the same bounded wait every pipelined kernel uses.
+ */
+int ic_selftest_wait_timeout(int timeout_us, ic_stream_t stream);
+
+/*
  * Step a1 — lightning indexer scores (digest Abstract; review Introduction:
  * the indexer scores all preceding tokens).
  *   q_idx  [B, Lq, H_I, d_I] bf16     k_idx [B, Lk, d_I] bf16

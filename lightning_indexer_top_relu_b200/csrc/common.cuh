@@ -86,17 +86,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Returns false
-// (and reports DEV_ERR_TIMEOUT) when it does not within WAIT_LIMIT_NS.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// (and reports DEV_ERR_TIMEOUT) when it does not within limit_ns.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          unsigned long long limit_ns = WAIT_LIMIT_NS) {
     if (mbar_try_wait(bar, parity)) return true;
     unsigned long long t0 = global_ns();
     for (;;) {
         for (int i = 0; i < 64; ++i)
             if (mbar_try_wait(bar, parity)) return true;
-        if (global_ns() - t0 > WAIT_LIMIT_NS) {
+        if (global_ns() - t0 > limit_ns) {
             report(DEV_ERR_TIMEOUT);
             return false;
         }
+    }
+}
+
+// Failure-detection self test: one thread waits on an mbarrier that nothing
+// arrives on; the bounded wait gives up and reports DEV_ERR_TIMEOUT.
+__global__ void selftest_wait_timeout_kernel(unsigned long long limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+        mbar_wait(&bar, 0, limit_ns);
     }
 }
 

@@ -84,22 +84,6 @@ int make_tmap_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uin
     return IC_OK;
 }
 
-// 2-D bf16 tensor {d0 (contiguous), d1} with 128-byte swizzled boxes {64, box1}.
-int make_tmap_2d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint32_t box1) {
-    int rc = get_encode();
-    if (rc) return rc;
-    cuuint64_t dims[2] = {d0, d1};
-    cuuint64_t strides[1] = {d0 * 2};
-    cuuint32_t box[2] = {64, box1};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
-                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return fail(IC_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
-    return IC_OK;
-}
-
 // ---------------------------------------------------------------- indexer
 
 struct IndexerGeom {
@@ -231,7 +215,7 @@ int launch_topk(const float* scores, long long ld, long long row_base, long long
 int attn_splits(long long n_rows, int k_slots, int sms) {
     if (n_rows >= 2LL * sms) return 1;
     long long s = (2LL * sms + n_rows - 1) / n_rows;
-    s = std::min<long long>(s, (k_slots + 4 * ic::SA_BLOCK - 1) / (4 * ic::SA_BLOCK));
+    s = std::min<long long>(s, (k_slots + ic::SA_WARPS * ic::SA_BLOCK - 1) / (ic::SA_WARPS * ic::SA_BLOCK));
     s = std::min<long long>(s, 64);
     return (int)std::max<long long>(1, s);
 }
@@ -393,6 +377,18 @@ int ic_get_last_device_error(ic_stream_t stream) {
         return fail(IC_ERR_CUDA, "a kernel's aligned shared-memory layout did not fit; it did no work");
     if (v & ic::DEV_ERR_BAD_INDEX)
         return fail(IC_ERR_INVALID_ARG, "an attention index outside [0, t] was skipped");
+    return IC_OK;
+}
+
+int ic_selftest_wait_timeout(int timeout_us, ic_stream_t stream) {
+    int dev, sms;
+    int rc = device_setup(&dev, &sms);
+    if (rc) return rc;
+    const long long us = std::min(2000000, std::max(1, timeout_us));
+    ic::selftest_wait_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        (unsigned long long)us * 1000ull);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "selftest launch");
     return IC_OK;
 }
 

@@ -25,10 +25,23 @@
 
 namespace ic {
 
-constexpr int SA_BLOCK = 16;                 // slots per warp iteration
-constexpr int SA_WARPS = 4;
+#ifndef IC_SA_BLOCK
+#define IC_SA_BLOCK 16
+#endif
+#ifndef IC_SA_WARPS
+#define IC_SA_WARPS 4
+#endif
+#ifndef IC_SA_STAGES
+#define IC_SA_STAGES 3
+#endif
+#ifndef IC_SA_MINB
+#define IC_SA_MINB 2
+#endif
+constexpr int SA_BLOCK = IC_SA_BLOCK;        // slots per warp iteration (16, 32 or 64)
+constexpr int SA_WARPS = IC_SA_WARPS;
 constexpr int SA_THREADS = 32 * SA_WARPS;
-constexpr int SA_STAGES = 3;
+constexpr int SA_STAGES = IC_SA_STAGES;
+static_assert(SA_BLOCK == 16 || SA_BLOCK == 32 || SA_BLOCK == 64, "block of 16, 32 or 64 slots");
 constexpr int SA_IDX_TILE = 2048;            // indices staged in shared memory at a time
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
@@ -111,7 +124,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(SA_THREADS, 2)
+__global__ void __launch_bounds__(SA_THREADS, IC_SA_MINB)
 sparse_attn_kernel(const SparseAttnArgs a) {
     using S = SaSmem<D>;
     constexpr int CPR = D / 8;                 // 16-byte chunks per row (16 or 8)
@@ -211,20 +224,27 @@ sparse_attn_kernel(const SparseAttnArgs a) {
             const int st = it % SA_STAGES;
             const uint32_t kbase = kv_base + st * S::STAGE;
             const uint32_t vbase = kbase + S::BLK;
-            float sc[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
+            constexpr int NT = SA_BLOCK / 8;            // S n-tiles of 8 slots
+            constexpr int KS = SA_BLOCK / 16;           // P.V k-steps of 16 slots
+            float sc[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.0f;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-                const int r = (lane & 7) + (lane >> 4) * 8;
-                const int c = 2 * kk + ((lane >> 3) & 1);
-                uint32_t b0, b1, b2, b3;
-                ldsm_x4(kbase + swz<D>(r, c), b0, b1, b2, b3);
-                mma_bf16(sc[0], qf[kk], b0, b1);
-                mma_bf16(sc[1], qf[kk], b2, b3);
+#pragma unroll
+                for (int np = 0; np < NT / 2; ++np) {
+                    const int r = np * 16 + (lane & 7) + (lane >> 4) * 8;
+                    const int c = 2 * kk + ((lane >> 3) & 1);
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4(kbase + swz<D>(r, c), b0, b1, b2, b3);
+                    mma_bf16(sc[2 * np], qf[kk], b0, b1);
+                    mma_bf16(sc[2 * np + 1], qf[kk], b2, b3);
+                }
             }
             const int* ids = idx_s + (warp + SA_WARPS * it) * SA_BLOCK;
             float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
+            for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     const bool valid = ids[nt * 8 + (lane & 3) * 2 + e] >= 0;
@@ -244,16 +264,18 @@ sparse_attn_kernel(const SparseAttnArgs a) {
             const float al0 = exp2f(m0 - base0), al1 = exp2f(m1 - base1);
             m0 = mn0;
             m1 = mn1;
-            float p[2][4];
             float rs0 = 0.0f, rs1 = 0.0f;
+            uint32_t pa[KS][4];
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                p[nt][0] = exp2f(sc[nt][0] - base0);
-                p[nt][1] = exp2f(sc[nt][1] - base0);
-                p[nt][2] = exp2f(sc[nt][2] - base1);
-                p[nt][3] = exp2f(sc[nt][3] - base1);
-                rs0 += p[nt][0] + p[nt][1];
-                rs1 += p[nt][2] + p[nt][3];
+            for (int nt = 0; nt < NT; ++nt) {
+                const float p0 = exp2f(sc[nt][0] - base0);
+                const float p1 = exp2f(sc[nt][1] - base0);
+                const float p2 = exp2f(sc[nt][2] - base1);
+                const float p3 = exp2f(sc[nt][3] - base1);
+                rs0 += p0 + p1;
+                rs1 += p2 + p3;
+                pa[nt >> 1][(nt & 1) * 2 + 0] = pack_bf16(p0, p1);
+                pa[nt >> 1][(nt & 1) * 2 + 1] = pack_bf16(p2, p3);
             }
             l0 = l0 * al0 + rs0;
             l1 = l1 * al1 + rs1;
@@ -266,19 +288,17 @@ sparse_attn_kernel(const SparseAttnArgs a) {
                     o[i][3] *= al1;
                 }
             }
-            uint32_t pa[4];
-            pa[0] = pack_bf16(p[0][0], p[0][1]);
-            pa[1] = pack_bf16(p[0][2], p[0][3]);
-            pa[2] = pack_bf16(p[1][0], p[1][1]);
-            pa[3] = pack_bf16(p[1][2], p[1][3]);
 #pragma unroll
-            for (int dn = 0; dn < D / 16; ++dn) {
-                const int r = (lane & 7) + ((lane >> 3) & 1) * 8;
-                const int c = 2 * dn + (lane >> 4);
-                uint32_t b0, b1, b2, b3;
-                ldsm_x4_t(vbase + swz<D>(r, c), b0, b1, b2, b3);
-                mma_bf16(o[2 * dn], pa, b0, b1);
-                mma_bf16(o[2 * dn + 1], pa, b2, b3);
+            for (int ks = 0; ks < KS; ++ks) {
+#pragma unroll
+                for (int dn = 0; dn < D / 16; ++dn) {
+                    const int r = ks * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+                    const int c = 2 * dn + (lane >> 4);
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4_t(vbase + swz<D>(r, c), b0, b1, b2, b3);
+                    mma_bf16(o[2 * dn], pa[ks], b0, b1);
+                    mma_bf16(o[2 * dn + 1], pa[ks], b2, b3);
+                }
             }
             __syncwarp();      // every lane is done with this stage before it is refilled
         }

@@ -32,7 +32,7 @@ STATUS = {0: "IC_OK", 1: "IC_ERR_INVALID_ARG", 2: "IC_ERR_UNSUPPORTED",
 EXPORTS = ("ic_status_string", "ic_last_error_message", "ic_get_last_device_error",
            "ic_indexer_scores", "ic_topk_select", "ic_sparse_attn",
            "ic_sparse_attn_workspace_bytes", "ic_layer_stack_workspace_bytes",
-           "ic_layer_stack_forward")
+           "ic_layer_stack_forward", "ic_layer_stack_forward_events", "ic_selftest_wait_timeout")
 
 
 class IndexCacheError(RuntimeError):
@@ -77,6 +77,11 @@ _lib.ic_sparse_attn_workspace_bytes.restype = _Z
 _lib.ic_sparse_attn_workspace_bytes.argtypes = [_I, _I, _I, _I, _I]
 _lib.ic_layer_stack_workspace_bytes.restype = _Z
 _lib.ic_layer_stack_workspace_bytes.argtypes = [ctypes.POINTER(ICDims), _I, ctypes.c_longlong]
+_lib.ic_selftest_wait_timeout.restype = _I
+_lib.ic_selftest_wait_timeout.argtypes = [_I, _P]
+_lib.ic_layer_stack_forward_events.restype = _I
+_lib.ic_layer_stack_forward_events.argtypes = [ctypes.c_char_p, _I, ctypes.POINTER(ICLayer),
+                                               ctypes.POINTER(ICDims), _P, _P, _Z, _P, _P]
 _lib.ic_layer_stack_forward.restype = _I
 _lib.ic_layer_stack_forward.argtypes = [ctypes.c_char_p, _I, ctypes.POINTER(ICLayer),
                                         ctypes.POINTER(ICDims), _P, _P, _Z, _P]
@@ -114,6 +119,11 @@ def _stream(stream) -> Optional[int]:
 def get_last_device_error(stream=None) -> int:
     """Synchronises the stream and returns (and clears) the device error status."""
     return int(_lib.ic_get_last_device_error(_stream(stream)))
+
+
+def selftest_wait_timeout(timeout_us: int = 20000, stream=None) -> None:
+    """Launches the bounded-wait self test (see include/indexcache.h)."""
+    _check(_lib.ic_selftest_wait_timeout(int(timeout_us), _stream(stream)), "ic_selftest_wait_timeout")
 
 
 def indexer_scores(q_idx, k_idx, w, q_offset: int = 0, out=None, stream=None) -> torch.Tensor:
@@ -212,10 +222,18 @@ class LayerStack:
                 _ptr(self.lses[i], torch.float32, "lse"), _ptr(self.dumps[i], torch.int32, "dump"))
         self._pattern_b = pattern.encode()
 
-    def forward(self, stream=None):
-        rc = _lib.ic_layer_stack_forward(self._pattern_b, len(self.layers), self.table,
-                                         ctypes.byref(self.dims), _ptr(self.idx_cache),
-                                         _ptr(self.ws), self.ws.numel(), _stream(stream))
+    def forward(self, stream=None, events=None):
+        """Runs the stack; `events` (a ctypes array of 4*n_layers cudaEvent_t
+        handles, or None) selects ic_layer_stack_forward_events."""
+        if events is None:
+            rc = _lib.ic_layer_stack_forward(self._pattern_b, len(self.layers), self.table,
+                                             ctypes.byref(self.dims), _ptr(self.idx_cache),
+                                             _ptr(self.ws), self.ws.numel(), _stream(stream))
+        else:
+            rc = _lib.ic_layer_stack_forward_events(
+                self._pattern_b, len(self.layers), self.table, ctypes.byref(self.dims),
+                _ptr(self.idx_cache), _ptr(self.ws), self.ws.numel(), _stream(stream),
+                ctypes.cast(events, ctypes.c_void_p))
         _check(rc, "ic_layer_stack_forward")
         return self.outs
 
