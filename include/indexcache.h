@@ -133,6 +133,33 @@ int ic_sparse_attn(const uint16_t *q, const uint16_t *k, const uint16_t *v, cons
 /* Workspace that lets ic_sparse_attn use its preferred slot split. */
 size_t ic_sparse_attn_workspace_bytes(int B, int Lq, int Hq, int d, int k_slots);
 
+/*
+ * ic_sparse_attn without a workspace argument and without any allocation.
+ * The paper has no counterpart: this entry point exists for callers that
+ * cannot allocate device memory — for example a host framework that owns all
+ * GPU memory and hands a plugin only its inputs and outputs, or a decode loop
+ * that must not call cudaMalloc (it can synchronise the device and its cost is
+ * unpredictable).  Same arguments, semantics and results as ic_sparse_attn.
+ * Rows that split their slots over several CTAs (decode) keep the per-split
+ * partial results in a fixed 4 MiB array inside the library instead of a
+ * workspace; every GPU that loads the library holds that array until the
+ * process exits.
+ *   - A call whose partial results would exceed 4 MiB (rows x splits x Hq x
+ *     (d + 1) x 4 bytes) is rejected with IC_ERR_WORKSPACE_TOO_SMALL before
+ *     anything is launched; ic_sparse_attn with a workspace handles it.
+ *   - The first call on a device looks up the array's device address (once per
+ *     device, with that device current); make that first call before any
+ *     stream capture.
+ *   - All calls share the one array and it keeps the last call's contents.
+ *     Every partial a call reads is written by the same call first, so nothing
+ *     needs clearing, but calls that overlap on the GPU (different streams,
+ *     or different host threads) race on the array: serialise them.
+ */
+int ic_sparse_attn_no_alloc(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                            const int32_t *idx, int B, int Lq, int Lk, int Hq, int Hkv, int d,
+                            int k_slots, int q_offset, float scale, uint16_t *out, float *lse,
+                            ic_stream_t stream);
+
 /* One layer of the stack.  S layers may leave q_idx, k_idx and w NULL. */
 typedef struct {
     const uint16_t *q;      /* [B, Lq, Hq, d] bf16 */

@@ -342,6 +342,33 @@ int check_positions(int B, int Lq, int Lk, int q_offset) {
 
 }  // namespace
 
+// Scratch for ic_sparse_attn_no_alloc: the per-split partial results (O / l and
+// the log2-sum-exp of each row, split and head) live in this fixed device
+// array instead of a caller workspace.  Every GPU that loads the library holds
+// it until the process exits.  Host code must never hand the symbol itself to
+// a kernel (on the host it is only a stand-in); the device address comes from
+// cudaGetSymbolAddress, looked up once per device.
+constexpr size_t NOALLOC_SCRATCH_BYTES = (size_t)4 << 20;   // 4 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
+
+namespace {
+void* g_noalloc_ptr[MAX_DEV];
+
+// Device address of g_noalloc_scratch on the current device (looked up on the
+// first call per device, with that device current).
+int noalloc_scratch(int dev, void** out) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || !p) return cuda_fail(e, "cudaGetSymbolAddress(g_noalloc_scratch)");
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return IC_OK;
+}
+}  // namespace
+
 // ======================================================================= C ABI
 
 extern "C" {
@@ -449,6 +476,35 @@ int ic_sparse_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, cons
     if ((rc = device_setup(&dev, &sms))) return rc;
     return launch_attn(q, k, v, idx, B, Lq, Lk, Hq, d, k_slots, q_offset, scale, out, lse, ws,
                        ws_bytes, false, sms, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int ic_sparse_attn_no_alloc(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                            const int32_t* idx, int B, int Lq, int Lk, int Hq, int Hkv, int d,
+                            int k_slots, int q_offset, float scale, uint16_t* out, float* lse,
+                            ic_stream_t stream) {
+    int rc = check_positions(B, Lq, Lk, q_offset);
+    if (rc) return rc;
+    if ((rc = check_attn_shape(Hq, Hkv, d))) return rc;
+    if (k_slots < 1) return fail(IC_ERR_INVALID_ARG, "k=%d", k_slots);
+    if (B == 0 || Lq == 0) return IC_OK;
+    if (!q || !k || !v || !idx || !out) return fail(IC_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v))
+        return fail(IC_ERR_UNSUPPORTED, "q, k and v must be 16-byte aligned");
+    if (!std::isfinite(scale)) return fail(IC_ERR_INVALID_ARG, "scale is not finite");
+    int dev, sms;
+    if ((rc = device_setup(&dev, &sms))) return rc;
+    const long long n_rows = (long long)B * Lq;
+    const int splits = attn_splits(n_rows, k_slots, sms);
+    const size_t need = attn_ws_bytes(n_rows, splits, Hq, d);
+    if (need > NOALLOC_SCRATCH_BYTES)
+        return fail(IC_ERR_WORKSPACE_TOO_SMALL,
+                    "%lld rows x %d slot splits need %zu bytes of scratch; the built-in scratch "
+                    "holds %zu bytes (call ic_sparse_attn with a workspace instead)",
+                    n_rows, splits, need, NOALLOC_SCRATCH_BYTES);
+    void* scratch = nullptr;
+    if ((rc = noalloc_scratch(dev, &scratch))) return rc;
+    return launch_attn(q, k, v, idx, B, Lq, Lk, Hq, d, k_slots, q_offset, scale, out, lse, scratch,
+                       NOALLOC_SCRATCH_BYTES, false, sms, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t ic_layer_stack_workspace_bytes(const ic_dims* dims, int n_layers, long long rows_per_chunk) {

@@ -32,7 +32,8 @@ STATUS = {0: "IC_OK", 1: "IC_ERR_INVALID_ARG", 2: "IC_ERR_UNSUPPORTED",
 EXPORTS = ("ic_status_string", "ic_last_error_message", "ic_get_last_device_error",
            "ic_indexer_scores", "ic_topk_select", "ic_sparse_attn",
            "ic_sparse_attn_workspace_bytes", "ic_layer_stack_workspace_bytes",
-           "ic_layer_stack_forward", "ic_layer_stack_forward_events", "ic_selftest_wait_timeout")
+           "ic_layer_stack_forward", "ic_layer_stack_forward_events", "ic_selftest_wait_timeout",
+           "ic_sparse_attn_no_alloc")
 
 
 class IndexCacheError(RuntimeError):
@@ -73,6 +74,9 @@ _lib.ic_topk_select.argtypes = [_P, _I, _I, _I, _I, _I, _P, _P]
 _lib.ic_sparse_attn.restype = _I
 _lib.ic_sparse_attn.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P,
                                 _Z, _P]
+_lib.ic_sparse_attn_no_alloc.restype = _I
+_lib.ic_sparse_attn_no_alloc.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P,
+                                         _P, _P]
 _lib.ic_sparse_attn_workspace_bytes.restype = _Z
 _lib.ic_sparse_attn_workspace_bytes.argtypes = [_I, _I, _I, _I, _I]
 _lib.ic_layer_stack_workspace_bytes.restype = _Z
@@ -175,6 +179,31 @@ def sparse_attn(q, k, v, idx, q_offset: int = 0, scale: float = 0.0, out=None, l
                              _ptr(ws, None, "ws"), 0 if ws is None else ws.numel() * ws.element_size(),
                              _stream(stream))
     _check(rc, "ic_sparse_attn")
+    return out, lse
+
+
+def sparse_attn_no_alloc(q, k, v, idx, q_offset: int = 0, scale: float = 0.0, out=None,
+                         lse=None, want_lse: bool = True, stream=None):
+    """ic_sparse_attn_no_alloc: the same attention without a workspace.
+
+    For callers that cannot hand the library device memory of its own (see
+    include/indexcache.h): split partials live in the library's fixed 4 MiB
+    device array; calls that overlap on the GPU race on it.
+    """
+    B, Lq, Hq, d = q.shape
+    Lk = k.shape[1]
+    Hkv = k.shape[2] if k.dim() == 4 else 1
+    kslots = idx.shape[-1]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(B, Lq, Hq, device=q.device, dtype=torch.float32)
+    rc = _lib.ic_sparse_attn_no_alloc(_ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
+                                      _ptr(v, torch.bfloat16, "v"), _ptr(idx, torch.int32, "idx"),
+                                      B, Lq, Lk, Hq, Hkv, d, kslots, q_offset, float(scale),
+                                      _ptr(out, torch.bfloat16, "out"),
+                                      _ptr(lse, torch.float32, "lse"), _stream(stream))
+    _check(rc, "ic_sparse_attn_no_alloc")
     return out, lse
 
 

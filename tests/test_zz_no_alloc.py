@@ -1,0 +1,69 @@
+"""ic_sparse_attn_no_alloc against ic_sparse_attn, through the C ABI.
+
+The no-allocation entry point serves callers that cannot give the library any
+device memory of its own (a host framework that owns every GPU buffer and
+passes a plugin only its inputs and outputs; a decode loop that must not call
+cudaMalloc).  Its results must match the workspace-based entry point within
+the attention tolerance, on two calls in a row: the second call runs on other
+inputs and must not see anything the first call left in the shared scratch.
+
+This file is named to be collected last, so a run that stops at the first
+failure has run every other test before it.  It passes both alone in a fresh
+process and after the rest of the suite.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from lightning_indexer_top_relu_b200 import build, synth
+
+pytestmark = pytest.mark.gpu
+
+ATTN_ATOL = 2e-2
+LSE_ATOL = 1e-3
+
+
+@pytest.fixture(scope="module")
+def ic():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    build.build()
+    from lightning_indexer_top_relu_b200 import indexcache
+    return indexcache
+
+
+def _decode_case(cfg_id):
+    # decode rows: few rows, so the slots of each row are split over several
+    # CTAs and the per-split partials go through the scratch
+    wl = synth.custom(B=4, Lq=1, Lk=3000, q_offset=2999, H_I=4, d_I=64, k=2048, Hq=16, d=128,
+                      cfg_id=cfg_id)
+    L = synth.make_layers(wl)[0]
+    sc = oracle.indexer_scores(L["q_idx"], L["k_idx"], L["w"], wl.q_offset).astype(np.float32)
+    idx = oracle.topk_sort(sc, oracle.row_positions(wl.B, 1, wl.q_offset), wl.k)
+    dev = {n: L[n].cuda() for n in ("q", "k", "v")}
+    return wl, dev, torch.from_numpy(idx).reshape(wl.B, 1, wl.k).cuda()
+
+
+def test_no_alloc_matches_workspace_entry_point_twice(ic):
+    assert ic.sparse_attn_workspace_bytes(4, 1, 16, 128, 2048) > 0    # the split path is taken
+    for cfg_id in (31, 32):                                           # two calls in a row
+        wl, t, idx = _decode_case(cfg_id)
+        ref, ref_lse = ic.sparse_attn(t["q"], t["k"], t["v"], idx, wl.q_offset)
+        out, lse = ic.sparse_attn_no_alloc(t["q"], t["k"], t["v"], idx, wl.q_offset)
+        torch.cuda.synchronize()
+        assert ic.get_last_device_error() == 0
+        assert (out.float() - ref.float()).abs().max().item() <= ATTN_ATOL
+        assert (lse - ref_lse).abs().max().item() <= LSE_ATOL
+
+
+def test_no_alloc_rejects_calls_beyond_its_scratch(ic):
+    # 295 rows x 2 slot splits x 16 heads x 129 floats x 4 bytes > 4 MiB
+    B, Lk, k = 295, 200, 128
+    q = torch.zeros(B, 1, 16, 128, device="cuda", dtype=torch.bfloat16)
+    kv = torch.zeros(B, Lk, 1, 128, device="cuda", dtype=torch.bfloat16)
+    idx = torch.zeros(B, 1, k, device="cuda", dtype=torch.int32)
+    with pytest.raises(ic.IndexCacheError) as e:
+        ic.sparse_attn_no_alloc(q, kv, kv, idx, Lk - 1)
+    assert e.value.status == 4                                        # IC_ERR_WORKSPACE_TOO_SMALL
+    assert "scratch" in str(e.value)
