@@ -164,56 +164,99 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- CPU oracle leg
 
-def oracle_rows_per_s(wl, pattern, layers_cpu, budget_s=15.0, seed=5):
-    """Times the oracle on a bounded sample of query rows; returns (rows/s, sample desc)."""
+def row_slice(wl, layers, r):
+    """Host copies of what the oracle needs for flattened query row r: that
+    row's query-side tensors and its sequence's keys (a one-row problem at
+    q_offset = t, the row's absolute position)."""
+    b, i = divmod(int(r), wl.Lq)
+    out = []
+    for L in layers:
+        d = {}
+        for key in ("q", "q_idx", "w"):
+            if key in L:
+                d[key] = L[key][b:b + 1, i:i + 1].contiguous().cpu()
+        for key in ("k", "v", "k_idx"):
+            if key in L:
+                d[key] = L[key][b:b + 1].contiguous().cpu()
+        out.append(d)
+    return out, wl.q_offset + i
+
+
+def _oracle_rows(wl, pattern, sl, workers):
+    """Runs the oracle on prepared one-row problems `sl`, one row per host
+    thread (one OpenMP thread each), and returns the wall time."""
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+
+    def one(item):
+        lay, t = item
+        oracle.set_num_threads(1)
+        oracle.layer_stack(pattern, lay, wl.k, q_offset=t)
+
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(max_workers=workers) as ex:
+        list(ex.map(one, sl))
+    return time.perf_counter() - t0
+
+
+def oracle_rows_per_s(wl, pattern, layers, budget_s=15.0, seed=5):
+    """Times the oracle on uniformly drawn query rows, one row per host core,
+    for about budget_s seconds; returns (rows/s, sample description, cores)."""
     import oracle
     rng = np.random.default_rng(seed)
     total = wl.B * wl.Lq
-    n = 8
-    elapsed, done = 0.0, 0
-    while True:
-        rows = np.sort(rng.choice(total, size=min(n, total), replace=False))
-        t0 = time.perf_counter()
-        oracle.layer_stack(pattern, layers_cpu, wl.k, wl.q_offset, rows=rows)
-        dt = time.perf_counter() - t0
+    workers = max(1, oracle.num_threads())
+    elapsed, done, n = 0.0, 0, workers
+    while elapsed < budget_s and done < total:
+        rows = rng.choice(total, size=min(n, total), replace=False)
+        sl = [row_slice(wl, layers, r) for r in rows]
+        dt = _oracle_rows(wl, pattern, sl, workers)
         elapsed += dt
         done += len(rows)
-        if elapsed >= 0.8 * budget_s or done >= total:
-            break
-        # next sample sized to land near the budget
-        rate = done / elapsed
-        n = int(min(total, max(8, rate * (budget_s - elapsed))))
-    return done / elapsed, f"{done} uniformly drawn query rows of {total}, all {len(pattern)} layers, {elapsed:.1f} s"
+        rate = len(rows) / max(dt, 1e-9)
+        n = int(max(workers, min(total, rate * max(budget_s - elapsed, 0.0))))
+    return done / elapsed, (f"{done} uniformly drawn query rows of {total}, each through all "
+                            f"{len(pattern)} layers, {elapsed:.1f} s"), workers
+
+
+def input_bytes(wl, indexer_for_all=True):
+    """Bytes of per-layer inputs the stack reads (bf16 q/K/V, indexer q_I/k_I, fp32 w)."""
+    n_f = wl.n_layers if indexer_for_all else sum(c in "F1" for c in wl.pattern)
+    attn = wl.B * (wl.Lq * wl.Hq * wl.d + 2 * wl.Lk * wl.d) * 2
+    idx = wl.B * (wl.Lq * wl.H_I * wl.d_I * 2 + wl.Lk * wl.d_I * 2 + wl.Lq * wl.H_I * 4)
+    return wl.n_layers * attn + n_f * idx
 
 
 def run_reference(args, wl, pattern):
-    """The CPU oracle as the reference arm (rank 0 only)."""
+    """The CPU oracle as the reference arm (rank 0 only): each step is a
+    bounded, uniformly drawn sample of --ref-rows query rows of the workload,
+    each row through every layer of the pattern."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     import oracle
-    layers = synth.make_layers(wl, indexer_for_all=False) if pattern == wl.pattern else \
-        synth.make_layers(wl)
+    big = input_bytes(wl, True) > 2 * 2 ** 30
+    dev = torch.device("cuda") if (big and torch.cuda.is_available()) else "cpu"
+    layers = synth.make_layers(wl, indexer_for_all=any(c in "F1" for c in pattern), device=dev)
     total = wl.B * wl.Lq
     rng = np.random.default_rng(11)
     n_rows = max(1, min(total, args.ref_rows))
-    for _ in range(args.warmup if args.warmup > 0 else 0):
-        pass  # the oracle has no warm-up state; warm-up steps are not repeated
+    workers = max(1, oracle.num_threads())
     times = []
     for s in range(args.steps):
-        rows = np.sort(rng.choice(total, size=n_rows, replace=False))
-        t0 = time.perf_counter()
-        oracle.layer_stack(pattern, layers, wl.k, wl.q_offset, rows=rows)
-        times.append(time.perf_counter() - t0)
+        rows = rng.choice(total, size=n_rows, replace=False)
+        sl = [row_slice(wl, layers, r) for r in rows]
+        times.append(_oracle_rows(wl, pattern, sl, workers))
     sec = float(np.sum(times))
     value = n_rows * args.steps / sec
-    sample = f"{n_rows} uniformly drawn query rows of {total} per step, all {len(pattern)} layers"
+    sample = (f"{n_rows} uniformly drawn query rows of {total} per step, each through all "
+              f"{len(pattern)} layers")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * sec / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_of(wl, pattern, args),
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": workers,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -260,9 +303,14 @@ def main():
     ap.add_argument("--no-all-f", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=64)
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
+    ap.add_argument("--rows-per-chunk", type=int, default=0,
+                    help="F-layer score rows per chunk (0: as many as 16 GiB of scores allow)")
     args = ap.parse_args()
     wl = synth.WORKLOADS[args.workload]
     pattern = args.pattern or wl.pattern
+    if len(pattern) != wl.n_layers:
+        import dataclasses
+        wl = dataclasses.replace(wl, n_layers=len(pattern), pattern=pattern)
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":
@@ -285,12 +333,21 @@ def main():
 
     peaks = load_peaks()
     need_all = (not args.no_all_f) and any(c in "S0" for c in pattern)
-    layers_cpu = synth.make_layers(wl, indexer_for_all=need_all)
-    pinned = [{k: v.pin_memory() for k, v in L.items()} for L in layers_cpu]
-    layers = [{k: v.to(dev, non_blocking=True) for k, v in L.items()} for L in pinned]
+    in_bytes = input_bytes(wl, need_all)
+    on_device = in_bytes > 2 * 2 ** 30          # too large to draw on the host
+    if on_device:
+        layers = synth.make_layers(wl, indexer_for_all=need_all, device=dev)
+        pinned = None
+    else:
+        layers_cpu = synth.make_layers(wl, indexer_for_all=need_all)
+        pinned = [{k: v.pin_memory() for k, v in L.items()} for L in layers_cpu]
+        layers = [{k: v.to(dev, non_blocking=True) for k, v in L.items()} for L in pinned]
     torch.cuda.synchronize()
     dims = ic.make_dims(wl.B, wl.Lq, wl.Lk, wl.q_offset, wl.H_I, wl.d_I, wl.Hq, wl.d, wl.k)
-    stack = ic.LayerStack(pattern, layers, dims)
+    rpc = args.rows_per_chunk
+    if rpc <= 0:
+        rpc = max(1, min(wl.B * wl.Lq, (16 * 2 ** 30) // (4 * wl.Lk)))
+    stack = ic.LayerStack(pattern, layers, dims, rows_per_chunk=rpc)
     stream = torch.cuda.current_stream()
     n = wl.n_layers
     flush = torch.empty(256 * 1024 * 1024 // 4, device=dev, dtype=torch.float32)
@@ -412,7 +469,7 @@ def main():
 
     # ---- the same stack with every layer Full, for the F/S speed-up
     if need_all:
-        stack_f = ic.LayerStack("F" * n, layers, dims)
+        stack_f = ic.LayerStack("F" * n, layers, dims, rows_per_chunk=rpc)
         for _ in range(2):
             stack_f.forward(stream)
         ts = []
@@ -432,7 +489,9 @@ def main():
         del stack_f
 
     # ---- end to end through the public API with host buffers
-    if not args.no_e2e:
+    if not args.no_e2e and pinned is None:
+        line["e2e"] = {"skipped": f"inputs of {in_bytes / 2**30:.1f} GiB are drawn on the device"}
+    if not args.no_e2e and pinned is not None:
         outs_host = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in stack.outs]
         h2d = sum(v.numel() * v.element_size() for i, L in enumerate(pinned) for k, v in L.items()
                   if k in ("q", "k", "v") or pattern[i] in "F1")
@@ -467,8 +526,8 @@ def main():
     # ---- CPU oracle baseline (rank 0, N=1 only)
     if not args.no_cpu_baseline and world == 1:
         import oracle
-        rps, sample = oracle_rows_per_s(wl, pattern, layers_cpu, budget_s=args.cpu_budget_s)
-        line["cpu_baseline"] = {"value": rps, "unit": "tokens/s", "cores": oracle.num_threads(),
+        rps, sample, cores = oracle_rows_per_s(wl, pattern, layers, budget_s=args.cpu_budget_s)
+        line["cpu_baseline"] = {"value": rps, "unit": "tokens/s", "cores": cores,
                                 "kind": "oracle", "sample": sample}
 
     if pg is not None:

@@ -14,7 +14,7 @@
 #include <cstring>
 #include <mutex>
 
-#include "../../include/indexcache.h"
+#include "indexcache.h"
 #include "common.cuh"
 #include "indexer_scores.cuh"
 #include "sparse_attn.cuh"

@@ -95,24 +95,25 @@ def custom(name: str = "custom", *, B=1, Lq, Lk=None, n_layers=1, H_I=4, d_I=64,
                     correlated)
 
 
-def _gen(seed: int) -> torch.Generator:
-    g = torch.Generator(device="cpu")
+def _gen(seed: int, device="cpu") -> torch.Generator:
+    g = torch.Generator(device=device)
     g.manual_seed(seed)
     return g
 
 
-def _randn(shape, seed: int) -> torch.Tensor:
-    return torch.randn(*shape, generator=_gen(seed), dtype=torch.float32)
+def _randn(shape, seed: int, device="cpu") -> torch.Tensor:
+    return torch.randn(*shape, generator=_gen(seed, device), dtype=torch.float32, device=device)
 
 
 def _seed(wl: Workload, layer: int, name: str) -> int:
     return 1000 * wl.cfg_id + 10 * layer + _TID[name]
 
 
-def _low_rank(rows: int, cols: int, wl: Workload, pname: str, batch: int) -> torch.Tensor:
+def _low_rank(rows: int, cols: int, wl: Workload, pname: str, batch: int,
+              device="cpu") -> torch.Tensor:
     """Unit-variance rank-16 matrix [batch, rows, cols] shared by every layer."""
-    a = _randn((batch, rows, RANK), _seed(wl, 99, "a"))
-    p = _randn((RANK, cols), _seed(wl, 99, pname))
+    a = _randn((batch, rows, RANK), _seed(wl, 99, "a"), device)
+    p = _randn((RANK, cols), _seed(wl, 99, pname), device)
     return (a @ p) / math.sqrt(RANK)
 
 
@@ -121,12 +122,14 @@ def _mix(shared: torch.Tensor, noise: torch.Tensor, rho: float) -> torch.Tensor:
 
 
 def make_layers(wl: Workload, layers: Optional[List[int]] = None, indexer_for_all: bool = True,
-                rho: float = RHO_INDEXER) -> List[Dict[str, torch.Tensor]]:
-    """Draw the per-layer inputs on the CPU (bf16 operands, fp32 head weights).
+                rho: float = RHO_INDEXER, device="cpu") -> List[Dict[str, torch.Tensor]]:
+    """Draw the per-layer inputs (bf16 operands, fp32 head weights).
 
     Returns a list of dicts with 'q', 'k', 'v' ([B,L,Hq,d] and [B,Lk,1,d]) and,
     for F layers (or every layer when indexer_for_all), 'q_idx' [B,Lq,H_I,d_I],
-    'k_idx' [B,Lk,d_I], 'w' [B,Lq,H_I].
+    'k_idx' [B,Lk,d_I], 'w' [B,Lq,H_I].  device='cuda' draws with device
+    generators (same seeds, different random streams than the CPU ones) for
+    workloads too large to draw on the host.
     """
     B, Lq, Lk = wl.B, wl.Lq, wl.Lk
     layers = list(range(wl.n_layers)) if layers is None else list(layers)
@@ -154,24 +157,25 @@ def make_layers(wl: Workload, layers: Optional[List[int]] = None, indexer_for_al
             out.append(d)
         return out
 
-    k_shared = _low_rank(Lk, wl.d_I, wl, "p_idx", B)
-    kv_k = _low_rank(Lk, wl.d, wl, "p_k", B)
-    kv_v = _low_rank(Lk, wl.d, wl, "p_v", B)
+    dev = device
+    k_shared = _low_rank(Lk, wl.d_I, wl, "p_idx", B, dev)
+    kv_k = _low_rank(Lk, wl.d, wl, "p_k", B, dev)
+    kv_v = _low_rank(Lk, wl.d, wl, "p_v", B, dev)
     q_shared = w_shared = None
     for l in layers:
         d: Dict[str, torch.Tensor] = {}
-        d["q"] = (_randn((B, Lq, wl.Hq, wl.d), _seed(wl, l, "q")) / math.sqrt(wl.d)).to(torch.bfloat16)
-        ek = _randn((B, Lk, wl.d), _seed(wl, l, "k"))
-        ev = _randn((B, Lk, wl.d), _seed(wl, l, "v"))
+        d["q"] = (_randn((B, Lq, wl.Hq, wl.d), _seed(wl, l, "q"), dev) / math.sqrt(wl.d)).to(torch.bfloat16)
+        ek = _randn((B, Lk, wl.d), _seed(wl, l, "k"), dev)
+        ev = _randn((B, Lk, wl.d), _seed(wl, l, "v"), dev)
         d["k"] = (_mix(kv_k, ek, RHO_KV) / math.sqrt(wl.d)).to(torch.bfloat16).reshape(B, Lk, 1, wl.d)
         d["v"] = (_mix(kv_v, ev, RHO_KV) / math.sqrt(wl.d)).to(torch.bfloat16).reshape(B, Lk, 1, wl.d)
         if indexer_for_all or wl.pattern[l] in "F1":
             if q_shared is None:
-                q_shared = _randn((B, Lq, wl.H_I, wl.d_I), _seed(wl, 99, "q_idx"))
-                w_shared = _randn((B, Lq, wl.H_I), _seed(wl, 99, "w"))
-            qi = _mix(q_shared, _randn((B, Lq, wl.H_I, wl.d_I), _seed(wl, l, "q_idx")), rho)
-            ki = _mix(k_shared, _randn((B, Lk, wl.d_I), _seed(wl, l, "k_idx")), rho)
-            wi = _mix(w_shared, _randn((B, Lq, wl.H_I), _seed(wl, l, "w")), rho)
+                q_shared = _randn((B, Lq, wl.H_I, wl.d_I), _seed(wl, 99, "q_idx"), dev)
+                w_shared = _randn((B, Lq, wl.H_I), _seed(wl, 99, "w"), dev)
+            qi = _mix(q_shared, _randn((B, Lq, wl.H_I, wl.d_I), _seed(wl, l, "q_idx"), dev), rho)
+            ki = _mix(k_shared, _randn((B, Lk, wl.d_I), _seed(wl, l, "k_idx"), dev), rho)
+            wi = _mix(w_shared, _randn((B, Lq, wl.H_I), _seed(wl, l, "w"), dev), rho)
             d["q_idx"] = (qi / math.sqrt(wl.d_I)).to(torch.bfloat16)
             d["k_idx"] = (ki / math.sqrt(wl.d_I)).to(torch.bfloat16)
             d["w"] = (wi / math.sqrt(wl.H_I)).contiguous()

@@ -64,6 +64,8 @@ def _load():
         for f in ("or_indexer_scores", "or_topk_sort", "or_topk_count", "or_sparse_attn",
                   "or_dense_attn", "or_num_threads"):
             getattr(lib, f).restype = ctypes.c_int
+        lib.or_set_num_threads.argtypes = [I]
+        lib.or_set_num_threads.restype = None
         _lib = lib
     return _lib
 
@@ -71,6 +73,11 @@ def _load():
 def num_threads() -> int:
     """Threads the oracle's OpenMP loops use."""
     return int(_load().or_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Threads this host thread's later oracle calls use."""
+    _load().or_set_num_threads(int(n))
 
 
 # ---------------------------------------------------------------- marshalling

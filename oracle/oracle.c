@@ -59,6 +59,17 @@ int or_num_threads(void)
 #endif
 }
 
+/* Threads the calling host thread's later oracle calls use (OpenMP's
+ * per-thread setting); lets a pool of host threads run one row each. */
+void or_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
 /*
  * Step a1, lightning indexer score (Abstract of the IndexCache digest; the
  * score form is the standard one stated in the header above).
