@@ -7,26 +7,37 @@
 // which later S layers reuse; the tie rule and the output order are this
 // library's reading, the pages do not state them).
 //
-// Method: scores map to order-preserving 32-bit keys (-0 folded onto +0, so
-// the order is the IEEE one).  Three radix passes (11, 11 and 10 bits, from
-// the top) find the exact key T of the k-th largest element and how many of
-// the k come from elements equal to T.  One last index-ordered pass emits
-// every element > T plus the first `need` elements == T, each at its output
-// slot found by a block-wide prefix count, so the output comes out sorted by
-// position with no sort.  Rows that fit in shared memory are read from HBM
-// once; longer rows are re-read from L2 on each pass.
+// Method (one CTA per row):
+//   1. One pass over the row maps every score to an order-preserving 32-bit
+//      key (-0 folded onto +0, so the order is the IEEE one), keeps the keys
+//      in shared memory when the row fits, and histograms the top 11 bits.
+//   2. A suffix scan of the 2048 bins finds the bin holding the k-th largest
+//      key.  Only that bin's keys (typically a few percent of the row) are
+//      gathered as candidates, with one shared atomic per warp (ballot +
+//      popc); two more radix passes (11 + 10 bits) over the candidates give
+//      the exact k-th key T and `need`, how many keys equal to T are kept.
+//   3. A final pass in position order emits every key > T and the first
+//      `need` keys == T: each warp owns a contiguous segment, counts it with
+//      ballots, one block-wide scan of the per-warp counts gives every
+//      warp's first output slot, and the warp writes its selections at
+//      ballot-prefix offsets -- sorted output, no sort.
+// Every pass loads a whole batch (up to TK_VB float4 per thread) before
+// using any of it, so a row costs one memory latency per batch instead of
+// one per element.  Rows too long for shared memory re-read their scores
+// from L2 in steps 2-3, batched the same way.
 #pragma once
 
 #include "common.cuh"
 
 namespace ic {
 
-constexpr int TK_THREADS = 512;
+constexpr int TK_THREADS = 256;
 constexpr int TK_WARPS = TK_THREADS / 32;
 constexpr int TK_BINS = 2048;
-constexpr int TK_ITEMS = 4;                                  // consecutive elements per thread
-constexpr int TK_SMEM_FIXED = TK_BINS * 4 + 64 * 8 + 64;     // histogram + scan scratch
-constexpr int TK_CACHE_MAX = 40960;                          // longest row kept in shared memory
+constexpr int TK_CAND = 2048;                                     // candidate keys kept in smem
+constexpr int TK_SMEM_FIXED = TK_BINS * 4 + TK_CAND * 4 + 256;    // hist + candidates + scratch
+constexpr int TK_CACHE_MAX = 45056;                               // longest row kept in smem
+constexpr int TK_VB = 8;                                          // float4 loads in flight per thread
 
 __device__ __forceinline__ uint32_t score_key(float f) {
     uint32_t u = __float_as_uint(f);
@@ -34,34 +45,42 @@ __device__ __forceinline__ uint32_t score_key(float f) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Block-wide exclusive scan of a 64-bit value; returns the exclusive prefix
-// and sets `total`.  Every thread of the block must call it.
-__device__ __forceinline__ unsigned long long tk_block_excl_scan(unsigned long long v,
-                                                                 unsigned long long* scratch,
-                                                                 unsigned long long& total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    unsigned long long x = v;
+// Suffix scan of the 2048-bin histogram: finds the bin b whose count makes
+// the running total (from the top bin down) reach `remaining`.  Writes
+// found[0] = b, found[1] = count of elements in bins above b.  All threads.
+__device__ __forceinline__ void tk_find_bin(const uint32_t* hist, int remaining, int* found,
+                                            unsigned* wsum) {
+    constexpr int PER = TK_BINS / TK_THREADS;      // 8 bins per thread, top bins first
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int hi = TK_BINS - 1 - PER * tid;
+    uint32_t h[PER];
+    uint32_t mine = 0;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+        h[e] = hist[hi - e];
+        mine += h[e];
+    }
+    uint32_t x = mine;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        unsigned long long y = __shfl_up_sync(0xffffffffu, x, o);
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
         if (lane >= o) x += y;
     }
-    if (lane == 31) scratch[warp] = x;
+    if (lane == 31) wsum[warp] = x;
     __syncthreads();
-    if (warp == 0) {
-        unsigned long long y = lane < TK_WARPS ? scratch[lane] : 0ull;
+    uint32_t before = 0;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            unsigned long long z = __shfl_up_sync(0xffffffffu, y, o);
-            if (lane >= o) y += z;
+    for (int w = 0; w < TK_WARPS; ++w) before += (w < warp) ? wsum[w] : 0u;
+    uint32_t above = before + x - mine;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+        if (above < (uint32_t)remaining && above + h[e] >= (uint32_t)remaining) {
+            found[0] = hi - e;
+            found[1] = (int)above;
         }
-        if (lane < TK_WARPS) scratch[32 + lane] = y;
+        above += h[e];
     }
     __syncthreads();
-    const unsigned long long before = warp > 0 ? scratch[32 + warp - 1] : 0ull;
-    total = scratch[32 + TK_WARPS - 1];
-    __syncthreads();
-    return before + x - v;
 }
 
 // Rows [row_base, row_base + n_rows) of a [B*Lq] flattened row space; score
@@ -73,11 +92,14 @@ topk_select_kernel(const float* __restrict__ scores, long long ld, long long row
                    int32_t* __restrict__ idx) {
     extern __shared__ __align__(16) uint8_t tk_smem[];
     uint32_t* hist = reinterpret_cast<uint32_t*>(tk_smem);
-    unsigned long long* scratch = reinterpret_cast<unsigned long long*>(tk_smem + TK_BINS * 4);
-    int* found = reinterpret_cast<int*>(tk_smem + TK_BINS * 4 + 64 * 8);
+    uint32_t* cand = reinterpret_cast<uint32_t*>(tk_smem + TK_BINS * 4);
+    int* found = reinterpret_cast<int*>(tk_smem + TK_BINS * 4 + TK_CAND * 4);      // [0..3]
+    unsigned* wsum = reinterpret_cast<unsigned*>(found + 4);                        // [TK_WARPS]
+    unsigned* wgt = wsum + TK_WARPS;                                                // [TK_WARPS]
+    unsigned* weq = wgt + TK_WARPS;                                                 // [TK_WARPS]
     uint32_t* keys = reinterpret_cast<uint32_t*>(tk_smem + TK_SMEM_FIXED);
 
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const long long rr = n_rows - 1 - (long long)blockIdx.x;   // longest rows first
     const long long r = row_base + rr;
     const int t = q_offset + (int)(r % Lq);
@@ -89,92 +111,165 @@ topk_select_kernel(const float* __restrict__ scores, long long ld, long long row
         return;
     }
     const float* src = scores + rr * ld;
-    if (CACHE) {
-        for (int i = tid; i < n; i += TK_THREADS) keys[i] = score_key(src[i]);
-    }
     auto key_at = [&](int i) -> uint32_t { return CACHE ? keys[i] : score_key(__ldg(src + i)); };
 
-    if (tid == 0) {
-        found[0] = 0;
-        found[1] = 0;
+    // ---- 1. keys + top-11-bit histogram in one pass
+    for (int b = tid; b < TK_BINS; b += TK_THREADS) hist[b] = 0;
+    if (tid == 0) found[2] = 0;                                // candidate count
+    __syncthreads();
+    const bool vec = ((reinterpret_cast<uintptr_t>(src) & 15) == 0);
+    const int nv = vec ? (n & ~3) : 0;
+    for (int base = 0; base < nv; base += TK_THREADS * 4 * TK_VB) {
+        float4 f[TK_VB];
+#pragma unroll
+        for (int u = 0; u < TK_VB; ++u) {           // all loads of the batch first
+            const int i = base + (u * TK_THREADS + tid) * 4;
+            f[u] = i < nv ? __ldg(reinterpret_cast<const float4*>(src + i))
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < TK_VB; ++u) {
+            const int i = base + (u * TK_THREADS + tid) * 4;
+            if (i < nv) {
+                const uint32_t k0 = score_key(f[u].x), k1 = score_key(f[u].y),
+                               k2 = score_key(f[u].z), k3 = score_key(f[u].w);
+                if (CACHE) *reinterpret_cast<uint4*>(keys + i) = make_uint4(k0, k1, k2, k3);
+                atomicAdd(&hist[k0 >> 21], 1u);
+                atomicAdd(&hist[k1 >> 21], 1u);
+                atomicAdd(&hist[k2 >> 21], 1u);
+                atomicAdd(&hist[k3 >> 21], 1u);
+            }
+        }
     }
-    uint32_t prefix = 0, pmask = 0;
-    int remaining = k;
-#pragma unroll 1
-    for (int pass = 0; pass < 3; ++pass) {
-        const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-        const uint32_t dmask = pass == 2 ? 0x3FFu : 0x7FFu;
+    for (int i = nv + tid; i < n; i += TK_THREADS) {
+        const uint32_t kk = score_key(__ldg(src + i));
+        if (CACHE) keys[i] = kk;
+        atomicAdd(&hist[kk >> 21], 1u);
+    }
+    __syncthreads();
+
+    tk_find_bin(hist, k, found, wsum);
+    const uint32_t b1 = (uint32_t)found[0];
+    int remaining = k - found[1];
+    const uint32_t cnt1 = hist[b1];
+    __syncthreads();                                           // hist is reused below
+
+    // ---- 2. candidates of the threshold bin, then two radix passes on them
+    uint32_t prefix = b1 << 21;
+    uint32_t pmask = 0x7FFu << 21;
+    const bool use_cand = cnt1 <= (uint32_t)TK_CAND;
+    if (use_cand) {
+        for (int gbase = warp * 32 * TK_VB; gbase < n; gbase += TK_THREADS * TK_VB) {
+            uint32_t kb[TK_VB];
+#pragma unroll
+            for (int u = 0; u < TK_VB; ++u) {
+                const int i = gbase + u * 32 + lane;
+                kb[u] = i < n ? key_at(i) : 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < TK_VB; ++u) {
+                const int i = gbase + u * 32 + lane;
+                const bool m = i < n && (kb[u] >> 21) == b1;
+                const unsigned bal = __ballot_sync(0xffffffffu, m);
+                if (bal) {
+                    unsigned pos0 = 0;
+                    if (lane == 0) pos0 = atomicAdd(reinterpret_cast<unsigned*>(&found[2]), __popc(bal));
+                    pos0 = __shfl_sync(0xffffffffu, pos0, 0);
+                    if (m) cand[pos0 + __popc(bal & ((1u << lane) - 1u))] = kb[u];
+                }
+            }
+        }
+    }
+    for (int pass = 1; pass < 3; ++pass) {
+        const int shift = pass == 1 ? 10 : 0;
+        const uint32_t dmask = pass == 1 ? 0x7FFu : 0x3FFu;
         for (int b = tid; b < TK_BINS; b += TK_THREADS) hist[b] = 0;
         __syncthreads();
-        for (int i = tid; i < n; i += TK_THREADS) {
-            const uint32_t key = key_at(i);
-            if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1u);
-        }
-        __syncthreads();
-        // Thread tid owns bins [hi-3, hi] with hi = 2047 - 4*tid (top bins first).
-        const int hi = TK_BINS - 1 - 4 * tid;
-        uint32_t h[4];
-        unsigned long long mine = 0;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            h[e] = hist[hi - e];
-            mine += h[e];
-        }
-        unsigned long long tot;
-        unsigned long long above = tk_block_excl_scan(mine, scratch, tot);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            if (above < (unsigned long long)remaining && above + h[e] >= (unsigned long long)remaining) {
-                found[0] = hi - e;
-                found[1] = (int)above;
+        if (use_cand) {
+            for (int i = tid; i < (int)cnt1; i += TK_THREADS) {
+                const uint32_t kk = cand[i];
+                if ((kk & pmask) == prefix) atomicAdd(&hist[(kk >> shift) & dmask], 1u);
             }
-            above += h[e];
+        } else {
+            for (int base = 0; base < n; base += TK_THREADS * TK_VB) {
+                uint32_t kb[TK_VB];
+#pragma unroll
+                for (int u = 0; u < TK_VB; ++u) {
+                    const int i = base + u * TK_THREADS + tid;
+                    kb[u] = i < n ? key_at(i) : 0u;
+                }
+#pragma unroll
+                for (int u = 0; u < TK_VB; ++u) {
+                    const int i = base + u * TK_THREADS + tid;
+                    if (i < n && (kb[u] & pmask) == prefix)
+                        atomicAdd(&hist[(kb[u] >> shift) & dmask], 1u);
+                }
+            }
         }
         __syncthreads();
-        const uint32_t digit = (uint32_t)found[0];
+        tk_find_bin(hist, remaining, found, wsum);
         remaining -= found[1];
-        prefix |= digit << shift;
+        prefix |= (uint32_t)found[0] << shift;
         pmask |= dmask << shift;
         __syncthreads();
     }
     const uint32_t T = prefix;
-    const int need = remaining;   // elements equal to T that are kept, lowest positions first
+    const int need = remaining;   // keys equal to T that are kept, lowest positions first
 
-    long long base_gt = 0, base_eq = 0;
-#pragma unroll 1
-    for (int tile = 0; tile < n; tile += TK_THREADS * TK_ITEMS) {
-        const int i0 = tile + tid * TK_ITEMS;
-        uint32_t kk[TK_ITEMS];
-        uint32_t cgt = 0, ceq = 0;
+    // ---- 3. emit in position order: warp w owns [w*seg, (w+1)*seg)
+    const int seg = ((n + TK_WARPS * 32 - 1) / (TK_WARPS * 32)) * 32;
+    const int s0 = min(n, warp * seg), s1 = min(n, s0 + seg);
+    unsigned cg = 0, ce = 0;
+    for (int gbase = s0; gbase < s1; gbase += 32 * TK_VB) {
+        uint32_t kb[TK_VB];
 #pragma unroll
-        for (int e = 0; e < TK_ITEMS; ++e) {
-            const int i = i0 + e;
-            kk[e] = i < n ? key_at(i) : 0u;
-            if (i < n) {
-                cgt += kk[e] > T;
-                ceq += kk[e] == T;
-            }
+        for (int u = 0; u < TK_VB; ++u) {
+            const int i = gbase + u * 32 + lane;
+            kb[u] = i < s1 ? key_at(i) : 0u;
         }
-        unsigned long long tot;
-        const unsigned long long ex =
-            tk_block_excl_scan(((unsigned long long)cgt << 32) | ceq, scratch, tot);
-        long long g = base_gt + (long long)(ex >> 32);
-        long long q = base_eq + (long long)(ex & 0xFFFFFFFFull);
 #pragma unroll
-        for (int e = 0; e < TK_ITEMS; ++e) {
-            const int i = i0 + e;
-            if (i >= n) break;
-            if (kk[e] > T) {
-                const long long pos = g + min(q, (long long)need);
-                if (pos < k) out[pos] = i;
-                ++g;
-            } else if (kk[e] == T) {
-                if (q < need && g + q < k) out[g + q] = i;
-                ++q;
-            }
+        for (int u = 0; u < TK_VB; ++u) {
+            const int i = gbase + u * 32 + lane;
+            cg += __popc(__ballot_sync(0xffffffffu, i < s1 && kb[u] > T));
+            ce += __popc(__ballot_sync(0xffffffffu, i < s1 && kb[u] == T));
         }
-        base_gt += (long long)(tot >> 32);
-        base_eq += (long long)(tot & 0xFFFFFFFFull);
+    }
+    if (lane == 0) {
+        wgt[warp] = cg;
+        weq[warp] = ce;
+    }
+    __syncthreads();
+    unsigned g = 0, e = 0;
+#pragma unroll
+    for (int w = 0; w < TK_WARPS; ++w) {
+        g += (w < warp) ? wgt[w] : 0u;
+        e += (w < warp) ? weq[w] : 0u;
+    }
+    const unsigned lt = (1u << lane) - 1u;
+    for (int gbase = s0; gbase < s1; gbase += 32 * TK_VB) {
+        uint32_t kb[TK_VB];
+#pragma unroll
+        for (int u = 0; u < TK_VB; ++u) {
+            const int i = gbase + u * 32 + lane;
+            kb[u] = i < s1 ? key_at(i) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < TK_VB; ++u) {
+            const int i = gbase + u * 32 + lane;
+            const unsigned mg = __ballot_sync(0xffffffffu, i < s1 && kb[u] > T);
+            const unsigned me = __ballot_sync(0xffffffffu, i < s1 && kb[u] == T);
+            const unsigned gi = g + __popc(mg & lt);
+            const unsigned ei = e + __popc(me & lt);
+            if ((mg >> lane) & 1u) {
+                const unsigned pos = gi + min(ei, (unsigned)need);
+                if (pos < (unsigned)k) out[pos] = i;
+            } else if (((me >> lane) & 1u) && ei < (unsigned)need) {
+                const unsigned pos = gi + ei;
+                if (pos < (unsigned)k) out[pos] = i;
+            }
+            g += __popc(mg);
+            e += __popc(me);
+        }
     }
 }
 
