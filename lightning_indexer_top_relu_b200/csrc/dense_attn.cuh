@@ -1,0 +1,347 @@
+// Sparse MQA attention for rows whose top-k covers a large share of their
+// visible positions, computed tile-dense on the tensor cores (sm_100a).
+//
+// The result is the same softmax over the selected positions as the gather
+// kernel (sparse_attn.cuh): a row's selection becomes a bitmask, and every
+// position outside it gets probability exactly 0.  When a row keeps k of
+// t+1 <= ~4k visible positions, sharing each K/V tile between the 8 queries
+// x 16 heads of a block and running the contractions on tcgen05 moves far
+// fewer bytes and runs far more flops per byte than gathering k rows per
+// query (IndexCache: every layer attends over the k cached positions; MQA).
+//
+// Per CTA: one block of 128/Hq queries x Hq heads = 128 rows (TMEM lanes);
+// two CTAs share an SM so one's MMAs overlap the other's softmax.
+//   warp 0      TMA: the Q block once; per 64-key tile, K[keys, d] and
+//               V^T[d, keys] (a per-layer transposed copy) into a 2-stage ring
+//   warp 1      TMEM allocation + MMA issue: S = Q K^T (M=128, N=64, K=d)
+//               into TMEM, then O += P V (A = P from shared memory, B = V^T
+//               tile; O accumulates in TMEM across tiles)
+//   warps 2..5  softmax: thread = row = TMEM lane.  Reads S twice (tile max,
+//               then exp2), masks it with the row's bitmask (prefetched one
+//               tile ahead), writes P as bf16 into a 128-byte-swizzled shared
+//               tile.  The running max is raised lazily: only when a tile's max
+//               exceeds it by more than 8 (log2 units) is O rescaled in TMEM,
+//               so P stays <= 2^8 and O / l is exact either way.
+// Scores are scaled in the log2 domain; masked positions contribute exactly 0.
+#pragma once
+
+#include "common.cuh"
+
+namespace ic {
+
+constexpr int DA_THREADS = 192;                  // 2 control warps + 4 softmax warps
+constexpr int DA_TILE = 64;                      // keys per tile
+constexpr float DA_RESCALE = 8.0f;               // lazy-max threshold (log2 units)
+
+struct DenseAttnArgs {
+    const uint32_t* mask;      // [B * Lq_d, W] bitmask of selected positions, row b*Lq_d + i
+    __nv_bfloat16* out;        // [B, Lq, Hq, 128]
+    float* lse;                // [B, Lq, Hq] or null
+    int Lq, Lk, Hq, q_offset;
+    int Lq_d;                  // rows i < Lq_d of each sequence take this path
+    int QBD;                   // queries per block (128 / Hq)
+    int nqb_d;                 // blocks per sequence on this path
+    int W;                     // mask words per row
+    int n_blocks;              // B * nqb_d
+    float scale_log2;
+};
+
+struct DenseSmem {
+    static constexpr int Q_BYTES = 128 * 128 * 2;            // 128 rows x 128 d (two 64-col boxes)
+    static constexpr int K_BYTES = 64 * 128 * 2;             // 64 keys x 128 d (two boxes)
+    static constexpr int V_BYTES = 128 * 64 * 2;             // 128 d x 64 keys (one box)
+    static constexpr int P_BYTES = 128 * 64 * 2;             // 128 rows x 64 keys (one box)
+    static constexpr int STAGE = K_BYTES + V_BYTES;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_ST = OFF_Q + Q_BYTES;           // 2 stages
+    static constexpr int OFF_P = OFF_ST + 2 * STAGE;
+    static constexpr int OFF_BAR = OFF_P + P_BYTES;
+    static constexpr int N_BARS = 1 + 2 + 2 + 3;
+    static constexpr int OFF_SLOT = OFF_BAR + N_BARS * 8;
+    static constexpr int BYTES = OFF_SLOT + 16;
+    // Up to 1024 B of slack for the 1024-B alignment of the swizzled tiles,
+    // capped so that two CTAs (plus their 1 KB reserved each) fit the SM's
+    // 228 KB; the kernel checks that the aligned layout fits.
+    static constexpr int PAIR_MAX = 233472 / 2 - 1024;
+    static constexpr int ALLOC = (BYTES + 1024) < PAIR_MAX ? (BYTES + 1024) : PAIR_MAX;
+    static_assert(BYTES <= PAIR_MAX, "two CTAs must fit one SM");
+};
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// tmap_q: q as 3-D {128, Lq*Hq, B}, box {64, 128, 1}; tmap_k: K as {128, Lk, B},
+// box {64, 64, 1}; tmap_vt: V^T as {Lk_d, 128, B} (rows padded), box {64, 128, 1}.
+__global__ void __launch_bounds__(DA_THREADS, 2)
+dense_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                  const __grid_constant__ CUtensorMap tmap_k,
+                  const __grid_constant__ CUtensorMap tmap_vt, const DenseAttnArgs a) {
+    using S = DenseSmem;
+    extern __shared__ uint8_t da_raw[];
+    uint8_t* smem = align_smem_1024(da_raw, S::BYTES);
+    if (smem == nullptr) return;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
+    uint64_t* q_full = bars;
+    uint64_t* kv_full = bars + 1;
+    uint64_t* kv_empty = bars + 3;
+    uint64_t* s_full = bars + 5;
+    uint64_t* p_full = bars + 6;
+    uint64_t* o_full = bars + 7;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::OFF_SLOT);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = a.n_blocks - 1 - (int)blockIdx.x;             // longest rows first
+    const int b = g / a.nqb_d;
+    const int i0 = (g % a.nqb_d) * a.QBD;
+    const int t_last = a.q_offset + i0 + a.QBD - 1;
+    const int nt = (min(t_last + 1, a.Lk) + DA_TILE - 1) / DA_TILE;
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&kv_full[i], 1);
+            mbar_init(&kv_empty[i], 1);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(p_full, 128);
+        mbar_init(o_full, 1);
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;          // S at +0 (64 cols), O at +64 (128 cols)
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tma_prefetch_desc(&tmap_q);
+            tma_prefetch_desc(&tmap_k);
+            tma_prefetch_desc(&tmap_vt);
+            mbar_arrive_expect_tx(q_full, (uint32_t)S::Q_BYTES);
+            for (int kb = 0; kb < 2; ++kb)
+                tma_load_3d(smem + S::OFF_Q + kb * 128 * 128, &tmap_q, q_full, kb * 64,
+                            i0 * a.Hq, b);
+            int j = 0;
+            for (; j < nt; ++j) {
+                const int st = j & 1;
+                if (!mbar_wait(&kv_empty[st], ((j >> 1) & 1) ^ 1)) break;
+                uint8_t* stg = smem + S::OFF_ST + st * S::STAGE;
+                mbar_arrive_expect_tx(&kv_full[st], (uint32_t)S::STAGE);
+                for (int kb = 0; kb < 2; ++kb)
+                    tma_load_3d(stg + kb * 64 * 128, &tmap_k, &kv_full[st], kb * 64, j * DA_TILE, b);
+                tma_load_3d(stg + S::K_BYTES, &tmap_vt, &kv_full[st], j * DA_TILE, 0, b);
+            }
+            mbar_wait(q_full, 0);
+            for (int c = (j > 2 ? j - 2 : 0); c < j; ++c) mbar_wait(&kv_full[c & 1], (c >> 1) & 1);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc_s = idesc_bf16_f32(128, DA_TILE);
+            const uint32_t idesc_o = idesc_bf16_f32(128, 128);
+            const uint32_t q_addr = smem_u32(smem + S::OFF_Q);
+            const uint32_t p_addr = smem_u32(smem + S::OFF_P);
+            bool ok = mbar_wait(q_full, 0);
+            for (int j = 0; j < nt && ok; ++j) {
+                const int st = j & 1;
+                if (!mbar_wait(&kv_full[st], (j >> 1) & 1)) break;
+                tc_fence_after();
+                const uint32_t k_addr = smem_u32(smem + S::OFF_ST + st * S::STAGE);
+                const uint32_t v_addr = k_addr + S::K_BYTES;
+                // S = Q K^T: the softmax warps read the previous S before they
+                // released the previous P, which this thread waited for.
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t qo = (uint32_t)((kk >> 2) * 128 * 128 + (kk & 3) * 32);
+                    const uint32_t ko = (uint32_t)((kk >> 2) * 64 * 128 + (kk & 3) * 32);
+                    tc_mma_f16(tmem, sw128_kmajor_desc(q_addr + qo), sw128_kmajor_desc(k_addr + ko),
+                               idesc_s, kk > 0 ? 1u : 0u);
+                }
+                tc_commit(s_full);
+                if (!mbar_wait(p_full, j & 1)) break;
+                tc_fence_after();
+                // O += P V   (A = P [rows x 64 keys], B = V^T tile [128 d x 64 keys])
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint32_t off = (uint32_t)(kk * 32);
+                    tc_mma_f16(tmem + 64, sw128_kmajor_desc(p_addr + off),
+                               sw128_kmajor_desc(v_addr + off), idesc_o,
+                               (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                tc_commit(o_full);
+                tc_commit(&kv_empty[st]);
+            }
+        }
+    } else {
+        // ---------------- softmax warps: thread = row r = (query r / Hq, head r % Hq)
+        const int wq = warp & 3;
+        const int r = wq * 32 + lane;
+        const int qi = r / a.Hq, h = r % a.Hq;
+        const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
+        const bool row_ok = i0 + qi < a.Lq_d;
+        const uint32_t* mrow = a.mask + (long long)(b * a.Lq_d + (row_ok ? i0 + qi : 0)) * a.W;
+        uint8_t* prow = smem + S::OFF_P + r * 128;
+        float m_used = -INFINITY, l_run = 0.0f;
+        bool ok = true;
+        auto load_mask = [&](int j, uint32_t& w0, uint32_t& w1) {
+            const int wi = j * 2;
+            w0 = (row_ok && wi < a.W) ? __ldg(mrow + wi) : 0u;
+            w1 = (row_ok && wi + 1 < a.W) ? __ldg(mrow + wi + 1) : 0u;
+        };
+        uint32_t nm0, nm1;
+        load_mask(0, nm0, nm1);
+        for (int j = 0; j < nt; ++j) {
+            const uint32_t mw[2] = {nm0, nm1};
+            if (j + 1 < nt) load_mask(j + 1, nm0, nm1);         // one tile ahead
+            if (!mbar_wait(s_full, j & 1)) { ok = false; break; }
+            tc_fence_after();
+            // pass 1: tile max over the selected positions
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tmem + lane_base + c * 32, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    if ((mw[c] >> e) & 1u) mx = fmaxf(mx, __uint_as_float(v[e]));
+            }
+            const float mxs = mx * a.scale_log2;
+            // O from the previous tile's P V must be complete before O is
+            // rescaled here or the next P V is let in.
+            if (j > 0) {
+                if (!mbar_wait(o_full, (j - 1) & 1)) { ok = false; break; }
+                tc_fence_after();
+            }
+            if (mxs > m_used + DA_RESCALE) {
+                const float alpha = exp2f(m_used - mxs);            // 0 on the first raise
+                if (j > 0) {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t v[32];
+                        tmem_ld_32x32b_x32(tmem + 64 + lane_base + c * 32, v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+                        tmem_st_32x32b_x32(tmem + 64 + lane_base + c * 32, v);
+                    }
+                    tmem_st_wait();
+                }
+                l_run *= alpha;
+                m_used = mxs;
+            }
+            const float base = m_used == -INFINITY ? 0.0f : m_used;
+            // pass 2: probabilities -> bf16 P tile (128-byte swizzled, K-major)
+            float rs = 0.0f;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tmem + lane_base + c * 32, v);
+                tmem_ld_wait();
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    const float p0 = ((mw[c] >> e) & 1u)
+                                         ? exp2f(__uint_as_float(v[e]) * a.scale_log2 - base) : 0.0f;
+                    const float p1 = ((mw[c] >> (e + 1)) & 1u)
+                                         ? exp2f(__uint_as_float(v[e + 1]) * a.scale_log2 - base) : 0.0f;
+                    rs += p0 + p1;
+                    __nv_bfloat162 pp = __floats2bfloat162_rn(p0, p1);
+                    pk[e >> 1] = *reinterpret_cast<uint32_t*>(&pp);
+                }
+                // keys c*32 .. c*32+31 = 16-byte chunks c*4 .. c*4+3
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int cc = c * 4 + u;
+                    *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) =
+                        make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+                }
+            }
+            l_run += rs;
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(p_full);
+        }
+        if (ok && nt > 0) {
+            ok = mbar_wait(o_full, (nt - 1) & 1);
+            tc_fence_after();
+        }
+        if (ok && i0 + qi < a.Lq) {
+            const long long orow = ((long long)b * a.Lq + i0 + qi) * a.Hq + h;
+            const float inv = l_run > 0.0f ? 1.0f / l_run : 0.0f;
+            uint4* dst = reinterpret_cast<uint4*>(a.out + orow * 128);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tmem + 64 + lane_base + c * 32, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        __nv_bfloat162 pp = __floats2bfloat162_rn(__uint_as_float(v[8 * u + 2 * e]) * inv,
+                                                                  __uint_as_float(v[8 * u + 2 * e + 1]) * inv);
+                        w[e] = *reinterpret_cast<uint32_t*>(&pp);
+                    }
+                    dst[c * 4 + u] = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+            if (a.lse) a.lse[orow] = l_run > 0.0f ? (m_used + log2f(l_run)) * LN2 : -INFINITY;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+// Bitmask of each row's selected positions: row p (= b*Lq_d + i, i < Lq_d)
+// of `mask` gets bit s set for every index s in idx[b, i, :] (-1 skipped).
+__global__ void build_mask_kernel(const int32_t* __restrict__ idx, int Lq, int k, int Lq_d, int W,
+                                  uint32_t* __restrict__ mask, long long n_rows) {
+    extern __shared__ uint32_t mk_smem[];
+    for (long long p = blockIdx.x; p < n_rows; p += gridDim.x) {
+        const long long b = p / Lq_d, i = p % Lq_d;
+        const int32_t* ir = idx + (b * Lq + i) * (long long)k;
+        for (int w = threadIdx.x; w < W; w += blockDim.x) mk_smem[w] = 0u;
+        __syncthreads();
+        for (int s = threadIdx.x; s < k; s += blockDim.x) {
+            const int id = __ldg(ir + s);
+            if (id >= 0 && (id >> 5) < W) atomicOr(&mk_smem[id >> 5], 1u << (id & 31));
+        }
+        __syncthreads();
+        for (int w = threadIdx.x; w < W; w += blockDim.x) mask[p * W + w] = mk_smem[w];
+        __syncthreads();
+    }
+}
+
+// V [B, Lk, 128] -> V^T [B, 128, ldt] for keys < Lk_d (64 keys x 128 d per CTA).
+__global__ void transpose_v_kernel(const __nv_bfloat16* __restrict__ v, int Lk, int Lk_d, int ldt,
+                                   __nv_bfloat16* __restrict__ vt) {
+    __shared__ __nv_bfloat16 tile[64][128 + 8];
+    const int b = blockIdx.y, s0 = blockIdx.x * 64;
+    const __nv_bfloat16* vb = v + (long long)b * Lk * 128;
+    for (int e = threadIdx.x; e < 64 * 16; e += blockDim.x) {
+        const int s = e / 16, c = e % 16;
+        uint4 val = make_uint4(0, 0, 0, 0);
+        if (s0 + s < Lk_d) val = *reinterpret_cast<const uint4*>(vb + (long long)(s0 + s) * 128 + c * 8);
+        *reinterpret_cast<uint4*>(&tile[s][c * 8]) = val;
+    }
+    __syncthreads();
+    __nv_bfloat16* tb = vt + (long long)b * 128 * ldt;
+    for (int e = threadIdx.x; e < 128 * 64; e += blockDim.x) {
+        const int d = e / 64, s = e % 64;
+        if (s0 + s < ldt) tb[(long long)d * ldt + s0 + s] = tile[s][d];
+    }
+}
+
+}  // namespace ic

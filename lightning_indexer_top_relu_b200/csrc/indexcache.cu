@@ -16,6 +16,7 @@
 
 #include "indexcache.h"
 #include "common.cuh"
+#include "dense_attn.cuh"
 #include "indexer_scores.cuh"
 #include "sparse_attn.cuh"
 #include "topk_select.cuh"
@@ -225,11 +226,14 @@ size_t attn_ws_bytes(long long n_rows, int splits, int Hq, int d) {
     return (size_t)n_rows * splits * (size_t)Hq * (d + 1) * sizeof(float);
 }
 
+// Gather attention over rows i in [row_i0, row_i0 + rows_per_b) of every
+// sequence (rows_per_b < 0: all rows).
 int launch_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* idx,
                 int B, int Lq, int Lk, int Hq, int d, int k_slots, int q_offset, float scale,
                 uint16_t* out, float* lse, void* ws, size_t ws_bytes, bool trim, int sms,
-                cudaStream_t st) {
-    const long long n_rows = (long long)B * Lq;
+                cudaStream_t st, int row_i0 = 0, int rows_per_b = -1) {
+    if (rows_per_b < 0) rows_per_b = Lq - row_i0;
+    const long long n_rows = (long long)B * rows_per_b;
     if (n_rows <= 0) return IC_OK;
     int splits = attn_splits(n_rows, k_slots, sms);
     while (splits > 1 && (ws == nullptr || attn_ws_bytes(n_rows, splits, Hq, d) > ws_bytes))
@@ -255,6 +259,8 @@ int launch_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, const i
     const float sc = scale > 0.0f ? scale : 1.0f / std::sqrt((float)d);
     a.scale_log2 = sc * ic::LOG2E;
     a.n_rows = n_rows;
+    a.rows_per_b = rows_per_b;
+    a.row_i0 = row_i0;
     dim3 grid((unsigned)n_rows, (unsigned)splits);
     if (d == 64) {
         ic::sparse_attn_kernel<64><<<grid, ic::SA_THREADS, ic::SaSmem<64>::BYTES, st>>>(a);
@@ -272,6 +278,91 @@ int launch_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, const i
         if (e != cudaSuccess) return cuda_fail(e, "sparse_attn combine launch");
     }
     return IC_OK;
+}
+
+// ---------------------------------------------------------------- dense-masked attention
+
+// Rows whose top-k covers at least 1/DENSE_FACTOR of their visible positions
+// (t < DENSE_FACTOR * k) attend tile-dense on the tensor cores; the others
+// gather.  Only used inside the layer stack, whose index rows hold distinct
+// positions (a bitmask cannot count a repeated index twice).
+constexpr int DENSE_FACTOR = 4;
+
+struct DenseGeom {
+    bool on = false;
+    int QBD = 0, Lq_d = 0, nqb_d = 0, W = 0, Lk_d = 0, ldt = 0;
+    size_t mask_bytes = 0, vt_bytes = 0, total = 0;
+};
+
+DenseGeom dense_geom(const ic_dims& D) {
+    DenseGeom g;
+    if (D.d != 128 || (128 % D.Hq) != 0) return g;
+    g.QBD = 128 / D.Hq;
+    long long lim = (long long)DENSE_FACTOR * D.k - D.q_offset;     // rows i with t < 4k
+    lim = std::min<long long>(lim, D.Lq);
+    if (lim < g.QBD) return g;
+    g.Lq_d = (int)(lim / g.QBD) * g.QBD;
+    g.nqb_d = g.Lq_d / g.QBD;
+    g.Lk_d = std::min(D.Lk, D.q_offset + g.Lq_d);
+    g.W = (g.Lk_d + 31) / 32;
+    g.ldt = ((g.Lk_d + 63) / 64) * 64;
+    g.mask_bytes = (((size_t)D.B * g.Lq_d * g.W * 4) + 1023) / 1024 * 1024;
+    g.vt_bytes = (size_t)D.B * 128 * g.ldt * 2;
+    g.total = g.mask_bytes + g.vt_bytes;
+    g.on = true;
+    return g;
+}
+
+int launch_build_mask(const DenseGeom& g, const ic_dims& D, const int32_t* idx, uint32_t* mask,
+                      cudaStream_t st) {
+    const long long n = (long long)D.B * g.Lq_d;
+    const int grid = (int)std::min<long long>(n, 65535);
+    ic::build_mask_kernel<<<grid, 256, g.W * 4, st>>>(idx, D.Lq, D.k, g.Lq_d, g.W, mask, n);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? IC_OK : cuda_fail(e, "build_mask launch");
+}
+
+int launch_dense_attn(const DenseGeom& g, const ic_dims& D, const ic_layer& L,
+                      const uint32_t* mask, uint16_t* vt, cudaStream_t st) {
+    // V^T of this layer's keys < Lk_d, zero-padded to ldt columns
+    dim3 tg((unsigned)(g.ldt / 64), (unsigned)D.B);
+    ic::transpose_v_kernel<<<tg, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(L.v), D.Lk,
+                                                g.Lk_d, g.ldt, reinterpret_cast<__nv_bfloat16*>(vt));
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "transpose_v launch");
+    CUtensorMap tq, tk, tv;
+    int rc = make_tmap_3d(&tq, L.q, 128, (uint64_t)D.Lq * D.Hq, (uint64_t)D.B, 128);
+    if (!rc) rc = make_tmap_3d(&tk, L.k, 128, (uint64_t)D.Lk, (uint64_t)D.B, ic::DA_TILE);
+    if (!rc) rc = get_encode();
+    if (rc) return rc;
+    {
+        cuuint64_t dims[3] = {(cuuint64_t)g.Lk_d, 128, (cuuint64_t)D.B};
+        cuuint64_t strides[2] = {(cuuint64_t)g.ldt * 2, (cuuint64_t)g.ldt * 2 * 128};
+        cuuint32_t box[3] = {64, 128, 1};
+        cuuint32_t estr[3] = {1, 1, 1};
+        CUresult r = g_encode(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, vt, dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return fail(IC_ERR_CUDA, "cuTensorMapEncodeTiled (V^T) failed (%d)", (int)r);
+    }
+    ic::DenseAttnArgs a;
+    a.mask = mask;
+    a.out = reinterpret_cast<__nv_bfloat16*>(L.out);
+    a.lse = L.lse;
+    a.Lq = D.Lq;
+    a.Lk = D.Lk;
+    a.Hq = D.Hq;
+    a.q_offset = D.q_offset;
+    a.Lq_d = g.Lq_d;
+    a.QBD = g.QBD;
+    a.nqb_d = g.nqb_d;
+    a.W = g.W;
+    a.n_blocks = D.B * g.nqb_d;
+    const float sc = D.scale > 0.0f ? D.scale : 1.0f / std::sqrt(128.0f);
+    a.scale_log2 = sc * ic::LOG2E;
+    ic::dense_attn_kernel<<<a.n_blocks, ic::DA_THREADS, ic::DenseSmem::ALLOC, st>>>(tq, tk, tv, a);
+    e = cudaGetLastError();
+    return e == cudaSuccess ? IC_OK : cuda_fail(e, "dense_attn launch");
 }
 
 // ---------------------------------------------------------------- per-device setup
@@ -300,6 +391,8 @@ int device_setup(int* dev_out, int* sms_out) {
         cudaFuncSetAttribute(ic::topk_select_kernel<true>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              ic::TK_SMEM_FIXED + ic::TK_CACHE_MAX * 4);
+        cudaFuncSetAttribute(ic::dense_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             ic::DenseSmem::ALLOC);
         cudaFuncSetAttribute(ic::sparse_attn_kernel<64>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, ic::SaSmem<64>::BYTES);
         cudaFuncSetAttribute(ic::sparse_attn_kernel<128>,
@@ -519,8 +612,9 @@ size_t ic_layer_stack_workspace_bytes(const ic_dims* dims, int n_layers, long lo
         blocks = std::min(blocks, std::max(1LL, (rows_per_chunk + geo.QB - 1) / geo.QB));
     const size_t scores = (size_t)blocks * geo.QB * (size_t)dims->Lk * sizeof(float);
     const size_t attn = ic_sparse_attn_workspace_bytes(dims->B, dims->Lq, dims->Hq, dims->d, dims->k);
+    const DenseGeom dg = dense_geom(*dims);
     (void)n_rows;
-    return std::max(scores, attn);
+    return std::max(std::max(scores, attn), dg.on ? dg.total + attn : (size_t)0);
 }
 
 static int stack_forward(const char* pattern, int n_layers, const ic_layer* layers,
@@ -582,6 +676,13 @@ static int stack_forward(const char* pattern, int n_layers, const ic_layer* laye
         return e == cudaSuccess ? IC_OK : cuda_fail(e, "cudaEventRecord");
     };
     const bool one_chunk = blocks_per_chunk >= n_blocks;
+    // Dense-masked attention for rows with t < 4k when the workspace holds
+    // its mask and V^T buffers (they reuse the score region: an F layer's
+    // scores are dead once its top-k is done).
+    const DenseGeom dg = dense_geom(D);
+    const bool dense = dg.on && dg.total <= ws_bytes;
+    uint32_t* dmask = reinterpret_cast<uint32_t*>(ws);
+    uint16_t* dvt = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(ws) + dg.mask_bytes);
     for (int l = 0; l < n_layers; ++l) {
         const ic_layer& L = layers[l];
         const bool full = pattern[l] == 'F' || pattern[l] == '1';
@@ -599,10 +700,21 @@ static int stack_forward(const char* pattern, int n_layers, const ic_layer* laye
                 if (rc) return rc;
             }
         }
+        if (dense && full && (rc = launch_build_mask(dg, D, idx_cache, dmask, st))) return rc;
         if (!(full && one_chunk) && (rc = mark(l, 1))) return rc;
         if ((rc = mark(l, 2))) return rc;
-        rc = launch_attn(L.q, L.k, L.v, idx_cache, D.B, D.Lq, D.Lk, D.Hq, D.d, D.k, D.q_offset,
-                         D.scale, L.out, L.lse, ws, ws_bytes, true, sms, st);
+        if (dense) {
+            if ((rc = launch_dense_attn(dg, D, L, dmask, dvt, st))) return rc;
+            if (dg.Lq_d < D.Lq) {
+                rc = launch_attn(L.q, L.k, L.v, idx_cache, D.B, D.Lq, D.Lk, D.Hq, D.d, D.k,
+                                 D.q_offset, D.scale, L.out, L.lse,
+                                 reinterpret_cast<uint8_t*>(ws) + dg.total, ws_bytes - dg.total,
+                                 true, sms, st, dg.Lq_d, D.Lq - dg.Lq_d);
+            }
+        } else {
+            rc = launch_attn(L.q, L.k, L.v, idx_cache, D.B, D.Lq, D.Lk, D.Hq, D.d, D.k, D.q_offset,
+                             D.scale, L.out, L.lse, ws, ws_bytes, true, sms, st);
+        }
         if (rc) return rc;
         if ((rc = mark(l, 3))) return rc;
         if (L.idx_dump) {

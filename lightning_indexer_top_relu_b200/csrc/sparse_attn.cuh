@@ -43,8 +43,6 @@ constexpr int SA_THREADS = 32 * SA_WARPS;
 constexpr int SA_STAGES = IC_SA_STAGES;
 static_assert(SA_BLOCK == 16 || SA_BLOCK == 32 || SA_BLOCK == 64, "block of 16, 32 or 64 slots");
 constexpr int SA_IDX_TILE = 2048;            // indices staged in shared memory at a time
-constexpr float LOG2E = 1.4426950408889634f;
-constexpr float LN2 = 0.6931471805599453f;
 
 struct SparseAttnArgs {
     const __nv_bfloat16* q;    // [B, Lq, Hq, D]
@@ -59,8 +57,16 @@ struct SparseAttnArgs {
     int splits, slots_per_split;
     int trim;                  // slots past min(k, t+1) are known empty
     float scale_log2;
-    long long n_rows;
+    long long n_rows;          // rows processed: B * rows_per_b
+    int rows_per_b;            // rows i in [row_i0, row_i0 + rows_per_b) of each sequence
+    int row_i0;
 };
+
+// Processing index p -> flattened query row b*Lq + i.
+__device__ __forceinline__ long long sa_row(const SparseAttnArgs& a, long long p) {
+    const long long b = p / a.rows_per_b;
+    return b * a.Lq + a.row_i0 + (p % a.rows_per_b);
+}
 
 template <int D>
 struct SaSmem {
@@ -133,7 +139,8 @@ sparse_attn_kernel(const SparseAttnArgs a) {
     const uint32_t sbase = smem_u32(sa_smem);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const long long row = a.n_rows - 1 - (long long)blockIdx.x;     // longest rows first
+    const long long pidx = a.n_rows - 1 - (long long)blockIdx.x;    // longest rows first
+    const long long row = sa_row(a, pidx);
     const int split = blockIdx.y;
     const int b = (int)(row / a.Lq);
     const int t = a.q_offset + (int)(row % a.Lq);
@@ -354,7 +361,7 @@ sparse_attn_kernel(const SparseAttnArgs a) {
             a.out[(row * a.Hq + h) * D + dcol] = __float2bfloat16_rn(val);
             if (a.lse && dcol == 0) a.lse[row * a.Hq + h] = lse2 * LN2;
         } else {
-            const long long pr = (row * a.splits + split) * a.Hq + h;
+            const long long pr = (pidx * a.splits + split) * a.Hq + h;
             a.part_o[pr * D + dcol] = val;
             if (dcol == 0) a.part_lse[pr] = lse2;
         }
@@ -364,16 +371,17 @@ sparse_attn_kernel(const SparseAttnArgs a) {
 // Merges the per-split partial results of each row (log2-sum-exp weights).
 template <int D>
 __global__ void sparse_attn_combine_kernel(const SparseAttnArgs a) {
-    const long long row = blockIdx.x;
+    const long long pidx = blockIdx.x;
+    const long long row = sa_row(a, pidx);
     for (int e = threadIdx.x; e < a.Hq * D; e += blockDim.x) {
         const int h = e / D, dcol = e % D;
         float M = -INFINITY;
         for (int s = 0; s < a.splits; ++s)
-            M = fmaxf(M, a.part_lse[(row * a.splits + s) * a.Hq + h]);
+            M = fmaxf(M, a.part_lse[(pidx * a.splits + s) * a.Hq + h]);
         float W = 0.0f, acc = 0.0f;
         if (M != -INFINITY) {
             for (int s = 0; s < a.splits; ++s) {
-                const long long pr = (row * a.splits + s) * a.Hq + h;
+                const long long pr = (pidx * a.splits + s) * a.Hq + h;
                 const float f = exp2f(a.part_lse[pr] - M);
                 W += f;
                 acc += f * a.part_o[pr * D + dcol];
