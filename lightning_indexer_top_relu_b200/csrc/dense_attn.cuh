@@ -11,15 +11,20 @@
 //
 // Per CTA: one block of 128/Hq queries x Hq heads = 128 rows (TMEM lanes);
 // two CTAs share an SM so one's MMAs overlap the other's softmax.
-//   warp 0      TMA: the Q block once; per 64-key tile, K[keys, d] and
-//               V^T[d, keys] (a per-layer transposed copy) into a 2-stage ring
-//   warp 1      TMEM allocation + MMA issue: S = Q K^T (M=128, N=64, K=d)
-//               into TMEM, then O += P V (A = P from shared memory, B = V^T
-//               tile; O accumulates in TMEM across tiles)
-//   warps 2..5  softmax: thread = row = TMEM lane.  Reads S twice (tile max,
-//               then exp2), masks it with the row's bitmask (prefetched one
-//               tile ahead), writes P as bf16 into a 128-byte-swizzled shared
-//               tile.  The running max is raised lazily: only when a tile's max
+//   warp 0      TMA: the Q block once; per 64-key tile K[keys, d] into a
+//               2-stage K ring and V^T[d, keys] (a per-layer transposed copy)
+//               into a 2-stage V ring.  One thread polls both rings and
+//               refills whichever stage is released first.
+//   warp 1      TMEM allocation + MMA issue.  S(j) = Q K(j)^T (M=128, N=64,
+//               K=d) goes to one of two TMEM score buffers, so S(j+1) is
+//               computed while the softmax works on S(j); O += P(j) V(j)
+//               (A = P from shared memory, B = V^T tile) accumulates in TMEM.
+//   warps 2..5  softmax: thread = row = TMEM lane.  Loads S(j) once into
+//               registers, masks it with the row's bitmask (prefetched one
+//               tile ahead), takes the tile max, computes the probabilities,
+//               and only then waits for P(j-1) V(j-1) to finish before it
+//               writes P(j) as bf16 into a 128-byte-swizzled shared tile.
+//               The running max is raised lazily: only when a tile's max
 //               exceeds it by more than 8 (log2 units) is O rescaled in TMEM,
 //               so P stays <= 2^8 and O / l is exact either way.
 // Scores are scaled in the log2 domain; masked positions contribute exactly 0.
@@ -51,12 +56,12 @@ struct DenseSmem {
     static constexpr int K_BYTES = 64 * 128 * 2;             // 64 keys x 128 d (two boxes)
     static constexpr int V_BYTES = 128 * 64 * 2;             // 128 d x 64 keys (one box)
     static constexpr int P_BYTES = 128 * 64 * 2;             // 128 rows x 64 keys (one box)
-    static constexpr int STAGE = K_BYTES + V_BYTES;
     static constexpr int OFF_Q = 0;
-    static constexpr int OFF_ST = OFF_Q + Q_BYTES;           // 2 stages
-    static constexpr int OFF_P = OFF_ST + 2 * STAGE;
+    static constexpr int OFF_K = OFF_Q + Q_BYTES;            // 2 stages
+    static constexpr int OFF_V = OFF_K + 2 * K_BYTES;        // 2 stages
+    static constexpr int OFF_P = OFF_V + 2 * V_BYTES;
     static constexpr int OFF_BAR = OFF_P + P_BYTES;
-    static constexpr int N_BARS = 1 + 2 + 2 + 3;
+    static constexpr int N_BARS = 16;
     static constexpr int OFF_SLOT = OFF_BAR + N_BARS * 8;
     static constexpr int BYTES = OFF_SLOT + 16;
     // Up to 1024 B of slack for the 1024-B alignment of the swizzled tiles,
@@ -67,8 +72,19 @@ struct DenseSmem {
     static_assert(BYTES <= PAIR_MAX, "two CTAs must fit one SM");
 };
 
+// TMEM columns of one CTA: two 64-column score buffers, then O (128 columns).
+constexpr uint32_t DA_TMEM_COLS = 256;
+constexpr uint32_t DA_O_COL = 128;
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 2^x on the MUFU unit (flush-to-zero; exactly 0 for x = -inf).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 // tmap_q: q as 3-D {128, Lq*Hq, B}, box {64, 128, 1}; tmap_k: K as {128, Lk, B},
@@ -83,11 +99,14 @@ dense_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
     if (smem == nullptr) return;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
     uint64_t* q_full = bars;
-    uint64_t* kv_full = bars + 1;
-    uint64_t* kv_empty = bars + 3;
-    uint64_t* s_full = bars + 5;
-    uint64_t* p_full = bars + 6;
-    uint64_t* o_full = bars + 7;
+    uint64_t* k_full = bars + 1;       // [2]
+    uint64_t* k_empty = bars + 3;      // [2]
+    uint64_t* v_full = bars + 5;       // [2]
+    uint64_t* v_empty = bars + 7;      // [2]
+    uint64_t* s_full = bars + 9;       // [2]
+    uint64_t* p_full = bars + 11;
+    uint64_t* o_full = bars + 12;
+    uint64_t* mma_done = bars + 13;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::OFF_SLOT);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -100,22 +119,25 @@ dense_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&kv_full[i], 1);
-            mbar_init(&kv_empty[i], 1);
+            mbar_init(&k_full[i], 1);
+            mbar_init(&k_empty[i], 1);
+            mbar_init(&v_full[i], 1);
+            mbar_init(&v_empty[i], 1);
+            mbar_init(&s_full[i], 1);
         }
-        mbar_init(s_full, 1);
         mbar_init(p_full, 128);
         mbar_init(o_full, 1);
+        mbar_init(mma_done, 1);
         fence_barrier_init();
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, 256);
+        tmem_alloc(tmem_slot, DA_TMEM_COLS);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *tmem_slot;          // S at +0 (64 cols), O at +64 (128 cols)
+    const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
         if (lane == 0) {
@@ -126,18 +148,42 @@ dense_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
             for (int kb = 0; kb < 2; ++kb)
                 tma_load_3d(smem + S::OFF_Q + kb * 128 * 128, &tmap_q, q_full, kb * 64,
                             i0 * a.Hq, b);
-            int j = 0;
-            for (; j < nt; ++j) {
-                const int st = j & 1;
-                if (!mbar_wait(&kv_empty[st], ((j >> 1) & 1) ^ 1)) break;
-                uint8_t* stg = smem + S::OFF_ST + st * S::STAGE;
-                mbar_arrive_expect_tx(&kv_full[st], (uint32_t)S::STAGE);
-                for (int kb = 0; kb < 2; ++kb)
-                    tma_load_3d(stg + kb * 64 * 128, &tmap_k, &kv_full[st], kb * 64, j * DA_TILE, b);
-                tma_load_3d(stg + S::K_BYTES, &tmap_vt, &kv_full[st], j * DA_TILE, 0, b);
+            // Refill whichever ring frees a stage first; V never runs ahead of K.
+            int jk = 0, jv = 0, spins = 0;
+            unsigned long long t0 = global_ns();
+            while (jk < nt || jv < nt) {
+                bool moved = false;
+                if (jk < nt && mbar_try_wait(&k_empty[jk & 1], ((jk >> 1) & 1) ^ 1)) {
+                    uint8_t* dst = smem + S::OFF_K + (jk & 1) * S::K_BYTES;
+                    mbar_arrive_expect_tx(&k_full[jk & 1], (uint32_t)S::K_BYTES);
+                    for (int kb = 0; kb < 2; ++kb)
+                        tma_load_3d(dst + kb * 64 * 128, &tmap_k, &k_full[jk & 1], kb * 64,
+                                    jk * DA_TILE, b);
+                    ++jk;
+                    moved = true;
+                }
+                if (jv < jk && mbar_try_wait(&v_empty[jv & 1], ((jv >> 1) & 1) ^ 1)) {
+                    mbar_arrive_expect_tx(&v_full[jv & 1], (uint32_t)S::V_BYTES);
+                    tma_load_3d(smem + S::OFF_V + (jv & 1) * S::V_BYTES, &tmap_vt, &v_full[jv & 1],
+                                jv * DA_TILE, 0, b);
+                    ++jv;
+                    moved = true;
+                }
+                if (moved) {
+                    spins = 0;
+                    t0 = global_ns();
+                } else if (++spins == 64) {
+                    spins = 0;
+                    if (global_ns() - t0 > WAIT_LIMIT_NS) {
+                        report(DEV_ERR_TIMEOUT);
+                        break;
+                    }
+                }
             }
+            // never leave with copies in flight
             mbar_wait(q_full, 0);
-            for (int c = (j > 2 ? j - 2 : 0); c < j; ++c) mbar_wait(&kv_full[c & 1], (c >> 1) & 1);
+            for (int c = (jk > 2 ? jk - 2 : 0); c < jk; ++c) mbar_wait(&k_full[c & 1], (c >> 1) & 1);
+            for (int c = (jv > 2 ? jv - 2 : 0); c < jv; ++c) mbar_wait(&v_full[c & 1], (c >> 1) & 1);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -146,35 +192,45 @@ dense_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
             const uint32_t q_addr = smem_u32(smem + S::OFF_Q);
             const uint32_t p_addr = smem_u32(smem + S::OFF_P);
             bool ok = mbar_wait(q_full, 0);
-            for (int j = 0; j < nt && ok; ++j) {
-                const int st = j & 1;
-                if (!mbar_wait(&kv_full[st], (j >> 1) & 1)) break;
-                tc_fence_after();
-                const uint32_t k_addr = smem_u32(smem + S::OFF_ST + st * S::STAGE);
-                const uint32_t v_addr = k_addr + S::K_BYTES;
-                // S = Q K^T: the softmax warps read the previous S before they
-                // released the previous P, which this thread waited for.
+            // iteration j issues S(j), then P(j-1) V(j-1): S(j) overwrites the
+            // buffer of S(j-2), which the softmax released with P(j-2).
+            for (int j = 0; j <= nt && ok; ++j) {
+                if (j < nt) {
+                    const int st = j & 1;
+                    if (!(ok = mbar_wait(&k_full[st], (j >> 1) & 1))) break;
+                    tc_fence_after();
+                    const uint32_t k_addr = smem_u32(smem + S::OFF_K + st * S::K_BYTES);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t qo = (uint32_t)((kk >> 2) * 128 * 128 + (kk & 3) * 32);
-                    const uint32_t ko = (uint32_t)((kk >> 2) * 64 * 128 + (kk & 3) * 32);
-                    tc_mma_f16(tmem, sw128_kmajor_desc(q_addr + qo), sw128_kmajor_desc(k_addr + ko),
-                               idesc_s, kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t qo = (uint32_t)((kk >> 2) * 128 * 128 + (kk & 3) * 32);
+                        const uint32_t ko = (uint32_t)((kk >> 2) * 64 * 128 + (kk & 3) * 32);
+                        tc_mma_f16(tmem + (uint32_t)(st * DA_TILE), sw128_kmajor_desc(q_addr + qo),
+                                   sw128_kmajor_desc(k_addr + ko), idesc_s, kk > 0 ? 1u : 0u);
+                    }
+                    tc_commit(&s_full[st]);
+                    tc_commit(&k_empty[st]);
                 }
-                tc_commit(s_full);
-                if (!mbar_wait(p_full, j & 1)) break;
-                tc_fence_after();
-                // O += P V   (A = P [rows x 64 keys], B = V^T tile [128 d x 64 keys])
+                if (j > 0) {
+                    const int jp = j - 1, st = jp & 1;
+                    if (!(ok = mbar_wait(p_full, jp & 1))) break;
+                    if (!(ok = mbar_wait(&v_full[st], (jp >> 1) & 1))) break;
+                    tc_fence_after();
+                    const uint32_t v_addr = smem_u32(smem + S::OFF_V + st * S::V_BYTES);
+                    // O += P V   (A = P [rows x 64 keys], B = V^T tile [128 d x 64 keys])
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint32_t off = (uint32_t)(kk * 32);
-                    tc_mma_f16(tmem + 64, sw128_kmajor_desc(p_addr + off),
-                               sw128_kmajor_desc(v_addr + off), idesc_o,
-                               (j > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint32_t off = (uint32_t)(kk * 32);
+                        tc_mma_f16(tmem + DA_O_COL, sw128_kmajor_desc(p_addr + off),
+                                   sw128_kmajor_desc(v_addr + off), idesc_o,
+                                   (jp > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    tc_commit(o_full);
+                    tc_commit(&v_empty[st]);
                 }
-                tc_commit(o_full);
-                tc_commit(&kv_empty[st]);
             }
+            // the MMAs this thread issued are done before TMEM is freed
+            tc_commit(mma_done);
+            mbar_wait(mma_done, 0);
         }
     } else {
         // ---------------- softmax warps: thread = row r = (query r / Hq, head r % Hq)
@@ -185,6 +241,7 @@ dense_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
         const bool row_ok = i0 + qi < a.Lq_d;
         const uint32_t* mrow = a.mask + (long long)(b * a.Lq_d + (row_ok ? i0 + qi : 0)) * a.W;
         uint8_t* prow = smem + S::OFF_P + r * 128;
+        const float sc = a.scale_log2;
         float m_used = -INFINITY, l_run = 0.0f;
         bool ok = true;
         auto load_mask = [&](int j, uint32_t& w0, uint32_t& w1) {
@@ -195,74 +252,81 @@ dense_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
         uint32_t nm0, nm1;
         load_mask(0, nm0, nm1);
         for (int j = 0; j < nt; ++j) {
-            const uint32_t mw[2] = {nm0, nm1};
+            const uint32_t mw0 = nm0, mw1 = nm1;
             if (j + 1 < nt) load_mask(j + 1, nm0, nm1);         // one tile ahead
-            if (!mbar_wait(s_full, j & 1)) { ok = false; break; }
+            if (!mbar_wait(&s_full[j & 1], (j >> 1) & 1)) { ok = false; break; }
             tc_fence_after();
-            // pass 1: tile max over the selected positions
-            float mx = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(tmem + lane_base + c * 32, v);
+            uint32_t v[64];
+            {
+                uint32_t (&v0)[32] = *reinterpret_cast<uint32_t (*)[32]>(&v[0]);
+                uint32_t (&v1)[32] = *reinterpret_cast<uint32_t (*)[32]>(&v[32]);
+                const uint32_t sb = tmem + lane_base + (uint32_t)((j & 1) * DA_TILE);
+                tmem_ld_32x32b_x32(sb, v0);
+                tmem_ld_32x32b_x32(sb + 32, v1);
                 tmem_ld_wait();
-#pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    if ((mw[c] >> e) & 1u) mx = fmaxf(mx, __uint_as_float(v[e]));
             }
-            const float mxs = mx * a.scale_log2;
-            // O from the previous tile's P V must be complete before O is
-            // rescaled here or the next P V is let in.
+            // positions outside the selection become -inf; tile max as a tree
+            float s[64];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                s[e] = ((mw0 >> e) & 1u) ? __uint_as_float(v[e]) : -INFINITY;
+                s[32 + e] = ((mw1 >> e) & 1u) ? __uint_as_float(v[32 + e]) : -INFINITY;
+            }
+            float mx[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) mx[e] = fmaxf(s[e], s[e + 32]);
+#pragma unroll
+            for (int w = 16; w >= 1; w >>= 1)
+#pragma unroll
+                for (int e = 0; e < w; ++e) mx[e] = fmaxf(mx[e], mx[e + w]);
+            const float mxs = mx[0] * sc;
+            const bool raise = mxs > m_used + DA_RESCALE;
+            const float m_new = raise ? mxs : m_used;
+            const float base = m_new == -INFINITY ? 0.0f : m_new;
+            // probabilities (bf16 pairs) and their sum
+            uint32_t pk[32];
+            float2 rs2[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+            const float2 sc2 = make_float2(sc, sc), nb2 = make_float2(-base, -base);
+#pragma unroll
+            for (int e = 0; e < 64; e += 2) {
+                const float2 x = __ffma2_rn(make_float2(s[e], s[e + 1]), sc2, nb2);
+                const float2 p = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                rs2[(e >> 1) & 3] = __fadd2_rn(rs2[(e >> 1) & 3], p);
+                __nv_bfloat162 pp = __floats2bfloat162_rn(p.x, p.y);
+                pk[e >> 1] = *reinterpret_cast<uint32_t*>(&pp);
+            }
+            const float2 r01 = __fadd2_rn(rs2[0], rs2[1]), r23 = __fadd2_rn(rs2[2], rs2[3]);
+            const float2 rsum = __fadd2_rn(r01, r23);
+            const float rs = rsum.x + rsum.y;
+            // P(j-1) V(j-1) must be complete before O is rescaled or P is overwritten
             if (j > 0) {
                 if (!mbar_wait(o_full, (j - 1) & 1)) { ok = false; break; }
                 tc_fence_after();
             }
-            if (mxs > m_used + DA_RESCALE) {
-                const float alpha = exp2f(m_used - mxs);            // 0 on the first raise
+            if (raise) {
+                const float alpha = ex2_approx(m_used - m_new);     // 0 on the first raise
                 if (j > 0) {
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
-                        uint32_t v[32];
-                        tmem_ld_32x32b_x32(tmem + 64 + lane_base + c * 32, v);
+                        uint32_t o[32];
+                        tmem_ld_32x32b_x32(tmem + DA_O_COL + lane_base + c * 32, o);
                         tmem_ld_wait();
 #pragma unroll
                         for (int e = 0; e < 32; ++e)
-                            v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-                        tmem_st_32x32b_x32(tmem + 64 + lane_base + c * 32, v);
+                            o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                        tmem_st_32x32b_x32(tmem + DA_O_COL + lane_base + c * 32, o);
                     }
                     tmem_st_wait();
                 }
                 l_run *= alpha;
-                m_used = mxs;
-            }
-            const float base = m_used == -INFINITY ? 0.0f : m_used;
-            // pass 2: probabilities -> bf16 P tile (128-byte swizzled, K-major)
-            float rs = 0.0f;
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(tmem + lane_base + c * 32, v);
-                tmem_ld_wait();
-                uint32_t pk[16];
-#pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const float p0 = ((mw[c] >> e) & 1u)
-                                         ? exp2f(__uint_as_float(v[e]) * a.scale_log2 - base) : 0.0f;
-                    const float p1 = ((mw[c] >> (e + 1)) & 1u)
-                                         ? exp2f(__uint_as_float(v[e + 1]) * a.scale_log2 - base) : 0.0f;
-                    rs += p0 + p1;
-                    __nv_bfloat162 pp = __floats2bfloat162_rn(p0, p1);
-                    pk[e >> 1] = *reinterpret_cast<uint32_t*>(&pp);
-                }
-                // keys c*32 .. c*32+31 = 16-byte chunks c*4 .. c*4+3
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int cc = c * 4 + u;
-                    *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) =
-                        make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-                }
+                m_used = m_new;
             }
             l_run += rs;
+            // keys 8u .. 8u+7 = 16-byte chunk u of the row, stored at chunk u ^ (r & 7)
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                *reinterpret_cast<uint4*>(prow + ((u ^ (r & 7)) << 4)) =
+                    make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(p_full);
@@ -277,16 +341,16 @@ dense_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
             uint4* dst = reinterpret_cast<uint4*>(a.out + orow * 128);
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(tmem + 64 + lane_base + c * 32, v);
+                uint32_t o[32];
+                tmem_ld_32x32b_x32(tmem + DA_O_COL + lane_base + c * 32, o);
                 tmem_ld_wait();
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     uint32_t w[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        __nv_bfloat162 pp = __floats2bfloat162_rn(__uint_as_float(v[8 * u + 2 * e]) * inv,
-                                                                  __uint_as_float(v[8 * u + 2 * e + 1]) * inv);
+                        __nv_bfloat162 pp = __floats2bfloat162_rn(__uint_as_float(o[8 * u + 2 * e]) * inv,
+                                                                  __uint_as_float(o[8 * u + 2 * e + 1]) * inv);
                         w[e] = *reinterpret_cast<uint32_t*>(&pp);
                     }
                     dst[c * 4 + u] = make_uint4(w[0], w[1], w[2], w[3]);
@@ -300,7 +364,7 @@ dense_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, DA_TMEM_COLS);
     }
 }
 
