@@ -60,13 +60,28 @@ def load_peaks():
 
 # ---------------------------------------------------------------- algorithmic work
 
+DENSE_FACTOR = 4          # rows with t < 4k attend tile-dense (the library's dispatch rule)
+DA_TILE = 64              # keys per tile of the dense-masked kernel
+SFU_PER_CLK_SM = 16       # ex2 results per clock per SM (CUDA arithmetic-throughput table)
+
+
+def dense_rows(wl):
+    """Rows per sequence that the layer stack sends to the dense-masked kernel
+    (t < 4k, whole blocks of 128/Hq queries), and that block size."""
+    if wl.d != 128 or 128 % wl.Hq:
+        return 0, 0
+    qbd = 128 // wl.Hq
+    lim = min(DENSE_FACTOR * wl.k - wl.q_offset, wl.Lq)
+    return (lim // qbd * qbd if lim >= qbd else 0), qbd
+
+
 def work_per_layer(wl):
     """Algorithmic flops / bytes of each step of one layer (causal)."""
     B, Lq, Lk, q0, k = wl.B, wl.Lq, wl.Lk, wl.q_offset, wl.k
     t = np.arange(Lq, dtype=np.float64) + q0
     vis = np.minimum(t + 1, Lk)
+    sel_row = np.minimum(vis, k)
     sum_vis = B * vis.sum()                       # sum over rows of visible positions
-    sel = B * np.minimum(vis, k).sum()            # sum over rows of selected positions
     rows = B * Lq
     w = {}
     w["indexer_flops"] = 2.0 * wl.H_I * wl.d_I * sum_vis
@@ -74,15 +89,33 @@ def work_per_layer(wl):
     w["indexer_bytes"] = (rows * wl.H_I * wl.d_I * 2 + rows * wl.H_I * 4 + B * Lk * wl.d_I * 2
                           + 4 * sum_vis)
     w["topk_bytes"] = 4 * sum_vis + 4.0 * rows * k
-    w["attn_flops"] = 4.0 * wl.Hq * wl.d * sel
-    # gathered K and V rows + q + out + index rows
-    w["attn_bytes"] = 4.0 * wl.d * sel + 2 * 2.0 * rows * wl.Hq * wl.d + 4.0 * rows * k
+    lq_d, qbd = dense_rows(wl)
+    # dense-masked rows: useful flops are those of the selected positions;
+    # the kernel executes whole 64-key tiles of 128 rows up to each block's last t
+    sel_d = B * sel_row[:lq_d].sum()
+    w["dense_rows"] = B * lq_d
+    w["dense_flops"] = 4.0 * wl.Hq * wl.d * sel_d
+    if lq_d:
+        t_last = q0 + np.arange(0, lq_d, qbd) + qbd - 1
+        tiles = B * np.ceil(np.minimum(t_last + 1, Lk) / DA_TILE).sum()
+    else:
+        tiles = 0.0
+    w["dense_tiles"] = tiles
+    w["dense_exec_flops"] = tiles * 4.0 * 128 * DA_TILE * wl.d
+    w["dense_exec_exps"] = tiles * 128 * DA_TILE
+    # gathered rows: K and V rows of every selected slot + q + out + index rows
+    sel_g = B * sel_row[lq_d:].sum()
+    rows_g = B * (Lq - lq_d)
+    w["gather_rows"] = rows_g
+    w["gather_flops"] = 4.0 * wl.Hq * wl.d * sel_g
+    w["gather_bytes"] = 4.0 * wl.d * sel_g + 2 * 2.0 * rows_g * wl.Hq * wl.d + 4.0 * rows_g * k
     return w
 
 
 # ---------------------------------------------------------------- ncu traffic
 
 _KERNEL_SRC = {"sparse_attn": ("sparse_attn_kernel", "sparse_attn.cuh"),
+               "dense_attn": ("dense_attn_kernel", "dense_attn.cuh"),
                "indexer_scores": ("indexer_scores_kernel", "indexer_scores.cuh"),
                "topk_select": ("topk_select_kernel", "topk_select.cuh")}
 
@@ -352,12 +385,14 @@ def main():
     n = wl.n_layers
     flush = torch.empty(256 * 1024 * 1024 // 4, device=dev, dtype=torch.float32)
 
-    # per-kernel marks: 4 events per layer per step
+    # per-kernel marks: ic.MARKS_PER_LAYER events per layer per step
+    npl = ic.MARKS_PER_LAYER
+
     def new_marks():
-        evs = [torch.cuda.Event(enable_timing=True) for _ in range(4 * n)]
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(npl * n)]
         for e in evs:  # torch creates the CUDA event on first record
             e.record(stream)
-        arr = (ctypes.c_void_p * (4 * n))(*[e.cuda_event for e in evs])
+        arr = (ctypes.c_void_p * (npl * n))(*[e.cuda_event for e in evs])
         assert all(arr), "CUDA event handles must exist before they are handed to the library"
         return evs, arr
 
@@ -379,6 +414,7 @@ def main():
         pg.barrier()
     torch.cuda.synchronize()
     clocks.start()
+    launches0 = ic.kernel_launch_count()
     wall0 = time.perf_counter()
     for s in range(args.steps):
         flush.fill_(float(s))                    # L2 flush outside the step's events
@@ -387,6 +423,7 @@ def main():
         ends[s].record(stream)
     torch.cuda.synchronize()
     wall = time.perf_counter() - wall0
+    gpu_launches = ic.kernel_launch_count() - launches0
     if pg is not None:
         pg.barrier()
     torch.cuda.synchronize()
@@ -399,68 +436,91 @@ def main():
     ms_per_step, tokens, value = aggregate_over_ranks(local_ms, float(wl.B * wl.Lq), pg, dev)
 
     # ---- per-kernel breakdown from the marks
-    ki = {"indexer": [], "topk": [], "attn": []}
+    ki = {"indexer": [], "topk": [], "attn_dense": [], "attn_gather": []}
+    w = work_per_layer(wl)
     for evs, _ in marks:
         for l, c in enumerate(pattern):
+            e = evs[npl * l: npl * (l + 1)]
             if c in "F1":
-                ki["indexer"].append(evs[4 * l].elapsed_time(evs[4 * l + 1]))
-                ki["topk"].append(evs[4 * l + 1].elapsed_time(evs[4 * l + 2]))
-            ki["attn"].append(evs[4 * l + 2].elapsed_time(evs[4 * l + 3]))
-    w = work_per_layer(wl)
-    n_f = sum(c in "F1" for c in pattern)
+                ki["indexer"].append(e[0].elapsed_time(e[1]))
+                ki["topk"].append(e[1].elapsed_time(e[2]))
+            if w["dense_rows"]:
+                ki["attn_dense"].append(e[2].elapsed_time(e[3]))
+            if w["gather_rows"]:
+                ki["attn_gather"].append(e[3].elapsed_time(e[4]))
+    sm_mhz = (clk or {}).get("sm_mhz") or 1965.0
+    n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
     kernels = {}
     per_step = {}
     for name, vals in ki.items():
         if not vals:
             continue
         avg = float(np.mean(vals))
+        sec = avg * 1e-3
         per_step[name] = float(np.sum(vals)) / args.steps
         ent = {"launches_per_step": len(vals) // args.steps, "ms_per_launch": avg,
                "share": per_step[name] / ms_per_step}
         if name == "indexer":
-            ent["tflops"] = w["indexer_flops"] / (avg * 1e-3) / 1e12
+            ent["tflops"] = w["indexer_flops"] / sec / 1e12
             ent["frac_of_bf16_peak"] = ent["tflops"] / peaks["bf16_tflops"]
-            ent["gbs"] = w["indexer_bytes"] / (avg * 1e-3) / 1e9
+            ent["gbs"] = w["indexer_bytes"] / sec / 1e9
         elif name == "topk":
-            ent["gbs"] = w["topk_bytes"] / (avg * 1e-3) / 1e9
+            ent["covers"] = "top-k select (+ selection bitmask build for dense-masked rows)"
+            ent["gbs"] = w["topk_bytes"] / sec / 1e9
             ent["frac_of_hbm"] = ent["gbs"] / peaks["hbm_gbs"]
+        elif name == "attn_dense":
+            ent["covers"] = "V transpose + dense-masked tcgen05 attention, rows t < 4k"
+            ent["rows"] = int(w["dense_rows"])
+            ent["tflops"] = w["dense_flops"] / sec / 1e12
+            ent["frac_of_bf16_peak"] = ent["tflops"] / peaks["bf16_tflops"]
+            ent["executed_tflops"] = w["dense_exec_flops"] / sec / 1e12
+            ent["executed_frac_of_bf16_peak"] = ent["executed_tflops"] / peaks["bf16_tflops"]
+            sfu_peak = SFU_PER_CLK_SM * n_sms * sm_mhz * 1e6
+            ent["exp2_per_s"] = w["dense_exec_exps"] / sec
+            ent["frac_of_sfu_peak"] = ent["exp2_per_s"] / sfu_peak
         else:
-            ent["tflops"] = w["attn_flops"] / (avg * 1e-3) / 1e12
-            ent["logical_gbs"] = w["attn_bytes"] / (avg * 1e-3) / 1e9
+            ent["covers"] = "gather attention (+ split combine), rows t >= 4k"
+            ent["rows"] = int(w["gather_rows"])
+            ent["tflops"] = w["gather_flops"] / sec / 1e12
+            ent["logical_gbs"] = w["gather_bytes"] / sec / 1e9
             ent["frac_of_hbm"] = ent["logical_gbs"] / peaks["hbm_gbs"]
         kernels[name] = ent
     dom = max(kernels, key=lambda k: kernels[k]["share"])
+    kd = kernels[dom]
     if dom == "indexer":
-        ach = kernels[dom]["tflops"]
-        roof = {"kernel": "indexer_scores", "bound": "tensor", "achieved": ach,
-                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"],
-                "traffic": None,
+        roof = {"kernel": "indexer_scores", "bound": "tensor", "achieved": kd["tflops"],
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": kd["tflops"] / peaks["bf16_tflops"],
                 "algorithmic_per_launch": w["indexer_flops"]}
     elif dom == "topk":
-        ach = kernels[dom]["gbs"]
-        roof = {"kernel": "topk_select", "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": ach / peaks["hbm_gbs"], "traffic": None,
+        roof = {"kernel": "topk_select", "bound": "hbm", "achieved": kd["gbs"],
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": kd["gbs"] / peaks["hbm_gbs"],
                 "algorithmic_per_launch": w["topk_bytes"]}
+    elif dom == "attn_dense":
+        roof = {"kernel": "dense_attn", "bound": "tensor", "achieved": kd["tflops"],
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": kd["tflops"] / peaks["bf16_tflops"],
+                "algorithmic_per_launch": w["dense_flops"],
+                "executed_frac": kd["executed_frac_of_bf16_peak"],
+                "sfu_frac": kd["frac_of_sfu_peak"],
+                "note": ("achieved counts the flops of the selected positions only (4*Hq*d per "
+                         "slot); the kernel runs whole 64-key tiles, whose flops give "
+                         "executed_frac, and one exp2 per tile element on the SFUs "
+                         "(16/clk/SM), whose rate gives sfu_frac")}
     else:
-        ach = kernels[dom]["logical_gbs"]
-        roof = {"kernel": "sparse_attn", "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": ach / peaks["hbm_gbs"], "traffic": None,
-                "algorithmic_per_launch": w["attn_bytes"]}
+        roof = {"kernel": "sparse_attn", "bound": "hbm", "achieved": kd["logical_gbs"],
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": kd["logical_gbs"] / peaks["hbm_gbs"],
+                "algorithmic_per_launch": w["gather_bytes"],
+                "note": ("achieved counts the logical K/V gather bytes; when a layer's K/V stay "
+                         "L2-resident, DRAM traffic (`traffic`) is far below them")}
     roof["peak_source"] = peaks["source"]
     roof["traffic"] = profile_traffic(roof["kernel"], wl.name)
-    if roof["kernel"] == "sparse_attn":
-        roof["note"] = ("achieved counts the logical K/V gather bytes; at this size a layer's K/V "
-                        "stay L2-resident, so DRAM traffic (`traffic`) is far below them")
-
-    launches_per_step = 0
-    for c in pattern:
-        launches_per_step += (2 if c in "F1" else 0) + 1   # indexer + top-k, attention
 
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded Gaussian, correlated layers)",
-            "config": config_of(wl, pattern, args), "gpu_launches": launches_per_step * args.steps,
+            "config": config_of(wl, pattern, args), "gpu_launches": int(gpu_launches),
             "kernels": kernels, "roofline": roof,
             "indexer_share": (per_step.get("indexer", 0) + per_step.get("topk", 0)) / ms_per_step,
             "wall_s_timed": wall}

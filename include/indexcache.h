@@ -207,17 +207,35 @@ int ic_layer_stack_forward(const char *pattern, int n_layers, const ic_layer *la
                            const ic_dims *dims, int32_t *idx_cache, void *ws, size_t ws_bytes,
                            ic_stream_t stream);
 
+/* Timing marks ic_layer_stack_forward_events records per layer. */
+#define IC_MARKS_PER_LAYER 5
+
 /*
  * ic_layer_stack_forward with per-layer timing marks: the same launches,
- * plus cudaEventRecord on `stream` of events[4*l + j] (each a cudaEvent_t;
- * NULL entries are skipped) at j=0 layer start, j=1 after the indexer
- * (when the layer's scores take one chunk; otherwise after indexer + top-k),
- * j=2 before the attention, j=3 after the attention.  For S layers j=0..2
- * coincide.  events holds 4*n_layers entries.
+ * plus cudaEventRecord on `stream` of events[IC_MARKS_PER_LAYER*l + j] (each
+ * a cudaEvent_t; NULL entries are skipped) at
+ *   j=0 layer start,
+ *   j=1 after the indexer (when the layer's scores take one chunk; otherwise
+ *       after indexer + top-k),
+ *   j=2 before the attention (after the top-k and, on F layers whose rows
+ *       take the dense-masked path, the bitmask build),
+ *   j=3 after the dense-masked attention of the rows with t < 4k (the
+ *       transposed V copy included; equal to j=2 when no row takes it),
+ *   j=4 after the attention.
+ * For S layers j=0..2 coincide.  events holds IC_MARKS_PER_LAYER*n_layers
+ * entries.
  */
 int ic_layer_stack_forward_events(const char *pattern, int n_layers, const ic_layer *layers,
                                   const ic_dims *dims, int32_t *idx_cache, void *ws,
                                   size_t ws_bytes, ic_stream_t stream, void *const *events);
+
+/*
+ * Kernel launches this library has issued in this process so far (every
+ * entry point, every device).  A host-side counter: reading it never
+ * synchronises.  Callers take the difference around a region to count the
+ * launches inside it.
+ */
+unsigned long long ic_kernel_launch_count(void);
 
 #ifdef __cplusplus
 }

@@ -12,6 +12,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "indexcache.h"
@@ -35,6 +36,16 @@ int fail(int code, const char* fmt, ...) {
 
 int cuda_fail(cudaError_t e, const char* what) {
     return fail(IC_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// Kernel launches this library has issued, over the process (all devices).
+std::atomic<unsigned long long> g_launches{0};
+
+// Status of the launch just made; counts it when it went in.
+int launched(cudaError_t e, const char* what) {
+    if (e != cudaSuccess) return cuda_fail(e, what);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return IC_OK;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -179,14 +190,14 @@ int launch_indexer(const uint16_t* q_idx, const uint16_t* k_idx, const float* w,
     if (grid <= 0) return IC_OK;
     cudaError_t e = dI == 64 ? launch_indexer_h<64>(H, tq, tk, a, grid, st)
                              : launch_indexer_h<128>(H, tq, tk, a, grid, st);
-    if (e != cudaSuccess) return cuda_fail(e, "indexer_scores launch");
+    if (launched(e, "indexer_scores launch")) return IC_ERR_CUDA;
     if (fill_masked) {
         const long long n_rows = block_row_start(geo, Lq, g1) - a.row_base;
         const int fg = (int)std::min<long long>(n_rows, 65535);
         ic::indexer_fill_masked_kernel<<<fg, 256, 0, st>>>(scores, ld, Lq, Lk, q_offset, geo.QB,
                                                            a.row_base, n_rows);
         e = cudaGetLastError();
-        if (e != cudaSuccess) return cuda_fail(e, "indexer fill launch");
+        if (launched(e, "indexer fill launch")) return IC_ERR_CUDA;
     }
     return IC_OK;
 }
@@ -207,7 +218,7 @@ int launch_topk(const float* scores, long long ld, long long row_base, long long
             scores, ld, row_base, n_rows, Lq, Lk, q_offset, k, idx);
     }
     e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "topk_select launch");
+    if (launched(e, "topk_select launch")) return IC_ERR_CUDA;
     return IC_OK;
 }
 
@@ -268,14 +279,14 @@ int launch_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, const i
         ic::sparse_attn_kernel<128><<<grid, ic::SA_THREADS, ic::SaSmem<128>::BYTES, st>>>(a);
     }
     cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "sparse_attn launch");
+    if (launched(e, "sparse_attn launch")) return IC_ERR_CUDA;
     if (splits > 1) {
         if (d == 64)
             ic::sparse_attn_combine_kernel<64><<<(unsigned)n_rows, 256, 0, st>>>(a);
         else
             ic::sparse_attn_combine_kernel<128><<<(unsigned)n_rows, 256, 0, st>>>(a);
         e = cudaGetLastError();
-        if (e != cudaSuccess) return cuda_fail(e, "sparse_attn combine launch");
+        if (launched(e, "sparse_attn combine launch")) return IC_ERR_CUDA;
     }
     return IC_OK;
 }
@@ -319,7 +330,7 @@ int launch_build_mask(const DenseGeom& g, const ic_dims& D, const int32_t* idx, 
     const int grid = (int)std::min<long long>(n, 65535);
     ic::build_mask_kernel<<<grid, 256, g.W * 4, st>>>(idx, D.Lq, D.k, g.Lq_d, g.W, mask, n);
     cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? IC_OK : cuda_fail(e, "build_mask launch");
+    return launched(e, "build_mask launch");
 }
 
 int launch_dense_attn(const DenseGeom& g, const ic_dims& D, const ic_layer& L,
@@ -329,7 +340,7 @@ int launch_dense_attn(const DenseGeom& g, const ic_dims& D, const ic_layer& L,
     ic::transpose_v_kernel<<<tg, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(L.v), D.Lk,
                                                 g.Lk_d, g.ldt, reinterpret_cast<__nv_bfloat16*>(vt));
     cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "transpose_v launch");
+    if (launched(e, "transpose_v launch")) return IC_ERR_CUDA;
     CUtensorMap tq, tk, tv;
     int rc = make_tmap_3d(&tq, L.q, 128, (uint64_t)D.Lq * D.Hq, (uint64_t)D.B, 128);
     if (!rc) rc = make_tmap_3d(&tk, L.k, 128, (uint64_t)D.Lk, (uint64_t)D.B, ic::DA_TILE);
@@ -362,7 +373,7 @@ int launch_dense_attn(const DenseGeom& g, const ic_dims& D, const ic_layer& L,
     a.scale_log2 = sc * ic::LOG2E;
     ic::dense_attn_kernel<<<a.n_blocks, ic::DA_THREADS, ic::DenseSmem::ALLOC, st>>>(tq, tk, tv, a);
     e = cudaGetLastError();
-    return e == cudaSuccess ? IC_OK : cuda_fail(e, "dense_attn launch");
+    return launched(e, "dense_attn launch");
 }
 
 // ---------------------------------------------------------------- per-device setup
@@ -500,6 +511,10 @@ int ic_get_last_device_error(ic_stream_t stream) {
     return IC_OK;
 }
 
+unsigned long long ic_kernel_launch_count(void) {
+    return g_launches.load(std::memory_order_relaxed);
+}
+
 int ic_selftest_wait_timeout(int timeout_us, ic_stream_t stream) {
     int dev, sms;
     int rc = device_setup(&dev, &sms);
@@ -508,7 +523,7 @@ int ic_selftest_wait_timeout(int timeout_us, ic_stream_t stream) {
     ic::selftest_wait_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
         (unsigned long long)us * 1000ull);
     cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "selftest launch");
+    if (launched(e, "selftest launch")) return IC_ERR_CUDA;
     return IC_OK;
 }
 
@@ -671,8 +686,9 @@ static int stack_forward(const char* pattern, int n_layers, const ic_layer* laye
     float* sc = reinterpret_cast<float*>(ws);
 
     auto mark = [&](int l, int slot) -> int {
-        if (!events || !events[4 * l + slot]) return IC_OK;
-        cudaError_t e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(events[4 * l + slot]), st);
+        if (!events || !events[IC_MARKS_PER_LAYER * l + slot]) return IC_OK;
+        cudaError_t e = cudaEventRecord(
+            reinterpret_cast<cudaEvent_t>(events[IC_MARKS_PER_LAYER * l + slot]), st);
         return e == cudaSuccess ? IC_OK : cuda_fail(e, "cudaEventRecord");
     };
     const bool one_chunk = blocks_per_chunk >= n_blocks;
@@ -705,6 +721,7 @@ static int stack_forward(const char* pattern, int n_layers, const ic_layer* laye
         if ((rc = mark(l, 2))) return rc;
         if (dense) {
             if ((rc = launch_dense_attn(dg, D, L, dmask, dvt, st))) return rc;
+            if ((rc = mark(l, 3))) return rc;
             if (dg.Lq_d < D.Lq) {
                 rc = launch_attn(L.q, L.k, L.v, idx_cache, D.B, D.Lq, D.Lk, D.Hq, D.d, D.k,
                                  D.q_offset, D.scale, L.out, L.lse,
@@ -712,11 +729,12 @@ static int stack_forward(const char* pattern, int n_layers, const ic_layer* laye
                                  true, sms, st, dg.Lq_d, D.Lq - dg.Lq_d);
             }
         } else {
+            if ((rc = mark(l, 3))) return rc;
             rc = launch_attn(L.q, L.k, L.v, idx_cache, D.B, D.Lq, D.Lk, D.Hq, D.d, D.k, D.q_offset,
                              D.scale, L.out, L.lse, ws, ws_bytes, true, sms, st);
         }
         if (rc) return rc;
-        if ((rc = mark(l, 3))) return rc;
+        if ((rc = mark(l, 4))) return rc;
         if (L.idx_dump) {
             cudaError_t e = cudaMemcpyAsync(L.idx_dump, idx_cache,
                                             (size_t)n_rows * D.k * sizeof(int32_t),

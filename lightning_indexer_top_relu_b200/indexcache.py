@@ -33,7 +33,9 @@ EXPORTS = ("ic_status_string", "ic_last_error_message", "ic_get_last_device_erro
            "ic_indexer_scores", "ic_topk_select", "ic_sparse_attn",
            "ic_sparse_attn_workspace_bytes", "ic_layer_stack_workspace_bytes",
            "ic_layer_stack_forward", "ic_layer_stack_forward_events", "ic_selftest_wait_timeout",
-           "ic_sparse_attn_no_alloc")
+           "ic_sparse_attn_no_alloc", "ic_kernel_launch_count")
+
+MARKS_PER_LAYER = 5        # IC_MARKS_PER_LAYER
 
 
 class IndexCacheError(RuntimeError):
@@ -86,6 +88,8 @@ _lib.ic_selftest_wait_timeout.argtypes = [_I, _P]
 _lib.ic_layer_stack_forward_events.restype = _I
 _lib.ic_layer_stack_forward_events.argtypes = [ctypes.c_char_p, _I, ctypes.POINTER(ICLayer),
                                                ctypes.POINTER(ICDims), _P, _P, _Z, _P, _P]
+_lib.ic_kernel_launch_count.restype = ctypes.c_ulonglong
+_lib.ic_kernel_launch_count.argtypes = []
 _lib.ic_layer_stack_forward.restype = _I
 _lib.ic_layer_stack_forward.argtypes = [ctypes.c_char_p, _I, ctypes.POINTER(ICLayer),
                                         ctypes.POINTER(ICDims), _P, _P, _Z, _P]
@@ -123,6 +127,11 @@ def _stream(stream) -> Optional[int]:
 def get_last_device_error(stream=None) -> int:
     """Synchronises the stream and returns (and clears) the device error status."""
     return int(_lib.ic_get_last_device_error(_stream(stream)))
+
+
+def kernel_launch_count() -> int:
+    """Kernel launches the library has issued in this process so far."""
+    return int(_lib.ic_kernel_launch_count())
 
 
 def selftest_wait_timeout(timeout_us: int = 20000, stream=None) -> None:
@@ -252,8 +261,8 @@ class LayerStack:
         self._pattern_b = pattern.encode()
 
     def forward(self, stream=None, events=None):
-        """Runs the stack; `events` (a ctypes array of 4*n_layers cudaEvent_t
-        handles, or None) selects ic_layer_stack_forward_events."""
+        """Runs the stack; `events` (a ctypes array of MARKS_PER_LAYER*n_layers
+        cudaEvent_t handles, or None) selects ic_layer_stack_forward_events."""
         if events is None:
             rc = _lib.ic_layer_stack_forward(self._pattern_b, len(self.layers), self.table,
                                              ctypes.byref(self.dims), _ptr(self.idx_cache),

@@ -118,3 +118,16 @@ def test_workspace_query(ic):
     one_block = ic.layer_stack_workspace_bytes(d, 4, rows_per_chunk=1)
     assert 0 < one_block < full
     assert ic.layer_stack_workspace_bytes(_dims(ic, d_I=96), 4) == 0
+
+
+def test_rejected_calls_launch_nothing(ic):
+    before = ic.kernel_launch_count()
+    assert _stack_call(ic, "SF", _dims(ic)) == 3                   # leading S
+    assert _stack_call(ic, "FX", _dims(ic)) == 1                   # bad pattern character
+    assert ic.kernel_launch_count() == before
+
+
+def test_marks_per_layer_matches_header(ic):
+    text = open(HEADER).read()
+    m = re.search(r"#define\s+IC_MARKS_PER_LAYER\s+(\d+)", text)
+    assert m and int(m.group(1)) == ic.MARKS_PER_LAYER

@@ -12,6 +12,7 @@ Bars (stated for bf16 inputs with fp32 accumulation):
     oracle's own scores, attention outputs within 2e-2 on the rows whose
     sets agree, S-layer indices bitwise equal to their F layer's.
 """
+import ctypes
 import math
 
 import numpy as np
@@ -275,12 +276,39 @@ def test_stack_chunking_and_pattern_spelling_do_not_change_results(ic):
     wl = synth.custom(Lq=700, n_layers=4, H_I=32, d_I=128, k=96, Hq=16, d=128,
                       pattern="FSFS", cfg_id=24)
     layers = synth.make_layers(wl)
+    n0 = ic.kernel_launch_count()
     a = _run_stack(ic, wl, layers)
+    assert ic.kernel_launch_count() > n0
     b = _run_stack(ic, wl, layers, pattern="1010", rows_per_chunk=1)   # one query block per chunk
     for l in range(4):
         assert torch.equal(a.outs[l], b.outs[l])
         assert torch.equal(a.dumps[l], b.dumps[l])
     _compare_stack(a, wl, layers, None)
+
+
+def test_stack_timing_marks_are_recorded_in_order(ic):
+    # rows t < 4k take the dense-masked kernel, the rest gather: every mark
+    # of every layer is recorded, in stream order
+    wl = synth.custom(Lq=700, n_layers=2, H_I=32, d_I=128, k=96, Hq=16, d=128, pattern="FS",
+                      cfg_id=26)
+    layers = synth.make_layers(wl)
+    dims = ic.make_dims(wl.B, wl.Lq, wl.Lk, wl.q_offset, wl.H_I, wl.d_I, wl.Hq, wl.d, wl.k)
+    st = ic.LayerStack(wl.pattern, [_cuda(L) for L in layers], dims)
+    stream = torch.cuda.current_stream()
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(ic.MARKS_PER_LAYER * 2)]
+    for e in evs:
+        e.record(stream)
+    arr = (ctypes.c_void_p * len(evs))(*[e.cuda_event for e in evs])
+    torch.cuda.synchronize()
+    st.forward(stream, events=arr)
+    torch.cuda.synchronize()
+    assert ic.get_last_device_error() == 0
+    gaps = [evs[i].elapsed_time(evs[i + 1]) for i in range(len(evs) - 1)]
+    assert min(gaps) >= 0.0
+    npl = ic.MARKS_PER_LAYER
+    assert evs[2].elapsed_time(evs[3]) > 0.0          # layer 0: dense-masked rows
+    assert evs[3].elapsed_time(evs[4]) > 0.0          # layer 0: gathered rows
+    assert evs[npl + 3].elapsed_time(evs[npl + 4]) > 0.0
 
 
 def test_stack_leading_shared_layer_fails_before_launch(ic):
