@@ -160,6 +160,29 @@ int ic_sparse_attn_no_alloc(const uint16_t *q, const uint16_t *k, const uint16_t
                             int k_slots, int q_offset, float scale, uint16_t *out, float *lse,
                             ic_stream_t stream);
 
+/*
+ * Step a4 as the layer stack runs it, for index rows that hold every position
+ * at most once (top-k output always does).  Same arguments, layout and
+ * results as ic_sparse_attn, except that a position repeated within a row
+ * counts once here (ic_sparse_attn counts every slot).  Rows whose selection
+ * can cover a quarter of their visible positions (t < 4k, in whole blocks of
+ * 128/Hq queries; d = 128 and Hq dividing 128; at most 65536 visible keys)
+ * attend tile-dense on the tensor cores under a bitmask of the selection --
+ * probability exactly 0 outside it -- when ws holds at least
+ * ic_sparse_attn_unique_workspace_bytes(...) bytes; the other rows, and all
+ * rows with a smaller workspace, gather.  Slots outside [0, t] are skipped and
+ * flag IC_ERR_INVALID_ARG in the device error word, as in ic_sparse_attn.
+ */
+int ic_sparse_attn_unique(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                          const int32_t *idx, int B, int Lq, int Lk, int Hq, int Hkv, int d,
+                          int k_slots, int q_offset, float scale, uint16_t *out, float *lse,
+                          void *ws, size_t ws_bytes, ic_stream_t stream);
+
+/* Workspace with which ic_sparse_attn_unique takes the dense-masked path
+ * where it applies (0 for invalid sizes). */
+size_t ic_sparse_attn_unique_workspace_bytes(int B, int Lq, int Lk, int q_offset, int Hq, int d,
+                                             int k_slots);
+
 /* One layer of the stack.  S layers may leave q_idx, k_idx and w NULL. */
 typedef struct {
     const uint16_t *q;      /* [B, Lq, Hq, d] bf16 */

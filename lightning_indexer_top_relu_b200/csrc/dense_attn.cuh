@@ -369,18 +369,24 @@ dense_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
 }
 
 // Bitmask of each row's selected positions: row p (= b*Lq_d + i, i < Lq_d)
-// of `mask` gets bit s set for every index s in idx[b, i, :] (-1 skipped).
-__global__ void build_mask_kernel(const int32_t* __restrict__ idx, int Lq, int k, int Lq_d, int W,
-                                  uint32_t* __restrict__ mask, long long n_rows) {
+// of `mask` gets bit s set for every index s in idx[b, i, :] with
+// 0 <= s <= t = q_offset + i (-1 skipped; any other value is skipped and
+// reported as DEV_ERR_BAD_INDEX, like the gather kernel does).
+__global__ void build_mask_kernel(const int32_t* __restrict__ idx, int Lq, int k, int q_offset,
+                                  int Lq_d, int W, uint32_t* __restrict__ mask, long long n_rows) {
     extern __shared__ uint32_t mk_smem[];
     for (long long p = blockIdx.x; p < n_rows; p += gridDim.x) {
         const long long b = p / Lq_d, i = p % Lq_d;
+        const int t = q_offset + (int)i;
         const int32_t* ir = idx + (b * Lq + i) * (long long)k;
         for (int w = threadIdx.x; w < W; w += blockDim.x) mk_smem[w] = 0u;
         __syncthreads();
         for (int s = threadIdx.x; s < k; s += blockDim.x) {
             const int id = __ldg(ir + s);
-            if (id >= 0 && (id >> 5) < W) atomicOr(&mk_smem[id >> 5], 1u << (id & 31));
+            if (id >= 0 && id <= t && (id >> 5) < W)
+                atomicOr(&mk_smem[id >> 5], 1u << (id & 31));
+            else if (id != -1)
+                report(DEV_ERR_BAD_INDEX);
         }
         __syncthreads();
         for (int w = threadIdx.x; w < W; w += blockDim.x) mask[p * W + w] = mk_smem[w];

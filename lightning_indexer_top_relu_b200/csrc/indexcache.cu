@@ -298,6 +298,9 @@ int launch_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, const i
 // gather.  Only used inside the layer stack, whose index rows hold distinct
 // positions (a bitmask cannot count a repeated index twice).
 constexpr int DENSE_FACTOR = 4;
+// Keys a dense-masked row may see (bounds the bitmask row: 8 KB of shared
+// memory in the mask build, and the transposed V copy).
+constexpr int DENSE_MAX_KEYS = 65536;
 
 struct DenseGeom {
     bool on = false;
@@ -310,6 +313,7 @@ DenseGeom dense_geom(const ic_dims& D) {
     if (D.d != 128 || (128 % D.Hq) != 0) return g;
     g.QBD = 128 / D.Hq;
     long long lim = (long long)DENSE_FACTOR * D.k - D.q_offset;     // rows i with t < 4k
+    lim = std::min<long long>(lim, (long long)DENSE_MAX_KEYS - D.q_offset);
     lim = std::min<long long>(lim, D.Lq);
     if (lim < g.QBD) return g;
     g.Lq_d = (int)(lim / g.QBD) * g.QBD;
@@ -328,7 +332,8 @@ int launch_build_mask(const DenseGeom& g, const ic_dims& D, const int32_t* idx, 
                       cudaStream_t st) {
     const long long n = (long long)D.B * g.Lq_d;
     const int grid = (int)std::min<long long>(n, 65535);
-    ic::build_mask_kernel<<<grid, 256, g.W * 4, st>>>(idx, D.Lq, D.k, g.Lq_d, g.W, mask, n);
+    ic::build_mask_kernel<<<grid, 256, g.W * 4, st>>>(idx, D.Lq, D.k, D.q_offset, g.Lq_d, g.W,
+                                                       mask, n);
     cudaError_t e = cudaGetLastError();
     return launched(e, "build_mask launch");
 }
@@ -374,6 +379,38 @@ int launch_dense_attn(const DenseGeom& g, const ic_dims& D, const ic_layer& L,
     ic::dense_attn_kernel<<<a.n_blocks, ic::DA_THREADS, ic::DenseSmem::ALLOC, st>>>(tq, tk, tv, a);
     e = cudaGetLastError();
     return launched(e, "dense_attn launch");
+}
+
+// Attention of one layer over index rows that hold each position at most
+// once: rows with t < 4k (whole blocks) on the dense-masked kernel when the
+// workspace holds its buffers, the rest gathered.  `mask_ready` says the
+// workspace already holds this index cache's bitmask (S layers of the stack);
+// `trim` says slots past min(k, t+1) are empty (top-k output); `mid` (may be
+// null) is recorded between the two parts.
+int attn_step(const ic_dims& D, const ic_layer& L, const int32_t* idx, bool mask_ready, bool trim,
+              void* ws, size_t ws_bytes, int sms, cudaStream_t st, cudaEvent_t mid) {
+    const DenseGeom dg = dense_geom(D);
+    const bool dense = dg.on && dg.total <= ws_bytes;
+    auto mark = [&]() -> int {
+        if (!mid) return IC_OK;
+        cudaError_t e = cudaEventRecord(mid, st);
+        return e == cudaSuccess ? IC_OK : cuda_fail(e, "cudaEventRecord");
+    };
+    int rc;
+    if (!dense) {
+        if ((rc = mark())) return rc;
+        return launch_attn(L.q, L.k, L.v, idx, D.B, D.Lq, D.Lk, D.Hq, D.d, D.k, D.q_offset,
+                           D.scale, L.out, L.lse, ws, ws_bytes, trim, sms, st);
+    }
+    uint32_t* dmask = reinterpret_cast<uint32_t*>(ws);
+    uint16_t* dvt = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(ws) + dg.mask_bytes);
+    if (!mask_ready && (rc = launch_build_mask(dg, D, idx, dmask, st))) return rc;
+    if ((rc = launch_dense_attn(dg, D, L, dmask, dvt, st))) return rc;
+    if ((rc = mark())) return rc;
+    if (dg.Lq_d >= D.Lq) return IC_OK;
+    return launch_attn(L.q, L.k, L.v, idx, D.B, D.Lq, D.Lk, D.Hq, D.d, D.k, D.q_offset, D.scale,
+                       L.out, L.lse, reinterpret_cast<uint8_t*>(ws) + dg.total, ws_bytes - dg.total,
+                       trim, sms, st, dg.Lq_d, D.Lq - dg.Lq_d);
 }
 
 // ---------------------------------------------------------------- per-device setup
@@ -615,6 +652,43 @@ int ic_sparse_attn_no_alloc(const uint16_t* q, const uint16_t* k, const uint16_t
                        NOALLOC_SCRATCH_BYTES, false, sms, reinterpret_cast<cudaStream_t>(stream));
 }
 
+size_t ic_sparse_attn_unique_workspace_bytes(int B, int Lq, int Lk, int q_offset, int Hq, int d,
+                                             int k_slots) {
+    if (B <= 0 || Lq <= 0 || Hq <= 0 || d <= 0 || k_slots <= 0) return 0;
+    if (check_positions(B, Lq, Lk, q_offset)) return 0;
+    ic_dims D{};
+    D.B = B; D.Lq = Lq; D.Lk = Lk; D.q_offset = q_offset; D.Hq = Hq; D.Hkv = 1; D.d = d;
+    D.k = k_slots;
+    const DenseGeom dg = dense_geom(D);
+    const size_t attn = ic_sparse_attn_workspace_bytes(B, Lq, Hq, d, k_slots);
+    return dg.on ? dg.total + attn : attn;
+}
+
+int ic_sparse_attn_unique(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                          const int32_t* idx, int B, int Lq, int Lk, int Hq, int Hkv, int d,
+                          int k_slots, int q_offset, float scale, uint16_t* out, float* lse,
+                          void* ws, size_t ws_bytes, ic_stream_t stream) {
+    int rc = check_positions(B, Lq, Lk, q_offset);
+    if (rc) return rc;
+    if ((rc = check_attn_shape(Hq, Hkv, d))) return rc;
+    if (k_slots < 1) return fail(IC_ERR_INVALID_ARG, "k=%d", k_slots);
+    if (B == 0 || Lq == 0) return IC_OK;
+    if (!q || !k || !v || !idx || !out) return fail(IC_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v))
+        return fail(IC_ERR_UNSUPPORTED, "q, k and v must be 16-byte aligned");
+    if (!std::isfinite(scale)) return fail(IC_ERR_INVALID_ARG, "scale is not finite");
+    if (ws_bytes > 0 && !ws) return fail(IC_ERR_INVALID_ARG, "ws is NULL but ws_bytes > 0");
+    int dev, sms;
+    if ((rc = device_setup(&dev, &sms))) return rc;
+    ic_dims D{};
+    D.B = B; D.Lq = Lq; D.Lk = Lk; D.q_offset = q_offset; D.Hq = Hq; D.Hkv = Hkv; D.d = d;
+    D.k = k_slots; D.scale = scale;
+    ic_layer L{};
+    L.q = q; L.k = k; L.v = v; L.out = out; L.lse = lse;
+    return attn_step(D, L, idx, false, false, ws, ws_bytes, sms,
+                     reinterpret_cast<cudaStream_t>(stream), nullptr);
+}
+
 size_t ic_layer_stack_workspace_bytes(const ic_dims* dims, int n_layers, long long rows_per_chunk) {
     if (!dims || n_layers < 1) return 0;
     if (check_positions(dims->B, dims->Lq, dims->Lk, dims->q_offset) ||
@@ -692,13 +766,9 @@ static int stack_forward(const char* pattern, int n_layers, const ic_layer* laye
         return e == cudaSuccess ? IC_OK : cuda_fail(e, "cudaEventRecord");
     };
     const bool one_chunk = blocks_per_chunk >= n_blocks;
-    // Dense-masked attention for rows with t < 4k when the workspace holds
-    // its mask and V^T buffers (they reuse the score region: an F layer's
-    // scores are dead once its top-k is done).
-    const DenseGeom dg = dense_geom(D);
-    const bool dense = dg.on && dg.total <= ws_bytes;
-    uint32_t* dmask = reinterpret_cast<uint32_t*>(ws);
-    uint16_t* dvt = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(ws) + dg.mask_bytes);
+    // The dense-masked attention's bitmask and V^T reuse the score region: an
+    // F layer's scores are dead once its top-k is done.  The bitmask is built
+    // once per F layer and read by the S layers after it.
     for (int l = 0; l < n_layers; ++l) {
         const ic_layer& L = layers[l];
         const bool full = pattern[l] == 'F' || pattern[l] == '1';
@@ -716,24 +786,15 @@ static int stack_forward(const char* pattern, int n_layers, const ic_layer* laye
                 if (rc) return rc;
             }
         }
-        if (dense && full && (rc = launch_build_mask(dg, D, idx_cache, dmask, st))) return rc;
+        const DenseGeom dg = dense_geom(D);
+        if (full && dg.on && dg.total <= ws_bytes &&
+            (rc = launch_build_mask(dg, D, idx_cache, reinterpret_cast<uint32_t*>(ws), st)))
+            return rc;
         if (!(full && one_chunk) && (rc = mark(l, 1))) return rc;
         if ((rc = mark(l, 2))) return rc;
-        if (dense) {
-            if ((rc = launch_dense_attn(dg, D, L, dmask, dvt, st))) return rc;
-            if ((rc = mark(l, 3))) return rc;
-            if (dg.Lq_d < D.Lq) {
-                rc = launch_attn(L.q, L.k, L.v, idx_cache, D.B, D.Lq, D.Lk, D.Hq, D.d, D.k,
-                                 D.q_offset, D.scale, L.out, L.lse,
-                                 reinterpret_cast<uint8_t*>(ws) + dg.total, ws_bytes - dg.total,
-                                 true, sms, st, dg.Lq_d, D.Lq - dg.Lq_d);
-            }
-        } else {
-            if ((rc = mark(l, 3))) return rc;
-            rc = launch_attn(L.q, L.k, L.v, idx_cache, D.B, D.Lq, D.Lk, D.Hq, D.d, D.k, D.q_offset,
-                             D.scale, L.out, L.lse, ws, ws_bytes, true, sms, st);
-        }
-        if (rc) return rc;
+        cudaEvent_t mid = events ? reinterpret_cast<cudaEvent_t>(events[IC_MARKS_PER_LAYER * l + 3])
+                                 : nullptr;
+        if ((rc = attn_step(D, L, idx_cache, true, true, ws, ws_bytes, sms, st, mid))) return rc;
         if ((rc = mark(l, 4))) return rc;
         if (L.idx_dump) {
             cudaError_t e = cudaMemcpyAsync(L.idx_dump, idx_cache,

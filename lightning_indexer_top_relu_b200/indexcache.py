@@ -33,7 +33,8 @@ EXPORTS = ("ic_status_string", "ic_last_error_message", "ic_get_last_device_erro
            "ic_indexer_scores", "ic_topk_select", "ic_sparse_attn",
            "ic_sparse_attn_workspace_bytes", "ic_layer_stack_workspace_bytes",
            "ic_layer_stack_forward", "ic_layer_stack_forward_events", "ic_selftest_wait_timeout",
-           "ic_sparse_attn_no_alloc", "ic_kernel_launch_count")
+           "ic_sparse_attn_no_alloc", "ic_kernel_launch_count", "ic_sparse_attn_unique",
+           "ic_sparse_attn_unique_workspace_bytes")
 
 MARKS_PER_LAYER = 5        # IC_MARKS_PER_LAYER
 
@@ -79,6 +80,11 @@ _lib.ic_sparse_attn.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, 
 _lib.ic_sparse_attn_no_alloc.restype = _I
 _lib.ic_sparse_attn_no_alloc.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P,
                                          _P, _P]
+_lib.ic_sparse_attn_unique.restype = _I
+_lib.ic_sparse_attn_unique.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P,
+                                       _P, _Z, _P]
+_lib.ic_sparse_attn_unique_workspace_bytes.restype = _Z
+_lib.ic_sparse_attn_unique_workspace_bytes.argtypes = [_I, _I, _I, _I, _I, _I, _I]
 _lib.ic_sparse_attn_workspace_bytes.restype = _Z
 _lib.ic_sparse_attn_workspace_bytes.argtypes = [_I, _I, _I, _I, _I]
 _lib.ic_layer_stack_workspace_bytes.restype = _Z
@@ -188,6 +194,39 @@ def sparse_attn(q, k, v, idx, q_offset: int = 0, scale: float = 0.0, out=None, l
                              _ptr(ws, None, "ws"), 0 if ws is None else ws.numel() * ws.element_size(),
                              _stream(stream))
     _check(rc, "ic_sparse_attn")
+    return out, lse
+
+
+def sparse_attn_unique_workspace_bytes(B: int, Lq: int, Lk: int, q_offset: int, Hq: int, d: int,
+                                       k: int) -> int:
+    return int(_lib.ic_sparse_attn_unique_workspace_bytes(B, Lq, Lk, q_offset, Hq, d, k))
+
+
+def sparse_attn_unique(q, k, v, idx, q_offset: int = 0, scale: float = 0.0, out=None, lse=None,
+                       want_lse: bool = True, ws=None, stream=None):
+    """ic_sparse_attn_unique: the layer stack's attention step for index rows
+    that hold each position at most once (dense-masked rows t < 4k when the
+    workspace allows, gathered rows otherwise).  ws=None allocates the full
+    workspace; pass an empty tensor to force the gather path."""
+    B, Lq, Hq, d = q.shape
+    Lk = k.shape[1]
+    Hkv = k.shape[2] if k.dim() == 4 else 1
+    kslots = idx.shape[-1]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(B, Lq, Hq, device=q.device, dtype=torch.float32)
+    if ws is None:
+        nbytes = sparse_attn_unique_workspace_bytes(B, Lq, Lk, q_offset, Hq, d, kslots)
+        ws = torch.empty(max(nbytes, 1), device=q.device, dtype=torch.uint8) if nbytes else None
+    nws = 0 if ws is None else ws.numel() * ws.element_size()
+    rc = _lib.ic_sparse_attn_unique(_ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
+                                    _ptr(v, torch.bfloat16, "v"), _ptr(idx, torch.int32, "idx"),
+                                    B, Lq, Lk, Hq, Hkv, d, kslots, q_offset, float(scale),
+                                    _ptr(out, torch.bfloat16, "out"),
+                                    _ptr(lse, torch.float32, "lse"),
+                                    _ptr(ws, None, "ws") if nws else None, nws, _stream(stream))
+    _check(rc, "ic_sparse_attn_unique")
     return out, lse
 
 

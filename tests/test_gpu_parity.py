@@ -232,6 +232,72 @@ def test_sparse_attn_with_holes_and_bad_indices(ic):
     assert ic.get_last_device_error() == 0
 
 
+DENSE_CASES = [
+    # B, Lq, Lk, q_offset, Hq, d, k   (rows t < 4k take the dense-masked kernel)
+    (1, 700, 700, 0, 16, 128, 96),          # 48 dense blocks, 316 gathered rows
+    (2, 1000, 1000, 0, 16, 128, 256),       # all dense, B = 2, ragged last key tile
+    (1, 300, 1324, 1024, 16, 128, 512),     # mid-sequence chunk, 4 gathered tail rows
+    (1, 500, 500, 0, 8, 128, 128),          # 16 queries per block
+]
+
+
+@pytest.mark.parametrize("B,Lq,Lk,q_offset,Hq,d,k", DENSE_CASES)
+def test_unique_attn_dense_and_gathered_rows_match_oracle(ic, B, Lq, Lk, q_offset, Hq, d, k):
+    wl = synth.custom(B=B, Lq=Lq, Lk=Lk, q_offset=q_offset, H_I=4, d_I=64, k=k, Hq=Hq, d=d,
+                      cfg_id=27)
+    L = synth.make_layers(wl)[0]
+    idx = _oracle_idx(L, k, q_offset)
+    ref, ref_lse = oracle.sparse_attn(L["q"], L["k"], L["v"], idx, q_offset)
+    t = {n: L[n].cuda() for n in ("q", "k", "v")}
+    idx_d = torch.from_numpy(idx).reshape(B, Lq, k).cuda()
+    n0 = ic.kernel_launch_count()
+    out, lse = ic.sparse_attn_unique(t["q"], t["k"], t["v"], idx_d, q_offset)
+    n_dense = ic.kernel_launch_count() - n0
+    assert ic.get_last_device_error() == 0
+    assert n_dense >= 3                                  # mask build, V^T, dense kernel
+    got = out.float().cpu().numpy().reshape(B * Lq, Hq, d)
+    assert np.abs(got - ref).max() <= ATTN_ATOL
+    assert np.abs(lse.cpu().numpy().reshape(B * Lq, Hq) - ref_lse).max() <= LSE_ATOL
+    # without the workspace every row gathers: the same results
+    out_g, lse_g = ic.sparse_attn_unique(t["q"], t["k"], t["v"], idx_d, q_offset,
+                                         ws=torch.empty(0, device="cuda", dtype=torch.uint8))
+    assert ic.get_last_device_error() == 0
+    assert (out_g.float() - out.float()).abs().max().item() <= ATTN_ATOL
+    assert (lse_g - lse).abs().max().item() <= LSE_ATOL
+
+
+def test_unique_attn_dense_rows_with_holes_and_bad_indices(ic):
+    """The dense-masked kernel sees the selection only as a bitmask: -1 slots
+    anywhere, unsorted rows, and an index beyond t (skipped and reported)."""
+    B, L, Hq, d, k = 1, 160, 16, 128, 40                 # every row t < 4k = 160
+    wl = synth.custom(B=B, Lq=L, H_I=4, d_I=64, k=k, Hq=Hq, d=d, cfg_id=28)
+    lay = synth.make_layers(wl)[0]
+    rng = np.random.default_rng(5)
+    idx = np.full((L, k), -1, dtype=np.int32)
+    for t in range(L):
+        cand = rng.choice(t + 1, size=min(k, t + 1), replace=False)
+        keep = rng.random(len(cand)) < 0.7
+        idx[t, : len(cand)] = np.where(keep, cand, -1)
+    rng.shuffle(idx, axis=1)
+    ref, ref_lse = oracle.sparse_attn(lay["q"], lay["k"], lay["v"], idx)
+    q, kk, v = lay["q"].cuda(), lay["k"].cuda(), lay["v"].cuda()
+    out, lse = ic.sparse_attn_unique(q, kk, v, torch.from_numpy(idx).reshape(1, L, k).cuda())
+    assert ic.get_last_device_error() == 0
+    assert np.abs(out.float().cpu().numpy().reshape(L, Hq, d) - ref).max() <= ATTN_ATOL
+    fin = np.isfinite(ref_lse)
+    g_lse = lse.cpu().numpy().reshape(L, Hq)
+    assert np.array_equal(np.isfinite(g_lse), fin)
+    assert np.abs(g_lse[fin] - ref_lse[fin]).max() <= LSE_ATOL
+
+    bad = idx.copy()
+    slot = int(np.flatnonzero(bad[100] == -1)[0])
+    bad[100, slot] = 150                                  # beyond t = 100
+    out2, _ = ic.sparse_attn_unique(q, kk, v, torch.from_numpy(bad).reshape(1, L, k).cuda())
+    assert ic.get_last_device_error() == 1                # IC_ERR_INVALID_ARG, context usable
+    assert np.abs(out2.float().cpu().numpy().reshape(L, Hq, d) - ref).max() <= ATTN_ATOL
+    assert ic.get_last_device_error() == 0
+
+
 # ------------------------------------------------------------------ a3/a5 layer stack
 
 def _run_stack(ic, wl, layers, pattern=None, **kw):
