@@ -465,7 +465,7 @@ def main():
             ent["frac_of_bf16_peak"] = ent["tflops"] / peaks["bf16_tflops"]
             ent["gbs"] = w["indexer_bytes"] / sec / 1e9
         elif name == "topk":
-            ent["covers"] = "top-k select (+ selection bitmask build for dense-masked rows)"
+            ent["covers"] = "top-k select (also writes the selection bitmask of dense-masked rows)"
             ent["gbs"] = w["topk_bytes"] / sec / 1e9
             ent["frac_of_hbm"] = ent["gbs"] / peaks["hbm_gbs"]
         elif name == "attn_dense":

@@ -205,17 +205,18 @@ int launch_indexer(const uint16_t* q_idx, const uint16_t* k_idx, const float* w,
 // ---------------------------------------------------------------- top-k
 
 int launch_topk(const float* scores, long long ld, long long row_base, long long n_rows, int Lq,
-                int Lk, int q_offset, int k, int32_t* idx, cudaStream_t st) {
+                int Lk, int q_offset, int k, int32_t* idx, cudaStream_t st,
+                uint32_t* mask = nullptr, int Lq_d = 0, int W = 0) {
     if (n_rows <= 0) return IC_OK;
     const int n_max = std::min(Lk, q_offset + Lq);
     cudaError_t e;
     if (n_max <= ic::TK_CACHE_MAX) {
         const int smem = ic::TK_SMEM_FIXED + n_max * 4;
         ic::topk_select_kernel<true><<<(unsigned)n_rows, ic::TK_THREADS, smem, st>>>(
-            scores, ld, row_base, n_rows, Lq, Lk, q_offset, k, idx);
+            scores, ld, row_base, n_rows, Lq, Lk, q_offset, k, idx, mask, Lq_d, W);
     } else {
         ic::topk_select_kernel<false><<<(unsigned)n_rows, ic::TK_THREADS, ic::TK_SMEM_FIXED, st>>>(
-            scores, ld, row_base, n_rows, Lq, Lk, q_offset, k, idx);
+            scores, ld, row_base, n_rows, Lq, Lk, q_offset, k, idx, mask, Lq_d, W);
     }
     e = cudaGetLastError();
     if (launched(e, "topk_select launch")) return IC_ERR_CUDA;
@@ -381,30 +382,37 @@ int launch_dense_attn(const DenseGeom& g, const ic_dims& D, const ic_layer& L,
     return launched(e, "dense_attn launch");
 }
 
+// How the attention step treats rows with t < 4k.
+enum AttnMode {
+    ATTN_GATHER = 0,        // every row gathers
+    ATTN_MASK_READY = 1,    // dense-masked; the workspace already holds the bitmask
+    ATTN_BUILD_MASK = 2,    // dense-masked; build the bitmask from idx first
+};
+
 // Attention of one layer over index rows that hold each position at most
-// once: rows with t < 4k (whole blocks) on the dense-masked kernel when the
-// workspace holds its buffers, the rest gathered.  `mask_ready` says the
-// workspace already holds this index cache's bitmask (S layers of the stack);
-// `trim` says slots past min(k, t+1) are empty (top-k output); `mid` (may be
-// null) is recorded between the two parts.
-int attn_step(const ic_dims& D, const ic_layer& L, const int32_t* idx, bool mask_ready, bool trim,
+// once.  Dense modes (the caller checked dense_geom(D).on and that ws holds
+// dense_geom(D).total bytes): rows with t < 4k, whole blocks, on the
+// dense-masked kernel -- bitmask at ws, V^T after it, the gathered rows'
+// split partials after both -- and the rest gathered.  `trim` says slots past
+// min(k, t+1) are empty (top-k output); `mid` (may be null) is recorded
+// between the two parts.
+int attn_step(const ic_dims& D, const ic_layer& L, const int32_t* idx, AttnMode mode, bool trim,
               void* ws, size_t ws_bytes, int sms, cudaStream_t st, cudaEvent_t mid) {
-    const DenseGeom dg = dense_geom(D);
-    const bool dense = dg.on && dg.total <= ws_bytes;
     auto mark = [&]() -> int {
         if (!mid) return IC_OK;
         cudaError_t e = cudaEventRecord(mid, st);
         return e == cudaSuccess ? IC_OK : cuda_fail(e, "cudaEventRecord");
     };
     int rc;
-    if (!dense) {
+    if (mode == ATTN_GATHER) {
         if ((rc = mark())) return rc;
         return launch_attn(L.q, L.k, L.v, idx, D.B, D.Lq, D.Lk, D.Hq, D.d, D.k, D.q_offset,
                            D.scale, L.out, L.lse, ws, ws_bytes, trim, sms, st);
     }
+    const DenseGeom dg = dense_geom(D);
     uint32_t* dmask = reinterpret_cast<uint32_t*>(ws);
     uint16_t* dvt = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(ws) + dg.mask_bytes);
-    if (!mask_ready && (rc = launch_build_mask(dg, D, idx, dmask, st))) return rc;
+    if (mode == ATTN_BUILD_MASK && (rc = launch_build_mask(dg, D, idx, dmask, st))) return rc;
     if ((rc = launch_dense_attn(dg, D, L, dmask, dvt, st))) return rc;
     if ((rc = mark())) return rc;
     if (dg.Lq_d >= D.Lq) return IC_OK;
@@ -685,7 +693,9 @@ int ic_sparse_attn_unique(const uint16_t* q, const uint16_t* k, const uint16_t* 
     D.k = k_slots; D.scale = scale;
     ic_layer L{};
     L.q = q; L.k = k; L.v = v; L.out = out; L.lse = lse;
-    return attn_step(D, L, idx, false, false, ws, ws_bytes, sms,
+    const DenseGeom dg = dense_geom(D);
+    const AttnMode mode = (dg.on && dg.total <= ws_bytes) ? ATTN_BUILD_MASK : ATTN_GATHER;
+    return attn_step(D, L, idx, mode, false, ws, ws_bytes, sms,
                      reinterpret_cast<cudaStream_t>(stream), nullptr);
 }
 
@@ -703,7 +713,10 @@ size_t ic_layer_stack_workspace_bytes(const ic_dims* dims, int n_layers, long lo
     const size_t attn = ic_sparse_attn_workspace_bytes(dims->B, dims->Lq, dims->Hq, dims->d, dims->k);
     const DenseGeom dg = dense_geom(*dims);
     (void)n_rows;
-    return std::max(std::max(scores, attn), dg.on ? dg.total + attn : (size_t)0);
+    // dense-masked rows: the bitmask (written by the top-k) sits before the
+    // score chunk; V^T and the gathered rows' partials reuse the score region
+    if (dg.on) return std::max(dg.mask_bytes + scores, dg.total + attn);
+    return std::max(scores, attn);
 }
 
 static int stack_forward(const char* pattern, int n_layers, const ic_layer* layers,
@@ -756,8 +769,18 @@ static int stack_forward(const char* pattern, int n_layers, const ic_layer* laye
         return fail(IC_ERR_WORKSPACE_TOO_SMALL,
                     "workspace of %zu bytes is below one query block of scores (%zu bytes)",
                     ws_bytes, block_bytes);
-    const long long blocks_per_chunk = std::min<long long>(n_blocks, (long long)(ws_bytes / block_bytes));
-    float* sc = reinterpret_cast<float*>(ws);
+    // Rows with t < 4k attend dense-masked when the workspace holds the
+    // bitmask (which the top-k writes, ahead of the score chunk) plus one
+    // block of scores, and V^T (which, like the gathered rows' partials,
+    // reuses the score region once the layer's top-k is done).  The bitmask
+    // of an F layer is read by the S layers after it.
+    const DenseGeom dg = dense_geom(D);
+    const bool dense = dg.on && ws_bytes >= dg.mask_bytes + std::max(block_bytes, dg.vt_bytes);
+    const size_t sc_off = dense ? dg.mask_bytes : 0;
+    const long long blocks_per_chunk =
+        std::min<long long>(n_blocks, (long long)((ws_bytes - sc_off) / block_bytes));
+    float* sc = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + sc_off);
+    uint32_t* dmask = dense ? reinterpret_cast<uint32_t*>(ws) : nullptr;
 
     auto mark = [&](int l, int slot) -> int {
         if (!events || !events[IC_MARKS_PER_LAYER * l + slot]) return IC_OK;
@@ -766,9 +789,6 @@ static int stack_forward(const char* pattern, int n_layers, const ic_layer* laye
         return e == cudaSuccess ? IC_OK : cuda_fail(e, "cudaEventRecord");
     };
     const bool one_chunk = blocks_per_chunk >= n_blocks;
-    // The dense-masked attention's bitmask and V^T reuse the score region: an
-    // F layer's scores are dead once its top-k is done.  The bitmask is built
-    // once per F layer and read by the S layers after it.
     for (int l = 0; l < n_layers; ++l) {
         const ic_layer& L = layers[l];
         const bool full = pattern[l] == 'F' || pattern[l] == '1';
@@ -782,19 +802,18 @@ static int stack_forward(const char* pattern, int n_layers, const ic_layer* laye
                 if (one_chunk && (rc = mark(l, 1))) return rc;
                 const long long r0 = block_row_start(geo, D.Lq, g0);
                 const long long r1 = block_row_start(geo, D.Lq, g1);
-                rc = launch_topk(sc, D.Lk, r0, r1 - r0, D.Lq, D.Lk, D.q_offset, D.k, idx_cache, st);
+                rc = launch_topk(sc, D.Lk, r0, r1 - r0, D.Lq, D.Lk, D.q_offset, D.k, idx_cache, st,
+                                 dmask, dg.Lq_d, dg.W);
                 if (rc) return rc;
             }
         }
-        const DenseGeom dg = dense_geom(D);
-        if (full && dg.on && dg.total <= ws_bytes &&
-            (rc = launch_build_mask(dg, D, idx_cache, reinterpret_cast<uint32_t*>(ws), st)))
-            return rc;
         if (!(full && one_chunk) && (rc = mark(l, 1))) return rc;
         if ((rc = mark(l, 2))) return rc;
         cudaEvent_t mid = events ? reinterpret_cast<cudaEvent_t>(events[IC_MARKS_PER_LAYER * l + 3])
                                  : nullptr;
-        if ((rc = attn_step(D, L, idx_cache, true, true, ws, ws_bytes, sms, st, mid))) return rc;
+        rc = attn_step(D, L, idx_cache, dense ? ATTN_MASK_READY : ATTN_GATHER, true, ws, ws_bytes,
+                       sms, st, mid);
+        if (rc) return rc;
         if ((rc = mark(l, 4))) return rc;
         if (L.idx_dump) {
             cudaError_t e = cudaMemcpyAsync(L.idx_dump, idx_cache,

@@ -85,11 +85,15 @@ __device__ __forceinline__ void tk_find_bin(const uint32_t* hist, int remaining,
 
 // Rows [row_base, row_base + n_rows) of a [B*Lq] flattened row space; score
 // row r lives at scores + (r - row_base) * ld; output row r at idx + r * k.
+// With `mask` non-null, rows i < Lq_d of each sequence also write their
+// selection as a bitmask: row b*Lq_d + i of `mask` ([*, W] words) gets bit s
+// set for every selected position s (words past the row's visible positions
+// are zero).  The emit pass builds it from the ballots it already takes.
 template <bool CACHE>
 __global__ void __launch_bounds__(TK_THREADS)
 topk_select_kernel(const float* __restrict__ scores, long long ld, long long row_base,
                    long long n_rows, int Lq, int Lk, int q_offset, int k,
-                   int32_t* __restrict__ idx) {
+                   int32_t* __restrict__ idx, uint32_t* __restrict__ mask, int Lq_d, int W) {
     extern __shared__ __align__(16) uint8_t tk_smem[];
     uint32_t* hist = reinterpret_cast<uint32_t*>(tk_smem);
     uint32_t* cand = reinterpret_cast<uint32_t*>(tk_smem + TK_BINS * 4);
@@ -105,9 +109,18 @@ topk_select_kernel(const float* __restrict__ scores, long long ld, long long row
     const int t = q_offset + (int)(r % Lq);
     const int n = min(t + 1, Lk);
     int32_t* out = idx + r * (long long)k;
+    uint32_t* mrow = nullptr;
+    if (mask != nullptr && (int)(r % Lq) < Lq_d)
+        mrow = mask + ((r / Lq) * Lq_d + r % Lq) * (long long)W;
+    const int nw = (n + 31) >> 5;                                 // words with visible positions
+    if (mrow != nullptr)
+        for (int w = nw + tid; w < W; w += TK_THREADS) mrow[w] = 0u;
 
     if (n <= k) {
         for (int i = tid; i < k; i += TK_THREADS) out[i] = i < n ? i : -1;
+        if (mrow != nullptr)
+            for (int w = tid; w < nw && w < W; w += TK_THREADS)
+                mrow[w] = (32 * w + 32 <= n) ? 0xffffffffu : ((1u << (n - 32 * w)) - 1u);
         return;
     }
     const float* src = scores + rr * ld;
@@ -260,12 +273,25 @@ topk_select_kernel(const float* __restrict__ scores, long long ld, long long row
             const unsigned me = __ballot_sync(0xffffffffu, i < s1 && kb[u] == T);
             const unsigned gi = g + __popc(mg & lt);
             const unsigned ei = e + __popc(me & lt);
+            bool sel = false;
             if ((mg >> lane) & 1u) {
                 const unsigned pos = gi + min(ei, (unsigned)need);
-                if (pos < (unsigned)k) out[pos] = i;
+                if (pos < (unsigned)k) {
+                    out[pos] = i;
+                    sel = true;
+                }
             } else if (((me >> lane) & 1u) && ei < (unsigned)need) {
                 const unsigned pos = gi + ei;
-                if (pos < (unsigned)k) out[pos] = i;
+                if (pos < (unsigned)k) {
+                    out[pos] = i;
+                    sel = true;
+                }
+            }
+            if (mrow != nullptr) {
+                // 32 consecutive positions starting at a multiple of 32
+                const unsigned word = __ballot_sync(0xffffffffu, sel);
+                const int w0 = (gbase + u * 32) >> 5;
+                if (lane == 0 && gbase + u * 32 < s1 && w0 < W) mrow[w0] = word;
             }
             g += __popc(mg);
             e += __popc(me);
