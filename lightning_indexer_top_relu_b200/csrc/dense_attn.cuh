@@ -15,19 +15,28 @@
 //               2-stage K ring and V^T[d, keys] (a per-layer transposed copy)
 //               into a 2-stage V ring.  One thread polls both rings and
 //               refills whichever stage is released first.
-//   warp 1      TMEM allocation + MMA issue.  S(j) = Q K(j)^T (M=128, N=64,
-//               K=d) goes to one of two TMEM score buffers, so S(j+1) is
-//               computed while the softmax works on S(j); O += P(j) V(j)
-//               (A = P from shared memory, B = V^T tile) accumulates in TMEM.
+//   warp 1      TMEM allocation + MMA issue.  S(j) = bias + Q K(j)^T (M=128,
+//               N=64) goes to one of two TMEM score buffers, so S(j+1) is
+//               computed while the softmax works on S(j).  The bias term is one
+//               extra K=16 step: a one-hot matrix (row -> its query) times the
+//               tile's bias matrix (key x query: 0 where the key is selected,
+//               -2^100 where it is not), so unselected scores arrive at about
+//               -2^100 and their probabilities are exactly 0.  O += P(j) V(j)
+//               reads P from TMEM (A operand) and the V^T tile from shared
+//               memory; O accumulates in TMEM.
 //   warps 2..5  softmax: thread = row = TMEM lane.  Loads S(j) once into
-//               registers, masks it with the row's bitmask (prefetched one
-//               tile ahead), takes the tile max, computes the probabilities,
-//               and only then waits for P(j-1) V(j-1) to finish before it
-//               writes P(j) as bf16 into a 128-byte-swizzled shared tile.
+//               registers, computes the probabilities against the running
+//               max, and only then waits for P(j-1) V(j-1) to finish before
+//               it writes P(j) as bf16 over the columns of S(j) it has read.
 //               The running max is raised lazily: only when a tile's max
 //               exceeds it by more than 8 (log2 units) is O rescaled in TMEM,
-//               so P stays <= 2^8 and O / l is exact either way.
-// Scores are scaled in the log2 domain; masked positions contribute exactly 0.
+//               so P stays <= 2^8 and O / l is exact either way.  A tile whose
+//               probabilities sum to at most 2^8 cannot hold a larger one, so
+//               the tile max is only taken (and the tile redone) when the sum
+//               is larger or no selected key has been seen yet.  Each thread
+//               also writes its share of the bias matrix two tiles ahead from
+//               the selection bitmask of its query.
+// Scores are scaled in the log2 domain.
 #pragma once
 
 #include "common.cuh"
@@ -37,6 +46,8 @@ namespace ic {
 constexpr int DA_THREADS = 192;                  // 2 control warps + 4 softmax warps
 constexpr int DA_TILE = 64;                      // keys per tile
 constexpr float DA_RESCALE = 8.0f;               // lazy-max threshold (log2 units)
+constexpr uint16_t DA_BIAS_OFF = 0xF180u;        // bf16 -2^100: an unselected key's bias
+constexpr float DA_NONE = -1.0e29f;              // scores below this are unselected
 
 struct DenseAttnArgs {
     const uint32_t* mask;      // [B * Lq_d, W] bitmask of selected positions, row b*Lq_d + i
@@ -51,16 +62,27 @@ struct DenseAttnArgs {
     float scale_log2;
 };
 
+// No-swizzle K-major operand of K = 16 bf16: 8-row x 16-byte core matrices,
+// the two along K 128 bytes apart, 8-row groups 256 bytes apart.
+constexpr int DA_NS_LBO = 128;
+constexpr int DA_NS_SBO = 256;
+
+__device__ __forceinline__ uint32_t ns_offset(int row, int col) {
+    return (uint32_t)((row >> 3) * DA_NS_SBO + (col >> 3) * DA_NS_LBO + (row & 7) * 16 + (col & 7) * 2);
+}
+
 struct DenseSmem {
     static constexpr int Q_BYTES = 128 * 128 * 2;            // 128 rows x 128 d (two 64-col boxes)
     static constexpr int K_BYTES = 64 * 128 * 2;             // 64 keys x 128 d (two boxes)
     static constexpr int V_BYTES = 128 * 64 * 2;             // 128 d x 64 keys (one box)
-    static constexpr int P_BYTES = 128 * 64 * 2;             // 128 rows x 64 keys (one box)
+    static constexpr int BIAS_BYTES = 64 * 16 * 2;           // 64 keys x 16 queries, no swizzle
+    static constexpr int ONEHOT_BYTES = 128 * 16 * 2;        // 128 rows x 16 queries, no swizzle
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + Q_BYTES;            // 2 stages
     static constexpr int OFF_V = OFF_K + 2 * K_BYTES;        // 2 stages
-    static constexpr int OFF_P = OFF_V + 2 * V_BYTES;
-    static constexpr int OFF_BAR = OFF_P + P_BYTES;
+    static constexpr int OFF_BIAS = OFF_V + 2 * V_BYTES;     // 2 stages
+    static constexpr int OFF_ONEHOT = OFF_BIAS + 2 * BIAS_BYTES;
+    static constexpr int OFF_BAR = OFF_ONEHOT + ONEHOT_BYTES;
     static constexpr int N_BARS = 16;
     static constexpr int OFF_SLOT = OFF_BAR + N_BARS * 8;
     static constexpr int BYTES = OFF_SLOT + 16;
@@ -72,7 +94,8 @@ struct DenseSmem {
     static_assert(BYTES <= PAIR_MAX, "two CTAs must fit one SM");
 };
 
-// TMEM columns of one CTA: two 64-column score buffers, then O (128 columns).
+// TMEM columns of one CTA: two 64-column score buffers (P(j) overwrites the
+// first 32 columns of S(j) as packed bf16 pairs), then O (128 columns).
 constexpr uint32_t DA_TMEM_COLS = 256;
 constexpr uint32_t DA_O_COL = 128;
 
@@ -85,6 +108,28 @@ __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// Shared-memory descriptor of a no-swizzle K-major operand (layout code 0).
+__device__ __forceinline__ uint64_t ns_kmajor_desc(uint32_t smem_addr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_addr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)(DA_NS_LBO >> 4) << 16;
+    d |= (uint64_t)(DA_NS_SBO >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    return d;
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]^T, kind::f16; A is M x K bf16 in TMEM (lane =
+// row, two K elements per 32-bit column).
+__device__ __forceinline__ void tc_mma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                  uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
 }
 
 // tmap_q: q as 3-D {128, Lq*Hq, B}, box {64, 128, 1}; tmap_k: K as {128, Lk, B},
@@ -107,6 +152,7 @@ dense_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
     uint64_t* p_full = bars + 11;
     uint64_t* o_full = bars + 12;
     uint64_t* mma_done = bars + 13;
+    uint64_t* bias_full = bars + 14;   // [2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::OFF_SLOT);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -124,11 +170,25 @@ dense_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
             mbar_init(&v_full[i], 1);
             mbar_init(&v_empty[i], 1);
             mbar_init(&s_full[i], 1);
+            mbar_init(&bias_full[i], 128);
         }
         mbar_init(p_full, 128);
         mbar_init(o_full, 1);
         mbar_init(mma_done, 1);
         fence_barrier_init();
+    }
+    // one-hot rows (row r -> query r / Hq) and zeroed bias stages (the query
+    // columns past QBD stay 0)
+    {
+        uint32_t* z = reinterpret_cast<uint32_t*>(smem + S::OFF_BIAS);
+        for (int i = threadIdx.x; i < (2 * S::BIAS_BYTES + S::ONEHOT_BYTES) / 4; i += DA_THREADS)
+            z[i] = 0u;
+        __syncthreads();
+        if (threadIdx.x < 128) {
+            const int r = threadIdx.x;
+            *reinterpret_cast<uint16_t*>(smem + S::OFF_ONEHOT + ns_offset(r, r / a.Hq)) = 0x3F80u;
+        }
+        fence_proxy_async_smem();
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, DA_TMEM_COLS);
@@ -190,22 +250,30 @@ dense_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
             const uint32_t idesc_s = idesc_bf16_f32(128, DA_TILE);
             const uint32_t idesc_o = idesc_bf16_f32(128, 128);
             const uint32_t q_addr = smem_u32(smem + S::OFF_Q);
-            const uint32_t p_addr = smem_u32(smem + S::OFF_P);
+            const uint64_t onehot_desc = ns_kmajor_desc(smem_u32(smem + S::OFF_ONEHOT));
             bool ok = mbar_wait(q_full, 0);
-            // iteration j issues S(j), then P(j-1) V(j-1): S(j) overwrites the
-            // buffer of S(j-2), which the softmax released with P(j-2).
+            // iteration j issues S(j), then P(j-1) V(j-1).  S(j) overwrites the
+            // buffer of S(j-2) and P(j-2): the softmax released S(j-2) with
+            // P(j-2), and P(j-2) V(j-2), which reads P(j-2) from there, has
+            // completed before S(j) is issued.
             for (int j = 0; j <= nt && ok; ++j) {
                 if (j < nt) {
                     const int st = j & 1;
                     if (!(ok = mbar_wait(&k_full[st], (j >> 1) & 1))) break;
+                    if (!(ok = mbar_wait(&bias_full[st], (j >> 1) & 1))) break;
+                    if (j >= 2 && !(ok = mbar_wait(o_full, (j - 2) & 1))) break;
                     tc_fence_after();
                     const uint32_t k_addr = smem_u32(smem + S::OFF_K + st * S::K_BYTES);
+                    const uint32_t s_col = tmem + (uint32_t)(st * DA_TILE);
+                    tc_mma_f16(s_col, onehot_desc,
+                               ns_kmajor_desc(smem_u32(smem + S::OFF_BIAS + st * S::BIAS_BYTES)),
+                               idesc_s, 0u);
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
                         const uint32_t qo = (uint32_t)((kk >> 2) * 128 * 128 + (kk & 3) * 32);
                         const uint32_t ko = (uint32_t)((kk >> 2) * 64 * 128 + (kk & 3) * 32);
-                        tc_mma_f16(tmem + (uint32_t)(st * DA_TILE), sw128_kmajor_desc(q_addr + qo),
-                                   sw128_kmajor_desc(k_addr + ko), idesc_s, kk > 0 ? 1u : 0u);
+                        tc_mma_f16(s_col, sw128_kmajor_desc(q_addr + qo),
+                                   sw128_kmajor_desc(k_addr + ko), idesc_s, 1u);
                     }
                     tc_commit(&s_full[st]);
                     tc_commit(&k_empty[st]);
@@ -216,14 +284,13 @@ dense_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     if (!(ok = mbar_wait(&v_full[st], (jp >> 1) & 1))) break;
                     tc_fence_after();
                     const uint32_t v_addr = smem_u32(smem + S::OFF_V + st * S::V_BYTES);
-                    // O += P V   (A = P [rows x 64 keys], B = V^T tile [128 d x 64 keys])
+                    const uint32_t p_col = tmem + (uint32_t)(st * DA_TILE);
+                    // O += P V   (A = P [rows x 64 keys] in TMEM, B = V^T tile [128 d x 64 keys])
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint32_t off = (uint32_t)(kk * 32);
-                        tc_mma_f16(tmem + DA_O_COL, sw128_kmajor_desc(p_addr + off),
-                                   sw128_kmajor_desc(v_addr + off), idesc_o,
-                                   (jp > 0 || kk > 0) ? 1u : 0u);
-                    }
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc_mma_f16_tmem_a(tmem + DA_O_COL, p_col + (uint32_t)(kk * 8),
+                                          sw128_kmajor_desc(v_addr + (uint32_t)(kk * 32)), idesc_o,
+                                          (jp > 0 || kk > 0) ? 1u : 0u);
                     tc_commit(o_full);
                     tc_commit(&v_empty[st]);
                 }
@@ -240,65 +307,90 @@ dense_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
         const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
         const bool row_ok = i0 + qi < a.Lq_d;
         const uint32_t* mrow = a.mask + (long long)(b * a.Lq_d + (row_ok ? i0 + qi : 0)) * a.W;
-        uint8_t* prow = smem + S::OFF_P + r * 128;
         const float sc = a.scale_log2;
+        // bias share: keys [kb0, kb0 + kpt) of each tile for query qi
+        const int kpt = DA_TILE / a.Hq;
+        const int kb0 = h * kpt;
+        auto bias_word = [&](int jj) -> uint32_t {
+            const int wi = (jj * DA_TILE + kb0) >> 5;
+            return (row_ok && wi < a.W) ? __ldg(mrow + wi) : 0u;
+        };
+        auto write_bias = [&](int jj, uint32_t word) {
+            uint8_t* bt = smem + S::OFF_BIAS + (jj & 1) * S::BIAS_BYTES;
+            const int sh = kb0 & 31;
+            for (int e = 0; e < kpt; ++e)
+                *reinterpret_cast<uint16_t*>(bt + ns_offset(kb0 + e, qi)) =
+                    ((word >> (sh + e)) & 1u) ? (uint16_t)0u : DA_BIAS_OFF;
+            fence_proxy_async_smem();
+            mbar_arrive(&bias_full[jj & 1]);
+        };
         float m_used = -INFINITY, l_run = 0.0f;
         bool ok = true;
-        auto load_mask = [&](int j, uint32_t& w0, uint32_t& w1) {
-            const int wi = j * 2;
-            w0 = (row_ok && wi < a.W) ? __ldg(mrow + wi) : 0u;
-            w1 = (row_ok && wi + 1 < a.W) ? __ldg(mrow + wi + 1) : 0u;
-        };
-        uint32_t nm0, nm1;
-        load_mask(0, nm0, nm1);
+        if (nt > 0) write_bias(0, bias_word(0));
+        if (nt > 1) write_bias(1, bias_word(1));
+        uint32_t nbw = nt > 2 ? bias_word(2) : 0u;
         for (int j = 0; j < nt; ++j) {
-            const uint32_t mw0 = nm0, mw1 = nm1;
-            if (j + 1 < nt) load_mask(j + 1, nm0, nm1);         // one tile ahead
             if (!mbar_wait(&s_full[j & 1], (j >> 1) & 1)) { ok = false; break; }
             tc_fence_after();
+            // S(j+2) overwrites bias stage j&1 only after S(j) is complete
+            if (j + 2 < nt) {
+                write_bias(j + 2, nbw);
+                if (j + 3 < nt) nbw = bias_word(j + 3);
+            }
+            const uint32_t sb = tmem + lane_base + (uint32_t)((j & 1) * DA_TILE);
             uint32_t v[64];
             {
                 uint32_t (&v0)[32] = *reinterpret_cast<uint32_t (*)[32]>(&v[0]);
                 uint32_t (&v1)[32] = *reinterpret_cast<uint32_t (*)[32]>(&v[32]);
-                const uint32_t sb = tmem + lane_base + (uint32_t)((j & 1) * DA_TILE);
                 tmem_ld_32x32b_x32(sb, v0);
                 tmem_ld_32x32b_x32(sb + 32, v1);
                 tmem_ld_wait();
             }
-            // positions outside the selection become -inf; tile max as a tree
-            float s[64];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                s[e] = ((mw0 >> e) & 1u) ? __uint_as_float(v[e]) : -INFINITY;
-                s[32 + e] = ((mw1 >> e) & 1u) ? __uint_as_float(v[32 + e]) : -INFINITY;
-            }
-            float mx[32];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) mx[e] = fmaxf(s[e], s[e + 32]);
-#pragma unroll
-            for (int w = 16; w >= 1; w >>= 1)
-#pragma unroll
-                for (int e = 0; e < w; ++e) mx[e] = fmaxf(mx[e], mx[e + w]);
-            const float mxs = mx[0] * sc;
-            const bool raise = mxs > m_used + DA_RESCALE;
-            const float m_new = raise ? mxs : m_used;
-            const float base = m_new == -INFINITY ? 0.0f : m_new;
-            // probabilities (bf16 pairs) and their sum
+            // probabilities (bf16 pairs) against `base`, and their sum
             uint32_t pk[32];
-            float2 rs2[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
-            const float2 sc2 = make_float2(sc, sc), nb2 = make_float2(-base, -base);
+            float rs;
+            auto softmax_tile = [&](float base) {
+                float2 rs2[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+                const float2 sc2 = make_float2(sc, sc), nb2 = make_float2(-base, -base);
 #pragma unroll
-            for (int e = 0; e < 64; e += 2) {
-                const float2 x = __ffma2_rn(make_float2(s[e], s[e + 1]), sc2, nb2);
-                const float2 p = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-                rs2[(e >> 1) & 3] = __fadd2_rn(rs2[(e >> 1) & 3], p);
-                __nv_bfloat162 pp = __floats2bfloat162_rn(p.x, p.y);
-                pk[e >> 1] = *reinterpret_cast<uint32_t*>(&pp);
+                for (int e = 0; e < 64; e += 2) {
+                    const float2 x = __ffma2_rn(
+                        make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), sc2, nb2);
+                    const float2 p = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                    rs2[(e >> 1) & 3] = __fadd2_rn(rs2[(e >> 1) & 3], p);
+                    __nv_bfloat162 pp = __floats2bfloat162_rn(p.x, p.y);
+                    pk[e >> 1] = *reinterpret_cast<uint32_t*>(&pp);
+                }
+                const float2 r01 = __fadd2_rn(rs2[0], rs2[1]), r23 = __fadd2_rn(rs2[2], rs2[3]);
+                const float2 rsum = __fadd2_rn(r01, r23);
+                rs = rsum.x + rsum.y;
+            };
+            // Against the running max first: a sum <= 2^8 means every
+            // probability is <= 2^8, so the running max stands (the lazy
+            // rule).  Otherwise -- or before any selected key was seen -- take
+            // the tile max (unselected keys sit near -2^100) and redo the tile.
+            bool raise = false;
+            float m_new = m_used;
+            bool need_max = m_used == -INFINITY;
+            if (!need_max) {
+                softmax_tile(m_used);
+                need_max = !(rs <= 256.0f);
             }
-            const float2 r01 = __fadd2_rn(rs2[0], rs2[1]), r23 = __fadd2_rn(rs2[2], rs2[3]);
-            const float2 rsum = __fadd2_rn(r01, r23);
-            const float rs = rsum.x + rsum.y;
-            // P(j-1) V(j-1) must be complete before O is rescaled or P is overwritten
+            if (need_max) {
+                float mx[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    mx[e] = fmaxf(__uint_as_float(v[e]), __uint_as_float(v[e + 32]));
+#pragma unroll
+                for (int w = 16; w >= 1; w >>= 1)
+#pragma unroll
+                    for (int e = 0; e < w; ++e) mx[e] = fmaxf(mx[e], mx[e + w]);
+                const float mxs = mx[0] > DA_NONE ? mx[0] * sc : -INFINITY;
+                raise = mxs > m_used + DA_RESCALE;
+                m_new = raise ? mxs : m_used;
+                softmax_tile(m_new == -INFINITY ? 0.0f : m_new);
+            }
+            // P(j-1) V(j-1) must be complete before O is rescaled
             if (j > 0) {
                 if (!mbar_wait(o_full, (j - 1) & 1)) { ok = false; break; }
                 tc_fence_after();
@@ -316,18 +408,14 @@ dense_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
                             o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
                         tmem_st_32x32b_x32(tmem + DA_O_COL + lane_base + c * 32, o);
                     }
-                    tmem_st_wait();
                 }
                 l_run *= alpha;
                 m_used = m_new;
             }
             l_run += rs;
-            // keys 8u .. 8u+7 = 16-byte chunk u of the row, stored at chunk u ^ (r & 7)
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-                *reinterpret_cast<uint4*>(prow + ((u ^ (r & 7)) << 4)) =
-                    make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-            fence_proxy_async_smem();
+            // P(j) over the first 32 columns of S(j), already read
+            tmem_st_32x32b_x32(sb, pk);
+            tmem_st_wait();
             tc_fence_before();
             mbar_arrive(p_full);
         }
