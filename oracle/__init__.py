@@ -61,8 +61,9 @@ def _load():
         lib.or_topk_count.argtypes = [P, P, L, I, I, P]
         lib.or_sparse_attn.argtypes = [P, P, P, P, I, I, I, I, I, I, I, D, P, L, P, P]
         lib.or_dense_attn.argtypes = [P, P, P, I, I, I, I, I, I, D, P, L, P, P]
+        lib.or_index_overlap.argtypes = [P, P, L, I, I, P]
         for f in ("or_indexer_scores", "or_topk_sort", "or_topk_count", "or_sparse_attn",
-                  "or_dense_attn", "or_num_threads"):
+                  "or_dense_attn", "or_num_threads", "or_index_overlap"):
             getattr(lib, f).restype = ctypes.c_int
         lib.or_set_num_threads.argtypes = [I]
         lib.or_set_num_threads.restype = None
@@ -211,6 +212,34 @@ def dense_attn(q, K, V, q_offset: int = 0, scale: float = 0.0, rows=None):
     if rc:
         raise ValueError(f"or_dense_attn failed ({rc})")
     return out, lse
+
+
+def index_overlap(idx_a, idx_b, Lk: int) -> np.ndarray:
+    """Per row of two index tensors ([n_rows, k] int32, -1 = empty), the set
+    sizes (|A & B|, |A|, |B|) as int32 [n_rows, 3] (skill page, Step 1)."""
+    a, b = _i32(idx_a), _i32(idx_b)
+    if a.shape != b.shape:
+        raise ValueError("index tensors differ in shape")
+    k = a.shape[-1]
+    a = a.reshape(-1, k)
+    b = b.reshape(-1, k)
+    out = np.empty((a.shape[0], 3), dtype=np.int32)
+    rc = _load().or_index_overlap(_ptr(a), _ptr(b), a.shape[0], k, int(Lk), _ptr(out))
+    if rc:
+        raise ValueError(f"or_index_overlap failed ({rc})")
+    return out
+
+
+def overlap_fraction(counts, k: int) -> np.ndarray:
+    """|A & B| / k per row: the share of a layer's k selections another layer
+    also selects (kualia.ai review: adjacent layers share 70-100%)."""
+    return np.asarray(counts)[:, 0] / float(k)
+
+
+def jaccard(counts) -> np.ndarray:
+    """|A & B| / (|A | B| + 1e-8) per row (skill page, Step 1)."""
+    c = np.asarray(counts, dtype=np.float64)
+    return c[:, 0] / (c[:, 1] + c[:, 2] - c[:, 0] + 1e-8)
 
 
 def is_full(c: str) -> bool:

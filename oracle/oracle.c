@@ -285,3 +285,46 @@ int or_dense_attn(const uint16_t *q, const uint16_t *K, const uint16_t *V,
     }
     return rc;
 }
+
+/*
+ * Cross-layer index overlap ("IndexCache ... Cross-Layer Index Reuse", skill
+ * page, Step 1 "Analyze Index Correlation Across Layers": the top-k sets of
+ * consecutive layers are compared per query position as sets; kualia.ai
+ * review, "The Redundancy That Was Sitting There": adjacent layers share
+ * 70-100% of their selected tokens).
+ * Row r of a and of b holds k slots; -1 is an empty slot and every other
+ * value must lie in [0, Lk).  A row is read as the SET of its valid entries
+ * (a repeated position counts once).  out3[3r+0] = |A & B|, out3[3r+1] = |A|,
+ * out3[3r+2] = |B|.  Returns -1 on a size error, -2 on an entry outside
+ * [-1, Lk) (the row's counts then ignore that entry).
+ */
+int or_index_overlap(const int32_t *a, const int32_t *b, int64_t n_rows, int k, int Lk,
+                     int32_t *out3)
+{
+    if (n_rows < 0 || k < 1 || Lk < 1) return -1;
+    int rc = 0;
+#pragma omp parallel for schedule(dynamic, 16) reduction(min : rc)
+    for (int64_t r = 0; r < n_rows; ++r) {
+        unsigned char *in_a = (unsigned char *)calloc((size_t)Lk, 1);
+        unsigned char *in_b = (unsigned char *)calloc((size_t)Lk, 1);
+        for (int s = 0; s < k; ++s) {
+            int32_t x = a[r * (int64_t)k + s], y = b[r * (int64_t)k + s];
+            if (x >= 0 && x < Lk) in_a[x] = 1;
+            else if (x != -1) rc = rc < -2 ? rc : -2;
+            if (y >= 0 && y < Lk) in_b[y] = 1;
+            else if (y != -1) rc = rc < -2 ? rc : -2;
+        }
+        int32_t both = 0, na = 0, nb = 0;
+        for (int s = 0; s < Lk; ++s) {
+            na += in_a[s];
+            nb += in_b[s];
+            both += in_a[s] & in_b[s];
+        }
+        out3[3 * r] = both;
+        out3[3 * r + 1] = na;
+        out3[3 * r + 2] = nb;
+        free(in_a);
+        free(in_b);
+    }
+    return rc;
+}

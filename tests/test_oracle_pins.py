@@ -313,3 +313,38 @@ def test_synthetic_layers_overlap_in_the_reported_band():
         ids.append(oracle.topk_sort(sc.astype(np.float32), tpos, 128))
     ov = [len(set(a) & set(b)) / 128 for a, b in zip(ids[0], ids[1])]
     assert 0.6 <= np.mean(ov) <= 1.0
+
+
+# ------------------------------------------------------------------ cross-layer overlap (f2)
+
+def test_overlap_hand_example():
+    # A = {0, 3, 5, 9}, B = {3, 4, 5} (+ holes): |A&B| = 2, |A| = 4, |B| = 3,
+    # overlap 2/4, Jaccard 2/5
+    a = np.array([[0, 3, 5, 9]], dtype=np.int32)
+    b = np.array([[5, -1, 3, 4]], dtype=np.int32)
+    c = oracle.index_overlap(a, b, 10)
+    assert c.tolist() == [[2, 4, 3]]
+    assert oracle.overlap_fraction(c, 4)[0] == 0.5
+    assert abs(oracle.jaccard(c)[0] - 0.4) < 1e-9
+
+
+def test_overlap_matches_python_sets_and_is_symmetric():
+    rng = np.random.default_rng(7)
+    k, Lk, n = 24, 60, 200
+    a = rng.integers(-1, Lk, size=(n, k)).astype(np.int32)     # holes and repeats
+    b = rng.integers(-1, Lk, size=(n, k)).astype(np.int32)
+    c = oracle.index_overlap(a, b, Lk)
+    for r in range(n):
+        sa, sb = set(a[r]) - {-1}, set(b[r]) - {-1}
+        assert c[r].tolist() == [len(sa & sb), len(sa), len(sb)]
+    c2 = oracle.index_overlap(b, a, Lk)
+    assert np.array_equal(c2[:, 0], c[:, 0]) and np.array_equal(c2[:, 1:], c[:, 2:0:-1])
+
+
+def test_overlap_identity_disjoint_and_bad_entries():
+    a = np.array([[1, 2, 3], [4, 5, -1]], dtype=np.int32)
+    assert oracle.index_overlap(a, a, 8).tolist() == [[3, 3, 3], [2, 2, 2]]
+    b = np.array([[5, 6, 7], [0, 1, 2]], dtype=np.int32)
+    assert oracle.index_overlap(a, b, 8)[:, 0].tolist() == [0, 0]
+    with pytest.raises(ValueError):
+        oracle.index_overlap(np.array([[8, 1, 2]], dtype=np.int32), a[:1], 8)
