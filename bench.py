@@ -313,6 +313,47 @@ def aggregate_over_ranks(ms_per_step: float, tokens_per_step: float, dist_mod=No
     return ms, tok, tok / (ms / 1e3)
 
 
+def cross_layer_overlap(ic, wl, layers, dims, rpc, stream, peaks, n):
+    """Untimed: every layer run as F with its index cache dumped, then the
+    top-k overlap of each adjacent pair on the device (ic_index_overlap).
+    Reports the statistic the pages quote for real models (adjacent layers
+    share 70-100% of their selections) for these synthetic inputs, over rows
+    with t >= k (earlier rows select every visible position), and the
+    overlap kernel's own rate."""
+    stack = ic.LayerStack("F" * n, layers, dims, dump_idx=True, rows_per_chunk=rpc)
+    stack.forward(stream)
+    torch.cuda.synchronize()
+    t = np.arange(wl.Lq) + wl.q_offset
+    keep = np.tile(t >= wl.k, wl.B)
+    ov, jac, times = [], [], []
+    counts = None
+    for l in range(n - 1):
+        a, b = stack.dumps[l], stack.dumps[l + 1]
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        counts = ic.index_overlap(a, b, wl.Lk, counts=counts, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+        c = counts.cpu().numpy().astype(np.float64)[keep]
+        if len(c):
+            ov.append(float(np.mean(c[:, 0] / wl.k)))
+            jac.append(float(np.mean(c[:, 0] / (c[:, 1] + c[:, 2] - c[:, 0] + 1e-8))))
+    if ic.get_last_device_error() != 0:
+        raise RuntimeError("device error in the overlap pass")
+    del stack
+    ms = float(np.median(times)) if times else 0.0
+    nbytes = 2 * 4.0 * wl.B * wl.Lq * wl.k + 12.0 * wl.B * wl.Lq
+    out = {"pairs": n - 1, "rows": "t >= k", "ms_per_launch": ms,
+           "gbs": nbytes / (ms * 1e-3) / 1e9 if ms > 0 else None}
+    if out["gbs"]:
+        out["frac_of_hbm"] = out["gbs"] / peaks["hbm_gbs"]
+    if ov:
+        out.update({"mean_overlap": float(np.mean(ov)), "min_pair_overlap": float(np.min(ov)),
+                    "mean_jaccard": float(np.mean(jac))})
+    return out
+
+
 def config_of(wl, pattern, args):
     return {"workload": wl.name, "B": wl.B, "L": wl.Lq, "Lk": wl.Lk, "q_offset": wl.q_offset,
             "layers": wl.n_layers, "pattern": pattern, "H_I": wl.H_I, "d_I": wl.d_I,
@@ -547,6 +588,8 @@ def main():
                          "value": vf,
                          "speedup_of_pattern": msf / ms_per_step}
         del stack_f
+        line["cross_layer_overlap"] = cross_layer_overlap(ic, wl, layers, dims, rpc, stream,
+                                                          peaks, n)
 
     # ---- end to end through the public API with host buffers
     if not args.no_e2e and pinned is None:

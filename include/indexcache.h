@@ -253,6 +253,22 @@ int ic_layer_stack_forward_events(const char *pattern, int n_layers, const ic_la
                                   size_t ws_bytes, ic_stream_t stream, void *const *events);
 
 /*
+ * Next step f2 -- cross-layer overlap of two layers' index sets (skill page,
+ * Step 1 "Analyze Index Correlation Across Layers": top-k sets of
+ * consecutive layers compared per query position; kualia.ai review: adjacent
+ * layers share 70-100% of their selected tokens).
+ *   idx_a, idx_b [n_rows, k] int32 (device; -1 = empty slot; every other
+ *   entry in [0, Lk))   counts [n_rows, 3] int32 (device, written)
+ * Row r gets counts[r] = { |A & B|, |A|, |B| } with each row read as the set
+ * of its valid entries (a position repeated in a row counts once); the
+ * overlap fraction is |A & B| / k and the Jaccard index |A & B| / |A | B|.
+ * Entries outside [-1, Lk) are skipped and flag IC_ERR_INVALID_ARG in the
+ * device error word.  Lk up to 262144.  Asynchronous on `stream`.
+ */
+int ic_index_overlap(const int32_t *idx_a, const int32_t *idx_b, long long n_rows, int k, int Lk,
+                     int32_t *counts, ic_stream_t stream);
+
+/*
  * Kernel launches this library has issued in this process so far (every
  * entry point, every device).  A host-side counter: reading it never
  * synchronises.  Callers take the difference around a region to count the

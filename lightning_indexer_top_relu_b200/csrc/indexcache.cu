@@ -18,6 +18,7 @@
 #include "indexcache.h"
 #include "common.cuh"
 #include "dense_attn.cuh"
+#include "index_overlap.cuh"
 #include "indexer_scores.cuh"
 #include "sparse_attn.cuh"
 #include "topk_select.cuh"
@@ -212,11 +213,12 @@ int launch_topk(const float* scores, long long ld, long long row_base, long long
     cudaError_t e;
     if (n_max <= ic::TK_CACHE_MAX) {
         const int smem = ic::TK_SMEM_FIXED + n_max * 4;
-        ic::topk_select_kernel<true><<<(unsigned)n_rows, ic::TK_THREADS, smem, st>>>(
+        ic::topk_select_kernel<ic::TK_THREADS, true><<<(unsigned)n_rows, ic::TK_THREADS, smem, st>>>(
             scores, ld, row_base, n_rows, Lq, Lk, q_offset, k, idx, mask, Lq_d, W);
     } else {
-        ic::topk_select_kernel<false><<<(unsigned)n_rows, ic::TK_THREADS, ic::TK_SMEM_FIXED, st>>>(
-            scores, ld, row_base, n_rows, Lq, Lk, q_offset, k, idx, mask, Lq_d, W);
+        ic::topk_select_kernel<ic::TK_THREADS_LONG, false>
+            <<<(unsigned)n_rows, ic::TK_THREADS_LONG, ic::TK_SMEM_FIXED, st>>>(
+                scores, ld, row_base, n_rows, Lq, Lk, q_offset, k, idx, mask, Lq_d, W);
     }
     e = cudaGetLastError();
     if (launched(e, "topk_select launch")) return IC_ERR_CUDA;
@@ -444,11 +446,13 @@ int device_setup(int* dev_out, int* sms_out) {
         set_indexer_attr<32, 64>();  set_indexer_attr<32, 128>();
         set_indexer_attr<64, 64>();  set_indexer_attr<64, 128>();
         set_indexer_attr<128, 64>(); set_indexer_attr<128, 128>();
-        cudaFuncSetAttribute(ic::topk_select_kernel<true>,
+        cudaFuncSetAttribute(ic::topk_select_kernel<ic::TK_THREADS, true>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              ic::TK_SMEM_FIXED + ic::TK_CACHE_MAX * 4);
         cudaFuncSetAttribute(ic::dense_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              ic::DenseSmem::ALLOC);
+        cudaFuncSetAttribute(ic::index_overlap_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             2 * (ic::OV_MAX_LK / 32) * 4);
         cudaFuncSetAttribute(ic::sparse_attn_kernel<64>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, ic::SaSmem<64>::BYTES);
         cudaFuncSetAttribute(ic::sparse_attn_kernel<128>,
@@ -697,6 +701,23 @@ int ic_sparse_attn_unique(const uint16_t* q, const uint16_t* k, const uint16_t* 
     const AttnMode mode = (dg.on && dg.total <= ws_bytes) ? ATTN_BUILD_MASK : ATTN_GATHER;
     return attn_step(D, L, idx, mode, false, ws, ws_bytes, sms,
                      reinterpret_cast<cudaStream_t>(stream), nullptr);
+}
+
+int ic_index_overlap(const int32_t* idx_a, const int32_t* idx_b, long long n_rows, int k, int Lk,
+                     int32_t* counts, ic_stream_t stream) {
+    if (n_rows < 0 || k < 1) return fail(IC_ERR_INVALID_ARG, "n_rows=%lld k=%d", n_rows, k);
+    if (Lk < 1 || Lk > ic::OV_MAX_LK)
+        return fail(IC_ERR_UNSUPPORTED, "Lk=%d (supported: 1..%d)", Lk, ic::OV_MAX_LK);
+    if (n_rows == 0) return IC_OK;
+    if (!idx_a || !idx_b || !counts) return fail(IC_ERR_INVALID_ARG, "null pointer");
+    int dev, sms;
+    int rc = device_setup(&dev, &sms);
+    if (rc) return rc;
+    const int W = (Lk + 31) / 32;
+    const int grid = (int)std::min<long long>(n_rows, (long long)sms * 8);
+    ic::index_overlap_kernel<<<grid, ic::OV_THREADS, 2 * W * 4, reinterpret_cast<cudaStream_t>(stream)>>>(
+        idx_a, idx_b, n_rows, k, Lk, counts);
+    return launched(cudaGetLastError(), "index_overlap launch");
 }
 
 size_t ic_layer_stack_workspace_bytes(const ic_dims* dims, int n_layers, long long rows_per_chunk) {

@@ -31,11 +31,14 @@
 
 namespace ic {
 
+// Threads per row.  Rows longer than TK_CACHE_MAX re-read their scores from
+// L2/HBM; measured at L=65536, eight 256-thread CTAs per SM beat 2 x 512 and
+// 1 x 1024 threads (more rows in flight outweigh keeping them in L2).
 constexpr int TK_THREADS = 256;
-constexpr int TK_WARPS = TK_THREADS / 32;
+constexpr int TK_THREADS_LONG = 256;
 constexpr int TK_BINS = 2048;
 constexpr int TK_CAND = 2048;                                     // candidate keys kept in smem
-constexpr int TK_SMEM_FIXED = TK_BINS * 4 + TK_CAND * 4 + 256;    // hist + candidates + scratch
+constexpr int TK_SMEM_FIXED = TK_BINS * 4 + TK_CAND * 4 + 512;    // hist + candidates + scratch
 constexpr int TK_CACHE_MAX = 45056;                               // longest row kept in smem
 constexpr int TK_VB = 8;                                          // float4 loads in flight per thread
 
@@ -48,9 +51,10 @@ __device__ __forceinline__ uint32_t score_key(float f) {
 // Suffix scan of the 2048-bin histogram: finds the bin b whose count makes
 // the running total (from the top bin down) reach `remaining`.  Writes
 // found[0] = b, found[1] = count of elements in bins above b.  All threads.
+template <int NT>
 __device__ __forceinline__ void tk_find_bin(const uint32_t* hist, int remaining, int* found,
                                             unsigned* wsum) {
-    constexpr int PER = TK_BINS / TK_THREADS;      // 8 bins per thread, top bins first
+    constexpr int PER = TK_BINS / NT;              // bins per thread, top bins first
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int hi = TK_BINS - 1 - PER * tid;
     uint32_t h[PER];
@@ -70,7 +74,7 @@ __device__ __forceinline__ void tk_find_bin(const uint32_t* hist, int remaining,
     __syncthreads();
     uint32_t before = 0;
 #pragma unroll
-    for (int w = 0; w < TK_WARPS; ++w) before += (w < warp) ? wsum[w] : 0u;
+    for (int w = 0; w < NT / 32; ++w) before += (w < warp) ? wsum[w] : 0u;
     uint32_t above = before + x - mine;
 #pragma unroll
     for (int e = 0; e < PER; ++e) {
@@ -89,18 +93,20 @@ __device__ __forceinline__ void tk_find_bin(const uint32_t* hist, int remaining,
 // selection as a bitmask: row b*Lq_d + i of `mask` ([*, W] words) gets bit s
 // set for every selected position s (words past the row's visible positions
 // are zero).  The emit pass builds it from the ballots it already takes.
-template <bool CACHE>
-__global__ void __launch_bounds__(TK_THREADS)
+template <int NT, bool CACHE>
+__global__ void __launch_bounds__(NT)
 topk_select_kernel(const float* __restrict__ scores, long long ld, long long row_base,
                    long long n_rows, int Lq, int Lk, int q_offset, int k,
                    int32_t* __restrict__ idx, uint32_t* __restrict__ mask, int Lq_d, int W) {
+    constexpr int NW = NT / 32;
+    static_assert(4 + 3 * NW <= 128, "scratch words");
     extern __shared__ __align__(16) uint8_t tk_smem[];
     uint32_t* hist = reinterpret_cast<uint32_t*>(tk_smem);
     uint32_t* cand = reinterpret_cast<uint32_t*>(tk_smem + TK_BINS * 4);
     int* found = reinterpret_cast<int*>(tk_smem + TK_BINS * 4 + TK_CAND * 4);      // [0..3]
-    unsigned* wsum = reinterpret_cast<unsigned*>(found + 4);                        // [TK_WARPS]
-    unsigned* wgt = wsum + TK_WARPS;                                                // [TK_WARPS]
-    unsigned* weq = wgt + TK_WARPS;                                                 // [TK_WARPS]
+    unsigned* wsum = reinterpret_cast<unsigned*>(found + 4);                        // [NW]
+    unsigned* wgt = wsum + NW;                                                // [NW]
+    unsigned* weq = wgt + NW;                                                 // [NW]
     uint32_t* keys = reinterpret_cast<uint32_t*>(tk_smem + TK_SMEM_FIXED);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -114,12 +120,12 @@ topk_select_kernel(const float* __restrict__ scores, long long ld, long long row
         mrow = mask + ((r / Lq) * Lq_d + r % Lq) * (long long)W;
     const int nw = (n + 31) >> 5;                                 // words with visible positions
     if (mrow != nullptr)
-        for (int w = nw + tid; w < W; w += TK_THREADS) mrow[w] = 0u;
+        for (int w = nw + tid; w < W; w += NT) mrow[w] = 0u;
 
     if (n <= k) {
-        for (int i = tid; i < k; i += TK_THREADS) out[i] = i < n ? i : -1;
+        for (int i = tid; i < k; i += NT) out[i] = i < n ? i : -1;
         if (mrow != nullptr)
-            for (int w = tid; w < nw && w < W; w += TK_THREADS)
+            for (int w = tid; w < nw && w < W; w += NT)
                 mrow[w] = (32 * w + 32 <= n) ? 0xffffffffu : ((1u << (n - 32 * w)) - 1u);
         return;
     }
@@ -127,22 +133,22 @@ topk_select_kernel(const float* __restrict__ scores, long long ld, long long row
     auto key_at = [&](int i) -> uint32_t { return CACHE ? keys[i] : score_key(__ldg(src + i)); };
 
     // ---- 1. keys + top-11-bit histogram in one pass
-    for (int b = tid; b < TK_BINS; b += TK_THREADS) hist[b] = 0;
+    for (int b = tid; b < TK_BINS; b += NT) hist[b] = 0;
     if (tid == 0) found[2] = 0;                                // candidate count
     __syncthreads();
     const bool vec = ((reinterpret_cast<uintptr_t>(src) & 15) == 0);
     const int nv = vec ? (n & ~3) : 0;
-    for (int base = 0; base < nv; base += TK_THREADS * 4 * TK_VB) {
+    for (int base = 0; base < nv; base += NT * 4 * TK_VB) {
         float4 f[TK_VB];
 #pragma unroll
         for (int u = 0; u < TK_VB; ++u) {           // all loads of the batch first
-            const int i = base + (u * TK_THREADS + tid) * 4;
+            const int i = base + (u * NT + tid) * 4;
             f[u] = i < nv ? __ldg(reinterpret_cast<const float4*>(src + i))
                           : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
         for (int u = 0; u < TK_VB; ++u) {
-            const int i = base + (u * TK_THREADS + tid) * 4;
+            const int i = base + (u * NT + tid) * 4;
             if (i < nv) {
                 const uint32_t k0 = score_key(f[u].x), k1 = score_key(f[u].y),
                                k2 = score_key(f[u].z), k3 = score_key(f[u].w);
@@ -154,14 +160,14 @@ topk_select_kernel(const float* __restrict__ scores, long long ld, long long row
             }
         }
     }
-    for (int i = nv + tid; i < n; i += TK_THREADS) {
+    for (int i = nv + tid; i < n; i += NT) {
         const uint32_t kk = score_key(__ldg(src + i));
         if (CACHE) keys[i] = kk;
         atomicAdd(&hist[kk >> 21], 1u);
     }
     __syncthreads();
 
-    tk_find_bin(hist, k, found, wsum);
+    tk_find_bin<NT>(hist, k, found, wsum);
     const uint32_t b1 = (uint32_t)found[0];
     int remaining = k - found[1];
     const uint32_t cnt1 = hist[b1];
@@ -172,7 +178,7 @@ topk_select_kernel(const float* __restrict__ scores, long long ld, long long row
     uint32_t pmask = 0x7FFu << 21;
     const bool use_cand = cnt1 <= (uint32_t)TK_CAND;
     if (use_cand) {
-        for (int gbase = warp * 32 * TK_VB; gbase < n; gbase += TK_THREADS * TK_VB) {
+        for (int gbase = warp * 32 * TK_VB; gbase < n; gbase += NT * TK_VB) {
             uint32_t kb[TK_VB];
 #pragma unroll
             for (int u = 0; u < TK_VB; ++u) {
@@ -196,31 +202,31 @@ topk_select_kernel(const float* __restrict__ scores, long long ld, long long row
     for (int pass = 1; pass < 3; ++pass) {
         const int shift = pass == 1 ? 10 : 0;
         const uint32_t dmask = pass == 1 ? 0x7FFu : 0x3FFu;
-        for (int b = tid; b < TK_BINS; b += TK_THREADS) hist[b] = 0;
+        for (int b = tid; b < TK_BINS; b += NT) hist[b] = 0;
         __syncthreads();
         if (use_cand) {
-            for (int i = tid; i < (int)cnt1; i += TK_THREADS) {
+            for (int i = tid; i < (int)cnt1; i += NT) {
                 const uint32_t kk = cand[i];
                 if ((kk & pmask) == prefix) atomicAdd(&hist[(kk >> shift) & dmask], 1u);
             }
         } else {
-            for (int base = 0; base < n; base += TK_THREADS * TK_VB) {
+            for (int base = 0; base < n; base += NT * TK_VB) {
                 uint32_t kb[TK_VB];
 #pragma unroll
                 for (int u = 0; u < TK_VB; ++u) {
-                    const int i = base + u * TK_THREADS + tid;
+                    const int i = base + u * NT + tid;
                     kb[u] = i < n ? key_at(i) : 0u;
                 }
 #pragma unroll
                 for (int u = 0; u < TK_VB; ++u) {
-                    const int i = base + u * TK_THREADS + tid;
+                    const int i = base + u * NT + tid;
                     if (i < n && (kb[u] & pmask) == prefix)
                         atomicAdd(&hist[(kb[u] >> shift) & dmask], 1u);
                 }
             }
         }
         __syncthreads();
-        tk_find_bin(hist, remaining, found, wsum);
+        tk_find_bin<NT>(hist, remaining, found, wsum);
         remaining -= found[1];
         prefix |= (uint32_t)found[0] << shift;
         pmask |= dmask << shift;
@@ -230,7 +236,7 @@ topk_select_kernel(const float* __restrict__ scores, long long ld, long long row
     const int need = remaining;   // keys equal to T that are kept, lowest positions first
 
     // ---- 3. emit in position order: warp w owns [w*seg, (w+1)*seg)
-    const int seg = ((n + TK_WARPS * 32 - 1) / (TK_WARPS * 32)) * 32;
+    const int seg = ((n + NW * 32 - 1) / (NW * 32)) * 32;
     const int s0 = min(n, warp * seg), s1 = min(n, s0 + seg);
     unsigned cg = 0, ce = 0;
     for (int gbase = s0; gbase < s1; gbase += 32 * TK_VB) {
@@ -254,7 +260,7 @@ topk_select_kernel(const float* __restrict__ scores, long long ld, long long row
     __syncthreads();
     unsigned g = 0, e = 0;
 #pragma unroll
-    for (int w = 0; w < TK_WARPS; ++w) {
+    for (int w = 0; w < NW; ++w) {
         g += (w < warp) ? wgt[w] : 0u;
         e += (w < warp) ? weq[w] : 0u;
     }

@@ -34,7 +34,7 @@ EXPORTS = ("ic_status_string", "ic_last_error_message", "ic_get_last_device_erro
            "ic_sparse_attn_workspace_bytes", "ic_layer_stack_workspace_bytes",
            "ic_layer_stack_forward", "ic_layer_stack_forward_events", "ic_selftest_wait_timeout",
            "ic_sparse_attn_no_alloc", "ic_kernel_launch_count", "ic_sparse_attn_unique",
-           "ic_sparse_attn_unique_workspace_bytes")
+           "ic_sparse_attn_unique_workspace_bytes", "ic_index_overlap")
 
 MARKS_PER_LAYER = 5        # IC_MARKS_PER_LAYER
 
@@ -94,6 +94,8 @@ _lib.ic_selftest_wait_timeout.argtypes = [_I, _P]
 _lib.ic_layer_stack_forward_events.restype = _I
 _lib.ic_layer_stack_forward_events.argtypes = [ctypes.c_char_p, _I, ctypes.POINTER(ICLayer),
                                                ctypes.POINTER(ICDims), _P, _P, _Z, _P, _P]
+_lib.ic_index_overlap.restype = _I
+_lib.ic_index_overlap.argtypes = [_P, _P, ctypes.c_longlong, _I, _I, _P, _P]
 _lib.ic_kernel_launch_count.restype = ctypes.c_ulonglong
 _lib.ic_kernel_launch_count.argtypes = []
 _lib.ic_layer_stack_forward.restype = _I
@@ -133,6 +135,22 @@ def _stream(stream) -> Optional[int]:
 def get_last_device_error(stream=None) -> int:
     """Synchronises the stream and returns (and clears) the device error status."""
     return int(_lib.ic_get_last_device_error(_stream(stream)))
+
+
+def index_overlap(idx_a, idx_b, Lk: int, counts=None, stream=None):
+    """Per-row (|A & B|, |A|, |B|) of two [..., k] int32 index tensors on the
+    device, as int32 [n_rows, 3] (ic_index_overlap)."""
+    if idx_a.shape != idx_b.shape:
+        raise ValueError("index tensors differ in shape")
+    k = idx_a.shape[-1]
+    n_rows = idx_a.numel() // k
+    if counts is None:
+        counts = torch.empty(n_rows, 3, device=idx_a.device, dtype=torch.int32)
+    rc = _lib.ic_index_overlap(_ptr(idx_a, torch.int32, "idx_a"), _ptr(idx_b, torch.int32, "idx_b"),
+                               n_rows, k, int(Lk), _ptr(counts, torch.int32, "counts"),
+                               _stream(stream))
+    _check(rc, "ic_index_overlap")
+    return counts
 
 
 def kernel_launch_count() -> int:

@@ -131,3 +131,15 @@ def test_marks_per_layer_matches_header(ic):
     text = open(HEADER).read()
     m = re.search(r"#define\s+IC_MARKS_PER_LAYER\s+(\d+)", text)
     assert m and int(m.group(1)) == ic.MARKS_PER_LAYER
+
+
+def test_index_overlap_rejects_bad_sizes_before_launch(ic):
+    lib = ic.lib()
+    before = ic.kernel_launch_count()
+    assert lib.ic_index_overlap(0x1000, 0x1000, 4, 0, 100, 0x2000, None) == 1     # k = 0
+    assert lib.ic_index_overlap(0x1000, 0x1000, -1, 8, 100, 0x2000, None) == 1    # n_rows < 0
+    assert lib.ic_index_overlap(0x1000, 0x1000, 4, 8, 0, 0x2000, None) == 2       # Lk = 0
+    assert lib.ic_index_overlap(0x1000, 0x1000, 4, 8, 1 << 19, 0x2000, None) == 2 # Lk too large
+    assert lib.ic_index_overlap(None, 0x1000, 4, 8, 100, 0x2000, None) == 1       # null
+    assert lib.ic_index_overlap(None, None, 0, 8, 100, None, None) == 0           # nothing to do
+    assert ic.kernel_launch_count() == before
