@@ -144,9 +144,9 @@ size_t ic_sparse_attn_workspace_bytes(int B, int Lq, int Hq, int d, int k_slots)
  * partial results in a fixed 4 MiB array inside the library instead of a
  * workspace; every GPU that loads the library holds that array until the
  * process exits.
- *   - A call whose partial results would exceed 4 MiB (rows x splits x Hq x
- *     (d + 1) x 4 bytes) is rejected with IC_ERR_WORKSPACE_TOO_SMALL before
- *     anything is launched; ic_sparse_attn with a workspace handles it.
+ *   - A call whose preferred split would need more than 4 MiB of partials
+ *     (rows x splits x Hq x (d + 1) x 4 bytes) runs with fewer splits (one
+ *     split needs none), so every valid call runs; results are the same.
  *   - The first call on a device looks up the array's device address (once per
  *     device, with that device current); make that first call before any
  *     stream capture.

@@ -7,9 +7,11 @@
 // (-1 = empty slot, a repeated position counts once), from which the overlap
 // fraction |A & B| / k and the Jaccard index |A & B| / |A | B| follow.
 //
-// One CTA per row (grid-stride): both rows become bitmaps over [0, Lk) in
-// shared memory (one atomicOr per slot), then one pass of popcounts over the
-// words counts |A|, |B| and |A & B|.  Bound: HBM, 8 bytes read per slot pair.
+// Both rows become bitmaps over [0, Lk) in shared memory (one atomicOr per
+// slot), then one pass of popcounts over the words counts |A|, |B| and
+// |A & B|.  Up to OV_WARP_MAX_LK positions one warp handles a row (its two
+// bitmaps in its own slice of shared memory, so a CTA has 8 rows in flight);
+// longer rows take a whole CTA each.  Bound: HBM, 8 bytes read per slot pair.
 #pragma once
 
 #include "common.cuh"
@@ -18,6 +20,64 @@ namespace ic {
 
 constexpr int OV_THREADS = 256;
 constexpr int OV_MAX_LK = 262144;                  // two bitmaps of 32 KB
+constexpr int OV_WARP_MAX_LK = 16384;              // per-warp bitmaps: 2 x 2 KB
+constexpr int OV_VB = 8;                           // loads in flight per lane
+
+// One warp per row (grid-stride over rows, 8 warps per CTA).
+__global__ void __launch_bounds__(OV_THREADS)
+index_overlap_warp_kernel(const int32_t* __restrict__ a, const int32_t* __restrict__ b,
+                          long long n_rows, int k, int Lk, int32_t* __restrict__ counts) {
+    extern __shared__ uint32_t ovw_smem[];
+    const int W = (Lk + 31) >> 5;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t* bm_a = ovw_smem + warp * 2 * W;
+    uint32_t* bm_b = bm_a + W;
+    for (long long r = (long long)blockIdx.x * (OV_THREADS / 32) + warp; r < n_rows;
+         r += (long long)gridDim.x * (OV_THREADS / 32)) {
+        for (int w = lane; w < 2 * W; w += 32) bm_a[w] = 0u;
+        __syncwarp();
+        const int32_t* ra = a + r * (long long)k;
+        const int32_t* rb = b + r * (long long)k;
+        for (int s0 = 0; s0 < k; s0 += 32 * OV_VB) {
+            int x[OV_VB], y[OV_VB];
+#pragma unroll
+            for (int u = 0; u < OV_VB; ++u) {          // the whole batch in flight first
+                const int s = s0 + u * 32 + lane;
+                x[u] = s < k ? __ldg(ra + s) : -1;
+                y[u] = s < k ? __ldg(rb + s) : -1;
+            }
+#pragma unroll
+            for (int u = 0; u < OV_VB; ++u) {
+                if (x[u] >= 0 && x[u] < Lk) atomicOr(&bm_a[x[u] >> 5], 1u << (x[u] & 31));
+                else if (x[u] != -1) report(DEV_ERR_BAD_INDEX);
+                if (y[u] >= 0 && y[u] < Lk) atomicOr(&bm_b[y[u] >> 5], 1u << (y[u] & 31));
+                else if (y[u] != -1) report(DEV_ERR_BAD_INDEX);
+            }
+        }
+        __syncwarp();
+        int both = 0, na = 0, nb = 0;
+        for (int w = lane; w < W; w += 32) {
+            const uint32_t u = bm_a[w], v = bm_b[w];
+            na += __popc(u);
+            nb += __popc(v);
+            both += __popc(u & v);
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            both += __shfl_xor_sync(0xffffffffu, both, o);
+            na += __shfl_xor_sync(0xffffffffu, na, o);
+            nb += __shfl_xor_sync(0xffffffffu, nb, o);
+        }
+        if (lane == 0) {
+            counts[3 * r] = both;
+            counts[3 * r + 1] = na;
+            counts[3 * r + 2] = nb;
+        }
+        __syncwarp();
+    }
+}
+
+// One CTA per row (grid-stride), for rows over more than OV_WARP_MAX_LK positions.
 
 __global__ void __launch_bounds__(OV_THREADS)
 index_overlap_kernel(const int32_t* __restrict__ a, const int32_t* __restrict__ b,

@@ -206,12 +206,23 @@ int launch_indexer(const uint16_t* q_idx, const uint16_t* k_idx, const float* w,
 // ---------------------------------------------------------------- top-k
 
 int launch_topk(const float* scores, long long ld, long long row_base, long long n_rows, int Lq,
-                int Lk, int q_offset, int k, int32_t* idx, cudaStream_t st,
+                int Lk, int q_offset, int k, int32_t* idx, int sms, cudaStream_t st,
                 uint32_t* mask = nullptr, int Lq_d = 0, int W = 0) {
     if (n_rows <= 0) return IC_OK;
     const int n_max = std::min(Lk, q_offset + Lq);
     cudaError_t e;
-    if (n_max <= ic::TK_CACHE_MAX) {
+    if (n_rows < 2LL * sms && n_max > 4096) {
+        // few long rows (decode): a 1024-thread CTA per row, one per SM
+        if (n_max <= ic::TK_CACHE_MAX) {
+            ic::topk_select_kernel<ic::TK_THREADS_FEW, true>
+                <<<(unsigned)n_rows, ic::TK_THREADS_FEW, ic::TK_SMEM_FIXED + n_max * 4, st>>>(
+                    scores, ld, row_base, n_rows, Lq, Lk, q_offset, k, idx, mask, Lq_d, W);
+        } else {
+            ic::topk_select_kernel<ic::TK_THREADS_FEW, false>
+                <<<(unsigned)n_rows, ic::TK_THREADS_FEW, ic::TK_SMEM_FIXED, st>>>(
+                    scores, ld, row_base, n_rows, Lq, Lk, q_offset, k, idx, mask, Lq_d, W);
+        }
+    } else if (n_max <= ic::TK_CACHE_MAX) {
         const int smem = ic::TK_SMEM_FIXED + n_max * 4;
         ic::topk_select_kernel<ic::TK_THREADS, true><<<(unsigned)n_rows, ic::TK_THREADS, smem, st>>>(
             scores, ld, row_base, n_rows, Lq, Lk, q_offset, k, idx, mask, Lq_d, W);
@@ -228,8 +239,9 @@ int launch_topk(const float* scores, long long ld, long long row_base, long long
 // ---------------------------------------------------------------- sparse attention
 
 int attn_splits(long long n_rows, int k_slots, int sms) {
+    // rows x splits CTAs fill the 2 CTAs per SM that fit, in one wave
     if (n_rows >= 2LL * sms) return 1;
-    long long s = (2LL * sms + n_rows - 1) / n_rows;
+    long long s = (2LL * sms) / n_rows;
     s = std::min<long long>(s, (k_slots + ic::SA_WARPS * ic::SA_BLOCK - 1) / (ic::SA_WARPS * ic::SA_BLOCK));
     s = std::min<long long>(s, 64);
     return (int)std::max<long long>(1, s);
@@ -284,10 +296,11 @@ int launch_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, const i
     cudaError_t e = cudaGetLastError();
     if (launched(e, "sparse_attn launch")) return IC_ERR_CUDA;
     if (splits > 1) {
+        const dim3 cg((unsigned)n_rows, (unsigned)Hq);
         if (d == 64)
-            ic::sparse_attn_combine_kernel<64><<<(unsigned)n_rows, 256, 0, st>>>(a);
+            ic::sparse_attn_combine_kernel<64><<<cg, 64, 0, st>>>(a);
         else
-            ic::sparse_attn_combine_kernel<128><<<(unsigned)n_rows, 256, 0, st>>>(a);
+            ic::sparse_attn_combine_kernel<128><<<cg, 128, 0, st>>>(a);
         e = cudaGetLastError();
         if (launched(e, "sparse_attn combine launch")) return IC_ERR_CUDA;
     }
@@ -446,6 +459,9 @@ int device_setup(int* dev_out, int* sms_out) {
         set_indexer_attr<32, 64>();  set_indexer_attr<32, 128>();
         set_indexer_attr<64, 64>();  set_indexer_attr<64, 128>();
         set_indexer_attr<128, 64>(); set_indexer_attr<128, 128>();
+        cudaFuncSetAttribute(ic::topk_select_kernel<ic::TK_THREADS_FEW, true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             ic::TK_SMEM_FIXED + ic::TK_CACHE_MAX * 4);
         cudaFuncSetAttribute(ic::topk_select_kernel<ic::TK_THREADS, true>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              ic::TK_SMEM_FIXED + ic::TK_CACHE_MAX * 4);
@@ -453,6 +469,9 @@ int device_setup(int* dev_out, int* sms_out) {
                              ic::DenseSmem::ALLOC);
         cudaFuncSetAttribute(ic::index_overlap_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              2 * (ic::OV_MAX_LK / 32) * 4);
+        cudaFuncSetAttribute(ic::index_overlap_warp_kernel,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (ic::OV_THREADS / 32) * 2 * (ic::OV_WARP_MAX_LK / 32) * 4);
         cudaFuncSetAttribute(ic::sparse_attn_kernel<64>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, ic::SaSmem<64>::BYTES);
         cudaFuncSetAttribute(ic::sparse_attn_kernel<128>,
@@ -604,7 +623,7 @@ int ic_topk_select(const float* scores, int B, int Lq, int Lk, int q_offset, int
     if (!scores || !idx) return fail(IC_ERR_INVALID_ARG, "null pointer");
     int dev, sms;
     if ((rc = device_setup(&dev, &sms))) return rc;
-    return launch_topk(scores, Lk, 0, (long long)B * Lq, Lq, Lk, q_offset, k, idx,
+    return launch_topk(scores, Lk, 0, (long long)B * Lq, Lq, Lk, q_offset, k, idx, sms,
                        reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -650,16 +669,10 @@ int ic_sparse_attn_no_alloc(const uint16_t* q, const uint16_t* k, const uint16_t
     if (!std::isfinite(scale)) return fail(IC_ERR_INVALID_ARG, "scale is not finite");
     int dev, sms;
     if ((rc = device_setup(&dev, &sms))) return rc;
-    const long long n_rows = (long long)B * Lq;
-    const int splits = attn_splits(n_rows, k_slots, sms);
-    const size_t need = attn_ws_bytes(n_rows, splits, Hq, d);
-    if (need > NOALLOC_SCRATCH_BYTES)
-        return fail(IC_ERR_WORKSPACE_TOO_SMALL,
-                    "%lld rows x %d slot splits need %zu bytes of scratch; the built-in scratch "
-                    "holds %zu bytes (call ic_sparse_attn with a workspace instead)",
-                    n_rows, splits, need, NOALLOC_SCRATCH_BYTES);
     void* scratch = nullptr;
     if ((rc = noalloc_scratch(dev, &scratch))) return rc;
+    // launch_attn halves the slot split until its partials fit the scratch
+    // (one split needs none), so every valid call runs.
     return launch_attn(q, k, v, idx, B, Lq, Lk, Hq, d, k_slots, q_offset, scale, out, lse, scratch,
                        NOALLOC_SCRATCH_BYTES, false, sms, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -714,9 +727,17 @@ int ic_index_overlap(const int32_t* idx_a, const int32_t* idx_b, long long n_row
     int rc = device_setup(&dev, &sms);
     if (rc) return rc;
     const int W = (Lk + 31) / 32;
-    const int grid = (int)std::min<long long>(n_rows, (long long)sms * 8);
-    ic::index_overlap_kernel<<<grid, ic::OV_THREADS, 2 * W * 4, reinterpret_cast<cudaStream_t>(stream)>>>(
-        idx_a, idx_b, n_rows, k, Lk, counts);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (Lk <= ic::OV_WARP_MAX_LK) {
+        const long long per_cta = ic::OV_THREADS / 32;
+        const int grid = (int)std::min<long long>((n_rows + per_cta - 1) / per_cta, (long long)sms * 8);
+        ic::index_overlap_warp_kernel<<<grid, ic::OV_THREADS, per_cta * 2 * W * 4, st>>>(
+            idx_a, idx_b, n_rows, k, Lk, counts);
+    } else {
+        const int grid = (int)std::min<long long>(n_rows, (long long)sms * 8);
+        ic::index_overlap_kernel<<<grid, ic::OV_THREADS, 2 * W * 4, st>>>(idx_a, idx_b, n_rows, k,
+                                                                          Lk, counts);
+    }
     return launched(cudaGetLastError(), "index_overlap launch");
 }
 
@@ -823,8 +844,8 @@ static int stack_forward(const char* pattern, int n_layers, const ic_layer* laye
                 if (one_chunk && (rc = mark(l, 1))) return rc;
                 const long long r0 = block_row_start(geo, D.Lq, g0);
                 const long long r1 = block_row_start(geo, D.Lq, g1);
-                rc = launch_topk(sc, D.Lk, r0, r1 - r0, D.Lq, D.Lk, D.q_offset, D.k, idx_cache, st,
-                                 dmask, dg.Lq_d, dg.W);
+                rc = launch_topk(sc, D.Lk, r0, r1 - r0, D.Lq, D.Lk, D.q_offset, D.k, idx_cache, sms,
+                                 st, dmask, dg.Lq_d, dg.W);
                 if (rc) return rc;
             }
         }

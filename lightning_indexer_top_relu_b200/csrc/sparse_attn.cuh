@@ -369,27 +369,42 @@ sparse_attn_kernel(const SparseAttnArgs a) {
 }
 
 // Merges the per-split partial results of each row (log2-sum-exp weights).
+// One CTA per (row, head), one thread per output column: the split weights
+// are computed once per head in shared memory.
 template <int D>
-__global__ void sparse_attn_combine_kernel(const SparseAttnArgs a) {
+__global__ void __launch_bounds__(D)
+sparse_attn_combine_kernel(const SparseAttnArgs a) {
+    __shared__ float wgt[64];
+    __shared__ float mw[2];
     const long long pidx = blockIdx.x;
+    const int h = blockIdx.y, dcol = threadIdx.x;
     const long long row = sa_row(a, pidx);
-    for (int e = threadIdx.x; e < a.Hq * D; e += blockDim.x) {
-        const int h = e / D, dcol = e % D;
+    const long long base = pidx * a.splits * a.Hq + h;               // split s at base + s*Hq
+    if (threadIdx.x < 32) {
         float M = -INFINITY;
-        for (int s = 0; s < a.splits; ++s)
-            M = fmaxf(M, a.part_lse[(pidx * a.splits + s) * a.Hq + h]);
-        float W = 0.0f, acc = 0.0f;
-        if (M != -INFINITY) {
-            for (int s = 0; s < a.splits; ++s) {
-                const long long pr = (pidx * a.splits + s) * a.Hq + h;
-                const float f = exp2f(a.part_lse[pr] - M);
-                W += f;
-                acc += f * a.part_o[pr * D + dcol];
-            }
+        for (int s = threadIdx.x; s < a.splits; s += 32) M = fmaxf(M, a.part_lse[base + (long long)s * a.Hq]);
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        float W = 0.0f;
+        for (int s = threadIdx.x; s < a.splits; s += 32) {
+            const float f = M == -INFINITY ? 0.0f : exp2f(a.part_lse[base + (long long)s * a.Hq] - M);
+            wgt[s] = f;
+            W += f;
         }
-        a.out[(row * a.Hq + h) * D + dcol] = __float2bfloat16_rn(W > 0.0f ? acc / W : 0.0f);
-        if (a.lse && dcol == 0) a.lse[row * a.Hq + h] = W > 0.0f ? (M + log2f(W)) * LN2 : -INFINITY;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) W += __shfl_xor_sync(0xffffffffu, W, o);
+        if (threadIdx.x == 0) {
+            mw[0] = M;
+            mw[1] = W;
+        }
     }
+    __syncthreads();
+    const float M = mw[0], W = mw[1];
+    float acc = 0.0f;
+    for (int s = 0; s < a.splits; ++s)
+        acc += wgt[s] * a.part_o[(base + (long long)s * a.Hq) * D + dcol];
+    a.out[(row * a.Hq + h) * D + dcol] = __float2bfloat16_rn(W > 0.0f ? acc / W : 0.0f);
+    if (a.lse && dcol == 0) a.lse[row * a.Hq + h] = W > 0.0f ? (M + log2f(W)) * LN2 : -INFINITY;
 }
 
 }  // namespace ic

@@ -36,6 +36,7 @@ namespace ic {
 // 1 x 1024 threads (more rows in flight outweigh keeping them in L2).
 constexpr int TK_THREADS = 256;
 constexpr int TK_THREADS_LONG = 256;
+constexpr int TK_THREADS_FEW = 1024;     // fewer rows than 2 x SMs (decode): more threads per row
 constexpr int TK_BINS = 2048;
 constexpr int TK_CAND = 2048;                                     // candidate keys kept in smem
 constexpr int TK_SMEM_FIXED = TK_BINS * 4 + TK_CAND * 4 + 512;    // hist + candidates + scratch
