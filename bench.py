@@ -60,18 +60,19 @@ def load_peaks():
 
 # ---------------------------------------------------------------- algorithmic work
 
-DENSE_FACTOR = 4          # rows with t < 4k attend tile-dense (the library's dispatch rule)
+DENSE_FACTOR = 8          # rows with t < 8k attend tile-dense (the library's dispatch rule)
+DENSE_MAX_KEYS = 65536    # ... and see at most this many keys
 DA_TILE = 64              # keys per tile of the dense-masked kernel
 SFU_PER_CLK_SM = 16       # ex2 results per clock per SM (CUDA arithmetic-throughput table)
 
 
 def dense_rows(wl):
     """Rows per sequence that the layer stack sends to the dense-masked kernel
-    (t < 4k, whole blocks of 128/Hq queries), and that block size."""
+    (t < 8k, whole blocks of 128/Hq queries), and that block size."""
     if wl.d != 128 or 128 % wl.Hq:
         return 0, 0
     qbd = 128 // wl.Hq
-    lim = min(DENSE_FACTOR * wl.k - wl.q_offset, wl.Lq)
+    lim = min(DENSE_FACTOR * wl.k - wl.q_offset, DENSE_MAX_KEYS - wl.q_offset, wl.Lq)
     return (lim // qbd * qbd if lim >= qbd else 0), qbd
 
 
@@ -510,7 +511,7 @@ def main():
             ent["gbs"] = w["topk_bytes"] / sec / 1e9
             ent["frac_of_hbm"] = ent["gbs"] / peaks["hbm_gbs"]
         elif name == "attn_dense":
-            ent["covers"] = "V transpose + dense-masked tcgen05 attention, rows t < 4k"
+            ent["covers"] = "V transpose + dense-masked tcgen05 attention, rows t < 8k"
             ent["rows"] = int(w["dense_rows"])
             ent["tflops"] = w["dense_flops"] / sec / 1e12
             ent["frac_of_bf16_peak"] = ent["tflops"] / peaks["bf16_tflops"]
@@ -520,7 +521,7 @@ def main():
             ent["exp2_per_s"] = w["dense_exec_exps"] / sec
             ent["frac_of_sfu_peak"] = ent["exp2_per_s"] / sfu_peak
         else:
-            ent["covers"] = "gather attention (+ split combine), rows t >= 4k"
+            ent["covers"] = "gather attention (+ split combine), rows t >= 8k"
             ent["rows"] = int(w["gather_rows"])
             ent["tflops"] = w["gather_flops"] / sec / 1e12
             ent["logical_gbs"] = w["gather_bytes"] / sec / 1e9

@@ -4,7 +4,7 @@
 // The result is the same softmax over the selected positions as the gather
 // kernel (sparse_attn.cuh): a row's selection becomes a bitmask, and every
 // position outside it gets probability exactly 0.  When a row keeps k of
-// t+1 <= ~4k visible positions, sharing each K/V tile between the 8 queries
+// t+1 <= ~8k visible positions, sharing each K/V tile between the 8 queries
 // x 16 heads of a block and running the contractions on tcgen05 moves far
 // fewer bytes and runs far more flops per byte than gathering k rows per
 // query (IndexCache: every layer attends over the k cached positions; MQA).

@@ -39,7 +39,8 @@ constexpr int TK_THREADS_LONG = 256;
 constexpr int TK_THREADS_FEW = 1024;     // fewer rows than 2 x SMs (decode): more threads per row
 constexpr int TK_BINS = 2048;
 constexpr int TK_CAND = 2048;                                     // candidate keys kept in smem
-constexpr int TK_SMEM_FIXED = TK_BINS * 4 + TK_CAND * 4 + 512;    // hist + candidates + scratch
+// hist + candidate keys + candidate warp ids + scratch
+constexpr int TK_SMEM_FIXED = TK_BINS * 4 + TK_CAND * 4 + TK_CAND + 1024;
 constexpr int TK_CACHE_MAX = 45056;                               // longest row kept in smem
 constexpr int TK_VB = 8;                                          // float4 loads in flight per thread
 
@@ -100,14 +101,18 @@ topk_select_kernel(const float* __restrict__ scores, long long ld, long long row
                    long long n_rows, int Lq, int Lk, int q_offset, int k,
                    int32_t* __restrict__ idx, uint32_t* __restrict__ mask, int Lq_d, int W) {
     constexpr int NW = NT / 32;
-    static_assert(4 + 3 * NW <= 128, "scratch words");
+    static_assert(4 + 6 * NW <= 256, "scratch words");
     extern __shared__ __align__(16) uint8_t tk_smem[];
     uint32_t* hist = reinterpret_cast<uint32_t*>(tk_smem);
     uint32_t* cand = reinterpret_cast<uint32_t*>(tk_smem + TK_BINS * 4);
-    int* found = reinterpret_cast<int*>(tk_smem + TK_BINS * 4 + TK_CAND * 4);      // [0..3]
+    uint8_t* cand_w = tk_smem + TK_BINS * 4 + TK_CAND * 4;                       // warp of each candidate
+    int* found = reinterpret_cast<int*>(tk_smem + TK_BINS * 4 + TK_CAND * 5);      // [0..3]
     unsigned* wsum = reinterpret_cast<unsigned*>(found + 4);                        // [NW]
-    unsigned* wgt = wsum + NW;                                                // [NW]
-    unsigned* weq = wgt + NW;                                                 // [NW]
+    unsigned* wgt = wsum + NW;                                                // [NW] keys > T
+    unsigned* weq = wgt + NW;                                                 // [NW] keys == T
+    unsigned* wdef = weq + NW;                                                // [NW] bins above b1
+    unsigned* cgt = wdef + NW;                                                // [NW] candidates > T
+    unsigned* ceq = cgt + NW;                                                 // [NW] candidates == T
     uint32_t* keys = reinterpret_cast<uint32_t*>(tk_smem + TK_SMEM_FIXED);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -174,30 +179,46 @@ topk_select_kernel(const float* __restrict__ scores, long long ld, long long row
     const uint32_t cnt1 = hist[b1];
     __syncthreads();                                           // hist is reused below
 
-    // ---- 2. candidates of the threshold bin, then two radix passes on them
+    // ---- 2. candidates of the threshold bin, then two radix passes on them.
+    // Warp w scans the positions [w*seg, (w+1)*seg) it also emits in step 3,
+    // counting the keys of higher bins (all kept) and gathering the bin's
+    // keys with its warp id, so that step 3 needs no counting pass.
+    const int seg = ((n + NW * 32 - 1) / (NW * 32)) * 32;
+    const int s0 = min(n, warp * seg), s1 = min(n, s0 + seg);
     uint32_t prefix = b1 << 21;
     uint32_t pmask = 0x7FFu << 21;
     const bool use_cand = cnt1 <= (uint32_t)TK_CAND;
     if (use_cand) {
-        for (int gbase = warp * 32 * TK_VB; gbase < n; gbase += NT * TK_VB) {
+        unsigned cdef = 0;
+        for (int gbase = s0; gbase < s1; gbase += 32 * TK_VB) {
             uint32_t kb[TK_VB];
 #pragma unroll
             for (int u = 0; u < TK_VB; ++u) {
                 const int i = gbase + u * 32 + lane;
-                kb[u] = i < n ? key_at(i) : 0u;
+                kb[u] = i < s1 ? key_at(i) : 0u;
             }
 #pragma unroll
             for (int u = 0; u < TK_VB; ++u) {
                 const int i = gbase + u * 32 + lane;
-                const bool m = i < n && (kb[u] >> 21) == b1;
+                cdef += __popc(__ballot_sync(0xffffffffu, i < s1 && (kb[u] >> 21) > b1));
+                const bool m = i < s1 && (kb[u] >> 21) == b1;
                 const unsigned bal = __ballot_sync(0xffffffffu, m);
                 if (bal) {
                     unsigned pos0 = 0;
                     if (lane == 0) pos0 = atomicAdd(reinterpret_cast<unsigned*>(&found[2]), __popc(bal));
                     pos0 = __shfl_sync(0xffffffffu, pos0, 0);
-                    if (m) cand[pos0 + __popc(bal & ((1u << lane) - 1u))] = kb[u];
+                    if (m) {
+                        const unsigned c = pos0 + __popc(bal & ((1u << lane) - 1u));
+                        cand[c] = kb[u];
+                        cand_w[c] = (uint8_t)warp;
+                    }
                 }
             }
+        }
+        if (lane == 0) {
+            wdef[warp] = cdef;
+            cgt[warp] = 0u;
+            ceq[warp] = 0u;
         }
     }
     for (int pass = 1; pass < 3; ++pass) {
@@ -236,27 +257,40 @@ topk_select_kernel(const float* __restrict__ scores, long long ld, long long row
     const uint32_t T = prefix;
     const int need = remaining;   // keys equal to T that are kept, lowest positions first
 
-    // ---- 3. emit in position order: warp w owns [w*seg, (w+1)*seg)
-    const int seg = ((n + NW * 32 - 1) / (NW * 32)) * 32;
-    const int s0 = min(n, warp * seg), s1 = min(n, s0 + seg);
-    unsigned cg = 0, ce = 0;
-    for (int gbase = s0; gbase < s1; gbase += 32 * TK_VB) {
-        uint32_t kb[TK_VB];
-#pragma unroll
-        for (int u = 0; u < TK_VB; ++u) {
-            const int i = gbase + u * 32 + lane;
-            kb[u] = i < s1 ? key_at(i) : 0u;
+    // ---- 3. emit in position order: warp w owns [w*seg, (w+1)*seg).  Per
+    // warp, keys > T = higher bins + candidates > T; keys == T = candidates
+    // == T (from the candidate list), or one counting pass without it.
+    if (use_cand) {
+        for (int c = tid; c < (int)cnt1; c += NT) {
+            const uint32_t kk = cand[c];
+            if (kk > T) atomicAdd(&cgt[cand_w[c]], 1u);
+            else if (kk == T) atomicAdd(&ceq[cand_w[c]], 1u);
         }
-#pragma unroll
-        for (int u = 0; u < TK_VB; ++u) {
-            const int i = gbase + u * 32 + lane;
-            cg += __popc(__ballot_sync(0xffffffffu, i < s1 && kb[u] > T));
-            ce += __popc(__ballot_sync(0xffffffffu, i < s1 && kb[u] == T));
+        __syncthreads();
+        if (tid < NW) {
+            wgt[tid] = wdef[tid] + cgt[tid];
+            weq[tid] = ceq[tid];
         }
-    }
-    if (lane == 0) {
-        wgt[warp] = cg;
-        weq[warp] = ce;
+    } else {
+        unsigned cg = 0, ce = 0;
+        for (int gbase = s0; gbase < s1; gbase += 32 * TK_VB) {
+            uint32_t kb[TK_VB];
+#pragma unroll
+            for (int u = 0; u < TK_VB; ++u) {
+                const int i = gbase + u * 32 + lane;
+                kb[u] = i < s1 ? key_at(i) : 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < TK_VB; ++u) {
+                const int i = gbase + u * 32 + lane;
+                cg += __popc(__ballot_sync(0xffffffffu, i < s1 && kb[u] > T));
+                ce += __popc(__ballot_sync(0xffffffffu, i < s1 && kb[u] == T));
+            }
+        }
+        if (lane == 0) {
+            wgt[warp] = cg;
+            weq[warp] = ce;
+        }
     }
     __syncthreads();
     unsigned g = 0, e = 0;

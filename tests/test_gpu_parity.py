@@ -233,8 +233,9 @@ def test_sparse_attn_with_holes_and_bad_indices(ic):
 
 
 DENSE_CASES = [
-    # B, Lq, Lk, q_offset, Hq, d, k   (rows t < 4k take the dense-masked kernel)
-    (1, 700, 700, 0, 16, 128, 96),          # 48 dense blocks, 316 gathered rows
+    # B, Lq, Lk, q_offset, Hq, d, k   (rows t < 8k take the dense-masked kernel)
+    (1, 700, 700, 0, 16, 128, 48),          # 48 dense blocks, 316 gathered rows
+    (1, 700, 700, 0, 16, 128, 96),          # 87 dense blocks, 4 gathered rows split over CTAs
     (2, 1000, 1000, 0, 16, 128, 256),       # all dense, B = 2, ragged last key tile
     (1, 300, 1324, 1024, 16, 128, 512),     # mid-sequence chunk, 4 gathered tail rows
     (1, 500, 500, 0, 8, 128, 128),          # 16 queries per block
@@ -269,7 +270,7 @@ def test_unique_attn_dense_and_gathered_rows_match_oracle(ic, B, Lq, Lk, q_offse
 def test_unique_attn_dense_rows_with_holes_and_bad_indices(ic):
     """The dense-masked kernel sees the selection only as a bitmask: -1 slots
     anywhere, unsorted rows, and an index beyond t (skipped and reported)."""
-    B, L, Hq, d, k = 1, 160, 16, 128, 40                 # every row t < 4k = 160
+    B, L, Hq, d, k = 1, 160, 16, 128, 40                 # every row t < 8k = 320
     wl = synth.custom(B=B, Lq=L, H_I=4, d_I=64, k=k, Hq=Hq, d=d, cfg_id=28)
     lay = synth.make_layers(wl)[0]
     rng = np.random.default_rng(5)
@@ -353,7 +354,7 @@ def test_stack_chunking_and_pattern_spelling_do_not_change_results(ic):
 
 
 def test_stack_timing_marks_are_recorded_in_order(ic):
-    # rows t < 4k take the dense-masked kernel, the rest gather: every mark
+    # rows t < 8k take the dense-masked kernel, the rest gather: every mark
     # of every layer is recorded, in stream order
     wl = synth.custom(Lq=700, n_layers=2, H_I=32, d_I=128, k=96, Hq=16, d=128, pattern="FS",
                       cfg_id=26)
