@@ -330,7 +330,8 @@ dense_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
         if (nt > 1) write_bias(1, bias_word(1));
         uint32_t nbw = nt > 2 ? bias_word(2) : 0u;
         for (int j = 0; j < nt; ++j) {
-            if (!mbar_wait(&s_full[j & 1], (j >> 1) & 1)) { ok = false; break; }
+            // waits are warp-uniform: the TMEM accesses below are warp-collective
+            if (!__all_sync(0xffffffffu, mbar_wait(&s_full[j & 1], (j >> 1) & 1))) { ok = false; break; }
             tc_fence_after();
             // S(j+2) overwrites bias stage j&1 only after S(j) is complete
             if (j + 2 < nt) {
@@ -392,23 +393,26 @@ dense_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
             }
             // P(j-1) V(j-1) must be complete before O is rescaled
             if (j > 0) {
-                if (!mbar_wait(o_full, (j - 1) & 1)) { ok = false; break; }
+                if (!__all_sync(0xffffffffu, mbar_wait(o_full, (j - 1) & 1))) { ok = false; break; }
                 tc_fence_after();
             }
-            if (raise) {
-                const float alpha = ex2_approx(m_used - m_new);     // 0 on the first raise
-                if (j > 0) {
+            // Rows raise their max independently, but TMEM loads and stores
+            // are warp-collective: when any row of the warp raises, every
+            // lane takes O through registers, the others with factor 1.
+            const float alpha = raise ? ex2_approx(m_used - m_new) : 1.0f;   // 0 on a first raise
+            if (j > 0 && __any_sync(0xffffffffu, raise)) {
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t o[32];
-                        tmem_ld_32x32b_x32(tmem + DA_O_COL + lane_base + c * 32, o);
-                        tmem_ld_wait();
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t o[32];
+                    tmem_ld_32x32b_x32(tmem + DA_O_COL + lane_base + c * 32, o);
+                    tmem_ld_wait();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                        tmem_st_32x32b_x32(tmem + DA_O_COL + lane_base + c * 32, o);
-                    }
+                    for (int e = 0; e < 32; ++e)
+                        o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    tmem_st_32x32b_x32(tmem + DA_O_COL + lane_base + c * 32, o);
                 }
+            }
+            if (raise) {
                 l_run *= alpha;
                 m_used = m_new;
             }
@@ -420,10 +424,11 @@ dense_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
             mbar_arrive(p_full);
         }
         if (ok && nt > 0) {
-            ok = mbar_wait(o_full, (nt - 1) & 1);
+            ok = __all_sync(0xffffffffu, mbar_wait(o_full, (nt - 1) & 1));
             tc_fence_after();
         }
-        if (ok && i0 + qi < a.Lq) {
+        if (ok) {                                   // uniform across the warp
+            const bool row_in = i0 + qi < a.Lq;
             const long long orow = ((long long)b * a.Lq + i0 + qi) * a.Hq + h;
             const float inv = l_run > 0.0f ? 1.0f / l_run : 0.0f;
             uint4* dst = reinterpret_cast<uint4*>(a.out + orow * 128);
@@ -432,6 +437,7 @@ dense_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 uint32_t o[32];
                 tmem_ld_32x32b_x32(tmem + DA_O_COL + lane_base + c * 32, o);
                 tmem_ld_wait();
+                if (!row_in) continue;
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     uint32_t w[4];
@@ -444,7 +450,7 @@ dense_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     dst[c * 4 + u] = make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }
-            if (a.lse) a.lse[orow] = l_run > 0.0f ? (m_used + log2f(l_run)) * LN2 : -INFINITY;
+            if (a.lse && row_in) a.lse[orow] = l_run > 0.0f ? (m_used + log2f(l_run)) * LN2 : -INFINITY;
         }
     }
 
