@@ -299,6 +299,37 @@ def test_unique_attn_dense_rows_with_holes_and_bad_indices(ic):
     assert ic.get_last_device_error() == 0
 
 
+def _first_tile_empty_idx(L, k, seed):
+    """Index rows where even queries past position 64 select nothing among
+    keys 0..63 and odd queries select key 0: within one warp (two queries x
+    16 heads) some rows raise their running max at the second key tile and
+    others do not."""
+    rng = np.random.default_rng(seed)
+    idx = np.full((L, k), -1, dtype=np.int32)
+    for t in range(L):
+        lo = 64 if (t % 2 == 0 and t >= 64 + k) else 0
+        pick = rng.choice(np.arange(lo, t + 1), size=min(k, t + 1 - lo), replace=False)
+        if lo == 0 and 0 not in pick:
+            pick[0] = 0
+        idx[t, : len(pick)] = np.sort(pick)
+    return idx
+
+
+def test_unique_attn_rows_raising_their_max_after_the_first_tile(ic):
+    """Rows of one warp raise the running max at different tiles; the O
+    rescale in TMEM is warp-collective and must stay correct for all rows."""
+    B, L, Hq, d, k = 1, 256, 16, 128, 40                  # every row t < 8k = 320
+    wl = synth.custom(B=B, Lq=L, H_I=4, d_I=64, k=k, Hq=Hq, d=d, cfg_id=30)
+    lay = synth.make_layers(wl)[0]
+    idx = _first_tile_empty_idx(L, k, 11)
+    ref, ref_lse = oracle.sparse_attn(lay["q"], lay["k"], lay["v"], idx)
+    out, lse = ic.sparse_attn_unique(lay["q"].cuda(), lay["k"].cuda(), lay["v"].cuda(),
+                                     torch.from_numpy(idx).reshape(1, L, k).cuda())
+    assert ic.get_last_device_error() == 0
+    assert np.abs(out.float().cpu().numpy().reshape(L, Hq, d) - ref).max() <= ATTN_ATOL
+    assert np.abs(lse.cpu().numpy().reshape(L, Hq) - ref_lse).max() <= LSE_ATOL
+
+
 # ------------------------------------------------------------------ a3/a5 layer stack
 
 def _run_stack(ic, wl, layers, pattern=None, **kw):
