@@ -60,24 +60,14 @@ def load_peaks():
 
 # ---------------------------------------------------------------- algorithmic work
 
-DENSE_FACTOR = 8          # rows with t < 8k attend tile-dense (the library's dispatch rule)
-DENSE_MAX_KEYS = 65536    # ... and see at most this many keys
 DA_TILE = 64              # keys per tile of the dense-masked kernel
 SFU_PER_CLK_SM = 16       # ex2 results per clock per SM (CUDA arithmetic-throughput table)
 
 
-def dense_rows(wl):
-    """Rows per sequence that the layer stack sends to the dense-masked kernel
-    (t < 8k, whole blocks of 128/Hq queries), and that block size."""
-    if wl.d != 128 or 128 % wl.Hq:
-        return 0, 0
-    qbd = 128 // wl.Hq
-    lim = min(DENSE_FACTOR * wl.k - wl.q_offset, DENSE_MAX_KEYS - wl.q_offset, wl.Lq)
-    return (lim // qbd * qbd if lim >= qbd else 0), qbd
-
-
-def work_per_layer(wl):
-    """Algorithmic flops / bytes of each step of one layer (causal)."""
+def work_per_layer(wl, lq_d: int = 0):
+    """Algorithmic flops / bytes of each step of one layer (causal).  The
+    first lq_d rows of each sequence take the dense-masked attention (as the
+    library reports for the stack's workspace), in blocks of 128/Hq queries."""
     B, Lq, Lk, q0, k = wl.B, wl.Lq, wl.Lk, wl.q_offset, wl.k
     t = np.arange(Lq, dtype=np.float64) + q0
     vis = np.minimum(t + 1, Lk)
@@ -90,7 +80,7 @@ def work_per_layer(wl):
     w["indexer_bytes"] = (rows * wl.H_I * wl.d_I * 2 + rows * wl.H_I * 4 + B * Lk * wl.d_I * 2
                           + 4 * sum_vis)
     w["topk_bytes"] = 4 * sum_vis + 4.0 * rows * k
-    lq_d, qbd = dense_rows(wl)
+    qbd = 128 // wl.Hq if lq_d else 0
     # dense-masked rows: useful flops are those of the selected positions;
     # the kernel executes whole 64-key tiles of 128 rows up to each block's last t
     sel_d = B * sel_row[:lq_d].sum()
@@ -423,6 +413,7 @@ def main():
     if rpc <= 0:
         rpc = max(1, min(wl.B * wl.Lq, (16 * 2 ** 30) // (4 * wl.Lk)))
     stack = ic.LayerStack(pattern, layers, dims, rows_per_chunk=rpc)
+    lq_d = ic.layer_stack_dense_rows(dims, stack.ws.numel())
     stream = torch.cuda.current_stream()
     n = wl.n_layers
     flush = torch.empty(256 * 1024 * 1024 // 4, device=dev, dtype=torch.float32)
@@ -479,7 +470,7 @@ def main():
 
     # ---- per-kernel breakdown from the marks
     ki = {"indexer": [], "topk": [], "attn_dense": [], "attn_gather": []}
-    w = work_per_layer(wl)
+    w = work_per_layer(wl, lq_d)
     for evs, _ in marks:
         for l, c in enumerate(pattern):
             e = evs[npl * l: npl * (l + 1)]

@@ -213,6 +213,16 @@ typedef struct {
 size_t ic_layer_stack_workspace_bytes(const ic_dims *dims, int n_layers, long long rows_per_chunk);
 
 /*
+ * Rows per sequence (the first ones, i < returned value) that
+ * ic_layer_stack_forward sends to the dense-masked attention for these dims
+ * and a workspace of ws_bytes: rows with t < 8k in whole blocks of 128/Hq
+ * queries, when d = 128, Hq divides 128, at most 65536 keys are visible and
+ * the workspace holds the selection bitmask next to one block of scores and
+ * the transposed V.  The other rows gather.  0 for invalid dims.
+ */
+int ic_layer_stack_dense_rows(const ic_dims *dims, size_t ws_bytes);
+
+/*
  * Steps a1-a5 — the IndexCache layer loop (skill page Step 3; technical
  * summary, Methodologie; review: "a single conditional branch").
  * pattern: n_layers characters, 'F' or '1' = Full layer, 'S' or '0' = Shared.

@@ -745,6 +745,19 @@ int ic_index_overlap(const int32_t* idx_a, const int32_t* idx_b, long long n_row
     return launched(cudaGetLastError(), "index_overlap launch");
 }
 
+int ic_layer_stack_dense_rows(const ic_dims* dims, size_t ws_bytes) {
+    if (!dims || check_positions(dims->B, dims->Lq, dims->Lk, dims->q_offset) ||
+        check_indexer_shape(dims->H_I, dims->d_I) || dims->k < 1 || dims->Lq < 1)
+        return 0;
+    const DenseGeom dg = dense_geom(*dims);
+    if (!dg.on) return 0;
+    // the same test stack_forward applies to its workspace
+    const IndexerGeom geo = indexer_geom(dims->Lq, dims->H_I);
+    const size_t block_bytes = (size_t)geo.QB * (size_t)dims->Lk * sizeof(float);
+    if (ws_bytes < dg.mask_bytes + std::max(block_bytes, dg.vt_bytes)) return 0;
+    return dg.Lq_d;
+}
+
 size_t ic_layer_stack_workspace_bytes(const ic_dims* dims, int n_layers, long long rows_per_chunk) {
     if (!dims || n_layers < 1) return 0;
     if (check_positions(dims->B, dims->Lq, dims->Lk, dims->q_offset) ||

@@ -34,7 +34,8 @@ EXPORTS = ("ic_status_string", "ic_last_error_message", "ic_get_last_device_erro
            "ic_sparse_attn_workspace_bytes", "ic_layer_stack_workspace_bytes",
            "ic_layer_stack_forward", "ic_layer_stack_forward_events", "ic_selftest_wait_timeout",
            "ic_sparse_attn_no_alloc", "ic_kernel_launch_count", "ic_sparse_attn_unique",
-           "ic_sparse_attn_unique_workspace_bytes", "ic_index_overlap")
+           "ic_sparse_attn_unique_workspace_bytes", "ic_index_overlap",
+           "ic_layer_stack_dense_rows")
 
 MARKS_PER_LAYER = 5        # IC_MARKS_PER_LAYER
 
@@ -87,6 +88,8 @@ _lib.ic_sparse_attn_unique_workspace_bytes.restype = _Z
 _lib.ic_sparse_attn_unique_workspace_bytes.argtypes = [_I, _I, _I, _I, _I, _I, _I]
 _lib.ic_sparse_attn_workspace_bytes.restype = _Z
 _lib.ic_sparse_attn_workspace_bytes.argtypes = [_I, _I, _I, _I, _I]
+_lib.ic_layer_stack_dense_rows.restype = _I
+_lib.ic_layer_stack_dense_rows.argtypes = [ctypes.POINTER(ICDims), _Z]
 _lib.ic_layer_stack_workspace_bytes.restype = _Z
 _lib.ic_layer_stack_workspace_bytes.argtypes = [ctypes.POINTER(ICDims), _I, ctypes.c_longlong]
 _lib.ic_selftest_wait_timeout.restype = _I
@@ -279,6 +282,11 @@ def make_dims(B, Lq, Lk, q_offset, H_I, d_I, Hq, d, k, scale=0.0, Hkv=1) -> ICDi
 
 def layer_stack_workspace_bytes(dims: ICDims, n_layers: int, rows_per_chunk: int = 0) -> int:
     return int(_lib.ic_layer_stack_workspace_bytes(ctypes.byref(dims), n_layers, rows_per_chunk))
+
+
+def layer_stack_dense_rows(dims: ICDims, ws_bytes: int) -> int:
+    """Rows per sequence the stack sends to the dense-masked attention."""
+    return int(_lib.ic_layer_stack_dense_rows(ctypes.byref(dims), int(ws_bytes)))
 
 
 class LayerStack:

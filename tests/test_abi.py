@@ -143,3 +143,24 @@ def test_index_overlap_rejects_bad_sizes_before_launch(ic):
     assert lib.ic_index_overlap(None, 0x1000, 4, 8, 100, 0x2000, None) == 1       # null
     assert lib.ic_index_overlap(None, None, 0, 8, 100, None, None) == 0           # nothing to do
     assert ic.kernel_launch_count() == before
+
+
+def test_layer_stack_dense_rows(ic):
+    """Rows t < 8k, whole blocks of 128/Hq queries, d = 128, with a workspace
+    that holds the bitmask, one block of scores and V^T; 0 otherwise."""
+    def rows(ws=None, **kw):
+        d = dict(B=1, Lq=700, Lk=700, q_offset=0, H_I=32, d_I=128, Hq=16, d=128, k=96)
+        d.update(kw)
+        dims = ic.make_dims(d["B"], d["Lq"], d["Lk"], d["q_offset"], d["H_I"], d["d_I"], d["Hq"],
+                            d["d"], d["k"])
+        if ws is None:
+            ws = ic.layer_stack_workspace_bytes(dims, 2)
+        return ic.layer_stack_dense_rows(dims, ws)
+    assert rows() == 696                       # min(8k, L) = 700 -> 87 blocks of 8
+    assert rows(k=48) == 384                   # 8k = 384
+    assert rows(Hq=8) == 688                   # blocks of 16 queries
+    assert rows(d=64, Hq=8) == 0               # the dense kernel needs d = 128
+    assert rows(Lq=1, Lk=32768, q_offset=32767, k=2048) == 0     # decode: t far beyond 8k
+    assert rows(Lq=300, Lk=1324, q_offset=1024, k=512) == 296    # mid-sequence chunk
+    assert rows(ws=1000) == 0                  # workspace too small: every row gathers
+    assert rows(d_I=96) == 0                   # invalid dims
