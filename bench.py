@@ -355,6 +355,68 @@ def config_of(wl, pattern, args):
 
 # ---------------------------------------------------------------- GPU leg
 
+def run_row_sharded(args, wl, pattern, ic, dev, world, rank, local, pg):
+    """--shard rows: the ranks split ONE workload's query rows (zig-zag row
+    chunks of the sequence for B = 1, whole sequences for B > 1); each step
+    every rank runs its shard of the stack, with no collective on the data
+    path.  value = the workload's tokens / max-over-ranks step time (strong
+    scaling).  Only the whole-step time is reported in this mode."""
+    from lightning_indexer_top_relu_b200 import sharding
+    layers = synth.make_layers(wl, indexer_for_all=False, device=dev)
+    torch.cuda.synchronize()
+    dims = ic.make_dims(wl.B, wl.Lq, wl.Lk, wl.q_offset, wl.H_I, wl.d_I, wl.Hq, wl.d, wl.k)
+    stack = sharding.ShardedStack(pattern, layers, dims, world, rank)
+    rows_here = sum(ch.nb * ch.n for ch in stack.chunks)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 * 1024 * 1024 // 4, device=dev, dtype=torch.float32)
+    for _ in range(args.warmup):
+        stack.forward(stream)
+    torch.cuda.synchronize()
+    if ic.get_last_device_error() != 0:
+        raise RuntimeError("device error during warm-up")
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    if pg is not None:
+        pg.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    launches0 = ic.kernel_launch_count()
+    for s in range(args.steps):
+        flush.fill_(float(s))
+        starts[s].record(stream)
+        stack.forward(stream)
+        ends[s].record(stream)
+    torch.cuda.synchronize()
+    launches = ic.kernel_launch_count() - launches0
+    if pg is not None:
+        pg.barrier()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if ic.get_last_device_error() != 0:
+        raise RuntimeError("device error during the timed steps")
+    local_ms = float(np.mean([starts[s].elapsed_time(ends[s]) for s in range(args.steps)]))
+    ms_per_step, tokens, value = aggregate_over_ranks(local_ms, float(rows_here), pg, dev)
+    cfg = config_of(wl, pattern, args)
+    cfg["parallelism"] = f"rows{world}" if wl.B == 1 else f"sequences{world}"
+    cfg["shard_rank0"] = [[ch.b0, ch.nb, ch.i0, ch.n] for ch in sharding.shard(wl.B, wl.Lq, world, 0)]
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded Gaussian, correlated layers)", "config": cfg,
+            "gpu_launches": int(launches), "roofline": None,
+            "note": "row-sharded mode: whole-step time only; the per-kernel breakdown and "
+                    "roofline come from the default (replica) mode"}
+    if clk is not None:
+        line["clocks"] = clk
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -368,6 +430,9 @@ def main():
     ap.add_argument("--no-all-f", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=64)
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "rows"],
+                    help="with N > 1 ranks: a replica of the workload per rank (weak scaling) "
+                         "or one workload's query rows split over the ranks (strong scaling)")
     ap.add_argument("--rows-per-chunk", type=int, default=0,
                     help="F-layer score rows per chunk (0: as many as 16 GiB of scores allow)")
     args = ap.parse_args()
@@ -395,6 +460,9 @@ def main():
         pg = dist
 
     from lightning_indexer_top_relu_b200 import indexcache as ic
+
+    if args.shard == "rows":
+        return run_row_sharded(args, wl, pattern, ic, dev, world, rank, local, pg)
 
     peaks = load_peaks()
     need_all = (not args.no_all_f) and any(c in "S0" for c in pattern)
