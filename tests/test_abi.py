@@ -164,3 +164,33 @@ def test_layer_stack_dense_rows(ic):
     assert rows(Lq=300, Lk=1324, q_offset=1024, k=512) == 296    # mid-sequence chunk
     assert rows(ws=1000) == 0                  # workspace too small: every row gathers
     assert rows(d_I=96) == 0                   # invalid dims
+
+
+def test_unique_attention_rejects_bad_arguments_before_launch(ic):
+    lib = ic.lib()
+    f = lib.ic_sparse_attn_unique
+    before = ic.kernel_launch_count()
+    ok = dict(q=0x1000, k=0x2000, v=0x3000, idx=0x4000, B=1, Lq=64, Lk=64, Hq=16, Hkv=1, d=128,
+              ks=32, q0=0, scale=0.0, out=0x5000, lse=None, ws=None, wsb=0)
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return f(a["q"], a["k"], a["v"], a["idx"], a["B"], a["Lq"], a["Lk"], a["Hq"], a["Hkv"],
+                 a["d"], a["ks"], a["q0"], a["scale"], a["out"], a["lse"], a["ws"], a["wsb"], None)
+    assert call(Hkv=2) == 2                      # MQA only
+    assert call(ks=0) == 1                       # k < 1
+    assert call(q0=10) == 1                      # q_offset + Lq > Lk
+    assert call(q=None) == 1                     # null operand
+    assert call(k=0x2008) == 2                   # K not 16-byte aligned
+    assert call(scale=float("nan")) == 1         # scale not finite
+    assert call(wsb=64) == 1                     # workspace size without a workspace
+    assert call(B=0) == 0                        # nothing to do
+    assert ic.kernel_launch_count() == before
+
+
+def test_unique_attention_workspace_query(ic):
+    q = ic.sparse_attn_unique_workspace_bytes
+    assert q(1, 700, 700, 0, 16, 128, 96) > 700 * 12 * 4        # bitmask + V^T at least
+    assert q(0, 700, 700, 0, 16, 128, 96) == 0
+    assert q(1, 700, 600, 0, 16, 128, 96) == 0                  # q_offset + Lq > Lk
