@@ -384,6 +384,31 @@ def test_stack_chunking_and_pattern_spelling_do_not_change_results(ic):
     _compare_stack(a, wl, layers, None)
 
 
+def test_stack_batch_of_two_with_dense_rows(ic):
+    # B = 2: the top-k writes each sequence's bitmask rows (b * rows + i) and
+    # the dense-masked kernel reads them back
+    wl = synth.custom(B=2, Lq=300, n_layers=2, H_I=32, d_I=128, k=64, Hq=16, d=128, pattern="FS",
+                      cfg_id=34)
+    layers = synth.make_layers(wl)
+    dims = ic.make_dims(wl.B, wl.Lq, wl.Lk, wl.q_offset, wl.H_I, wl.d_I, wl.Hq, wl.d, wl.k)
+    assert ic.layer_stack_dense_rows(dims, ic.layer_stack_workspace_bytes(dims, 2)) == 296
+    st = _run_stack(ic, wl, layers)
+    check_idx_valid(st.idx_cache, 0, wl.k)
+    _compare_stack(st, wl, layers, None)
+
+
+def test_stack_continuation_chunk_with_dense_rows(ic):
+    # rows 512..767 of a sequence whose first 512 positions are already cached
+    wl = synth.custom(Lq=256, Lk=768, q_offset=512, n_layers=2, H_I=32, d_I=128, k=128, Hq=16,
+                      d=128, pattern="FS", cfg_id=35)
+    layers = synth.make_layers(wl)
+    dims = ic.make_dims(wl.B, wl.Lq, wl.Lk, wl.q_offset, wl.H_I, wl.d_I, wl.Hq, wl.d, wl.k)
+    assert ic.layer_stack_dense_rows(dims, ic.layer_stack_workspace_bytes(dims, 2)) == 256
+    st = _run_stack(ic, wl, layers)
+    check_idx_valid(st.idx_cache, wl.q_offset, wl.k)
+    _compare_stack(st, wl, layers, None)
+
+
 def test_stack_timing_marks_are_recorded_in_order(ic):
     # rows t < 8k take the dense-masked kernel, the rest gather: every mark
     # of every layer is recorded, in stream order
