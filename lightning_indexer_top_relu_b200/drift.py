@@ -63,8 +63,8 @@ class DriftRefreshStack:
             if c not in "S0":
                 raise ValueError(f"pattern character {c!r} is neither F/1 nor S/0")
             if not run:
-                raise ValueError("layer 0 is Shared: no cached indices available before the "
-                                 "first F layer")
+                raise ValueError("the base pattern starts with a shared layer; the index cache "
+                                 "stays empty until a full layer has run")
             counts, t = self.backend.probe(l, self.probe_rows)
             keep = np.asarray(t) >= self.k
             ov = float(np.mean(np.asarray(counts)[keep, 0] / self.k)) if keep.any() else 1.0

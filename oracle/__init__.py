@@ -270,7 +270,8 @@ def layer_stack(pattern: str, layers: Sequence[dict], k: int, q_offset: int = 0,
             sc = indexer_scores(qi, L["k_idx"], L["w"], q_offset, rows)
             cached = topk_sort(sc.astype(np.float32), row_positions(B, Lq, q_offset, rows), k)
         elif cached is None:
-            raise NoCachedIndices("No cached indices available")
+            raise NoCachedIndices(f"layer {l} is shared, but no full layer before it has "
+                                  "filled the index cache")
         o, lse = sparse_attn(L["q"], L["k"], L["v"], cached, q_offset, scale, rows)
         outs.append(o)
         idxs.append(cached)

@@ -228,6 +228,22 @@ def test_attention_dominant_logit_picks_its_value_row():
     assert abs(lse[0, 0] - (64.0 + math.log1p(3 * math.exp(-64.0)))) < 1e-12
 
 
+def test_attention_row_sampling_matches_full():
+    """Row r of a sampled call is flattened row rows[r] of the full call, and
+    it reads index row r (one index row per requested row)."""
+    wl = synth.custom(B=2, Lq=30, Lk=50, q_offset=20, H_I=2, d_I=64, k=8, Hq=3, d=64)
+    L = synth.make_layers(wl)[0]
+    sc = oracle.indexer_scores(L["q_idx"], L["k_idx"], L["w"], q_offset=20)
+    idx = oracle.topk_sort(sc.astype(np.float32), oracle.row_positions(2, 30, 20), 8)
+    full, full_lse = oracle.sparse_attn(L["q"], L["k"], L["v"], idx, q_offset=20)
+    dense, dense_lse = oracle.dense_attn(L["q"], L["k"], L["v"], q_offset=20)
+    rows = [59, 0, 31, 7, 30]
+    part, part_lse = oracle.sparse_attn(L["q"], L["k"], L["v"], idx[rows], q_offset=20, rows=rows)
+    assert np.array_equal(part, full[rows]) and np.array_equal(part_lse, full_lse[rows])
+    dpart, dpart_lse = oracle.dense_attn(L["q"], L["k"], L["v"], q_offset=20, rows=rows)
+    assert np.array_equal(dpart, dense[rows]) and np.array_equal(dpart_lse, dense_lse[rows])
+
+
 def test_attention_empty_row_and_out_of_range_index():
     q = _bf16(np.ones((1, 1, 2, 4)))
     K = _bf16(np.ones((1, 3, 1, 4)))
@@ -326,6 +342,13 @@ def test_overlap_hand_example():
     assert c.tolist() == [[2, 4, 3]]
     assert oracle.overlap_fraction(c, 4)[0] == 0.5
     assert abs(oracle.jaccard(c)[0] - 0.4) < 1e-9
+    # a short row (t + 1 < k: holes at the tail): the fraction is still over
+    # the k slots of the cache, A = {1, 2}, B = {2, 3, 7} -> 1/4
+    c = oracle.index_overlap(np.array([[1, 2, -1, -1]], dtype=np.int32),
+                             np.array([[2, 3, 7, -1]], dtype=np.int32), 10)
+    assert c.tolist() == [[1, 2, 3]]
+    assert oracle.overlap_fraction(c, 4)[0] == 0.25
+    assert abs(oracle.jaccard(c)[0] - 0.25) < 1e-9
 
 
 def test_overlap_matches_python_sets_and_is_symmetric():
