@@ -799,7 +799,7 @@ static int stack_forward(const char* pattern, int n_layers, const ic_layer* laye
     }
     if (pattern[0] == 'S' || pattern[0] == '0')
         return fail(IC_ERR_NO_CACHED_INDICES,
-                    "layer 0 is Shared: no cached indices available before the first F layer");
+                    "layer 0 is Shared: the index cache is empty until a Full layer has run");
     const ic_dims& D = *dims;
     int rc = check_positions(D.B, D.Lq, D.Lk, D.q_offset);
     if (rc) return rc;

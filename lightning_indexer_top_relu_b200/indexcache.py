@@ -47,8 +47,10 @@ class IndexCacheError(RuntimeError):
         super().__init__(f"{where}: {STATUS.get(status, status)}: {msg}")
 
 
-class NoCachedIndices(IndexCacheError):
-    pass
+class NoCachedIndices(IndexCacheError, ValueError):
+    """A shared layer came before any full layer (IC_ERR_NO_CACHED_INDICES).
+    Also a ValueError: the failure a caller of a Python index-cache lookup
+    expects when no indices have been stored yet."""
 
 
 class ICLayer(ctypes.Structure):
