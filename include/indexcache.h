@@ -5,18 +5,17 @@
  *
  * Sources.  "IndexCache: Accelerating Sparse Attention via Cross-Layer Index
  * Reuse" (arXiv 2603.12201), as described by:
- *   - the fugumt digest, Abstract: a lightning indexer selects the top-k most
- *     relevant tokens per query, reducing core attention from O(L^2) to
- *     O(Lk); Full layers run their own indexers, Shared layers reuse the
- *     nearest Full layer's top-k indices;
+ *   - the fugumt digest, Abstract: per query, a lightning indexer ranks the
+ *     earlier tokens and only the k best-ranked enter core attention, which
+ *     then costs O(Lk) per sequence rather than O(L^2); a Full layer keeps its indexer, a
+ *     Shared layer takes the index set of the closest Full layer above it;
  *   - the kualia.ai review, "The Redundancy That Was Sitting There": the
- *     index cache is a temporary buffer holding only the current index tensor,
- *     overwritten at each F layer;
+ *     cache is one scratch tensor of indices that each F layer replaces;
  *   - the skill page, Step 3 (IndexCacheManager.get_indices_for_layer): an S
  *     layer with nothing cached is an error;
  *   - the knowledge note "Cross-Layer Index Reuse", How It Works: the anchor
- *     layer scores the visible positions; following layers run their own
- *     sparse attention over the stored positions.
+ *     layer scores the visible positions and stores its selection; each
+ *     layer after it attends sparsely over that stored selection.
  * The pages print no indexer formula; this library computes the standard
  * lightning-indexer score s[t,s] = sum_j w[t,j] * max(0, q_I[t,j] . k_I[s]).
  *
@@ -86,7 +85,7 @@ int ic_selftest_wait_timeout(int timeout_us, ic_stream_t stream);
 
 /*
  * Step a1 — lightning indexer scores (digest Abstract; review Introduction:
- * the indexer scores all preceding tokens).
+ * one indexer pass rates every earlier token of each query).
  *   q_idx  [B, Lq, H_I, d_I] bf16     k_idx [B, Lk, d_I] bf16
  *   w      [B, Lq, H_I]      fp32     scores [B, Lq, Lk] fp32 (written)
  * scores[b,i,s] = sum_j w[b,i,j] * max(0, q_idx[b,i,j,:] . k_idx[b,s,:]) for
@@ -98,8 +97,7 @@ int ic_indexer_scores(const uint16_t *q_idx, const uint16_t *k_idx, const float 
                       ic_stream_t stream);
 
 /*
- * Step a2 — per-row top-k (digest Abstract: the indexer selects the top-k
- * tokens per query).
+ * Step a2 — per-row top-k (digest Abstract: k tokens are kept per query).
  *   scores [B, Lq, Lk] fp32 (only s <= t is read)   idx [B, Lq, k] int32 (written)
  * Row (b, i) keeps the min(k, t+1) visible positions first in the order
  * (score descending, position ascending), written in ascending position
@@ -112,8 +110,8 @@ int ic_topk_select(const float *scores, int B, int Lq, int Lk, int q_offset, int
 
 /*
  * Step a4 — sparse attention over the cached positions (digest Abstract:
- * core attention over k tokens; knowledge note: each layer runs its own
- * sparse attention over the stored positions).  MQA: Hkv must be 1.
+ * core attention over k tokens; knowledge note: every later layer attends
+ * sparsely over the stored set).  MQA: Hkv must be 1.
  *   q [B, Lq, Hq, d] bf16   k, v [B, Lk, Hkv, d] bf16   idx [B, Lq, k] int32
  *   out [B, Lq, Hq, d] bf16 (written)   lse [B, Lq, Hq] fp32 (written; may be NULL)
  * For each (b, i, h) over the slots whose index lies in [0, t]:

@@ -15,8 +15,8 @@ into it, and runs the layer loop of the IndexCache inference path:
   returns the cached indices and fails when none exist yet.
 * Same paper (Dutch technical summary, Methodologie): S layers inherit the
   top-k indices of the nearest preceding F layer.
-* kualia.ai review ("The Redundancy That Was Sitting There"): the cache holds
-  only the current index tensor and is overwritten at each F layer.
+* kualia.ai review ("The Redundancy That Was Sitting There"): the cache is
+  one scratch tensor of indices that each F layer replaces.
 
 Pattern characters: 'F' or '1' = full layer, 'S' or '0' = shared layer (the
 skill page's code uses '1'/'0', the prose uses F/S).

@@ -8,14 +8,14 @@
  *
  * Sources (the pages describing IndexCache, arXiv 2603.12201):
  *  - "IndexCache: Accelerating Sparse Attention via Cross-Layer Index Reuse"
- *    (fugumt digest, Abstract): a lightning indexer selects the top-k most
- *    relevant tokens per query; core attention then runs over those k tokens.
+ *    (fugumt digest, Abstract): per query, a lightning indexer ranks the
+ *    earlier tokens; core attention then covers only the k best-ranked ones.
  *  - "When the Optimizer Becomes the Bottleneck: A Close Look at IndexCache"
- *    (kualia.ai, Introduction): the indexer scores all preceding tokens and
- *    keeps the top-k.
+ *    (kualia.ai, Introduction): one indexer pass rates every earlier token
+ *    of a query and the k highest-rated are kept.
  *  - "Cross-Layer Index Reuse" (knowledge note, How It Works): the anchor
- *    layer scores the visible positions and stores a top-k index set; the
- *    layers after it run their own sparse attention over those positions.
+ *    layer scores the visible positions and stores its k-position set; each
+ *    layer after it attends sparsely over that stored set.
  *  The pages print no formula for the indexer score.  The plainest standard
  *  form is used: s[t,s] = sum_j w[t,j] * max(0, q_I[t,j] . k_I[s]), with the
  *  visible set s <= t.
@@ -189,8 +189,8 @@ int or_topk_count(const float *scores, const int64_t *tpos, int64_t n_rows, int 
 /* ------------------------------------------------------------------ */
 /* Step a4, sparse attention over the cached positions (IndexCache      */
 /* digest, Abstract: core attention over k selected tokens; knowledge   */
-/* note, How It Works: each layer runs its own sparse attention over    */
-/* the stored positions).  MQA: every query head reads the one K/V head.*/
+/* note, How It Works: every later layer attends sparsely over the     */
+/* stored set).  MQA: every query head reads the one K/V head.          */
 /*   q [B,Lq,Hq,d]  K,V [B,Lk,d]  idx [n_rows,k], one row per requested  */
 /*   query row (-1 = empty slot)                                        */
 /* For row r and head h over the valid slots:                           */
