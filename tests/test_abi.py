@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+from hypothesis import given, settings, strategies as st
 
 from lightning_indexer_top_relu_b200 import build
 
@@ -164,6 +165,33 @@ def test_layer_stack_dense_rows(ic):
     assert rows(Lq=300, Lk=1324, q_offset=1024, k=512) == 296    # mid-sequence chunk
     assert rows(ws=1000) == 0                  # workspace too small: every row gathers
     assert rows(d_I=96) == 0                   # invalid dims
+
+
+@settings(max_examples=300, deadline=None)
+@given(Lq=st.integers(1, 20000), q0=st.integers(0, 70000), extra=st.integers(0, 1000),
+       k=st.integers(1, 4096), Hq=st.sampled_from([1, 2, 4, 8, 16, 32, 64, 128, 12, 48]),
+       d=st.sampled_from([64, 128]), B=st.integers(1, 3), rpc=st.sampled_from([0, 1, 200]))
+def test_layer_stack_dense_rows_rule_and_own_workspace(ic, Lq, q0, extra, k, Hq, d, B, rpc):
+    """The rule as stated (rows t < 8k, at most 65536 visible keys, whole
+    blocks of 128/Hq queries, d = 128) holds on random shapes, and the size
+    the workspace query returns always lets the stack take the dense path,
+    whatever the score chunking."""
+    Lk = q0 + Lq + extra
+    k = min(k, Lk)
+    dims = ic.make_dims(B, Lq, Lk, q0, 32, 128, Hq, d, k)
+    if d != 128 or 128 % Hq:
+        want = 0
+    else:
+        qbd = 128 // Hq
+        lim = min(8 * k - q0, 65536 - q0, Lq)
+        want = lim // qbd * qbd if lim >= qbd else 0
+    ws = ic.layer_stack_workspace_bytes(dims, 2, rpc)
+    assert ws > 0
+    assert ic.layer_stack_dense_rows(dims, ws) == want
+    assert ic.layer_stack_dense_rows(dims, 0) == 0
+    # a smaller score chunk never asks for more workspace
+    if rpc:
+        assert ws <= ic.layer_stack_workspace_bytes(dims, 2, 0)
 
 
 def test_unique_attention_rejects_bad_arguments_before_launch(ic):
