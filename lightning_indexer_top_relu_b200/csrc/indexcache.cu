@@ -67,18 +67,23 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-EncodeTiledFn g_encode = nullptr;
+// Looked up once; host threads may race on the first lookup (they store the
+// same pointer), so the slot is atomic.
+std::atomic<EncodeTiledFn> g_encode_fn{nullptr};
 
 int get_encode() {
-    if (g_encode) return IC_OK;
+    if (g_encode_fn.load(std::memory_order_acquire)) return IC_OK;
     void* fn = nullptr;
     cudaDriverEntryPointQueryResult q;
     cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
     if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
         return fail(IC_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
-    g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    g_encode_fn.store(reinterpret_cast<EncodeTiledFn>(fn), std::memory_order_release);
     return IC_OK;
 }
+
+// Valid after get_encode() returned IC_OK.
+EncodeTiledFn encoder() { return g_encode_fn.load(std::memory_order_acquire); }
 
 // 3-D bf16 tensor {d0 (contiguous), d1, d2}, 128-byte swizzled boxes {64, box1, 1}.
 int make_tmap_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
@@ -89,7 +94,7 @@ int make_tmap_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uin
     cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
     cuuint32_t box[3] = {64, box1, 1};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+    CUresult r = encoder()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -375,7 +380,7 @@ int launch_dense_attn(const DenseGeom& g, const ic_dims& D, const ic_layer& L,
         cuuint64_t strides[2] = {(cuuint64_t)g.ldt * 2, (cuuint64_t)g.ldt * 2 * 128};
         cuuint32_t box[3] = {64, 128, 1};
         cuuint32_t estr[3] = {1, 1, 1};
-        CUresult r = g_encode(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, vt, dims, strides, box, estr,
+        CUresult r = encoder()(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, vt, dims, strides, box, estr,
                               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return fail(IC_ERR_CUDA, "cuTensorMapEncodeTiled (V^T) failed (%d)", (int)r);
