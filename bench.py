@@ -223,13 +223,22 @@ def _oracle_rows(wl, pattern, sl, workers):
     return time.perf_counter() - t0
 
 
+def host_cores() -> int:
+    """Host cores this process may run on.  The oracle legs run one row per
+    core with one OpenMP thread each, so a launcher's OMP_NUM_THREADS (torchrun
+    sets 1) does not shrink the pool."""
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:
+        return max(1, os.cpu_count() or 1)
+
+
 def oracle_rows_per_s(wl, pattern, layers, budget_s=15.0, seed=5):
     """Times the oracle on uniformly drawn query rows, one row per host core,
     for about budget_s seconds; returns (rows/s, sample description, cores)."""
-    import oracle
     rng = np.random.default_rng(seed)
     total = wl.B * wl.Lq
-    workers = max(1, oracle.num_threads())
+    workers = host_cores()
     elapsed, done, n = 0.0, 0, workers
     while elapsed < budget_s and done < total:
         rows = rng.choice(total, size=min(n, total), replace=False)
@@ -258,25 +267,26 @@ def run_reference(args, wl, pattern):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    import oracle
     big = input_bytes(wl, True) > 2 * 2 ** 30
     dev = torch.device("cuda") if (big and torch.cuda.is_available()) else "cpu"
     layers = synth.make_layers(wl, indexer_for_all=any(c in "F1" for c in pattern), device=dev)
     total = wl.B * wl.Lq
     rng = np.random.default_rng(11)
     n_rows = max(1, min(total, args.ref_rows))
-    workers = max(1, oracle.num_threads())
+    workers = host_cores()
     times = []
-    for s in range(args.steps):
+    for s in range(args.warmup + args.steps):
         rows = rng.choice(total, size=n_rows, replace=False)
         sl = [row_slice(wl, layers, r) for r in rows]
-        times.append(_oracle_rows(wl, pattern, sl, workers))
+        dt = _oracle_rows(wl, pattern, sl, workers)
+        if s >= args.warmup:                       # warm-up steps are not timed
+            times.append(dt)
     sec = float(np.sum(times))
     value = n_rows * args.steps / sec
     sample = (f"{n_rows} uniformly drawn query rows of {total} per step, each through all "
-              f"{len(pattern)} layers")
+              f"{len(pattern)} layers, on {workers} host cores (no GPU work)")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
-            "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * sec / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_of(wl, pattern, args),
@@ -688,7 +698,7 @@ def main():
 
     # ---- CPU oracle baseline (rank 0, N=1 only)
     if not args.no_cpu_baseline and world == 1:
-        import oracle
+        import oracle  # noqa: F401  (built and loaded before its timed sample)
         rps, sample, cores = oracle_rows_per_s(wl, pattern, layers, budget_s=args.cpu_budget_s)
         line["cpu_baseline"] = {"value": rps, "unit": "tokens/s", "cores": cores,
                                 "kind": "oracle", "sample": sample}

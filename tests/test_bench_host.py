@@ -62,3 +62,50 @@ def test_input_bytes_and_device_drawing_threshold():
     assert bench.input_bytes(wl, True) == 8 * per_layer_attn + 8 * per_f_idx
     assert bench.input_bytes(wl, True) < 2 * 2 ** 30                       # drawn on the host
     assert bench.input_bytes(synth.WORKLOADS["prefill_64k"], True) > 2 * 2 ** 30
+
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _json_lines(out):
+    import json
+    return [json.loads(l) for l in out.splitlines() if l.startswith("{")]
+
+
+def test_reference_arm_prints_one_line_with_its_baseline():
+    """bench.py --impl reference: the oracle on host cores, W untimed
+    warm-up steps, the same metric and config keys as the GPU arm, and
+    cpu_baseline / e2e objects describing the run."""
+    import subprocess
+    import sys
+    env = dict(os.environ, OMP_NUM_THREADS="1")      # what torchrun sets; must not shrink the pool
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload",
+                        "tiny_prefill", "--steps", "2", "--warmup", "1", "--ref-rows", "4"],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = _json_lines(r.stdout)
+    assert len(lines) == 1
+    ln = lines[0]
+    assert ln["impl"] == "reference" and ln["metric"] == bench.METRIC
+    assert ln["unit"] == "tokens/s" and ln["higher_is_better"] is True and ln["value"] > 0
+    assert ln["steps"] == 2 and ln["warmup"] == 1 and ln["n_gpus"] == 1
+    assert ln["config"]["workload"] == "tiny_prefill"
+    assert ln["cpu_baseline"]["kind"] == "oracle"
+    assert ln["cpu_baseline"]["cores"] == bench.host_cores()
+    assert ln["cpu_baseline"]["value"] == ln["value"]
+    assert ln["e2e"] == {"value": ln["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                         "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_under_two_ranks_prints_from_rank_0_only():
+    import subprocess
+    import sys
+    r = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+                        "--nproc-per-node", "2", "--master-addr", "127.0.0.1",
+                        "--master-port", "29571", "bench.py", "--impl", "reference", "--gpus",
+                        "2", "--workload", "tiny_prefill", "--steps", "1", "--warmup", "1",
+                        "--ref-rows", "2"],
+                       cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = _json_lines(r.stdout)
+    assert len(lines) == 1 and lines[0]["impl"] == "reference" and lines[0]["n_gpus"] == 2
