@@ -32,8 +32,13 @@
  *     Prefill: q_offset = 0, Lq = Lk.  Decode: Lq = 1, q_offset = Lk - 1.
  *   - Supported shapes: d_I in {64, 128}; H_I a power of two in [4, 128];
  *     d in {64, 128}; Hq in {8, 16}; Hkv == 1 (MQA); 1 <= k <= Lk.  Other
- *     shapes return IC_ERR_UNSUPPORTED.  bf16 buffers must be 16-byte
- *     aligned (IC_ERR_UNSUPPORTED otherwise).
+ *     shapes return IC_ERR_UNSUPPORTED.  Alignment:
+ *       - bf16 buffers, the indexer's head weights w and every workspace
+ *         must be 16-byte aligned: kernels read them with 16-byte vector,
+ *         bulk or TMA copies;
+ *       - the other fp32 / int32 buffers (scores, idx, lse, counts) must be
+ *         4-byte aligned.
+ *     A misaligned pointer returns IC_ERR_UNSUPPORTED before any launch.
  *   - Device-side faults are never raised on purpose: kernels report an
  *     out-of-range attention index or a timed-out wait into a device error
  *     word that ic_get_last_device_error() reads.

@@ -50,6 +50,8 @@ int launched(cudaError_t e, const char* what) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// fp32 / int32 buffers read and written element by element
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 
 // ---------------------------------------------------------------- device facts
@@ -611,8 +613,9 @@ int ic_indexer_scores(const uint16_t* q_idx, const uint16_t* k_idx, const float*
     if ((rc = check_indexer_shape(H_I, d_I))) return rc;
     if (B == 0 || Lq == 0) return IC_OK;
     if (!q_idx || !k_idx || !w || !scores) return fail(IC_ERR_INVALID_ARG, "null pointer");
-    if (!aligned16(q_idx) || !aligned16(k_idx))
-        return fail(IC_ERR_UNSUPPORTED, "q_idx and k_idx must be 16-byte aligned");
+    if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(w))
+        return fail(IC_ERR_UNSUPPORTED, "q_idx, k_idx and w must be 16-byte aligned");
+    if (!aligned4(scores)) return fail(IC_ERR_UNSUPPORTED, "scores must be 4-byte aligned");
     if ((long long)Lq * H_I > (1LL << 31)) return fail(IC_ERR_UNSUPPORTED, "Lq*H_I too large");
     int dev, sms;
     if ((rc = device_setup(&dev, &sms))) return rc;
@@ -629,6 +632,8 @@ int ic_topk_select(const float* scores, int B, int Lq, int Lk, int q_offset, int
     if (k < 1) return fail(IC_ERR_INVALID_ARG, "k=%d", k);
     if (B == 0 || Lq == 0) return IC_OK;
     if (!scores || !idx) return fail(IC_ERR_INVALID_ARG, "null pointer");
+    if (!aligned4(scores) || !aligned4(idx))
+        return fail(IC_ERR_UNSUPPORTED, "scores and idx must be 4-byte aligned");
     int dev, sms;
     if ((rc = device_setup(&dev, &sms))) return rc;
     return launch_topk(scores, Lk, 0, (long long)B * Lq, Lq, Lk, q_offset, k, idx, sms,
@@ -653,9 +658,12 @@ int ic_sparse_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, cons
     if (k_slots < 1) return fail(IC_ERR_INVALID_ARG, "k=%d", k_slots);
     if (B == 0 || Lq == 0) return IC_OK;
     if (!q || !k || !v || !idx || !out) return fail(IC_ERR_INVALID_ARG, "null pointer");
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v))
-        return fail(IC_ERR_UNSUPPORTED, "q, k and v must be 16-byte aligned");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+        return fail(IC_ERR_UNSUPPORTED, "q, k, v and out must be 16-byte aligned");
+    if (!aligned4(idx) || (lse && !aligned4(lse)))
+        return fail(IC_ERR_UNSUPPORTED, "idx and lse must be 4-byte aligned");
     if (!std::isfinite(scale)) return fail(IC_ERR_INVALID_ARG, "scale is not finite");
+    if (ws && !aligned16(ws)) return fail(IC_ERR_UNSUPPORTED, "ws must be 16-byte aligned");
     int dev, sms;
     if ((rc = device_setup(&dev, &sms))) return rc;
     return launch_attn(q, k, v, idx, B, Lq, Lk, Hq, d, k_slots, q_offset, scale, out, lse, ws,
@@ -672,8 +680,10 @@ int ic_sparse_attn_no_alloc(const uint16_t* q, const uint16_t* k, const uint16_t
     if (k_slots < 1) return fail(IC_ERR_INVALID_ARG, "k=%d", k_slots);
     if (B == 0 || Lq == 0) return IC_OK;
     if (!q || !k || !v || !idx || !out) return fail(IC_ERR_INVALID_ARG, "null pointer");
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v))
-        return fail(IC_ERR_UNSUPPORTED, "q, k and v must be 16-byte aligned");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+        return fail(IC_ERR_UNSUPPORTED, "q, k, v and out must be 16-byte aligned");
+    if (!aligned4(idx) || (lse && !aligned4(lse)))
+        return fail(IC_ERR_UNSUPPORTED, "idx and lse must be 4-byte aligned");
     if (!std::isfinite(scale)) return fail(IC_ERR_INVALID_ARG, "scale is not finite");
     int dev, sms;
     if ((rc = device_setup(&dev, &sms))) return rc;
@@ -708,10 +718,13 @@ int ic_sparse_attn_unique(const uint16_t* q, const uint16_t* k, const uint16_t* 
     if (k_slots < 1) return fail(IC_ERR_INVALID_ARG, "k=%d", k_slots);
     if (B == 0 || Lq == 0) return IC_OK;
     if (!q || !k || !v || !idx || !out) return fail(IC_ERR_INVALID_ARG, "null pointer");
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v))
-        return fail(IC_ERR_UNSUPPORTED, "q, k and v must be 16-byte aligned");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+        return fail(IC_ERR_UNSUPPORTED, "q, k, v and out must be 16-byte aligned");
+    if (!aligned4(idx) || (lse && !aligned4(lse)))
+        return fail(IC_ERR_UNSUPPORTED, "idx and lse must be 4-byte aligned");
     if (!std::isfinite(scale)) return fail(IC_ERR_INVALID_ARG, "scale is not finite");
     if (ws_bytes > 0 && !ws) return fail(IC_ERR_INVALID_ARG, "ws is NULL but ws_bytes > 0");
+    if (ws && !aligned16(ws)) return fail(IC_ERR_UNSUPPORTED, "ws must be 16-byte aligned");
     int dev, sms;
     if ((rc = device_setup(&dev, &sms))) return rc;
     ic_dims D{};
@@ -732,6 +745,8 @@ int ic_index_overlap(const int32_t* idx_a, const int32_t* idx_b, long long n_row
         return fail(IC_ERR_UNSUPPORTED, "Lk=%d (supported: 1..%d)", Lk, ic::OV_MAX_LK);
     if (n_rows == 0) return IC_OK;
     if (!idx_a || !idx_b || !counts) return fail(IC_ERR_INVALID_ARG, "null pointer");
+    if (!aligned4(idx_a) || !aligned4(idx_b) || !aligned4(counts))
+        return fail(IC_ERR_UNSUPPORTED, "idx_a, idx_b and counts must be 4-byte aligned");
     int dev, sms;
     int rc = device_setup(&dev, &sms);
     if (rc) return rc;
@@ -817,15 +832,20 @@ static int stack_forward(const char* pattern, int n_layers, const ic_layer* laye
         const bool full = pattern[l] == 'F' || pattern[l] == '1';
         if (!L.q || !L.k || !L.v || !L.out)
             return fail(IC_ERR_INVALID_ARG, "layer %d: null q/k/v/out", l);
-        if (!aligned16(L.q) || !aligned16(L.k) || !aligned16(L.v))
-            return fail(IC_ERR_UNSUPPORTED, "layer %d: q, k, v must be 16-byte aligned", l);
+        if (!aligned16(L.q) || !aligned16(L.k) || !aligned16(L.v) || !aligned16(L.out))
+            return fail(IC_ERR_UNSUPPORTED, "layer %d: q, k, v, out must be 16-byte aligned", l);
+        if (L.lse && !aligned4(L.lse))
+            return fail(IC_ERR_UNSUPPORTED, "layer %d: lse must be 4-byte aligned", l);
         if (full) {
             if (!L.q_idx || !L.k_idx || !L.w)
                 return fail(IC_ERR_INVALID_ARG, "layer %d is F but q_idx/k_idx/w is null", l);
-            if (!aligned16(L.q_idx) || !aligned16(L.k_idx))
-                return fail(IC_ERR_UNSUPPORTED, "layer %d: q_idx, k_idx must be 16-byte aligned", l);
+            if (!aligned16(L.q_idx) || !aligned16(L.k_idx) || !aligned16(L.w))
+                return fail(IC_ERR_UNSUPPORTED, "layer %d: q_idx, k_idx, w must be 16-byte aligned",
+                            l);
         }
     }
+    if (!aligned4(idx_cache)) return fail(IC_ERR_UNSUPPORTED, "idx_cache must be 4-byte aligned");
+    if (ws && !aligned16(ws)) return fail(IC_ERR_UNSUPPORTED, "ws must be 16-byte aligned");
     if (D.B == 0 || D.Lq == 0) return IC_OK;
     if ((long long)D.Lq * D.H_I > (1LL << 31)) return fail(IC_ERR_UNSUPPORTED, "Lq*H_I too large");
     int dev, sms;

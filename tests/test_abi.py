@@ -222,3 +222,65 @@ def test_unique_attention_workspace_query(ic):
     assert q(1, 700, 700, 0, 16, 128, 96) > 700 * 12 * 4        # bitmask + V^T at least
     assert q(0, 700, 700, 0, 16, 128, 96) == 0
     assert q(1, 700, 600, 0, 16, 128, 96) == 0                  # q_offset + Lq > Lk
+
+
+def test_misaligned_buffers_are_rejected_before_launch(ic):
+    """Every buffer a kernel reads with vector, bulk or TMA copies must be
+    16-byte aligned (bf16 tensors, w, the workspaces), every fp32 / int32
+    buffer 4-byte aligned: otherwise IC_ERR_UNSUPPORTED (2), not a device fault."""
+    lib = ic.lib()
+    before = ic.kernel_launch_count()
+    U = 2
+
+    def indexer(**kw):
+        a = dict(q=0x1000, k=0x2000, w=0x3000, s=0x4000)
+        a.update(kw)
+        return lib.ic_indexer_scores(a["q"], a["k"], a["w"], 1, 64, 64, 4, 64, 0, a["s"], None)
+    assert indexer(w=0x3004) == U                # head weights feed a 16-byte bulk copy
+    assert indexer(s=0x4002) == U
+    assert indexer(q=0x1008) == U
+
+    def topk(**kw):
+        a = dict(s=0x1000, i=0x2000)
+        a.update(kw)
+        return lib.ic_topk_select(a["s"], 1, 64, 64, 0, 8, a["i"], None)
+    assert topk(s=0x1002) == U and topk(i=0x2001) == U
+
+    attn_ok = dict(q=0x1000, k=0x2000, v=0x3000, idx=0x4000, out=0x5000, lse=None, ws=None, wsb=0)
+
+    def attn(f, with_ws, **kw):
+        a = dict(attn_ok)
+        a.update(kw)
+        head = (a["q"], a["k"], a["v"], a["idx"], 1, 64, 64, 16, 1, 128, 32, 0, 0.0, a["out"],
+                a["lse"])
+        return f(*head, a["ws"], a["wsb"], None) if with_ws else f(*head, None)
+    for f, with_ws in ((lib.ic_sparse_attn, True), (lib.ic_sparse_attn_unique, True),
+                       (lib.ic_sparse_attn_no_alloc, False)):
+        assert attn(f, with_ws, out=0x5008) == U     # the dense-masked kernel stores 16 bytes
+        assert attn(f, with_ws, idx=0x4002) == U
+        assert attn(f, with_ws, lse=0x6002) == U
+        if with_ws:
+            assert attn(f, with_ws, ws=0x7008, wsb=1 << 16) == U
+
+    assert lib.ic_index_overlap(0x1000, 0x2000, 4, 8, 100, 0x3002, None) == U
+    assert lib.ic_index_overlap(0x1001, 0x2000, 4, 8, 100, 0x3000, None) == U
+
+    d = _dims(ic)
+    layer = dict(q=0x1000, k=0x2000, v=0x3000, q_idx=0x4000, k_idx=0x5000, w=0x6000, out=0x7000,
+                 lse=None)
+
+    def stack(idx_cache=0x8000, ws=0x9000, **kw):
+        a = dict(layer)
+        a.update(kw)
+        table = (ic.ICLayer * 2)()
+        for i in range(2):
+            table[i] = ic.ICLayer(a["q"], a["k"], a["v"], a["q_idx"], a["k_idx"], a["w"], a["out"],
+                                  a["lse"], None)
+        return lib.ic_layer_stack_forward(b"FS", 2, table, ctypes.byref(d), idx_cache, ws, 1 << 20,
+                                          None)
+    assert stack(w=0x6004) == U
+    assert stack(out=0x7008) == U
+    assert stack(lse=0x8002) == U
+    assert stack(idx_cache=0x8002) == U
+    assert stack(ws=0x9008) == U
+    assert ic.kernel_launch_count() == before
