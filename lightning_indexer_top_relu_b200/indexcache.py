@@ -131,6 +131,34 @@ def _ptr(t: Optional[torch.Tensor], dtype=None, name="tensor") -> Optional[int]:
     return t.data_ptr()
 
 
+def _expect(t: Optional[torch.Tensor], shape, name: str) -> None:
+    """A caller tensor must have exactly the shape the call derives from its
+    leading operand: the C layer sees only pointers and sizes, so a smaller
+    tensor would let a kernel read or write past its end."""
+    if t is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _dims_of(t: torch.Tensor, n: int, name: str):
+    if t.dim() != n:
+        raise ValueError(f"{name} must have {n} dimensions, got shape {tuple(t.shape)}")
+    return tuple(t.shape)
+
+
+def _kv_shapes(q, k, v):
+    """(B, Lq, Hq, d, Lk, Hkv) of an attention call: q [B,Lq,Hq,d]; k and v
+    [B,Lk,Hkv,d] or [B,Lk,d] (one KV head), both the same."""
+    B, Lq, Hq, d = _dims_of(q, 4, "q")
+    if k.dim() == 4:
+        Lk, Hkv = k.shape[1], k.shape[2]
+        _expect(k, (B, Lk, Hkv, d), "k")
+    else:
+        Lk, Hkv = _dims_of(k, 3, "k")[1], 1
+        _expect(k, (B, Lk, d), "k")
+    _expect(v, tuple(k.shape), "v")
+    return B, Lq, Hq, d, Lk, Hkv
+
+
 def _stream(stream) -> Optional[int]:
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -151,6 +179,7 @@ def index_overlap(idx_a, idx_b, Lk: int, counts=None, stream=None):
     n_rows = idx_a.numel() // k
     if counts is None:
         counts = torch.empty(n_rows, 3, device=idx_a.device, dtype=torch.int32)
+    _expect(counts, (n_rows, 3), "counts")
     rc = _lib.ic_index_overlap(_ptr(idx_a, torch.int32, "idx_a"), _ptr(idx_b, torch.int32, "idx_b"),
                                n_rows, k, int(Lk), _ptr(counts, torch.int32, "counts"),
                                _stream(stream))
@@ -170,10 +199,13 @@ def selftest_wait_timeout(timeout_us: int = 20000, stream=None) -> None:
 
 def indexer_scores(q_idx, k_idx, w, q_offset: int = 0, out=None, stream=None) -> torch.Tensor:
     """scores [B,Lq,Lk] fp32 from q_idx [B,Lq,H_I,d_I] bf16, k_idx [B,Lk,d_I] bf16, w [B,Lq,H_I] fp32."""
-    B, Lq, H, dI = q_idx.shape
-    Lk = k_idx.shape[1]
+    B, Lq, H, dI = _dims_of(q_idx, 4, "q_idx")
+    Lk = _dims_of(k_idx, 3, "k_idx")[1]
+    _expect(k_idx, (B, Lk, dI), "k_idx")
+    _expect(w, (B, Lq, H), "w")
     if out is None:
         out = torch.empty(B, Lq, Lk, device=q_idx.device, dtype=torch.float32)
+    _expect(out, (B, Lq, Lk), "out")
     rc = _lib.ic_indexer_scores(_ptr(q_idx, torch.bfloat16, "q_idx"), _ptr(k_idx, torch.bfloat16, "k_idx"),
                                 _ptr(w, torch.float32, "w"), B, Lq, Lk, H, dI, q_offset,
                                 _ptr(out, torch.float32, "scores"), _stream(stream))
@@ -183,9 +215,10 @@ def indexer_scores(q_idx, k_idx, w, q_offset: int = 0, out=None, stream=None) ->
 
 def topk_select(scores, k: int, q_offset: int = 0, out=None, stream=None) -> torch.Tensor:
     """idx [B,Lq,k] int32 (ascending positions, -1 padded) from scores [B,Lq,Lk] fp32."""
-    B, Lq, Lk = scores.shape
+    B, Lq, Lk = _dims_of(scores, 3, "scores")
     if out is None:
         out = torch.empty(B, Lq, k, device=scores.device, dtype=torch.int32)
+    _expect(out, (B, Lq, k), "out")
     rc = _lib.ic_topk_select(_ptr(scores, torch.float32, "scores"), B, Lq, Lk, q_offset, k,
                              _ptr(out, torch.int32, "idx"), _stream(stream))
     _check(rc, "ic_topk_select")
@@ -199,14 +232,15 @@ def sparse_attn_workspace_bytes(B: int, Lq: int, Hq: int, d: int, k: int) -> int
 def sparse_attn(q, k, v, idx, q_offset: int = 0, scale: float = 0.0, out=None, lse=None,
                 want_lse: bool = True, ws=None, stream=None):
     """(out [B,Lq,Hq,d] bf16, lse [B,Lq,Hq] fp32) over the positions in idx [B,Lq,k] int32."""
-    B, Lq, Hq, d = q.shape
-    Lk = k.shape[1]
-    Hkv = k.shape[2] if k.dim() == 4 else 1
-    kslots = idx.shape[-1]
+    B, Lq, Hq, d, Lk, Hkv = _kv_shapes(q, k, v)
+    kslots = _dims_of(idx, 3, "idx")[2]
+    _expect(idx, (B, Lq, kslots), "idx")
     if out is None:
         out = torch.empty_like(q)
     if lse is None and want_lse:
         lse = torch.empty(B, Lq, Hq, device=q.device, dtype=torch.float32)
+    _expect(out, (B, Lq, Hq, d), "out")
+    _expect(lse, (B, Lq, Hq), "lse")
     if ws is None:
         nbytes = sparse_attn_workspace_bytes(B, Lq, Hq, d, kslots)
         ws = torch.empty(max(nbytes, 1), device=q.device, dtype=torch.uint8) if nbytes else None
@@ -231,14 +265,15 @@ def sparse_attn_unique(q, k, v, idx, q_offset: int = 0, scale: float = 0.0, out=
     that hold each position at most once (dense-masked rows t < 8k when the
     workspace allows, gathered rows otherwise).  ws=None allocates the full
     workspace; pass an empty tensor to force the gather path."""
-    B, Lq, Hq, d = q.shape
-    Lk = k.shape[1]
-    Hkv = k.shape[2] if k.dim() == 4 else 1
-    kslots = idx.shape[-1]
+    B, Lq, Hq, d, Lk, Hkv = _kv_shapes(q, k, v)
+    kslots = _dims_of(idx, 3, "idx")[2]
+    _expect(idx, (B, Lq, kslots), "idx")
     if out is None:
         out = torch.empty_like(q)
     if lse is None and want_lse:
         lse = torch.empty(B, Lq, Hq, device=q.device, dtype=torch.float32)
+    _expect(out, (B, Lq, Hq, d), "out")
+    _expect(lse, (B, Lq, Hq), "lse")
     if ws is None:
         nbytes = sparse_attn_unique_workspace_bytes(B, Lq, Lk, q_offset, Hq, d, kslots)
         ws = torch.empty(max(nbytes, 1), device=q.device, dtype=torch.uint8) if nbytes else None
@@ -261,14 +296,15 @@ def sparse_attn_no_alloc(q, k, v, idx, q_offset: int = 0, scale: float = 0.0, ou
     include/indexcache.h): split partials live in the library's fixed 4 MiB
     device array; calls that overlap on the GPU race on it.
     """
-    B, Lq, Hq, d = q.shape
-    Lk = k.shape[1]
-    Hkv = k.shape[2] if k.dim() == 4 else 1
-    kslots = idx.shape[-1]
+    B, Lq, Hq, d, Lk, Hkv = _kv_shapes(q, k, v)
+    kslots = _dims_of(idx, 3, "idx")[2]
+    _expect(idx, (B, Lq, kslots), "idx")
     if out is None:
         out = torch.empty_like(q)
     if lse is None and want_lse:
         lse = torch.empty(B, Lq, Hq, device=q.device, dtype=torch.float32)
+    _expect(out, (B, Lq, Hq, d), "out")
+    _expect(lse, (B, Lq, Hq), "lse")
     rc = _lib.ic_sparse_attn_no_alloc(_ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
                                       _ptr(v, torch.bfloat16, "v"), _ptr(idx, torch.int32, "idx"),
                                       B, Lq, Lk, Hq, Hkv, d, kslots, q_offset, float(scale),
@@ -303,6 +339,18 @@ class LayerStack:
         self.pattern = pattern
         self.dims = dims
         n = len(layers)
+        d = dims
+        for i, L in enumerate(layers):
+            _expect(L["q"], (d.B, d.Lq, d.Hq, d.d), f"layer {i} q")
+            kv = (d.B, d.Lk, d.Hkv, d.d) if L["k"].dim() == 4 else (d.B, d.Lk, d.d)
+            _expect(L["k"], kv, f"layer {i} k")
+            _expect(L["v"], kv, f"layer {i} v")
+            if i < len(pattern) and pattern[i] in "F1":
+                for name, shape in (("q_idx", (d.B, d.Lq, d.H_I, d.d_I)),
+                                    ("k_idx", (d.B, d.Lk, d.d_I)), ("w", (d.B, d.Lq, d.H_I))):
+                    if L.get(name) is None:
+                        raise ValueError(f"layer {i} is a full layer but has no {name}")
+                    _expect(L[name], shape, f"layer {i} {name}")
         dev = layers[0]["q"].device
         self.layers = list(layers)
         self.outs = [torch.empty_like(L["q"]) for L in layers]

@@ -284,3 +284,57 @@ def test_misaligned_buffers_are_rejected_before_launch(ic):
     assert stack(idx_cache=0x8002) == U
     assert stack(ws=0x9008) == U
     assert ic.kernel_launch_count() == before
+
+
+def test_binding_rejects_inconsistent_shapes_before_the_library(ic):
+    """The C layer sees pointers and sizes only, so the binding checks every
+    tensor against the sizes it derives from the leading operand; these CPU
+    tensors never reach the library (a consistent call fails later, on the
+    device check)."""
+    import torch
+    bf, f32, i32 = torch.bfloat16, torch.float32, torch.int32
+    q_idx, k_idx, w = (torch.zeros(1, 8, 4, 64, dtype=bf), torch.zeros(1, 8, 64, dtype=bf),
+                       torch.zeros(1, 8, 4, dtype=f32))
+    with pytest.raises(ValueError, match="CUDA"):
+        ic.indexer_scores(q_idx, k_idx, w)
+    with pytest.raises(ValueError, match="k_idx has shape"):
+        ic.indexer_scores(q_idx, torch.zeros(1, 8, 32, dtype=bf), w)
+    with pytest.raises(ValueError, match="k_idx has shape"):
+        ic.indexer_scores(q_idx, torch.zeros(2, 8, 64, dtype=bf), w)
+    with pytest.raises(ValueError, match="w has shape"):
+        ic.indexer_scores(q_idx, k_idx, torch.zeros(1, 8, 2, dtype=f32))
+    with pytest.raises(ValueError, match="out has shape"):
+        ic.indexer_scores(q_idx, k_idx, w, out=torch.zeros(1, 8, 7, dtype=f32))
+    with pytest.raises(ValueError, match="3 dimensions"):
+        ic.topk_select(torch.zeros(8, 8, dtype=f32), 4)
+    with pytest.raises(ValueError, match="out has shape"):
+        ic.topk_select(torch.zeros(1, 8, 8, dtype=f32), 4, out=torch.zeros(1, 8, 3, dtype=i32))
+
+    q, kv = torch.zeros(1, 8, 16, 128, dtype=bf), torch.zeros(1, 8, 1, 128, dtype=bf)
+    idx = torch.zeros(1, 8, 4, dtype=i32)
+    for f in (ic.sparse_attn, ic.sparse_attn_unique, ic.sparse_attn_no_alloc):
+        with pytest.raises(ValueError, match="CUDA"):
+            f(q, kv, kv, idx)
+        with pytest.raises(ValueError, match="v has shape"):
+            f(q, kv, torch.zeros(1, 9, 1, 128, dtype=bf), idx)
+        with pytest.raises(ValueError, match="k has shape"):
+            f(q, torch.zeros(1, 8, 1, 64, dtype=bf), kv, idx)
+        with pytest.raises(ValueError, match="idx has shape"):
+            f(q, kv, kv, torch.zeros(1, 7, 4, dtype=i32))
+        with pytest.raises(ValueError, match="out has shape"):
+            f(q, kv, kv, idx, out=torch.zeros(1, 8, 8, 128, dtype=bf))
+        with pytest.raises(ValueError, match="lse has shape"):
+            f(q, kv, kv, idx, lse=torch.zeros(1, 8, 8, dtype=f32))
+    with pytest.raises(ValueError, match="counts has shape"):
+        ic.index_overlap(idx, idx, 8, counts=torch.zeros(7, 3, dtype=i32))
+
+    dims = ic.make_dims(1, 8, 8, 0, 4, 64, 16, 128, 4)
+    full = {"q": q, "k": kv, "v": kv, "q_idx": q_idx, "k_idx": k_idx, "w": w}
+    with pytest.raises(ValueError, match="layer 1 w has shape"):
+        ic.LayerStack("FF", [full, dict(full, w=torch.zeros(1, 8, 8, dtype=f32))], dims)
+    with pytest.raises(ValueError, match="has no k_idx"):
+        ic.LayerStack("FF", [full, {n: t for n, t in full.items() if n != "k_idx"}], dims)
+    with pytest.raises(ValueError, match="layer 0 q has shape"):
+        ic.LayerStack("F", [dict(full, q=torch.zeros(1, 8, 8, 128, dtype=bf))], dims)
+    with pytest.raises(ValueError, match="CUDA"):             # S layers need no indexer inputs
+        ic.LayerStack("FS", [full, {"q": q, "k": kv, "v": kv}], dims)
