@@ -8,6 +8,7 @@ import socket
 
 import numpy as np
 import pytest
+from hypothesis import given, settings, strategies as st
 import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
@@ -25,6 +26,23 @@ def test_zigzag_chunks_cover_every_row_once(Lq, world):
             assert n > 0 and (i0 % 128 == 0)
             rows.extend(range(i0, i0 + n))
     assert sorted(rows) == list(range(Lq))
+
+
+@settings(max_examples=300, deadline=None)
+@given(B=st.integers(1, 40), Lq=st.integers(1, 20000), world=st.integers(1, 16),
+       align=st.sampled_from([1, 8, 64, 128]))
+def test_shards_partition_the_rows_of_every_sequence(B, Lq, world, align):
+    """Over all ranks every (sequence, row) pair is covered exactly once, each
+    chunk lies inside the problem, and row chunks start on `align` rows."""
+    seen = np.zeros((B, Lq), dtype=np.int32)
+    for r in range(world):
+        for ch in sharding.shard(B, Lq, world, r, align):
+            assert ch.nb > 0 and ch.n > 0
+            assert 0 <= ch.b0 and ch.b0 + ch.nb <= B and 0 <= ch.i0 and ch.i0 + ch.n <= Lq
+            if B == 1:
+                assert ch.i0 % align == 0
+            seen[ch.b0:ch.b0 + ch.nb, ch.i0:ch.i0 + ch.n] += 1
+    assert np.all(seen == 1)
 
 
 @pytest.mark.parametrize("world", [2, 4, 8])
