@@ -99,6 +99,26 @@ MUTANTS = [
        "return np.asarray(counts)[:, 0] / np.asarray(counts)[:, 1]")]),
     ("jaccard_over_the_sum", "__init__.py",
      [("c[:, 0] / (c[:, 1] + c[:, 2] - c[:, 0] + 1e-8)", "c[:, 0] / (c[:, 1] + c[:, 2] + 1e-8)")]),
+    ("bf16_sign_dropped", "oracle.c",
+     [("uint32_t u = ((uint32_t)h) << 16;", "uint32_t u = ((uint32_t)(h & 0x7fffu)) << 16;")]),
+    ("count_form_off_by_one", "oracle.c",
+     [("if (beat < k) o[m++] = (int32_t)s;", "if (beat <= k && m < k) o[m++] = (int32_t)s;")]),
+    ("softmax_in_base_2", "oracle.c",
+     [("double e = exp(z[i] - m);", "double e = exp2(z[i] - m);")]),
+    ("default_scale_over_d", "oracle.c",
+     [("if (scale <= 0.0) scale = 1.0 / sqrt((double)d);",
+       "if (scale <= 0.0) scale = 1.0 / (double)d;", 2)]),
+    ("dense_attention_without_the_query_position", "oracle.c",
+     [("for (int64_t s = 0; s <= t; ++s) all[s] = (int32_t)s;",
+       "for (int64_t s = 0; s <= t; ++s) all[s] = (int32_t)(s < t ? s : -1);")]),
+    ("overlap_ignores_bad_entries", "oracle.c",
+     [("else if (x != -1) rc = rc < -2 ? rc : -2;", ""),
+      ("else if (y != -1) rc = rc < -2 ? rc : -2;", "")]),
+    ("row_positions_of_the_sequence_index", "__init__.py",
+     [("return (r % Lq) + q_offset", "return (r // Lq) + q_offset")]),
+    ("stack_attention_ignores_the_row_sample", "__init__.py",
+     [('o, lse = sparse_attn(L["q"], L["k"], L["v"], cached, q_offset, scale, rows)',
+       'o, lse = sparse_attn(L["q"], L["k"], L["v"], cached, q_offset, scale)')]),
     # ---- a3 / a5 layer stack
     ("shared_layers_keep_the_first_full_layer", "__init__.py",
      [("            cached = topk_sort(sc.astype(np.float32), row_positions(B, Lq, q_offset, rows), k)",

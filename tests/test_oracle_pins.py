@@ -284,6 +284,21 @@ def test_stack_shared_layers_reuse_nearest_full_layer():
     assert np.array_equal(o2, outs[2])
 
 
+def test_stack_on_sampled_rows_equals_the_full_stack_there():
+    """The layer loop on a row sample (what the full-size checks use) gives,
+    row for row, the full run's indices, outputs and log-sum-exps."""
+    wl = synth.custom(B=2, Lq=40, Lk=60, q_offset=20, n_layers=3, H_I=2, d_I=64, k=8, Hq=2,
+                      d=64, pattern="FSF")
+    layers = synth.make_layers(wl)
+    outs, idxs, lses = oracle.layer_stack(wl.pattern, layers, wl.k, q_offset=20)
+    rows = [79, 3, 40, 0, 55]
+    o2, i2, l2 = oracle.layer_stack(wl.pattern, layers, wl.k, q_offset=20, rows=rows)
+    for l in range(3):
+        assert np.array_equal(i2[l], idxs[l][rows])
+        assert np.array_equal(o2[l], outs[l][rows])
+        assert np.array_equal(l2[l], lses[l][rows])
+
+
 def test_stack_leading_shared_layer_is_an_error():
     wl = synth.custom(Lq=8, n_layers=2, k=4, pattern="SF")
     layers = synth.make_layers(wl)
