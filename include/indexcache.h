@@ -236,8 +236,9 @@ int ic_layer_stack_dense_rows(const ic_dims *dims, size_t ws_bytes);
  * (IC_ERR_NO_CACHED_INDICES otherwise, before any launch).
  * ws: device workspace of ws_bytes; F-layer scores are produced in row
  * chunks that fit in it; fewer than one query block of rows returns
- * IC_ERR_WORKSPACE_TOO_SMALL.  No host synchronisation happens inside, so
- * the whole call can be captured into a CUDA graph.
+ * IC_ERR_WORKSPACE_TOO_SMALL.  Nothing inside synchronises the host or
+ * allocates, so the call is meant to be capturable into a CUDA graph; no
+ * test captures it yet.
  */
 int ic_layer_stack_forward(const char *pattern, int n_layers, const ic_layer *layers,
                            const ic_dims *dims, int32_t *idx_cache, void *ws, size_t ws_bytes,
