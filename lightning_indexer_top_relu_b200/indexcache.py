@@ -388,6 +388,9 @@ class LayerStack:
                                              ctypes.byref(self.dims), _ptr(self.idx_cache),
                                              _ptr(self.ws), self.ws.numel(), _stream(stream))
         else:
+            need = MARKS_PER_LAYER * len(self.layers)
+            if len(events) < need:
+                raise ValueError(f"events holds {len(events)} handles, the stack records {need}")
             rc = _lib.ic_layer_stack_forward_events(
                 self._pattern_b, len(self.layers), self.table, ctypes.byref(self.dims),
                 _ptr(self.idx_cache), _ptr(self.ws), self.ws.numel(), _stream(stream),
