@@ -1,0 +1,102 @@
+"""The layer stack at the full sizes of the benchmarked long-context prefill
+(B=1, L=65536, 8 layers FSSSFSSS, indexer 64 x 128, k=2048, attention
+16 x 128) and decode (B=32 sequences of one query over 32768 cached
+positions, 16 layers (FSSS)x4), in the configuration bench.py times.
+
+Every row of every layer is checked on the device:
+
+* its index row is valid: min(k, t+1) strictly ascending positions <= t,
+  then -1;
+* S layers hold exactly their F layer's rows.
+
+A bounded sample of rows is checked against the oracle:
+
+* top-k set overlap >= 0.99 against the oracle's own scores;
+* attention within the tolerance against the oracle's attention over the
+  GPU's own index rows.  At 64K a row rarely has exactly the oracle's set,
+  so every sampled row is compared this way.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from lightning_indexer_top_relu_b200 import build, synth
+
+pytestmark = pytest.mark.gpu
+
+ATTN_ATOL = 2e-2
+LSE_ATOL = 1e-3
+
+
+@pytest.fixture(scope="module")
+def ic():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    build.build()
+    from lightning_indexer_top_relu_b200 import indexcache
+    return indexcache
+
+
+def _valid_rows(idx: torch.Tensor, q_offset: int, k: int) -> bool:
+    B, Lq, _ = idx.shape
+    t = torch.arange(Lq, device=idx.device) + q_offset
+    m = torch.clamp(t + 1, max=k)
+    slot = torch.arange(k, device=idx.device)
+    valid = slot[None, :] < m[:, None]
+    ok = torch.all(torch.where(valid[None], (idx >= 0) & (idx <= t[None, :, None]), idx == -1))
+    d = idx[..., 1:] - idx[..., :-1]
+    return bool(ok) and bool(torch.all(torch.where(valid[None, :, 1:], d > 0, True)))
+
+
+def check_sampled(ic, wl, layers, ref_layers, ref_wl, rows, ref_rows, sync):
+    """Runs the stack on `layers` (device tensors) and checks it as the
+    module docstring says.  The oracle runs on `ref_layers` (CPU tensors of
+    the problem `ref_wl`, the same sequences or a sub-batch of them): its
+    flattened row ref_rows[j] is the stack's row rows[j]."""
+    dims = ic.make_dims(wl.B, wl.Lq, wl.Lk, wl.q_offset, wl.H_I, wl.d_I, wl.Hq, wl.d, wl.k)
+    st = ic.LayerStack(wl.pattern, layers, dims, want_lse=True, dump_idx=True)
+    st.forward()
+    sync()
+    assert ic.get_last_device_error() == 0
+    src = 0
+    for l, c in enumerate(wl.pattern):
+        if c in "F1":
+            src = l
+        assert _valid_rows(st.dumps[l], wl.q_offset, wl.k), l
+        assert torch.equal(st.dumps[l], st.dumps[src]), l
+    _, ref_idx, _ = oracle.layer_stack(ref_wl.pattern, ref_layers, ref_wl.k, ref_wl.q_offset,
+                                       rows=ref_rows)
+    sel = torch.as_tensor(np.asarray(rows, dtype=np.int64), device=st.dumps[0].device)
+    for l in range(wl.n_layers):
+        gidx = st.dumps[l].reshape(-1, wl.k)[sel].cpu().numpy()
+        ov = [len(set(a[a >= 0].tolist()) & set(b[b >= 0].tolist())) / max(int((b >= 0).sum()), 1)
+              for a, b in zip(gidx, ref_idx[l])]
+        assert np.mean(ov) >= 0.99, (l, np.mean(ov), min(ov))
+        L = ref_layers[l]
+        ref, ref_lse = oracle.sparse_attn(L["q"], L["k"], L["v"], gidx, ref_wl.q_offset,
+                                          rows=ref_rows)
+        out = st.outs[l].reshape(-1, wl.Hq, wl.d)[sel].float().cpu().numpy()
+        lse = st.lses[l].reshape(-1, wl.Hq)[sel].cpu().numpy()
+        assert np.abs(out - ref).max() <= ATTN_ATOL, l
+        assert np.abs(lse - ref_lse).max() <= LSE_ATOL, l
+
+
+def test_prefill_64k_stack_full_size_sampled_rows(ic):
+    wl = synth.WORKLOADS["prefill_64k"]
+    layers = synth.make_layers(wl, indexer_for_all=False, device="cuda")   # drawn as bench.py does
+    ref_layers = [{n: t.cpu() for n, t in L.items()} for L in layers]
+    rows = synth.sample_rows(wl, 24)
+    check_sampled(ic, wl, layers, ref_layers, wl, rows, rows, torch.cuda.synchronize)
+
+
+def test_decode_32k_stack_full_size_sampled_rows(ic):
+    wl = synth.WORKLOADS["decode_32k"]
+    layers = synth.make_layers(wl, indexer_for_all=False, device="cuda")
+    seqs = list(range(0, wl.B, 4))                        # the oracle sees 8 of the 32 sequences
+    ref_layers = [{n: t[seqs].cpu() for n, t in L.items()} for L in layers]
+    ref_wl = dataclasses.replace(wl, B=len(seqs))
+    check_sampled(ic, wl, layers, ref_layers, ref_wl, seqs, list(range(len(seqs))),
+                  torch.cuda.synchronize)
