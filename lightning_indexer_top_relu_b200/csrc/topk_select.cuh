@@ -14,13 +14,20 @@
 //   2. A suffix scan of the 2048 bins finds the bin holding the k-th largest
 //      key.  Only that bin's keys (typically a few percent of the row) are
 //      gathered as candidates, with one shared atomic per warp (ballot +
-//      popc); two more radix passes (11 + 10 bits) over the candidates give
-//      the exact k-th key T and `need`, how many keys equal to T are kept.
+//      popc).  Each candidate is tagged with the warp whose step-3 segment
+//      holds it.  The same pass counts each segment's keys of higher bins,
+//      all of which are kept.  Two more radix passes (11 + 10 bits) over the
+//      candidates give the exact k-th key T and `need`, how many keys equal
+//      to T are kept.  A bin of more than TK_CAND keys (long tied rows) gets
+//      no candidate list; the radix passes and the counts of step 3 then
+//      read the whole row.
 //   3. A final pass in position order emits every key > T and the first
-//      `need` keys == T: each warp owns a contiguous segment, counts it with
-//      ballots, one block-wide scan of the per-warp counts gives every
-//      warp's first output slot, and the warp writes its selections at
-//      ballot-prefix offsets -- sorted output, no sort.
+//      `need` keys == T.  Each warp owns a contiguous segment; its counts of
+//      keys > T and == T come from the candidate list.  One block-wide scan
+//      of the per-warp counts gives every warp's first output slot, and the
+//      warp writes its selections at ballot-prefix offsets -- sorted output,
+//      no sort.  Rows that attend dense-masked also get their selection as
+//      a bitmask row: lane 0 stores each 32-position ballot as one word.
 // Every pass loads a whole batch (up to TK_VB float4 per thread) before
 // using any of it, so a row costs one memory latency per batch instead of
 // one per element.  Rows too long for shared memory re-read their scores
