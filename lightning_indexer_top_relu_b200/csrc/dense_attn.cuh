@@ -33,9 +33,13 @@
 //               so P stays <= 2^8 and O / l is exact either way.  A tile whose
 //               probabilities sum to at most 2^8 cannot hold a larger one, so
 //               the tile max is only taken (and the tile redone) when the sum
-//               is larger or no selected key has been seen yet.  Each thread
-//               also writes its share of the bias matrix two tiles ahead from
-//               the selection bitmask of its query.
+//               is larger or no selected key has been seen yet.  Rows raise
+//               their max independently, but tcgen05.ld/st are warp-collective,
+//               so the rescale is warp-uniform: when any row of a warp raises,
+//               every lane takes O through registers (the others with factor
+//               1).  Likewise every wait before a TMEM access is voted across
+//               the warp.  Each thread also writes its share of the bias matrix
+//               two tiles ahead from the selection bitmask of its query.
 // Scores are scaled in the log2 domain.
 #pragma once
 
