@@ -97,12 +97,19 @@ def test_reference_arm_prints_one_line_with_its_baseline():
                          "d2h_bytes_per_step": 0}
 
 
+def _free_port() -> int:
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
 def test_reference_arm_under_two_ranks_prints_from_rank_0_only():
     import subprocess
     import sys
     r = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
                         "--nproc-per-node", "2", "--master-addr", "127.0.0.1",
-                        "--master-port", "29571", "bench.py", "--impl", "reference", "--gpus",
+                        "--master-port", str(_free_port()), "bench.py", "--impl", "reference", "--gpus",
                         "2", "--workload", "tiny_prefill", "--steps", "1", "--warmup", "1",
                         "--ref-rows", "2"],
                        cwd=ROOT, capture_output=True, text=True, timeout=600)
