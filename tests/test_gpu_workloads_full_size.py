@@ -1,7 +1,13 @@
-"""The layer stack at the full sizes of the benchmarked long-context prefill
-(B=1, L=65536, 8 layers FSSSFSSS, indexer 64 x 128, k=2048, attention
-16 x 128) and decode (B=32 sequences of one query over 32768 cached
-positions, 16 layers (FSSS)x4), in the configuration bench.py times.
+"""The layer stack at the full sizes of the benchmarked long-context
+configurations, in the configuration bench.py times (inputs drawn on the
+device, score chunks as bench.py sizes them):
+
+* prefill: B=1, L=65536, 8 layers FSSSFSSS, indexer 64 x 128, k=2048,
+  attention 16 x 128;
+* decode: B=32 sequences of one query over 32768 cached positions, 16 layers
+  (FSSS)x4;
+* the longest single-layer sweep point: L=131072, whose scores take 4
+  workspace chunks.
 
 Every row of every layer is checked on the device:
 
@@ -51,13 +57,20 @@ def _valid_rows(idx: torch.Tensor, q_offset: int, k: int) -> bool:
     return bool(ok) and bool(torch.all(torch.where(valid[None, :, 1:], d > 0, True)))
 
 
+def bench_rows_per_chunk(wl) -> int:
+    """F-layer score rows per workspace chunk as bench.py sizes them: as many
+    as 16 GiB of fp32 scores hold."""
+    return max(1, min(wl.B * wl.Lq, (16 * 2 ** 30) // (4 * wl.Lk)))
+
+
 def check_sampled(ic, wl, layers, ref_layers, ref_wl, rows, ref_rows, sync):
     """Runs the stack on `layers` (device tensors) and checks it as the
     module docstring says.  The oracle runs on `ref_layers` (CPU tensors of
     the problem `ref_wl`, the same sequences or a sub-batch of them): its
     flattened row ref_rows[j] is the stack's row rows[j]."""
     dims = ic.make_dims(wl.B, wl.Lq, wl.Lk, wl.q_offset, wl.H_I, wl.d_I, wl.Hq, wl.d, wl.k)
-    st = ic.LayerStack(wl.pattern, layers, dims, want_lse=True, dump_idx=True)
+    st = ic.LayerStack(wl.pattern, layers, dims, want_lse=True, dump_idx=True,
+                       rows_per_chunk=bench_rows_per_chunk(wl))
     st.forward()
     sync()
     assert ic.get_last_device_error() == 0
@@ -100,3 +113,14 @@ def test_decode_32k_stack_full_size_sampled_rows(ic):
     ref_wl = dataclasses.replace(wl, B=len(seqs))
     check_sampled(ic, wl, layers, ref_layers, ref_wl, seqs, list(range(len(seqs))),
                   torch.cuda.synchronize)
+
+
+def test_sweep_128k_layer_full_size_chunked_scores(ic):
+    """One F layer at L = 131072: its scores exceed one 16 GiB workspace
+    chunk, so the indexer and top-k run over 4 chunks of 32768 rows."""
+    wl = synth.WORKLOADS["sweep_128k"]
+    assert bench_rows_per_chunk(wl) == 32768
+    layers = synth.make_layers(wl, device="cuda")
+    ref_layers = [{n: t.cpu() for n, t in L.items()} for L in layers]
+    rows = synth.sample_rows(wl, 24)
+    check_sampled(ic, wl, layers, ref_layers, wl, rows, rows, torch.cuda.synchronize)
