@@ -33,6 +33,7 @@ import math
 import os
 import subprocess
 import sys
+import threading
 import time
 
 import numpy as np
@@ -137,24 +138,33 @@ def profile_traffic(kernel: str, workload: str):
 # ---------------------------------------------------------------- clocks
 
 class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi every 200 ms
+    while the timed region runs; the samples are read through a pipe (a
+    thread drains it), so nothing is written to disk."""
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index: int):
-        self.dev = device_index
+    def __init__(self, device_index: int, cmd=None):
+        self.cmd = cmd or ["nvidia-smi", "-i", str(device_index), f"--query-gpu={self.QUERY}",
+                           "--format=csv,noheader,nounits", "-lms", "200"]
         self.proc = None
-        self.path = os.path.join("/tmp", f"ic_clocks_{os.getpid()}.csv")
+        self.thread = None
+        self.lines = []
+
+    def _drain(self):
+        for line in self.proc.stdout:
+            self.lines.append(line)
 
     def start(self):
         try:
-            self.fh = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=self.fh, stderr=subprocess.DEVNULL)
+            self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+            return
+        self.thread = threading.Thread(target=self._drain, daemon=True)
+        self.thread.start()
 
     def stop(self):
         if self.proc is None:
@@ -164,22 +174,21 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-        self.fh.close()
+            self.proc.wait()
+        self.thread.join(timeout=5)
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        with open(self.path) as f:
-            for row in csv.reader(f):
-                if len(row) < 9:
-                    continue
-                try:
-                    sm.append(float(row[1]))
-                    mx = float(row[2])
-                except ValueError:
-                    continue
-                for n, v in zip(names, row[5:9]):
-                    if v.strip().lower() == "active":
-                        reasons.add(n)
-        os.unlink(self.path)
+        for row in csv.reader(list(self.lines)):
+            if len(row) < 9:
+                continue
+            try:
+                sm.append(float(row[1]))
+                mx = float(row[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, row[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
         if not sm:
             return None
         return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),

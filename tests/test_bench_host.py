@@ -116,3 +116,24 @@ def test_reference_arm_under_two_ranks_prints_from_rank_0_only():
     assert r.returncode == 0, r.stderr[-2000:]
     lines = _json_lines(r.stdout)
     assert len(lines) == 1 and lines[0]["impl"] == "reference" and lines[0]["n_gpus"] == 2
+
+
+def test_clock_sampler_reads_samples_through_a_pipe():
+    """The sampler's parsing of nvidia-smi's CSV, fed by a stand-in command
+    that prints three samples and then idles until it is stopped."""
+    import sys
+    import time
+    rows = ["0, 1965, 1965, 512.3, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+            "0, 1950, 1965, 700.1, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+            "0, 1980, 1965, 650.0, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active"]
+    script = ("import sys, time\n" + "".join(f"print({r!r}, flush=True)\n" for r in rows)
+              + "time.sleep(60)\n")
+    cs = bench.ClockSampler(0, cmd=[sys.executable, "-c", script])
+    cs.start()
+    time.sleep(1.0)
+    out = cs.stop()
+    assert out == {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"],
+                   "samples": 3}
+    missing = bench.ClockSampler(0, cmd=["/nonexistent/nvidia-smi"])
+    missing.start()
+    assert missing.stop() is None
