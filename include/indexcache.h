@@ -236,7 +236,9 @@ int ic_layer_stack_dense_rows(const ic_dims *dims, size_t ws_bytes);
  * (IC_ERR_NO_CACHED_INDICES otherwise, before any launch).
  * ws: device workspace of ws_bytes; F-layer scores are produced in row
  * chunks that fit in it; fewer than one query block of rows returns
- * IC_ERR_WORKSPACE_TOO_SMALL.  Nothing inside synchronises the host or
+ * IC_ERR_WORKSPACE_TOO_SMALL.  Each layer is an NVTX range ("layer <l> F" or
+ * "layer <l> S", with nested ranges for the indexer + top-k and the
+ * attention) for profilers.  Nothing inside synchronises the host or
  * allocates, so the call is meant to be capturable into a CUDA graph; no
  * test captures it yet.
  */

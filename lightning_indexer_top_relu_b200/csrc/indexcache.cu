@@ -6,6 +6,7 @@
 // cached between calls except per-device launch attributes.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cmath>
@@ -48,6 +49,15 @@ int launched(cudaError_t e, const char* what) {
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return IC_OK;
 }
+
+// An NVTX range around host work, for profilers (a no-op unless one is
+// attached); the scope pops it on every return path.
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 // fp32 / int32 buffers read and written element by element
@@ -883,8 +893,12 @@ static int stack_forward(const char* pattern, int n_layers, const ic_layer* laye
     for (int l = 0; l < n_layers; ++l) {
         const ic_layer& L = layers[l];
         const bool full = pattern[l] == 'F' || pattern[l] == '1';
+        char label[32];
+        snprintf(label, sizeof label, "layer %d %c", l, full ? 'F' : 'S');
+        const NvtxRange layer_range(label);
         if ((rc = mark(l, 0))) return rc;
         if (full) {
+            const NvtxRange r("indexer + top-k");
             for (long long g0 = 0; g0 < n_blocks; g0 += blocks_per_chunk) {
                 const long long g1 = std::min(n_blocks, g0 + blocks_per_chunk);
                 rc = launch_indexer(L.q_idx, L.k_idx, L.w, D.B, D.Lq, D.Lk, D.H_I, D.d_I,
@@ -902,8 +916,11 @@ static int stack_forward(const char* pattern, int n_layers, const ic_layer* laye
         if ((rc = mark(l, 2))) return rc;
         cudaEvent_t mid = events ? reinterpret_cast<cudaEvent_t>(events[IC_MARKS_PER_LAYER * l + 3])
                                  : nullptr;
-        rc = attn_step(D, L, idx_cache, dense ? ATTN_MASK_READY : ATTN_GATHER, true, ws, ws_bytes,
-                       sms, st, mid);
+        {
+            const NvtxRange r("attention");
+            rc = attn_step(D, L, idx_cache, dense ? ATTN_MASK_READY : ATTN_GATHER, true, ws,
+                           ws_bytes, sms, st, mid);
+        }
         if (rc) return rc;
         if ((rc = mark(l, 4))) return rc;
         if (L.idx_dump) {
