@@ -227,7 +227,8 @@ int ic_layer_stack_dense_rows(const ic_dims *dims, size_t ws_bytes);
 
 /*
  * Steps a1-a5 — the IndexCache layer loop (skill page Step 3; technical
- * summary, Methodologie; review: "a single conditional branch").
+ * summary, Methodologie; review, "The Redundancy That Was Sitting There": the
+ * loop gains one branch per layer).
  * pattern: n_layers characters, 'F' or '1' = Full layer, 'S' or '0' = Shared.
  * For layer l: if F, the indexer scores and the top-k overwrite idx_cache
  * ([B, Lq, k] int32, caller-owned, the one index cache); then every layer
