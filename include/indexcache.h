@@ -272,8 +272,8 @@ int ic_layer_stack_forward_events(const char *pattern, int n_layers, const ic_la
 /*
  * Next step f2 -- cross-layer overlap of two layers' index sets (skill page,
  * Step 1 "Analyze Index Correlation Across Layers": top-k sets of
- * consecutive layers compared per query position; kualia.ai review: adjacent
- * layers share 70-100% of their selected tokens).
+ * consecutive layers compared per query position; kualia.ai review: in
+ * adjacent layers 70-100% of the k picks coincide).
  *   idx_a, idx_b [n_rows, k] int32 (device; -1 = empty slot; every other
  *   entry in [0, Lk))   counts [n_rows, 3] int32 (device, written)
  * Row r gets counts[r] = { |A & B|, |A|, |B| } with each row read as the set

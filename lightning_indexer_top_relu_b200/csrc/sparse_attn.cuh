@@ -2,8 +2,8 @@
 //
 // For query row t and head h, over the slots i whose index idx_i is valid:
 //   z_i = scale * q[t,h] . K[idx_i],  out = sum_i softmax(z)_i V[idx_i]
-// (IndexCache: every layer, F or S, runs its own sparse attention over the k
-// positions held in the index cache; all query heads share the one K/V head).
+// (IndexCache: every layer, F or S, attends sparsely over the k positions
+// held in the index cache; all query heads share the one K/V head).
 //
 // One CTA handles one query row (all heads) and one split of its slots.  The
 // CTA first stages up to 2048 of the row's indices in shared memory in one

@@ -290,8 +290,8 @@ int or_dense_attn(const uint16_t *q, const uint16_t *K, const uint16_t *V,
  * Cross-layer index overlap ("IndexCache ... Cross-Layer Index Reuse", skill
  * page, Step 1 "Analyze Index Correlation Across Layers": the top-k sets of
  * consecutive layers are compared per query position as sets; kualia.ai
- * review, "The Redundancy That Was Sitting There": adjacent layers share
- * 70-100% of their selected tokens).
+ * review, "The Redundancy That Was Sitting There": in adjacent layers 70-100%
+ * of the k picks coincide).
  * Row r of a and of b holds k slots; -1 is an empty slot and every other
  * value must lie in [0, Lk).  A row is read as the SET of its valid entries
  * (a repeated position counts once).  out3[3r+0] = |A & B|, out3[3r+1] = |A|,
