@@ -226,6 +226,7 @@ def _oracle_rows(wl, pattern, sl, workers):
         oracle.set_num_threads(1)
         oracle.layer_stack(pattern, lay, wl.k, q_offset=t)
 
+    oracle.num_threads()              # loads (building if needed) before the pool starts
     t0 = time.perf_counter()
     with ThreadPoolExecutor(max_workers=workers) as ex:
         list(ex.map(one, sl))

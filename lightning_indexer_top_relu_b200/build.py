@@ -43,13 +43,14 @@ def needs_build() -> bool:
 def build(force: bool = False, verbose: bool = False, extra=None) -> str:
     if not force and not needs_build():
         return LIB
+    tmp = f"{LIB}.{os.getpid()}.tmp"        # concurrent builds each replace the library whole
     cmd = [NVCC, *FLAGS, *(extra or []), "-I", os.path.join(ROOT, "include"),
-           "-o", LIB + ".tmp", os.path.join(CSRC, "indexcache.cu")]
+           "-o", tmp, os.path.join(CSRC, "indexcache.cu")]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)
-    os.replace(LIB + ".tmp", LIB)
+    os.replace(tmp, LIB)
     return LIB
 
 

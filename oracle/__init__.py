@@ -26,6 +26,7 @@ from __future__ import annotations
 import ctypes
 import os
 import subprocess
+import threading
 from typing import Optional, Sequence
 
 import numpy as np
@@ -34,6 +35,9 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 _lib = None
+# Host threads (a row-per-core pool) may ask for the library at the same time:
+# one of them builds and loads it, the others wait.
+_lock = threading.RLock()
 
 
 class NoCachedIndices(ValueError):
@@ -42,17 +46,25 @@ class NoCachedIndices(ValueError):
 
 def build(force: bool = False) -> str:
     """Compile oracle.c into liboracle.so next to it (gcc, -O2, OpenMP)."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-Wall",
-               "-o", _LIB + ".tmp", _SRC, "-lm"]
-        subprocess.run(cmd, check=True)
-        os.replace(_LIB + ".tmp", _LIB)
+    with _lock:
+        if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+            # a name of this process and thread: concurrent builds (several
+            # processes) each replace the library atomically with a whole file
+            tmp = f"{_LIB}.{os.getpid()}.{threading.get_ident()}.tmp"
+            cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-Wall",
+                   "-o", tmp, _SRC, "-lm"]
+            subprocess.run(cmd, check=True)
+            os.replace(tmp, _LIB)
     return _LIB
 
 
 def _load():
     global _lib
-    if _lib is None:
+    if _lib is not None:
+        return _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
         build()
         lib = ctypes.CDLL(_LIB)
         P, I, L, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_double

@@ -208,3 +208,18 @@ def test_unmodified_copy_passes_every_pin(tmp_path):
 def test_planted_mistake_fails_a_pin(tmp_path, tag, fname, edits):
     mod = _mutant_oracle(tmp_path, tag, fname, edits)
     assert _failing_pins(mod, stop_at_first=True), f"no pin catches the slip {tag!r}"
+
+
+def test_concurrent_first_use_builds_and_loads_once(tmp_path):
+    """Host threads of a row-per-core pool may all make the first oracle call
+    at once; a fresh copy (no library built yet) must come up in every one."""
+    from concurrent.futures import ThreadPoolExecutor
+    mod_dir = tmp_path / "oracle_fresh"
+    mod_dir.mkdir()
+    for f in ("oracle.c", "__init__.py"):
+        shutil.copy(os.path.join(ROOT, "oracle", f), mod_dir / f)
+    mod = _load_module("oracle_fresh", str(mod_dir / "__init__.py"), str(mod_dir))
+    with ThreadPoolExecutor(max_workers=8) as ex:
+        got = list(ex.map(lambda _: mod.num_threads(), range(8)))
+    assert all(n >= 1 for n in got)
+    assert sorted(p.name for p in mod_dir.iterdir() if p.suffix == ".tmp") == []
