@@ -124,3 +124,52 @@ def test_sweep_128k_layer_full_size_chunked_scores(ic):
     ref_layers = [{n: t.cpu() for n, t in L.items()} for L in layers]
     rows = synth.sample_rows(wl, 24)
     check_sampled(ic, wl, layers, ref_layers, wl, rows, rows, torch.cuda.synchronize)
+
+
+def _score_rel_err(gpu: np.ndarray, ref: np.ndarray, tpos) -> float:
+    """Largest |gpu - ref| / max(|ref|, 1e-3 * max |ref row|) over visible
+    positions (the floor keeps sign-mixed rows from dividing by ~0)."""
+    worst = 0.0
+    for r, t in enumerate(tpos):
+        g, f = gpu[r, : t + 1].astype(np.float64), ref[r, : t + 1]
+        floor = 1e-3 * max(np.abs(f).max(), 1e-30)
+        worst = max(worst, float((np.abs(g - f) / np.maximum(np.abs(f), floor)).max()))
+    return worst
+
+
+def check_kernels_one_by_one(ic, wl, L, sync):
+    """Each step on its own over a whole layer (`L`, device tensors): indexer
+    scores within 2e-2 of the oracle's (invisible positions exactly -inf),
+    top-k bit-exact on the GPU's own scores, gather attention within the
+    attention tolerance on the GPU's own index rows -- on sampled rows."""
+    rows = synth.sample_rows(wl, 24)
+    dev = L["q"].device
+    sel = torch.as_tensor(np.asarray(rows, dtype=np.int64), device=dev)
+    tpos = oracle.row_positions(wl.B, wl.Lq, wl.q_offset, rows)
+    cpu = {n: t.cpu() for n, t in L.items()}
+
+    scores = ic.indexer_scores(L["q_idx"], L["k_idx"], L["w"], wl.q_offset)
+    sync()
+    got = scores.reshape(-1, wl.Lk)[sel].cpu().numpy()
+    ref = oracle.indexer_scores(cpu["q_idx"], cpu["k_idx"], cpu["w"], wl.q_offset, rows=rows)
+    assert _score_rel_err(got, ref, tpos) <= 2e-2
+    for r, t in enumerate(tpos):
+        assert np.all(np.isneginf(got[r, t + 1:]))
+
+    idx = ic.topk_select(scores, wl.k, wl.q_offset)
+    del scores
+    gidx = idx.reshape(-1, wl.k)[sel].cpu().numpy()
+    assert np.array_equal(gidx, oracle.topk_sort(got, tpos, wl.k))
+
+    out, lse = ic.sparse_attn(L["q"], L["k"], L["v"], idx, wl.q_offset)
+    assert ic.get_last_device_error() == 0
+    ref_o, ref_lse = oracle.sparse_attn(cpu["q"], cpu["k"], cpu["v"], gidx, wl.q_offset, rows=rows)
+    assert np.abs(out.reshape(-1, wl.Hq, wl.d)[sel].float().cpu().numpy() - ref_o).max() <= ATTN_ATOL
+    assert np.abs(lse.reshape(-1, wl.Hq)[sel].cpu().numpy() - ref_lse).max() <= LSE_ATOL
+
+
+@pytest.mark.parametrize("name", ["prefill_8k", "prefill_64k"])
+def test_kernels_one_by_one_full_size_sampled_rows(ic, name):
+    wl = synth.WORKLOADS[name]
+    L = synth.make_layers(wl, layers=[0], device="cuda")[0]
+    check_kernels_one_by_one(ic, wl, L, torch.cuda.synchronize)
