@@ -137,3 +137,33 @@ def test_clock_sampler_reads_samples_through_a_pipe():
     missing = bench.ClockSampler(0, cmd=["/nonexistent/nvidia-smi"])
     missing.start()
     assert missing.stop() is None
+
+
+@pytest.mark.parametrize("name,a1_tflop,a2_gb,a4_tflop,gather_gb", [
+    ("prefill_8k", 0.275, 0.201, 0.120, 7.5),
+    ("prefill_64k", 35.2, 9.1, 1.08, 67.7),
+    ("sweep_128k", 140.7, 35.4, 2.18, 136.0),
+    ("sweep_4k", 0.1375, None, 0.052, 3.2),
+    ("sweep_16k", 2.20, None, 0.258, 16.1),
+    ("decode_32k", 0.0172, 0.0045, 0.00054, 0.0335),
+])
+def test_work_model_matches_the_per_layer_work_table(name, a1_tflop, a2_gb, a4_tflop, gather_gb):
+    """The roofline numerators against the per-layer algorithmic work
+    tabulated for each configuration (indexer flops 2*H_I*d_I*sum(t+1), top-k
+    bytes 4*sum(t+1) + 4*L*k, attention flops 4*Hq*d*V_k, logical K/V gather
+    4*d*V_k; values rounded to about 3 digits)."""
+    wl = synth.WORKLOADS[name]
+    w = bench.work_per_layer(wl, 0)                      # every row counted as gathered
+    t = np.arange(wl.Lq) + wl.q_offset
+    vk = wl.B * np.minimum(np.minimum(t + 1, wl.Lk), wl.k).sum()
+
+    def close(x, want):
+        return abs(x - want) <= 0.015 * want
+    assert close(w["indexer_flops"] / 1e12, a1_tflop)
+    if a2_gb is not None:
+        assert close(w["topk_bytes"] / 1e9, a2_gb)
+    assert close(w["gather_flops"] / 1e12, a4_tflop)
+    assert close(4.0 * wl.d * vk / 1e9, gather_gb)
+    # the gather bytes add q, out and the index rows to the K/V rows
+    extra = 2 * 2.0 * wl.B * wl.Lq * wl.Hq * wl.d + 4.0 * wl.B * wl.Lq * wl.k
+    assert w["gather_bytes"] == pytest.approx(4.0 * wl.d * vk + extra)
