@@ -49,14 +49,19 @@ L2_BYTES = 126 * 1024 * 1024
 
 
 def load_peaks():
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(p):
-        with open(p) as f:
+    """Roofline denominators: the copy bandwidth and bf16 GEMM rates measured
+    on this machine's B200s (MEASURED_PEAKS.json), else an earlier measurement
+    on the same pool, labelled "fallback"."""
+    fallback = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             d = json.load(f)
-        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
-                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
-    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
-            "source": "fallback"}
+        out = {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+               "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    except (OSError, ValueError, KeyError, TypeError):
+        return fallback
+    return out if out["hbm_gbs"] > 0 and out["bf16_tflops"] > 0 else fallback
 
 
 # ---------------------------------------------------------------- algorithmic work

@@ -167,3 +167,19 @@ def test_work_model_matches_the_per_layer_work_table(name, a1_tflop, a2_gb, a4_t
     # the gather bytes add q, out and the index rows to the K/V rows
     extra = 2 * 2.0 * wl.B * wl.Lq * wl.Hq * wl.d + 4.0 * wl.B * wl.Lq * wl.k
     assert w["gather_bytes"] == pytest.approx(4.0 * wl.d * vk + extra)
+
+
+def test_peaks_come_from_the_measured_file_else_the_fallback(tmp_path, monkeypatch):
+    import json
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.load_peaks()["source"] == "fallback"                     # no file
+    f = tmp_path / "MEASURED_PEAKS.json"
+    f.write_text("{not json")
+    assert bench.load_peaks()["source"] == "fallback"
+    f.write_text(json.dumps({"hbm_gbs": 6545.0}))                          # a key missing
+    assert bench.load_peaks()["source"] == "fallback"
+    f.write_text(json.dumps({"hbm_gbs": 6545.0, "bf16_tflops": 1652.8,
+                             "bf16_tflops_sustained": 1386.2}))
+    p = bench.load_peaks()
+    assert p == {"hbm_gbs": 6545.0, "bf16_tflops": 1652.8, "bf16_tflops_sustained": 1386.2,
+                 "source": "measured"}
