@@ -64,6 +64,24 @@ def test_indexer_nonnegative_dots_reduce_to_matvec():
             assert np.all(np.isneginf(sc[b, t, t + 1:]))
 
 
+def test_indexer_matches_a_library_evaluation_of_the_formula():
+    """Mixed-sign q_I, k_I and w, B > 1, a row offset: the score equals an
+    fp64 torch evaluation of sum_j w[t,j] * relu(q_I[t,j] . k_I[s]) for
+    s <= t (an independent routine: einsum, clamp, a weighted head sum)."""
+    rng = np.random.default_rng(9)
+    B, Lq, Lk, H, dI, q0 = 2, 23, 40, 5, 16, 17
+    q = _bf16(rng.normal(size=(B, Lq, H, dI)))
+    k = _bf16(rng.normal(size=(B, Lk, dI)))
+    w = torch.tensor(rng.normal(size=(B, Lq, H)), dtype=torch.float32)
+    sc = oracle.indexer_scores(q, k, w, q_offset=q0).reshape(B, Lq, Lk)
+    dots = torch.einsum("bthc,bsc->bths", q.double(), k.double())
+    ref = (w.double()[..., None] * dots.clamp(min=0)).sum(dim=2).numpy()
+    t = np.arange(Lq)[:, None] + q0
+    vis = np.arange(Lk)[None, :] <= t
+    assert np.allclose(sc[:, vis], ref[:, vis], rtol=1e-12, atol=1e-12)
+    assert np.all(np.isneginf(sc[:, ~vis]))
+
+
 def test_indexer_negative_dots_give_zero():
     """Every q_I . k_I < 0 -> every visible score is exactly 0 (ReLU clips)."""
     rng = np.random.default_rng(2)
