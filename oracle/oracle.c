@@ -84,6 +84,7 @@ int or_indexer_scores(const uint16_t *qI, const uint16_t *kI, const float *w,
 {
     if (B < 0 || Lq < 0 || Lk < 0 || H <= 0 || dI <= 0 || q_offset < 0)
         return -1;
+    if ((int64_t)q_offset + Lq > Lk) return -1;   /* a query past the last key */
     int bad = 0;
 #pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
     for (int64_t r = 0; r < n_rows; ++r) {
@@ -243,6 +244,7 @@ int or_sparse_attn(const uint16_t *q, const uint16_t *K, const uint16_t *V, cons
                    const int64_t *rows, int64_t n_rows, double *out, double *lse)
 {
     if (B < 0 || Lq < 0 || Lk < 0 || Hq <= 0 || d <= 0 || k <= 0 || q_offset < 0) return -1;
+    if ((int64_t)q_offset + Lq > Lk) return -1;   /* a query past the last key */
     if (scale <= 0.0) scale = 1.0 / sqrt((double)d);
     int rc = 0;
 #pragma omp parallel for schedule(dynamic, 1) reduction(min : rc)
@@ -251,7 +253,6 @@ int or_sparse_attn(const uint16_t *q, const uint16_t *K, const uint16_t *V, cons
         if (rid < 0 || rid >= (int64_t)B * Lq) { rc = rc < -1 ? rc : -1; continue; }
         int64_t b = rid / Lq, i = rid % Lq;
         int64_t t = (int64_t)q_offset + i;
-        if (t >= Lk) t = Lk - 1;
         int e = attend_row(q + rid * (int64_t)Hq * d, K + b * (int64_t)Lk * d,
                            V + b * (int64_t)Lk * d, idx + r * (int64_t)k, k, Hq, d, scale, t,
                            out + r * (int64_t)Hq * d, lse ? lse + r * (int64_t)Hq : NULL);
@@ -266,6 +267,7 @@ int or_dense_attn(const uint16_t *q, const uint16_t *K, const uint16_t *V,
                   const int64_t *rows, int64_t n_rows, double *out, double *lse)
 {
     if (B < 0 || Lq < 0 || Lk <= 0 || Hq <= 0 || d <= 0 || q_offset < 0) return -1;
+    if ((int64_t)q_offset + Lq > Lk) return -1;   /* a query past the last key */
     if (scale <= 0.0) scale = 1.0 / sqrt((double)d);
     int rc = 0;
 #pragma omp parallel for schedule(dynamic, 1) reduction(min : rc)
@@ -274,7 +276,6 @@ int or_dense_attn(const uint16_t *q, const uint16_t *K, const uint16_t *V,
         if (rid < 0 || rid >= (int64_t)B * Lq) { rc = rc < -1 ? rc : -1; continue; }
         int64_t b = rid / Lq, i = rid % Lq;
         int64_t t = (int64_t)q_offset + i;
-        if (t >= Lk) t = Lk - 1;
         int32_t *all = (int32_t *)malloc(sizeof(int32_t) * (size_t)(t + 1));
         for (int64_t s = 0; s <= t; ++s) all[s] = (int32_t)s;
         int e = attend_row(q + rid * (int64_t)Hq * d, K + b * (int64_t)Lk * d,

@@ -272,6 +272,24 @@ def test_attention_empty_row_and_out_of_range_index():
         oracle.sparse_attn(q, K, V, np.array([[0, 2]], dtype=np.int32), q_offset=1)
 
 
+def test_queries_past_the_last_key_are_rejected():
+    """q_offset + Lq > Lk puts a query after the last key; the library
+    rejects that before any launch, and so does every oracle step (it used to
+    clamp t to Lk - 1 silently)."""
+    wl = synth.custom(Lq=4, Lk=6, q_offset=2, H_I=2, d_I=64, k=4, Hq=2, d=64)
+    L = synth.make_layers(wl)[0]
+    idx = np.zeros((4, 4), dtype=np.int32)
+    oracle.indexer_scores(L["q_idx"], L["k_idx"], L["w"], q_offset=2)        # t <= 5: fine
+    oracle.sparse_attn(L["q"], L["k"], L["v"], idx, q_offset=2)
+    oracle.dense_attn(L["q"], L["k"], L["v"], q_offset=2)
+    with pytest.raises(ValueError):
+        oracle.indexer_scores(L["q_idx"], L["k_idx"], L["w"], q_offset=3)
+    with pytest.raises(ValueError):
+        oracle.sparse_attn(L["q"], L["k"], L["v"], idx, q_offset=3)
+    with pytest.raises(ValueError):
+        oracle.dense_attn(L["q"], L["k"], L["v"], q_offset=3)
+
+
 # ------------------------------------------------------------------ layer stack (a3, a5)
 
 def _check_idx_valid(idx, tpos, k):
