@@ -1,18 +1,25 @@
 """Benchmark of the IndexCache sparse-attention layer stack on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload prefill_8k] [--pattern P] [--no-cpu-baseline]
+                    [--workload prefill_64k] [--pattern P] [--no-cpu-baseline]
+                    [--no-e2e] [--no-all-f] [--no-extras] [--sweep 4,16,64,128]
 
 One step = one pass of the whole hot path over one batch of synthetic input:
 the layer loop with the F-layer indexer + top-k and every layer's sparse
 attention (ic_layer_stack_forward), inputs resident in HBM.  The default
-workload is the 8K-token prefill: B=1, L=8192, 8 layers FSSSFSSS, indexer
-32 heads x 128, k=2048, attention 16 query heads / 1 KV head x 128.
+workload is the 64K-token prefill: B=1, L=65536, 8 layers FSSSFSSS, indexer
+64 heads x 128, k=2048, attention 16 query heads / 1 KV head x 128; the same
+inputs also run all-F (FFFFFFFF) for the F/S speed-up.
 
 Prints ONE JSON line (rank 0).  `value` is prefill tokens/s over the stack
 (B*L*N / max-over-ranks step time).  `kernels` breaks the step down per
 kernel from CUDA events recorded on the launching stream inside the timed
 steps; `roofline` is for the kernel with the largest share of the step.
+`e2e` is the same stack through the public call with pinned host buffers
+(inputs copied in and outputs copied out inside the timed region).  On one
+GPU the line also carries supplementary points: `sweep_16_layers` (B=1,
+L in {4K, 16K, 64K, 128K}, 16 layers all-F vs (FSSS)x4, indexer share of the
+step) and `decode_32k` (B=32 over a 32768-token cache, 16 layers).
 With N > 1 (torchrun) every rank runs an independent replica of the workload
 (the query rows of different sequences never interact), so scaling is weak
 and no collective is on the data path; the barrier and the max-over-ranks
@@ -202,20 +209,28 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- CPU oracle leg
 
-def row_slice(wl, layers, r):
+def row_slice(wl, layers, r, key_cache=None):
     """Host copies of what the oracle needs for flattened query row r: that
     row's query-side tensors and its sequence's keys (a one-row problem at
-    q_offset = t, the row's absolute position)."""
+    q_offset = t, the row's absolute position).  `key_cache` (a dict) keeps
+    the host copy of each sequence's K, V and k_I, so a sample of many rows
+    copies every key tensor to the host once."""
     b, i = divmod(int(r), wl.Lq)
     out = []
-    for L in layers:
+    for l, L in enumerate(layers):
         d = {}
         for key in ("q", "q_idx", "w"):
             if key in L:
                 d[key] = L[key][b:b + 1, i:i + 1].contiguous().cpu()
         for key in ("k", "v", "k_idx"):
             if key in L:
-                d[key] = L[key][b:b + 1].contiguous().cpu()
+                if key_cache is None:
+                    d[key] = L[key][b:b + 1].contiguous().cpu()
+                else:
+                    ck = (l, key, b)
+                    if ck not in key_cache:
+                        key_cache[ck] = L[key][b:b + 1].contiguous().cpu()
+                    d[key] = key_cache[ck]
         out.append(d)
     return out, wl.q_offset + i
 
@@ -255,9 +270,10 @@ def oracle_rows_per_s(wl, pattern, layers, budget_s=15.0, seed=5):
     total = wl.B * wl.Lq
     workers = host_cores()
     elapsed, done, n = 0.0, 0, workers
+    cache = {}
     while elapsed < budget_s and done < total:
         rows = rng.choice(total, size=min(n, total), replace=False)
-        sl = [row_slice(wl, layers, r) for r in rows]
+        sl = [row_slice(wl, layers, r, cache) for r in rows]
         dt = _oracle_rows(wl, pattern, sl, workers)
         elapsed += dt
         done += len(rows)
@@ -287,12 +303,14 @@ def run_reference(args, wl, pattern):
     layers = synth.make_layers(wl, indexer_for_all=any(c in "F1" for c in pattern), device=dev)
     total = wl.B * wl.Lq
     rng = np.random.default_rng(11)
-    n_rows = max(1, min(total, args.ref_rows))
+    want = args.ref_rows if args.ref_rows > 0 else (64 if wl.Lk <= 16384 else 32)
+    n_rows = max(1, min(total, want))
     workers = host_cores()
     times = []
+    cache = {}
     for s in range(args.warmup + args.steps):
         rows = rng.choice(total, size=n_rows, replace=False)
-        sl = [row_slice(wl, layers, r) for r in rows]
+        sl = [row_slice(wl, layers, r, cache) for r in rows]
         dt = _oracle_rows(wl, pattern, sl, workers)
         if s >= args.warmup:                       # warm-up steps are not timed
             times.append(dt)
@@ -442,18 +460,304 @@ def run_row_sharded(args, wl, pattern, ic, dev, world, rank, local, pg):
     return 0
 
 
+# ---------------------------------------------------------------- timing helpers
+
+def new_marks(stream, n_layers: int, npl: int):
+    """npl CUDA events per layer for ic_layer_stack_forward_events, created
+    (recorded once) so their handles exist before the library records them."""
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(npl * n_layers)]
+    for e in evs:  # torch creates the CUDA event on first record
+        e.record(stream)
+    arr = (ctypes.c_void_p * (npl * n_layers))(*[e.cuda_event for e in evs])
+    assert all(arr), "CUDA event handles must exist before they are handed to the library"
+    return evs, arr
+
+
+def time_stack(ic, stack, stream, flush, steps: int, warmup: int, with_marks: bool = True):
+    """`warmup` untimed steps, then `steps` steps each timed with CUDA events
+    on the launching stream, L2 flushed (a 256 MiB write) before each.
+    Returns (per-step ms, per-step timing marks or None)."""
+    n = len(stack.layers)
+    for _ in range(warmup):
+        stack.forward(stream)
+    torch.cuda.synchronize()
+    marks = [new_marks(stream, n, ic.MARKS_PER_LAYER) for _ in range(steps)] if with_marks else None
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    torch.cuda.synchronize()
+    for s in range(steps):
+        flush.fill_(float(s))
+        starts[s].record(stream)
+        stack.forward(stream, events=marks[s][1] if marks else None)
+        ends[s].record(stream)
+    torch.cuda.synchronize()
+    return [starts[s].elapsed_time(ends[s]) for s in range(steps)], marks
+
+
+def auto_steps(ic, stack, stream, flush, budget_ms: float, lo: int = 2, hi: int = 10) -> int:
+    """Timed steps for a supplementary point: enough to fill about budget_ms
+    (one untimed probe step gives the step time), clamped to [lo, hi]."""
+    ms, _ = time_stack(ic, stack, stream, flush, 1, 1, with_marks=False)
+    return int(min(hi, max(lo, math.ceil(budget_ms / max(ms[0], 1e-3)))))
+
+
+def kernel_times(wl, pattern, marks, steps: int, npl: int, w):
+    """Per-launch times (ms) of each kernel group from the stack's marks:
+    indexer (mark 0 -> 1), top-k (1 -> 2) on F layers; dense-masked attention
+    (2 -> 3) and gathered attention (3 -> 4) on every layer that has such rows."""
+    ki = {"indexer": [], "topk": [], "attn_dense": [], "attn_gather": []}
+    for evs, _ in marks:
+        for l, c in enumerate(pattern):
+            e = evs[npl * l: npl * (l + 1)]
+            if c in "F1":
+                ki["indexer"].append(e[0].elapsed_time(e[1]))
+                ki["topk"].append(e[1].elapsed_time(e[2]))
+            if w["dense_rows"]:
+                ki["attn_dense"].append(e[2].elapsed_time(e[3]))
+            if w["gather_rows"]:
+                ki["attn_gather"].append(e[3].elapsed_time(e[4]))
+    return {k: v for k, v in ki.items() if v}
+
+
+def kernel_breakdown(ki, w, steps: int, ms_per_step: float, peaks, sm_mhz: float, n_sms: int):
+    """Per-kernel rates and shares of the step from kernel_times() output."""
+    kernels, per_step = {}, {}
+    for name, vals in ki.items():
+        avg = float(np.mean(vals))
+        sec = avg * 1e-3
+        per_step[name] = float(np.sum(vals)) / steps
+        ent = {"launches_per_step": len(vals) // steps, "ms_per_launch": avg,
+               "share": per_step[name] / ms_per_step}
+        if name == "indexer":
+            ent["tflops"] = w["indexer_flops"] / sec / 1e12
+            ent["frac_of_bf16_peak"] = ent["tflops"] / peaks["bf16_tflops"]
+            if peaks.get("bf16_tflops_sustained"):
+                ent["frac_of_bf16_sustained"] = ent["tflops"] / peaks["bf16_tflops_sustained"]
+            ent["gbs"] = w["indexer_bytes"] / sec / 1e9
+        elif name == "topk":
+            ent["covers"] = "top-k select (also writes the selection bitmask of dense-masked rows)"
+            ent["gbs"] = w["topk_bytes"] / sec / 1e9
+            ent["frac_of_hbm"] = ent["gbs"] / peaks["hbm_gbs"]
+        elif name == "attn_dense":
+            ent["covers"] = "V transpose + dense-masked tcgen05 attention, rows t < 8k"
+            ent["rows"] = int(w["dense_rows"])
+            ent["tflops"] = w["dense_flops"] / sec / 1e12
+            ent["frac_of_bf16_peak"] = ent["tflops"] / peaks["bf16_tflops"]
+            ent["executed_tflops"] = w["dense_exec_flops"] / sec / 1e12
+            ent["executed_frac_of_bf16_peak"] = ent["executed_tflops"] / peaks["bf16_tflops"]
+            sfu_peak = SFU_PER_CLK_SM * n_sms * sm_mhz * 1e6
+            ent["exp2_per_s"] = w["dense_exec_exps"] / sec
+            ent["frac_of_sfu_peak"] = ent["exp2_per_s"] / sfu_peak
+        else:
+            ent["covers"] = "gather attention (+ split combine), rows t >= 8k"
+            ent["rows"] = int(w["gather_rows"])
+            ent["tflops"] = w["gather_flops"] / sec / 1e12
+            ent["logical_gbs"] = w["gather_bytes"] / sec / 1e9
+            ent["frac_of_hbm"] = ent["logical_gbs"] / peaks["hbm_gbs"]
+        kernels[name] = ent
+    return kernels, per_step
+
+
+def tensor_peak(peaks, clk):
+    """The bf16 denominator for a contraction timed inside the step: the
+    sustained (power-capped) cuBLAS rate when the clock record shows the SM
+    clock held down by the power cap (sw_power_cap active, or the median SM
+    clock under load below 95% of its maximum), else the burst rate.
+    Returns (peak, which)."""
+    sus = peaks.get("bf16_tflops_sustained")
+    capped = False
+    if clk:
+        mx = clk.get("sm_max_mhz") or 0.0
+        capped = "sw_power_cap" in clk.get("reasons", []) or (
+            mx > 0 and clk.get("sm_mhz", mx) < 0.95 * mx)
+    if capped and sus:
+        return float(sus), "sustained"
+    return float(peaks["bf16_tflops"]), "burst"
+
+
+def roofline_of(kernels, w, peaks, clk, workload: str):
+    """Roofline entry for the kernel with the largest share of the step."""
+    dom = max(kernels, key=lambda k: kernels[k]["share"])
+    kd = kernels[dom]
+    tpeak, tkind = tensor_peak(peaks, clk)
+    if dom == "indexer":
+        roof = {"kernel": "indexer_scores", "bound": "tensor", "achieved": kd["tflops"],
+                "peak": tpeak, "peak_kind": tkind, "unit": "TFLOP/s",
+                "frac": kd["tflops"] / tpeak,
+                "frac_of_burst": kd["tflops"] / peaks["bf16_tflops"],
+                "algorithmic_per_launch": w["indexer_flops"],
+                "note": "achieved = 2*H_I*d_I flops per (query, visible key) / event time"}
+    elif dom == "topk":
+        roof = {"kernel": "topk_select", "bound": "hbm", "achieved": kd["gbs"],
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": kd["gbs"] / peaks["hbm_gbs"],
+                "algorithmic_per_launch": w["topk_bytes"]}
+    elif dom == "attn_dense":
+        roof = {"kernel": "dense_attn", "bound": "tensor", "achieved": kd["tflops"],
+                "peak": tpeak, "peak_kind": tkind, "unit": "TFLOP/s",
+                "frac": kd["tflops"] / tpeak,
+                "frac_of_burst": kd["tflops"] / peaks["bf16_tflops"],
+                "algorithmic_per_launch": w["dense_flops"],
+                "executed_frac": kd["executed_tflops"] / tpeak,
+                "sfu_frac": kd["frac_of_sfu_peak"],
+                "note": ("achieved counts the flops of the selected positions only (4*Hq*d per "
+                         "slot); the kernel runs whole 64-key tiles, whose flops give "
+                         "executed_frac, and one exp2 per tile element on the SFUs "
+                         "(16/clk/SM), whose rate gives sfu_frac")}
+    else:
+        roof = {"kernel": "sparse_attn", "bound": "hbm", "achieved": kd["logical_gbs"],
+                "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": kd["logical_gbs"] / peaks["hbm_gbs"],
+                "algorithmic_per_launch": w["gather_bytes"],
+                "note": ("achieved counts the logical K/V gather bytes; when a layer's K/V stay "
+                         "L2-resident, DRAM traffic (`traffic`) is far below them")}
+    roof["peak_source"] = peaks["source"]
+    roof["traffic"] = profile_traffic(roof["kernel"], workload)
+    return roof
+
+
+def default_rows_per_chunk(wl) -> int:
+    """F-layer score rows per chunk: as many as 16 GiB of fp32 scores allow."""
+    return max(1, min(wl.B * wl.Lq, (16 * 2 ** 30) // (4 * wl.Lk)))
+
+
+def stack_point(ic, wl, pattern, layers, stream, flush, peaks, n_sms, clk, budget_ms,
+                rows_per_chunk=0, warmup=1):
+    """One supplementary stack measurement: step time, tokens/s, the indexer
+    share of the step and the indexer's tensor rate, from the stack's marks."""
+    dims = ic.make_dims(wl.B, wl.Lq, wl.Lk, wl.q_offset, wl.H_I, wl.d_I, wl.Hq, wl.d, wl.k)
+    rpc = rows_per_chunk or default_rows_per_chunk(wl)
+    stack = ic.LayerStack(pattern, layers, dims, rows_per_chunk=rpc)
+    lq_d = ic.layer_stack_dense_rows(dims, stack.ws.numel())
+    steps = auto_steps(ic, stack, stream, flush, budget_ms)
+    ms, marks = time_stack(ic, stack, stream, flush, steps, warmup)
+    if ic.get_last_device_error() != 0:
+        raise RuntimeError(f"device error in the {wl.name} {pattern} point")
+    w = work_per_layer(wl, lq_d)
+    msps = float(np.mean(ms))
+    ki = kernel_times(wl, pattern, marks, steps, ic.MARKS_PER_LAYER, w)
+    kern, per_step = kernel_breakdown(ki, w, steps, msps, peaks,
+                                      (clk or {}).get("sm_mhz") or 1965.0, n_sms)
+    out = {"pattern": pattern, "steps": steps, "ms_per_step": msps,
+           "tokens_per_s": wl.B * wl.Lq / (msps * 1e-3),
+           "indexer_share": (per_step.get("indexer", 0) + per_step.get("topk", 0)) / msps}
+    if "indexer" in kern:
+        out["indexer_ms_per_launch"] = kern["indexer"]["ms_per_launch"]
+        out["indexer_tflops"] = kern["indexer"]["tflops"]
+        out["indexer_frac_of_bf16_peak"] = kern["indexer"]["frac_of_bf16_peak"]
+    if "topk" in kern:
+        out["topk_ms_per_launch"] = kern["topk"]["ms_per_launch"]
+    for name in ("attn_dense", "attn_gather"):
+        if name in kern:
+            out[f"{name}_ms_per_launch"] = kern[name]["ms_per_launch"]
+    del stack
+    return out
+
+
+def sweep_points(ic, lengths_k, dev, stream, flush, peaks, n_sms, clk):
+    """The indexer + top-k sweep: B = 1, L in lengths (K tokens), indexer
+    64 x 128, k = 2048, a 16-layer stack run all-F and (FSSS)x4, each with the
+    indexer share of the step.  Inputs are drawn on the device."""
+    import dataclasses
+    out = {}
+    for lk in lengths_k:
+        base = synth.WORKLOADS[f"sweep_{lk}k"]
+        wl = dataclasses.replace(base, n_layers=16, pattern="FSSS" * 4)
+        layers = synth.make_layers(wl, indexer_for_all=True, device=dev)
+        torch.cuda.synchronize()
+        pt = {}
+        for pat in ("F" * 16, "FSSS" * 4):
+            pt["all_f" if pat == "F" * 16 else "fsss_x4"] = stack_point(
+                ic, wl, pat, layers, stream, flush, peaks, n_sms, clk, budget_ms=1500.0)
+        pt["speedup_of_pattern"] = pt["all_f"]["ms_per_step"] / pt["fsss_x4"]["ms_per_step"]
+        out[f"{lk}k"] = pt
+        del layers
+        torch.cuda.empty_cache()
+    return out
+
+
+def decode_point(ic, dev, stream, flush, peaks, n_sms, clk):
+    """decode_32k: B = 32 sequences, one new query each over a 32768-token
+    cache, 16 layers (FSSS)x4 vs all-F; tokens/s = 32 tokens per step."""
+    wl = synth.WORKLOADS["decode_32k"]
+    layers = synth.make_layers(wl, indexer_for_all=True, device=dev)
+    torch.cuda.synchronize()
+    pt = {"config": {"B": wl.B, "Lq": wl.Lq, "Lk": wl.Lk, "q_offset": wl.q_offset,
+                     "layers": wl.n_layers, "H_I": wl.H_I, "d_I": wl.d_I, "k": wl.k,
+                     "Hq": wl.Hq, "d": wl.d}}
+    for pat in (wl.pattern, "F" * wl.n_layers):
+        key = "all_f" if pat == "F" * wl.n_layers else "fsss_x4"
+        pt[key] = stack_point(ic, wl, pat, layers, stream, flush, peaks, n_sms, clk,
+                              budget_ms=500.0, warmup=3)
+    pt["speedup_of_pattern"] = pt["all_f"]["ms_per_step"] / pt["fsss_x4"]["ms_per_step"]
+    del layers
+    torch.cuda.empty_cache()
+    return pt
+
+
+def e2e_leg(ic, stack, layers, pattern, stream, steps: int, pg, dev, tokens: float):
+    """The same stack end to end through the public call with host buffers:
+    every step copies that step's inputs (every layer's q/K/V and the F
+    layers' q_I/k_I/w) from pinned host memory to the device, runs the stack,
+    and copies every layer's output back to pinned host memory, all inside
+    the timed region.  The host copies are made once from the device-drawn
+    inputs (drawing several GB on the host would take minutes)."""
+    used = [{k: v for k, v in L.items() if k in ("q", "k", "v") or pattern[i] in "F1"}
+            for i, L in enumerate(layers)]
+    pinned = []
+    for L in used:
+        d = {}
+        for k, v in L.items():
+            h = torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
+            h.copy_(v)
+            d[k] = h
+        pinned.append(d)
+    outs_host = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in stack.outs]
+    h2d = sum(v.numel() * v.element_size() for L in pinned for v in L.values())
+    d2h = sum(o.numel() * o.element_size() for o in stack.outs)
+
+    def e2e_step():
+        for i, L in enumerate(pinned):
+            for k, v in L.items():
+                layers[i][k].copy_(v, non_blocking=True)
+        stack.forward(stream)
+        for o, h in zip(stack.outs, outs_host):
+            h.copy_(o, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if pg is not None:
+        pg.barrier()
+    a.record(stream)
+    for _ in range(steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    e_ms, _, e_val = aggregate_over_ranks(a.elapsed_time(b) / steps, tokens, pg, dev)
+    del pinned, outs_host
+    return {"value": e_val, "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": e_ms, "steps": steps,
+            "note": "pinned host buffers; copies and the stack on one stream, in order"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="prefill_8k", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--workload", default="prefill_64k", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--pattern", default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-all-f", action="store_true")
-    ap.add_argument("--ref-rows", type=int, default=64)
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the supplementary points (16-layer sweep, decode_32k)")
+    ap.add_argument("--sweep", default="4,16,64,128",
+                    help="sweep lengths in K tokens for the 16-layer all-F vs (FSSS)x4 points")
+    ap.add_argument("--ref-rows", type=int, default=0,
+                    help="query rows per step of the reference arm (0: 64, or 32 above 16K "
+                         "tokens, where one row costs the oracle about 0.5 core-seconds)")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--shard", default="replicas", choices=["replicas", "rows"],
                     help="with N > 1 ranks: a replica of the workload per rank (weak scaling) "
@@ -491,47 +795,25 @@ def main():
 
     peaks = load_peaks()
     need_all = (not args.no_all_f) and any(c in "S0" for c in pattern)
-    in_bytes = input_bytes(wl, need_all)
-    on_device = in_bytes > 2 * 2 ** 30          # too large to draw on the host
-    if on_device:
-        layers = synth.make_layers(wl, indexer_for_all=need_all, device=dev)
-        pinned = None
-    else:
-        layers_cpu = synth.make_layers(wl, indexer_for_all=need_all)
-        pinned = [{k: v.pin_memory() for k, v in L.items()} for L in layers_cpu]
-        layers = [{k: v.to(dev, non_blocking=True) for k, v in L.items()} for L in pinned]
+    layers = synth.make_layers(wl, indexer_for_all=need_all, device=dev)
     torch.cuda.synchronize()
     dims = ic.make_dims(wl.B, wl.Lq, wl.Lk, wl.q_offset, wl.H_I, wl.d_I, wl.Hq, wl.d, wl.k)
-    rpc = args.rows_per_chunk
-    if rpc <= 0:
-        rpc = max(1, min(wl.B * wl.Lq, (16 * 2 ** 30) // (4 * wl.Lk)))
+    rpc = args.rows_per_chunk if args.rows_per_chunk > 0 else default_rows_per_chunk(wl)
     stack = ic.LayerStack(pattern, layers, dims, rows_per_chunk=rpc)
     lq_d = ic.layer_stack_dense_rows(dims, stack.ws.numel())
     stream = torch.cuda.current_stream()
     n = wl.n_layers
-    flush = torch.empty(256 * 1024 * 1024 // 4, device=dev, dtype=torch.float32)
-
-    # per-kernel marks: ic.MARKS_PER_LAYER events per layer per step
     npl = ic.MARKS_PER_LAYER
-
-    def new_marks():
-        evs = [torch.cuda.Event(enable_timing=True) for _ in range(npl * n)]
-        for e in evs:  # torch creates the CUDA event on first record
-            e.record(stream)
-        arr = (ctypes.c_void_p * (npl * n))(*[e.cuda_event for e in evs])
-        assert all(arr), "CUDA event handles must exist before they are handed to the library"
-        return evs, arr
-
-    def step(marks=None):
-        stack.forward(stream, events=marks)
+    flush = torch.empty(256 * 1024 * 1024 // 4, device=dev, dtype=torch.float32)
+    n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
 
     for _ in range(args.warmup):
-        step()
+        stack.forward(stream)
     torch.cuda.synchronize()
     if ic.get_last_device_error() != 0:
         raise RuntimeError("device error during warm-up")
 
-    marks = [new_marks() for _ in range(args.steps)]
+    marks = [new_marks(stream, n, npl) for _ in range(args.steps)]
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     torch.cuda.synchronize()
@@ -545,7 +827,7 @@ def main():
     for s in range(args.steps):
         flush.fill_(float(s))                    # L2 flush outside the step's events
         starts[s].record(stream)
-        step(marks[s][1])
+        stack.forward(stream, events=marks[s][1])
         ends[s].record(stream)
     torch.cuda.synchronize()
     wall = time.perf_counter() - wall0
@@ -561,86 +843,12 @@ def main():
     local_ms = float(np.sum(step_ms)) / args.steps
     ms_per_step, tokens, value = aggregate_over_ranks(local_ms, float(wl.B * wl.Lq), pg, dev)
 
-    # ---- per-kernel breakdown from the marks
-    ki = {"indexer": [], "topk": [], "attn_dense": [], "attn_gather": []}
     w = work_per_layer(wl, lq_d)
-    for evs, _ in marks:
-        for l, c in enumerate(pattern):
-            e = evs[npl * l: npl * (l + 1)]
-            if c in "F1":
-                ki["indexer"].append(e[0].elapsed_time(e[1]))
-                ki["topk"].append(e[1].elapsed_time(e[2]))
-            if w["dense_rows"]:
-                ki["attn_dense"].append(e[2].elapsed_time(e[3]))
-            if w["gather_rows"]:
-                ki["attn_gather"].append(e[3].elapsed_time(e[4]))
+    ki = kernel_times(wl, pattern, marks, args.steps, npl, w)
     sm_mhz = (clk or {}).get("sm_mhz") or 1965.0
-    n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    kernels = {}
-    per_step = {}
-    for name, vals in ki.items():
-        if not vals:
-            continue
-        avg = float(np.mean(vals))
-        sec = avg * 1e-3
-        per_step[name] = float(np.sum(vals)) / args.steps
-        ent = {"launches_per_step": len(vals) // args.steps, "ms_per_launch": avg,
-               "share": per_step[name] / ms_per_step}
-        if name == "indexer":
-            ent["tflops"] = w["indexer_flops"] / sec / 1e12
-            ent["frac_of_bf16_peak"] = ent["tflops"] / peaks["bf16_tflops"]
-            ent["gbs"] = w["indexer_bytes"] / sec / 1e9
-        elif name == "topk":
-            ent["covers"] = "top-k select (also writes the selection bitmask of dense-masked rows)"
-            ent["gbs"] = w["topk_bytes"] / sec / 1e9
-            ent["frac_of_hbm"] = ent["gbs"] / peaks["hbm_gbs"]
-        elif name == "attn_dense":
-            ent["covers"] = "V transpose + dense-masked tcgen05 attention, rows t < 8k"
-            ent["rows"] = int(w["dense_rows"])
-            ent["tflops"] = w["dense_flops"] / sec / 1e12
-            ent["frac_of_bf16_peak"] = ent["tflops"] / peaks["bf16_tflops"]
-            ent["executed_tflops"] = w["dense_exec_flops"] / sec / 1e12
-            ent["executed_frac_of_bf16_peak"] = ent["executed_tflops"] / peaks["bf16_tflops"]
-            sfu_peak = SFU_PER_CLK_SM * n_sms * sm_mhz * 1e6
-            ent["exp2_per_s"] = w["dense_exec_exps"] / sec
-            ent["frac_of_sfu_peak"] = ent["exp2_per_s"] / sfu_peak
-        else:
-            ent["covers"] = "gather attention (+ split combine), rows t >= 8k"
-            ent["rows"] = int(w["gather_rows"])
-            ent["tflops"] = w["gather_flops"] / sec / 1e12
-            ent["logical_gbs"] = w["gather_bytes"] / sec / 1e9
-            ent["frac_of_hbm"] = ent["logical_gbs"] / peaks["hbm_gbs"]
-        kernels[name] = ent
-    dom = max(kernels, key=lambda k: kernels[k]["share"])
-    kd = kernels[dom]
-    if dom == "indexer":
-        roof = {"kernel": "indexer_scores", "bound": "tensor", "achieved": kd["tflops"],
-                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": kd["tflops"] / peaks["bf16_tflops"],
-                "algorithmic_per_launch": w["indexer_flops"]}
-    elif dom == "topk":
-        roof = {"kernel": "topk_select", "bound": "hbm", "achieved": kd["gbs"],
-                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": kd["gbs"] / peaks["hbm_gbs"],
-                "algorithmic_per_launch": w["topk_bytes"]}
-    elif dom == "attn_dense":
-        roof = {"kernel": "dense_attn", "bound": "tensor", "achieved": kd["tflops"],
-                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": kd["tflops"] / peaks["bf16_tflops"],
-                "algorithmic_per_launch": w["dense_flops"],
-                "executed_frac": kd["executed_frac_of_bf16_peak"],
-                "sfu_frac": kd["frac_of_sfu_peak"],
-                "note": ("achieved counts the flops of the selected positions only (4*Hq*d per "
-                         "slot); the kernel runs whole 64-key tiles, whose flops give "
-                         "executed_frac, and one exp2 per tile element on the SFUs "
-                         "(16/clk/SM), whose rate gives sfu_frac")}
-    else:
-        roof = {"kernel": "sparse_attn", "bound": "hbm", "achieved": kd["logical_gbs"],
-                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": kd["logical_gbs"] / peaks["hbm_gbs"],
-                "algorithmic_per_launch": w["gather_bytes"],
-                "note": ("achieved counts the logical K/V gather bytes; when a layer's K/V stay "
-                         "L2-resident, DRAM traffic (`traffic`) is far below them")}
-    roof["peak_source"] = peaks["source"]
-    roof["traffic"] = profile_traffic(roof["kernel"], wl.name)
+    kernels, per_step = kernel_breakdown(ki, w, args.steps, ms_per_step, peaks, sm_mhz, n_sms)
+    roof = roofline_of(kernels, w, peaks, clk, wl.name)
+    del marks
 
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
@@ -656,60 +864,26 @@ def main():
     # ---- the same stack with every layer Full, for the F/S speed-up
     if need_all:
         stack_f = ic.LayerStack("F" * n, layers, dims, rows_per_chunk=rpc)
-        for _ in range(2):
-            stack_f.forward(stream)
-        ts = []
-        for s in range(max(3, args.steps // 2)):
-            flush.fill_(float(s))
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            stack_f.forward(stream)
-            b.record(stream)
-            torch.cuda.synchronize()
-            ts.append(a.elapsed_time(b))
-        msf = float(np.mean(ts))
+        k_f = max(3, args.steps // 2)
+        ms_f, marks_f = time_stack(ic, stack_f, stream, flush, k_f, 2)
+        msf = float(np.mean(ms_f))
+        ki_f = kernel_times(wl, "F" * n, marks_f, k_f, npl, w)
+        share_f = sum(float(np.sum(ki_f.get(k, [0.0]))) for k in ("indexer", "topk")) / k_f / msf
         msf, _, vf = aggregate_over_ranks(msf, float(wl.B * wl.Lq), pg, dev)
-        line["all_f"] = {"pattern": "F" * n, "ms_per_step": msf,
-                         "value": vf,
-                         "speedup_of_pattern": msf / ms_per_step}
-        del stack_f
+        line["all_f"] = {"pattern": "F" * n, "ms_per_step": msf, "value": vf, "steps": k_f,
+                         "indexer_share": share_f, "speedup_of_pattern": msf / ms_per_step}
+        del stack_f, marks_f
         line["cross_layer_overlap"] = cross_layer_overlap(ic, wl, layers, dims, rpc, stream,
                                                           peaks, n)
+        if ic.get_last_device_error() != 0:
+            raise RuntimeError("device error in the all-F leg")
 
     # ---- end to end through the public API with host buffers
-    if not args.no_e2e and pinned is None:
-        line["e2e"] = {"skipped": f"inputs of {in_bytes / 2**30:.1f} GiB are drawn on the device"}
-    if not args.no_e2e and pinned is not None:
-        outs_host = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in stack.outs]
-        h2d = sum(v.numel() * v.element_size() for i, L in enumerate(pinned) for k, v in L.items()
-                  if k in ("q", "k", "v") or pattern[i] in "F1")
-        d2h = sum(o.numel() * o.element_size() for o in stack.outs)
-
-        def e2e_step():
-            for i, L in enumerate(pinned):
-                for k, v in L.items():
-                    if k in ("q", "k", "v") or pattern[i] in "F1":
-                        layers[i][k].copy_(v, non_blocking=True)
-            stack.forward(stream)
-            for o, h in zip(stack.outs, outs_host):
-                h.copy_(o, non_blocking=True)
-
-        e2e_step()
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        if pg is not None:
-            pg.barrier()
-        a.record(stream)
-        k_e2e = max(3, args.steps // 2)
-        for _ in range(k_e2e):
-            e2e_step()
-        b.record(stream)
-        torch.cuda.synchronize()
-        e_ms, e_tok, e_val = aggregate_over_ranks(a.elapsed_time(b) / k_e2e, float(wl.B * wl.Lq),
-                                                  pg, dev)
-        line["e2e"] = {"value": e_val, "unit": "tokens/s",
-                       "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-                       "ms_per_step": e_ms}
+    if not args.no_e2e:
+        line["e2e"] = e2e_leg(ic, stack, layers, pattern, stream, max(3, args.steps // 2), pg,
+                              dev, float(wl.B * wl.Lq))
+        if ic.get_last_device_error() != 0:
+            raise RuntimeError("device error in the end-to-end leg")
 
     # ---- CPU oracle baseline (rank 0, N=1 only)
     if not args.no_cpu_baseline and world == 1:
@@ -717,6 +891,14 @@ def main():
         rps, sample, cores = oracle_rows_per_s(wl, pattern, layers, budget_s=args.cpu_budget_s)
         line["cpu_baseline"] = {"value": rps, "unit": "tokens/s", "cores": cores,
                                 "kind": "oracle", "sample": sample}
+
+    # ---- supplementary points (one GPU only): the 16-layer sweep and decode
+    if not args.no_extras and world == 1:
+        del stack, layers
+        torch.cuda.empty_cache()
+        lengths = [int(x) for x in args.sweep.split(",") if x.strip()]
+        line["sweep_16_layers"] = sweep_points(ic, lengths, dev, stream, flush, peaks, n_sms, clk)
+        line["decode_32k"] = decode_point(ic, dev, stream, flush, peaks, n_sms, clk)
 
     if pg is not None:
         pg.barrier()

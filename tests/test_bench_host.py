@@ -183,3 +183,64 @@ def test_peaks_come_from_the_measured_file_else_the_fallback(tmp_path, monkeypat
     p = bench.load_peaks()
     assert p == {"hbm_gbs": 6545.0, "bf16_tflops": 1652.8, "bf16_tflops_sustained": 1386.2,
                  "source": "measured"}
+
+
+def test_tensor_peak_is_sustained_only_when_the_power_cap_holds_clocks():
+    peaks = {"hbm_gbs": 6459.9, "bf16_tflops": 1725.8, "bf16_tflops_sustained": 1391.2,
+             "source": "measured"}
+    assert bench.tensor_peak(peaks, None) == (1725.8, "burst")
+    full = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": [], "samples": 20}
+    assert bench.tensor_peak(peaks, full) == (1725.8, "burst")
+    capped = dict(full, reasons=["sw_power_cap"], sm_mhz=1800.0)
+    assert bench.tensor_peak(peaks, capped) == (1391.2, "sustained")
+    slow = dict(full, sm_mhz=1700.0)
+    assert bench.tensor_peak(peaks, slow) == (1391.2, "sustained")
+    no_sus = dict(peaks, bf16_tflops_sustained=None)
+    assert bench.tensor_peak(no_sus, capped) == (1725.8, "burst")
+
+
+class _Ev:
+    def __init__(self, t):
+        self.t = t
+
+    def elapsed_time(self, other):
+        return other.t - self.t
+
+
+def test_kernel_breakdown_and_roofline_from_stack_marks():
+    """Two steps of a 2-layer FS stack with fake event times: the indexer,
+    top-k and attention groups come from the right marks, shares add up,
+    and the roofline names the largest share."""
+    wl = synth.custom("fake", Lq=4096, n_layers=2, H_I=64, d_I=128, k=2048, Hq=16, d=128,
+                      pattern="FS")
+    w = bench.work_per_layer(wl, 0)
+    npl = 5
+    marks = []
+    for s in range(2):
+        # layer 0 F: indexer 3 ms, top-k 1 ms, attention 2 ms; layer 1 S: attention 2 ms
+        t = [0, 3, 4, 4, 6, 6, 6, 6, 6, 8]
+        marks.append(([_Ev(x) for x in t], None))
+    ki = bench.kernel_times(wl, "FS", marks, 2, npl, w)
+    assert ki["indexer"] == [3, 3] and ki["topk"] == [1, 1]
+    assert ki["attn_gather"] == [2, 2, 2, 2] and "attn_dense" not in ki
+    peaks = {"hbm_gbs": 6459.9, "bf16_tflops": 1725.8, "bf16_tflops_sustained": 1391.2,
+             "source": "measured"}
+    kern, per_step = bench.kernel_breakdown(ki, w, 2, 8.0, peaks, 1965.0, 148)
+    assert abs(sum(k["share"] for k in kern.values()) - 1.0) < 1e-9
+    assert kern["attn_gather"]["launches_per_step"] == 2
+    assert abs(kern["indexer"]["tflops"] - w["indexer_flops"] / 3e-3 / 1e12) < 1e-6
+    roof = bench.roofline_of(kern, w, peaks, None, "fake")
+    assert roof["kernel"] == "sparse_attn" and roof["bound"] == "hbm"
+    assert abs(roof["frac"] - roof["achieved"] / 6459.9) < 1e-12
+    kern["indexer"]["share"] = 0.9
+    roof = bench.roofline_of(kern, w, peaks, {"sm_mhz": 1500.0, "sm_max_mhz": 1965.0,
+                                              "reasons": ["sw_power_cap"]}, "fake")
+    assert roof["kernel"] == "indexer_scores" and roof["peak_kind"] == "sustained"
+    assert abs(roof["frac_of_burst"] - roof["achieved"] / 1725.8) < 1e-12
+
+
+def test_default_workload_is_the_64k_prefill():
+    import inspect
+    src = inspect.getsource(bench.main)
+    assert 'default="prefill_64k"' in src
+    assert synth.WORKLOADS["prefill_64k"].pattern == "FSSSFSSS"
