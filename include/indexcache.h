@@ -147,12 +147,16 @@ size_t ic_sparse_attn_workspace_bytes(int B, int Lq, int Hq, int d, int k_slots)
  * partial results in a fixed 4 MiB array inside the library instead of a
  * workspace; every GPU that loads the library holds that array until the
  * process exits.
- *   - A call whose preferred split would need more than 4 MiB of partials
- *     (rows x splits x Hq x (d + 1) x 4 bytes) runs with fewer splits (one
- *     split needs none), so every valid call runs; results are the same.
+ *   - Rows split their slots only while rows x splits stays within two CTAs
+ *     per SM, so with the supported Hq <= 16 and d <= 128 the partials take
+ *     at most 2 x SMs x 16 x 129 x 4 bytes (2.4 MB on a 148-SM B200) and the
+ *     preferred split always fits.  On a GPU with more SMs the call would run
+ *     with fewer splits (one split needs no scratch); results are the same.
  *   - The first call on a device looks up the array's device address (once per
  *     device, with that device current); make that first call before any
- *     stream capture.
+ *     stream capture.  The library keeps that address, and its per-device
+ *     kernel attributes, for the life of the process: do not use it again on
+ *     a device after cudaDeviceReset.
  *   - All calls share the one array and it keeps the last call's contents.
  *     Every partial a call reads is written by the same call first, so nothing
  *     needs clearing, but calls that overlap on the GPU (different streams,
@@ -268,6 +272,64 @@ int ic_layer_stack_forward(const char *pattern, int n_layers, const ic_layer *la
 int ic_layer_stack_forward_events(const char *pattern, int n_layers, const ic_layer *layers,
                                   const ic_dims *dims, int32_t *idx_cache, void *ws,
                                   size_t ws_bytes, ic_stream_t stream, void *const *events);
+
+/*
+ * Options of ic_layer_stack_forward_opts (NULL = all defaults).
+ *   fused_topk  how an F layer turns scores into index rows (next step f1;
+ *               the kualia.ai review, "The Hidden Quadratic": the indexer's
+ *               O(L^2) work and its L x L score matrix dominate long
+ *               prefills):
+ *                 0  store each chunk's causal scores in the workspace, then
+ *                    run the top-k over them;
+ *                 1  fused: never store the score matrix.  A pass over every
+ *                    stride-th key tile (stride = max(1, key tiles / 16))
+ *                    gives each row a threshold -- the r-th largest sampled
+ *                    score, r = ceil(m p + z sqrt(m p (1 - p))) + 1 for m
+ *                    visible samples and p = k / (t + 1) -- then the indexer
+ *                    runs again keeping only scores at or above it (at most
+ *                    3k per row; rows with at most 3k visible positions keep
+ *                    them all), and an exact selection runs on those
+ *                    candidates.  A row with fewer than k candidates or more
+ *                    than 3k has its query block re-run the way of mode 0, so
+ *                    the index rows equal mode 0's bit for bit in every case.
+ *                    Needs k <= 4096 and Lk <= 262144 (IC_ERR_UNSUPPORTED
+ *                    otherwise);
+ *                -1  (default) the library's choice: fused when the longest
+ *                    row sees more than 6k positions and there are at least
+ *                    1024 query rows, else mode 0.
+ *   z           the threshold's margin in binomial standard deviations
+ *               (<= 0: 4).  Larger keeps more candidates and falls back less
+ *               often; the index rows do not depend on it.
+ */
+typedef struct {
+    int fused_topk;
+    float z;
+} ic_stack_options;
+
+/*
+ * ic_layer_stack_forward_events with options (opts may be NULL; events may be
+ * NULL).  On the fused path, timing mark j=1 is recorded after the candidate
+ * pass (sampled scores, thresholds and candidates), and j=2 after the exact
+ * selection and the fallback rounds.  The workspace from
+ * ic_layer_stack_workspace_bytes holds the fused path's chunk too; a smaller
+ * one is split into more chunks, and fused_topk = 1 with a workspace that
+ * holds no fused chunk returns IC_ERR_WORKSPACE_TOO_SMALL.
+ */
+int ic_layer_stack_forward_opts(const char *pattern, int n_layers, const ic_layer *layers,
+                                const ic_dims *dims, const ic_stack_options *opts,
+                                int32_t *idx_cache, void *ws, size_t ws_bytes,
+                                ic_stream_t stream, void *const *events);
+
+/*
+ * Diagnostic of the fused path: synchronises `stream` and writes to *blocks
+ * how many query blocks of the last F layer's last row chunk fell back to
+ * the plain indexer + top-k (read from the workspace of the last
+ * ic_layer_stack_forward_opts call with the same dims, options and
+ * workspace).  IC_ERR_INVALID_ARG when the stack does not fuse for them.
+ */
+int ic_layer_stack_fused_fallback_blocks(const ic_dims *dims, const ic_stack_options *opts,
+                                         const void *ws, size_t ws_bytes, ic_stream_t stream,
+                                         int *blocks);
 
 /*
  * Next step f2 -- cross-layer overlap of two layers' index sets (skill page,

@@ -19,6 +19,7 @@
 #include "indexcache.h"
 #include "common.cuh"
 #include "dense_attn.cuh"
+#include "fused_topk.cuh"
 #include "index_overlap.cuh"
 #include "indexer_scores.cuh"
 #include "sparse_attn.cuh"
@@ -134,37 +135,62 @@ long long block_row_start(const IndexerGeom& g, int Lq, long long gb) {
 
 template <int H, int DI>
 void set_indexer_attr() {
-    cudaFuncSetAttribute(ic::indexer_scores_kernel<H, DI>,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         ic::IndexerSmem<DI>::ALLOC);
+    cudaFuncSetAttribute(ic::indexer_scores_kernel<H, DI, ic::IDX_SCORES>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, ic::IndexerSmem<DI>::ALLOC);
+    cudaFuncSetAttribute(ic::indexer_scores_kernel<H, DI, ic::IDX_SAMPLE>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, ic::IndexerSmem<DI>::ALLOC);
+    cudaFuncSetAttribute(ic::indexer_scores_kernel<H, DI, ic::IDX_CAND>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, ic::IndexerSmem<DI>::ALLOC);
 }
 
 template <int H, int DI>
-cudaError_t launch_indexer_t(const CUtensorMap& tq, const CUtensorMap& tk,
+cudaError_t launch_indexer_t(int mode, const CUtensorMap& tq, const CUtensorMap& tk,
                              const ic::IndexerArgs& a, int grid, cudaStream_t st) {
-    ic::indexer_scores_kernel<H, DI>
-        <<<grid, ic::IDX_THREADS, ic::IndexerSmem<DI>::ALLOC, st>>>(tq, tk, a);
+    constexpr int SM = ic::IndexerSmem<DI>::ALLOC;
+    if (mode == ic::IDX_SAMPLE)
+        ic::indexer_scores_kernel<H, DI, ic::IDX_SAMPLE><<<grid, ic::IDX_THREADS, SM, st>>>(tq, tk, a);
+    else if (mode == ic::IDX_CAND)
+        ic::indexer_scores_kernel<H, DI, ic::IDX_CAND><<<grid, ic::IDX_THREADS, SM, st>>>(tq, tk, a);
+    else
+        ic::indexer_scores_kernel<H, DI, ic::IDX_SCORES><<<grid, ic::IDX_THREADS, SM, st>>>(tq, tk, a);
     return cudaGetLastError();
 }
 
 template <int DI>
-cudaError_t launch_indexer_h(int H, const CUtensorMap& tq, const CUtensorMap& tk,
+cudaError_t launch_indexer_h(int H, int mode, const CUtensorMap& tq, const CUtensorMap& tk,
                              const ic::IndexerArgs& a, int grid, cudaStream_t st) {
     switch (H) {
-        case 4: return launch_indexer_t<4, DI>(tq, tk, a, grid, st);
-        case 8: return launch_indexer_t<8, DI>(tq, tk, a, grid, st);
-        case 16: return launch_indexer_t<16, DI>(tq, tk, a, grid, st);
-        case 32: return launch_indexer_t<32, DI>(tq, tk, a, grid, st);
-        case 64: return launch_indexer_t<64, DI>(tq, tk, a, grid, st);
-        case 128: return launch_indexer_t<128, DI>(tq, tk, a, grid, st);
+        case 4: return launch_indexer_t<4, DI>(mode, tq, tk, a, grid, st);
+        case 8: return launch_indexer_t<8, DI>(mode, tq, tk, a, grid, st);
+        case 16: return launch_indexer_t<16, DI>(mode, tq, tk, a, grid, st);
+        case 32: return launch_indexer_t<32, DI>(mode, tq, tk, a, grid, st);
+        case 64: return launch_indexer_t<64, DI>(mode, tq, tk, a, grid, st);
+        case 128: return launch_indexer_t<128, DI>(mode, tq, tk, a, grid, st);
         default: return cudaErrorInvalidValue;
     }
 }
 
-// Scores query blocks [g0, g1) into `scores` (row = flattened row - row of g0).
+// What an indexer launch does besides storing every score of its blocks
+// (the default): the sampled tiles only, candidates above per-row
+// thresholds, and/or query blocks taken from a device list.
+struct IdxExtra {
+    int mode = ic::IDX_SCORES;
+    int stride = 1;                       // IDX_SAMPLE
+    const uint32_t* thr = nullptr;        // IDX_CAND
+    uint32_t* cnt = nullptr;
+    unsigned long long* cand = nullptr;
+    int cap = 0;
+    const int* blk_list = nullptr;        // block list (blocks of [g0, g1) only)
+    const int* blk_count = nullptr;
+    int list_off = 0, list_len = 0;
+};
+
+// Scores query blocks [g0, g1) into `scores` (row = flattened row - row of g0),
+// or does what `x` asks instead (sampled tiles, candidates, a block list).
 int launch_indexer(const uint16_t* q_idx, const uint16_t* k_idx, const float* w, int B, int Lq,
                    int Lk, int H, int dI, int q_offset, long long g0, long long g1, float* scores,
-                   long long ld, bool fill_masked, int sms, cudaStream_t st) {
+                   long long ld, bool fill_masked, int sms, cudaStream_t st,
+                   const IdxExtra& x = IdxExtra()) {
     const IndexerGeom geo = indexer_geom(Lq, H);
     CUtensorMap tq, tk;
     int rc = make_tmap_3d(&tq, q_idx, (uint64_t)dI, (uint64_t)Lq * H, (uint64_t)B, (uint32_t)geo.N);
@@ -172,22 +198,31 @@ int launch_indexer(const uint16_t* q_idx, const uint16_t* k_idx, const float* w,
     rc = make_tmap_3d(&tk, k_idx, (uint64_t)dI, (uint64_t)Lk, (uint64_t)B, (uint32_t)ic::IDX_BM);
     if (rc) return rc;
 
-    // Total key tiles of the range, to size work units.
+    // Key tiles visited over the range (every stride-th in IDX_SAMPLE), to size work units.
+    const int stride = x.mode == ic::IDX_SAMPLE ? std::max(1, x.stride) : 1;
     long long total = 0;
     int max_nt = 0;
     for (long long gb = g0; gb < g1; ++gb) {
         const int i0 = (int)(gb % geo.nqb) * geo.QB;
         const int nq = std::min(geo.QB, Lq - i0);
         const int n_vis = std::min(q_offset + i0 + nq, Lk);
-        const int nt = (n_vis + ic::IDX_BM - 1) / ic::IDX_BM;
+        const int nt = ((n_vis + ic::IDX_BM - 1) / ic::IDX_BM + stride - 1) / stride;
         total += nt;
         max_nt = std::max(max_nt, nt);
     }
+    const bool listed = x.blk_list != nullptr;
+    long long blocks = listed ? std::min<long long>(x.list_len, g1 - g0) : g1 - g0;
+    if (listed) {
+        // unknown until run time how many blocks are listed: units of a
+        // few tiles, so that even one long block spreads over many CTAs
+        total = (long long)blocks * max_nt;
+    }
     int tpu = (int)std::min<long long>(64, std::max<long long>(4, total / (6LL * sms)));
+    if (listed) tpu = std::max(4, std::min(tpu, max_nt / 8));
     tpu = std::min(tpu, std::max(1, max_nt));
     const int max_splits = (max_nt + tpu - 1) / tpu;
 
-    ic::IndexerArgs a;
+    ic::IndexerArgs a{};
     a.w = w;
     a.scores = scores;
     a.ld = ld;
@@ -203,11 +238,20 @@ int launch_indexer(const uint16_t* q_idx, const uint16_t* k_idx, const float* w,
     a.row_base = block_row_start(geo, Lq, g0);
     a.tpu = tpu;
     a.max_splits = max_splits;
-    const long long n_units = (g1 - g0) * (long long)max_splits;
+    a.stride = stride;
+    a.thr = x.thr;
+    a.cnt = x.cnt;
+    a.cand = x.cand;
+    a.cap = x.cap;
+    a.blk_list = x.blk_list;
+    a.blk_count = x.blk_count;
+    a.list_off = x.list_off;
+    a.list_len = (int)blocks;
+    const long long n_units = blocks * (long long)max_splits;
     const int grid = (int)std::min<long long>(n_units, sms);
     if (grid <= 0) return IC_OK;
-    cudaError_t e = dI == 64 ? launch_indexer_h<64>(H, tq, tk, a, grid, st)
-                             : launch_indexer_h<128>(H, tq, tk, a, grid, st);
+    cudaError_t e = dI == 64 ? launch_indexer_h<64>(H, x.mode, tq, tk, a, grid, st)
+                             : launch_indexer_h<128>(H, x.mode, tq, tk, a, grid, st);
     if (launched(e, "indexer_scores launch")) return IC_ERR_CUDA;
     if (fill_masked) {
         const long long n_rows = block_row_start(geo, Lq, g1) - a.row_base;
@@ -222,31 +266,38 @@ int launch_indexer(const uint16_t* q_idx, const uint16_t* k_idx, const float* w,
 
 // ---------------------------------------------------------------- top-k
 
+// Rows [row_base, row_base + n_rows) of `scores`, or (lst.blk_list non-null)
+// the rows of the listed blocks, whose scores sit in consecutive rows.
 int launch_topk(const float* scores, long long ld, long long row_base, long long n_rows, int Lq,
                 int Lk, int q_offset, int k, int32_t* idx, int sms, cudaStream_t st,
-                uint32_t* mask = nullptr, int Lq_d = 0, int W = 0) {
+                uint32_t* mask = nullptr, int Lq_d = 0, int W = 0,
+                const ic::TopkList& lst = ic::TopkList{}) {
     if (n_rows <= 0) return IC_OK;
     const int n_max = std::min(Lk, q_offset + Lq);
+    // one CTA per row; a listed launch loops a persistent grid over its rows
+    const unsigned grid = lst.blk_list != nullptr
+                              ? (unsigned)std::min<long long>(n_rows, 8LL * sms)
+                              : (unsigned)n_rows;
     cudaError_t e;
     if (n_rows < 2LL * sms && n_max > 4096) {
         // few long rows (decode): a 1024-thread CTA per row, one per SM
         if (n_max <= ic::TK_CACHE_MAX) {
             ic::topk_select_kernel<ic::TK_THREADS_FEW, true>
-                <<<(unsigned)n_rows, ic::TK_THREADS_FEW, ic::TK_SMEM_FIXED + n_max * 4, st>>>(
-                    scores, ld, row_base, n_rows, Lq, Lk, q_offset, k, idx, mask, Lq_d, W);
+                <<<grid, ic::TK_THREADS_FEW, ic::TK_SMEM_FIXED + n_max * 4, st>>>(
+                    scores, ld, row_base, n_rows, Lq, Lk, q_offset, k, idx, mask, Lq_d, W, lst);
         } else {
             ic::topk_select_kernel<ic::TK_THREADS_FEW, false>
-                <<<(unsigned)n_rows, ic::TK_THREADS_FEW, ic::TK_SMEM_FIXED, st>>>(
-                    scores, ld, row_base, n_rows, Lq, Lk, q_offset, k, idx, mask, Lq_d, W);
+                <<<grid, ic::TK_THREADS_FEW, ic::TK_SMEM_FIXED, st>>>(
+                    scores, ld, row_base, n_rows, Lq, Lk, q_offset, k, idx, mask, Lq_d, W, lst);
         }
     } else if (n_max <= ic::TK_CACHE_MAX) {
         const int smem = ic::TK_SMEM_FIXED + n_max * 4;
-        ic::topk_select_kernel<ic::TK_THREADS, true><<<(unsigned)n_rows, ic::TK_THREADS, smem, st>>>(
-            scores, ld, row_base, n_rows, Lq, Lk, q_offset, k, idx, mask, Lq_d, W);
+        ic::topk_select_kernel<ic::TK_THREADS, true><<<grid, ic::TK_THREADS, smem, st>>>(
+            scores, ld, row_base, n_rows, Lq, Lk, q_offset, k, idx, mask, Lq_d, W, lst);
     } else {
         ic::topk_select_kernel<ic::TK_THREADS_LONG, false>
-            <<<(unsigned)n_rows, ic::TK_THREADS_LONG, ic::TK_SMEM_FIXED, st>>>(
-                scores, ld, row_base, n_rows, Lq, Lk, q_offset, k, idx, mask, Lq_d, W);
+            <<<grid, ic::TK_THREADS_LONG, ic::TK_SMEM_FIXED, st>>>(
+                scores, ld, row_base, n_rows, Lq, Lk, q_offset, k, idx, mask, Lq_d, W, lst);
     }
     e = cudaGetLastError();
     if (launched(e, "topk_select launch")) return IC_ERR_CUDA;
@@ -456,6 +507,168 @@ int attn_step(const ic_dims& D, const ic_layer& L, const int32_t* idx, AttnMode 
                        trim, sms, st, dg.Lq_d, D.Lq - dg.Lq_d);
 }
 
+// ---------------------------------------------------------------- fused indexer -> top-k
+
+constexpr int FUSED_CAP_FACTOR = 3;     // candidates a row may keep: 3k
+constexpr float FUSED_Z = 4.0f;         // threshold margin in binomial standard deviations
+constexpr int FUSED_FB_DIV = 8;         // fallback scores: 1/8 of a chunk's blocks per round
+constexpr int FUSED_MAX_K = 4096;       // candidate list in shared memory: 3k x 8 bytes
+constexpr int FUSED_MAX_LK = 262144;    // bitmap of a row's positions in shared memory
+constexpr int FUSED_AUTO_MIN_ROWS = 1024;
+
+// Sizes of the fused path for given dims (ok = false when it cannot run).
+struct FusedGeom {
+    bool ok = false;
+    int stride = 1;          // sampled key tiles m * stride
+    int ns = 0;              // sampled tiles per row at most (<= 32)
+    int cap = 0;             // candidates kept per row
+    int n_max = 0;           // longest row's visible positions
+};
+
+FusedGeom fused_geom(const ic_dims& D) {
+    FusedGeom f;
+    if (D.k > FUSED_MAX_K || D.Lk > FUSED_MAX_LK || D.Lq < 1) return f;
+    f.n_max = std::min(D.Lk, D.q_offset + D.Lq);
+    const int nt_max = (f.n_max + ic::IDX_BM - 1) / ic::IDX_BM;
+    f.stride = std::max(1, nt_max / 16);
+    f.ns = (nt_max + f.stride - 1) / f.stride;
+    f.cap = FUSED_CAP_FACTOR * D.k;
+    f.ok = f.ns * ic::IDX_BM <= ic::FT_MAX_SAMPLES &&
+           ic::fused_select_smem(f.cap, D.Lk) <= (size_t)ic::MAX_DYN_SMEM;
+    return f;
+}
+
+// Whether the stack fuses the top-k into the indexer: `mode` 1 asks for it,
+// 0 refuses it, -1 leaves it to the library, which fuses when the longest
+// row is over twice the candidate capacity and there are many rows (prefill).
+bool fused_wanted(const FusedGeom& f, const ic_dims& D, int mode) {
+    if (!f.ok || mode == 0) return false;
+    if (mode == 1) return true;
+    return f.n_max > 2 * f.cap && (long long)D.B * D.Lq >= FUSED_AUTO_MIN_ROWS;
+}
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Workspace layout of one chunk of `blocks` query blocks on the fused path.
+struct FusedLayout {
+    size_t samp = 0, cand = 0, thr = 0, cnt = 0, flag = 0, list = 0, lcount = 0, fb = 0, total = 0;
+    long long fb_blocks = 0;
+};
+
+FusedLayout fused_layout(const FusedGeom& f, long long blocks, int QB, int Lk) {
+    FusedLayout L;
+    const size_t rows = (size_t)blocks * QB;
+    L.fb_blocks = (blocks + FUSED_FB_DIV - 1) / FUSED_FB_DIV;
+    size_t o = 0;
+    L.samp = o;   o = align256(o + rows * (size_t)f.ns * ic::IDX_BM * 4);
+    L.cand = o;   o = align256(o + rows * (size_t)f.cap * 8);
+    L.thr = o;    o = align256(o + rows * 4);
+    L.cnt = o;    o = align256(o + rows * 4);
+    L.flag = o;   o = align256(o + (size_t)blocks * 4);
+    L.list = o;   o = align256(o + (size_t)blocks * 4);
+    L.lcount = o; o = align256(o + 16);
+    L.fb = o;     o = align256(o + (size_t)L.fb_blocks * QB * (size_t)Lk * 4);
+    L.total = o;
+    return L;
+}
+
+// Most query blocks per chunk whose fused layout fits in `avail` bytes (0 if none).
+long long fused_blocks_fitting(const FusedGeom& f, long long n_blocks, int QB, int Lk,
+                               size_t avail) {
+    const FusedLayout one = fused_layout(f, 1, QB, Lk);
+    if (one.total > avail) return 0;
+    long long lo = 1, hi = n_blocks;
+    while (lo < hi) {                      // largest count that fits
+        const long long mid = lo + (hi - lo + 1) / 2;
+        if (fused_layout(f, mid, QB, Lk).total <= avail) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
+// One F layer's index rows of query blocks [g0, g1) on the fused path: the
+// sampled scores, the thresholds, the candidates, the exact selection, and
+// the fallback rounds over the flagged blocks (each round scores up to
+// lay.fb_blocks listed blocks into the fallback buffer and runs the plain
+// top-k on them; rounds past the list's length do nothing).  `mid` (may be
+// null) is recorded after the candidate pass.
+int fused_chunk(const ic_dims& D, const ic_layer& Lr, const IndexerGeom& geo, const FusedGeom& f,
+                long long g0, long long g1, uint8_t* base, int32_t* idx, uint32_t* dmask,
+                const DenseGeom& dg, float z, int sms, cudaStream_t st, cudaEvent_t mid) {
+    const FusedLayout lay = fused_layout(f, g1 - g0, geo.QB, D.Lk);
+    const long long r0 = block_row_start(geo, D.Lq, g0);
+    const long long r1 = block_row_start(geo, D.Lq, g1);
+    ic::FusedArgs fa{};
+    fa.row_base = r0;
+    fa.n_rows = r1 - r0;
+    fa.Lq = D.Lq;
+    fa.Lk = D.Lk;
+    fa.q_offset = D.q_offset;
+    fa.k = D.k;
+    fa.cap = f.cap;
+    fa.stride = f.stride;
+    fa.ns = f.ns;
+    fa.z = z;
+    fa.QB = geo.QB;
+    fa.nqb = geo.nqb;
+    fa.g0 = g0;
+    fa.n_blocks = g1 - g0;
+    fa.samp = reinterpret_cast<const float*>(base + lay.samp);
+    fa.thr = reinterpret_cast<uint32_t*>(base + lay.thr);
+    fa.cnt = reinterpret_cast<uint32_t*>(base + lay.cnt);
+    fa.cand = reinterpret_cast<const unsigned long long*>(base + lay.cand);
+    fa.bflag = reinterpret_cast<uint32_t*>(base + lay.flag);
+    fa.blist = reinterpret_cast<int*>(base + lay.list);
+    fa.list_count = reinterpret_cast<int*>(base + lay.lcount);
+    fa.idx = idx;
+    fa.mask = dmask;
+    fa.Lq_d = dg.Lq_d;
+    fa.W = dg.W;
+
+    IdxExtra xs;
+    xs.mode = ic::IDX_SAMPLE;
+    xs.stride = f.stride;
+    int rc = launch_indexer(Lr.q_idx, Lr.k_idx, Lr.w, D.B, D.Lq, D.Lk, D.H_I, D.d_I, D.q_offset,
+                            g0, g1, reinterpret_cast<float*>(base + lay.samp),
+                            (long long)f.ns * ic::IDX_BM, false, sms, st, xs);
+    if (rc) return rc;
+    const int tgrid = (int)std::min<long long>(fa.n_rows, 16LL * sms);
+    ic::fused_threshold_kernel<<<tgrid, ic::FT_THREADS, 0, st>>>(fa);
+    if (launched(cudaGetLastError(), "fused_threshold launch")) return IC_ERR_CUDA;
+    IdxExtra xc;
+    xc.mode = ic::IDX_CAND;
+    xc.thr = fa.thr;
+    xc.cnt = fa.cnt;
+    xc.cand = reinterpret_cast<unsigned long long*>(base + lay.cand);
+    xc.cap = f.cap;
+    rc = launch_indexer(Lr.q_idx, Lr.k_idx, Lr.w, D.B, D.Lq, D.Lk, D.H_I, D.d_I, D.q_offset, g0,
+                        g1, nullptr, 0, false, sms, st, xc);
+    if (rc) return rc;
+    if (mid) {
+        cudaError_t e = cudaEventRecord(mid, st);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    }
+    ic::fused_select_kernel<<<(unsigned)fa.n_rows, ic::FS_THREADS,
+                              ic::fused_select_smem(f.cap, D.Lk), st>>>(fa);
+    if (launched(cudaGetLastError(), "fused_select launch")) return IC_ERR_CUDA;
+    float* fb = reinterpret_cast<float*>(base + lay.fb);
+    for (long long off = 0; off < g1 - g0; off += lay.fb_blocks) {
+        IdxExtra xl;
+        xl.blk_list = fa.blist;
+        xl.blk_count = fa.list_count;
+        xl.list_off = (int)off;
+        xl.list_len = (int)lay.fb_blocks;
+        rc = launch_indexer(Lr.q_idx, Lr.k_idx, Lr.w, D.B, D.Lq, D.Lk, D.H_I, D.d_I, D.q_offset,
+                            g0, g1, fb, D.Lk, false, sms, st, xl);
+        if (rc) return rc;
+        ic::TopkList tl{fa.blist, fa.list_count, (int)off, (int)lay.fb_blocks, geo.QB, geo.nqb};
+        rc = launch_topk(fb, D.Lk, 0, lay.fb_blocks * geo.QB, D.Lq, D.Lk, D.q_offset, D.k, idx,
+                         sms, st, dmask, dg.Lq_d, dg.W, tl);
+        if (rc) return rc;
+    }
+    return IC_OK;
+}
+
 // ---------------------------------------------------------------- per-device setup
 
 int device_setup(int* dev_out, int* sms_out) {
@@ -487,6 +700,10 @@ int device_setup(int* dev_out, int* sms_out) {
                              ic::TK_SMEM_FIXED + ic::TK_CACHE_MAX * 4);
         cudaFuncSetAttribute(ic::dense_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              ic::DenseSmem::ALLOC);
+        cudaFuncSetAttribute(ic::fused_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)std::min<size_t>(ic::MAX_DYN_SMEM,
+                                                   ic::fused_select_smem(FUSED_CAP_FACTOR * FUSED_MAX_K,
+                                                                         FUSED_MAX_LK)));
         cudaFuncSetAttribute(ic::index_overlap_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              2 * (ic::OV_MAX_LK / 32) * 4);
         cudaFuncSetAttribute(ic::index_overlap_warp_kernel,
@@ -798,7 +1015,11 @@ size_t ic_layer_stack_workspace_bytes(const ic_dims* dims, int n_layers, long lo
     long long blocks = (long long)dims->B * geo.nqb;
     if (rows_per_chunk > 0)
         blocks = std::min(blocks, std::max(1LL, (rows_per_chunk + geo.QB - 1) / geo.QB));
-    const size_t scores = (size_t)blocks * geo.QB * (size_t)dims->Lk * sizeof(float);
+    size_t scores = (size_t)blocks * geo.QB * (size_t)dims->Lk * sizeof(float);
+    // the fused top-k's chunk (candidate lists, fallback buffer) in place of
+    // the score chunk, when the fused path can run for these dims
+    const FusedGeom fgeo = fused_geom(*dims);
+    if (fgeo.ok) scores = std::max(scores, fused_layout(fgeo, blocks, geo.QB, dims->Lk).total);
     const size_t attn = ic_sparse_attn_workspace_bytes(dims->B, dims->Lq, dims->Hq, dims->d, dims->k);
     const DenseGeom dg = dense_geom(*dims);
     (void)n_rows;
@@ -816,8 +1037,8 @@ size_t ic_layer_stack_workspace_bytes(const ic_dims* dims, int n_layers, long lo
 }
 
 static int stack_forward(const char* pattern, int n_layers, const ic_layer* layers,
-                         const ic_dims* dims, int32_t* idx_cache, void* ws, size_t ws_bytes,
-                         ic_stream_t stream, void* const* events) {
+                         const ic_dims* dims, const ic_stack_options* opts, int32_t* idx_cache,
+                         void* ws, size_t ws_bytes, ic_stream_t stream, void* const* events) {
     if (!pattern || !layers || !dims || !idx_cache || n_layers < 1)
         return fail(IC_ERR_INVALID_ARG, "null argument or n_layers < 1");
     if ((int)strnlen(pattern, (size_t)n_layers + 1) != n_layers)
@@ -837,6 +1058,11 @@ static int stack_forward(const char* pattern, int n_layers, const ic_layer* laye
     if ((rc = check_attn_shape(D.Hq, D.Hkv, D.d))) return rc;
     if (D.k < 1 || D.k > D.Lk) return fail(IC_ERR_INVALID_ARG, "k=%d outside [1, Lk]", D.k);
     if (!std::isfinite(D.scale)) return fail(IC_ERR_INVALID_ARG, "scale is not finite");
+    const int fuse_mode = opts ? opts->fused_topk : -1;
+    const FusedGeom fgeo = fused_geom(D);
+    if (fuse_mode == 1 && !fgeo.ok)
+        return fail(IC_ERR_UNSUPPORTED, "the fused top-k needs k <= %d and Lk <= %d",
+                    FUSED_MAX_K, FUSED_MAX_LK);
     for (int l = 0; l < n_layers; ++l) {
         const ic_layer& L = layers[l];
         const bool full = pattern[l] == 'F' || pattern[l] == '1';
@@ -878,8 +1104,25 @@ static int stack_forward(const char* pattern, int n_layers, const ic_layer* laye
     const DenseGeom dg = dense_geom(D);
     const bool dense = dg.on && ws_bytes >= dg.mask_bytes + std::max(block_bytes, dg.vt_bytes);
     const size_t sc_off = dense ? dg.mask_bytes : 0;
-    const long long blocks_per_chunk =
+    long long blocks_per_chunk =
         std::min<long long>(n_blocks, (long long)((ws_bytes - sc_off) / block_bytes));
+    // Fused indexer -> top-k: chunks as large as the workspace holds their
+    // candidate lists and fallback buffer; the score matrix is never stored.
+    const float z = (opts && opts->z > 0.0f) ? opts->z : FUSED_Z;
+    bool fused = fused_wanted(fgeo, D, fuse_mode);
+    if (fused) {
+        const long long fb =
+            fused_blocks_fitting(fgeo, n_blocks, geo.QB, D.Lk, ws_bytes - sc_off);
+        if (fb < 1) {
+            if (fuse_mode == 1)
+                return fail(IC_ERR_WORKSPACE_TOO_SMALL,
+                            "workspace of %zu bytes holds no query block of the fused top-k",
+                            ws_bytes);
+            fused = false;
+        } else {
+            blocks_per_chunk = fb;
+        }
+    }
     float* sc = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + sc_off);
     uint32_t* dmask = dense ? reinterpret_cast<uint32_t*>(ws) : nullptr;
 
@@ -901,6 +1144,15 @@ static int stack_forward(const char* pattern, int n_layers, const ic_layer* laye
             const NvtxRange r("indexer + top-k");
             for (long long g0 = 0; g0 < n_blocks; g0 += blocks_per_chunk) {
                 const long long g1 = std::min(n_blocks, g0 + blocks_per_chunk);
+                if (fused) {
+                    cudaEvent_t m1 = nullptr;
+                    if (one_chunk && events)
+                        m1 = reinterpret_cast<cudaEvent_t>(events[IC_MARKS_PER_LAYER * l + 1]);
+                    rc = fused_chunk(D, L, geo, fgeo, g0, g1, reinterpret_cast<uint8_t*>(sc),
+                                     idx_cache, dmask, dg, z, sms, st, m1);
+                    if (rc) return rc;
+                    continue;
+                }
                 rc = launch_indexer(L.q_idx, L.k_idx, L.w, D.B, D.Lq, D.Lk, D.H_I, D.d_I,
                                     D.q_offset, g0, g1, sc, D.Lk, false, sms, st);
                 if (rc) return rc;
@@ -936,13 +1188,57 @@ static int stack_forward(const char* pattern, int n_layers, const ic_layer* laye
 int ic_layer_stack_forward(const char* pattern, int n_layers, const ic_layer* layers,
                            const ic_dims* dims, int32_t* idx_cache, void* ws, size_t ws_bytes,
                            ic_stream_t stream) {
-    return stack_forward(pattern, n_layers, layers, dims, idx_cache, ws, ws_bytes, stream, nullptr);
+    return stack_forward(pattern, n_layers, layers, dims, nullptr, idx_cache, ws, ws_bytes, stream,
+                         nullptr);
 }
 
 int ic_layer_stack_forward_events(const char* pattern, int n_layers, const ic_layer* layers,
                                   const ic_dims* dims, int32_t* idx_cache, void* ws,
                                   size_t ws_bytes, ic_stream_t stream, void* const* events) {
-    return stack_forward(pattern, n_layers, layers, dims, idx_cache, ws, ws_bytes, stream, events);
+    return stack_forward(pattern, n_layers, layers, dims, nullptr, idx_cache, ws, ws_bytes, stream,
+                         events);
+}
+
+int ic_layer_stack_forward_opts(const char* pattern, int n_layers, const ic_layer* layers,
+                                const ic_dims* dims, const ic_stack_options* opts,
+                                int32_t* idx_cache, void* ws, size_t ws_bytes,
+                                ic_stream_t stream, void* const* events) {
+    if (opts && (opts->fused_topk < -1 || opts->fused_topk > 1 || !std::isfinite(opts->z)))
+        return fail(IC_ERR_INVALID_ARG, "options: fused_topk=%d z=%g", opts->fused_topk,
+                    (double)opts->z);
+    return stack_forward(pattern, n_layers, layers, dims, opts, idx_cache, ws, ws_bytes, stream,
+                         events);
+}
+
+int ic_layer_stack_fused_fallback_blocks(const ic_dims* dims, const ic_stack_options* opts,
+                                         const void* ws, size_t ws_bytes, ic_stream_t stream,
+                                         int* blocks) {
+    if (!dims || !ws || !blocks) return fail(IC_ERR_INVALID_ARG, "null argument");
+    if (check_positions(dims->B, dims->Lq, dims->Lk, dims->q_offset) ||
+        check_indexer_shape(dims->H_I, dims->d_I) || dims->k < 1 || dims->Lq < 1)
+        return fail(IC_ERR_INVALID_ARG, "invalid dims");
+    const ic_dims& D = *dims;
+    const IndexerGeom geo = indexer_geom(D.Lq, D.H_I);
+    const long long n_blocks = (long long)D.B * geo.nqb;
+    const size_t block_bytes = (size_t)geo.QB * (size_t)D.Lk * sizeof(float);
+    const DenseGeom dg = dense_geom(D);
+    const bool dense = dg.on && ws_bytes >= dg.mask_bytes + std::max(block_bytes, dg.vt_bytes);
+    const size_t sc_off = dense ? dg.mask_bytes : 0;
+    const FusedGeom fgeo = fused_geom(D);
+    if (!fused_wanted(fgeo, D, opts ? opts->fused_topk : -1) || ws_bytes < sc_off)
+        return fail(IC_ERR_INVALID_ARG, "the stack does not fuse the top-k for these dims");
+    const long long fb = fused_blocks_fitting(fgeo, n_blocks, geo.QB, D.Lk, ws_bytes - sc_off);
+    if (fb < 1) return fail(IC_ERR_WORKSPACE_TOO_SMALL, "no fused chunk fits the workspace");
+    const long long g_last = ((n_blocks - 1) / fb) * fb;          // the last chunk's first block
+    const FusedLayout lay = fused_layout(fgeo, std::min(fb, n_blocks - g_last), geo.QB, D.Lk);
+    int v = 0;
+    cudaError_t e = cudaMemcpyAsync(&v, reinterpret_cast<const uint8_t*>(ws) + sc_off + lay.lcount,
+                                    sizeof v, cudaMemcpyDeviceToHost,
+                                    reinterpret_cast<cudaStream_t>(stream));
+    if (e == cudaSuccess) e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "read the fallback block count");
+    *blocks = v;
+    return IC_OK;
 }
 
 }  // extern "C"

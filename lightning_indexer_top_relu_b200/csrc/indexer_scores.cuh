@@ -20,13 +20,30 @@
 //               k_I tiles (A operand) through a 3-stage ring
 //   warp 1      TMEM allocator + single-thread MMA issuer
 //   warps 2..9  epilogue: tcgen05.ld -> ReLU -> w-weighted head sum -> causal
-//               mask -> fp32 score stores.  Warp w reads TMEM lane quarter
-//               w % 4 and the half of the block's queries given by (w-2) / 4,
-//               so two warps share each SM sub-partition.  Two TMEM
-//               accumulators (2 x 256 columns) let the epilogue of tile j
-//               overlap the MMA of tile j+1.
+//               mask -> output.  Warp w reads TMEM lane quarter w % 4 and the
+//               half of the block's queries given by (w-2) / 4, so two warps
+//               share each SM sub-partition.  Two TMEM accumulators
+//               (2 x 256 columns) let the epilogue of tile j overlap the MMA
+//               of tile j+1.
 // A work unit is (query block, run of up to `tpu` key tiles); units are
 // walked longest-causal-row first and dealt round-robin to the CTAs.
+//
+// Epilogue modes (a template parameter; the MMA and the score arithmetic are
+// the same code in every mode, so a score is bit-identical whichever mode
+// produced it):
+//   IDX_SCORES  every score of the visited key tiles is stored (-inf where
+//               s > t);
+//   IDX_SAMPLE  only key tiles j = m * stride are visited, and their scores
+//               are stored compactly at column m*128 + lane of a sample row;
+//   IDX_CAND    nothing is stored but the scores whose order-preserving key
+//               is at least the row's threshold key: each is appended to the
+//               row's candidate list as (key << 32) | ~s, one 64-bit value
+//               whose unsigned order is (score descending, position
+//               ascending).  The row's counter counts every candidate, also
+//               those past the list's capacity (which are dropped).
+// With a block list (the exact fallback of the fused top-k), the launch's
+// query blocks are taken from a device array whose length is read on the
+// device, and scores go to consecutive buffer rows of those blocks.
 #pragma once
 
 #include "common.cuh"
@@ -39,9 +56,11 @@ constexpr int IDX_STAGES = 3;        // k_I tile ring depth
 constexpr int IDX_EPI_WARPS = 8;
 constexpr int IDX_THREADS = 64 + 32 * IDX_EPI_WARPS;
 
+enum : int { IDX_SCORES = 0, IDX_SAMPLE = 1, IDX_CAND = 2 };
+
 struct IndexerArgs {
     const float* w;        // [B, Lq, H]
-    float* scores;         // row (flattened query row - row_base), stride ld
+    float* scores;         // IDX_SCORES / IDX_SAMPLE: row (flattened query row - row_base), stride ld
     long long ld;
     int B, Lq, Lk, q_offset;
     int QB;                // queries per block
@@ -51,6 +70,18 @@ struct IndexerArgs {
     long long row_base;    // flattened row of the first row of block g0
     int tpu;               // key tiles per work unit
     int max_splits;        // work units per query block (some may be empty)
+    int stride;            // IDX_SAMPLE: key tiles j = m * stride are visited (1 otherwise)
+    // IDX_CAND: per row (flattened row - row_base)
+    const uint32_t* thr;   // threshold key
+    uint32_t* cnt;         // candidates found (may exceed cap)
+    unsigned long long* cand;   // [rows, cap]
+    int cap;
+    // block list: when blk_list is non-null the launch covers list entries
+    // [list_off, list_off + min(list_len, *blk_count - list_off)); score
+    // rows are (entry - list_off) * QB + query
+    const int* blk_list;
+    const int* blk_count;
+    int list_off, list_len;
 };
 
 template <int DI>
@@ -74,25 +105,46 @@ struct IndexerSmem {
 };
 
 struct UnitInfo {
-    int b, i0, nq, j0, j1;
+    int b, i0, nq, j0, j1;   // tiles visited: j0..j1-1 (sample index m in IDX_SAMPLE)
+    long long row0;          // output row of the block's first query
 };
 
+// Work units of this launch (in block-list mode the length is read on the device).
+__device__ __forceinline__ long long idx_units(const IndexerArgs& a) {
+    long long nb = (long long)(a.g1 - a.g0);
+    if (a.blk_list != nullptr) {
+        const long long have = (long long)__ldg(a.blk_count) - a.list_off;
+        nb = have < 0 ? 0 : (have < a.list_len ? have : a.list_len);
+    }
+    return nb * a.max_splits;
+}
+
+template <int MODE>
 __device__ __forceinline__ UnitInfo unit_info(const IndexerArgs& a, long long u) {
     UnitInfo r;
-    int g = a.g1 - 1 - (int)(u / a.max_splits);
-    int split = (int)(u % a.max_splits);
+    const int slot = (int)(u / a.max_splits);
+    int g;
+    if (a.blk_list != nullptr) {
+        g = __ldg(a.blk_list + a.list_off + slot);
+    } else {
+        g = a.g1 - 1 - slot;
+    }
+    const int split = (int)(u % a.max_splits);
     r.b = g / a.nqb;
     r.i0 = (g % a.nqb) * a.QB;
     r.nq = min(a.QB, a.Lq - r.i0);
+    r.row0 = a.blk_list != nullptr ? (long long)slot * a.QB
+                                   : (long long)r.b * a.Lq + r.i0 - a.row_base;
     int t_last = a.q_offset + r.i0 + r.nq - 1;
     int n_vis = min(t_last + 1, a.Lk);
     int nt = (n_vis + IDX_BM - 1) / IDX_BM;
+    if (MODE == IDX_SAMPLE) nt = (nt + a.stride - 1) / a.stride;
     r.j0 = split * a.tpu;
     r.j1 = min(r.j0 + a.tpu, nt);
     return r;
 }
 
-template <int H, int DI>
+template <int H, int DI, int MODE>
 __global__ void __launch_bounds__(IDX_THREADS, 1)
 indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
                       const __grid_constant__ CUtensorMap tmap_k, const IndexerArgs args) {
@@ -117,7 +169,8 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const long long n_units = (long long)(args.g1 - args.g0) * args.max_splits;
+    const long long n_units = idx_units(args);
+    const int kstride = MODE == IDX_SAMPLE ? args.stride : 1;   // key tile = visited index * kstride
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
@@ -153,7 +206,7 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
             uint32_t uq = 0, ta = 0;
             bool ok = true;
             for (long long u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-                UnitInfo ui = unit_info(args, u);
+                UnitInfo ui = unit_info<MODE>(args, u);
                 if (ui.j0 >= ui.j1) continue;
                 const int qb = uq & 1;
                 if (!mbar_wait(&q_empty[qb], ((uq >> 1) & 1) ^ 1)) { ok = false; break; }
@@ -173,7 +226,7 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     uint8_t* adst = a_s + st * S::A_BYTES;
                     for (int kb = 0; kb < KBOX; ++kb)
                         tma_load_3d(adst + kb * IDX_BM * 128, &tmap_k, &a_full[st], kb * 64,
-                                    j * IDX_BM, ui.b);
+                                    j * kstride * IDX_BM, ui.b);
                 }
             }
             // Drain: every load issued has landed before the CTA may retire.
@@ -189,7 +242,7 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
             uint32_t uq = 0, ta = 0;
             bool ok = true;
             for (long long u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-                UnitInfo ui = unit_info(args, u);
+                UnitInfo ui = unit_info<MODE>(args, u);
                 if (ui.j0 >= ui.j1) continue;
                 const int qb = uq & 1;
                 if (!mbar_wait(&q_full[qb], (uq >> 1) & 1)) { ok = false; break; }
@@ -225,10 +278,11 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
         const int cg = (warp - 2) >> 2;           // which half of the block's queries
         const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
         constexpr int QH = (QBMAX + 1) / 2;       // queries per half at most
+        const unsigned lt = (1u << lane) - 1u;
         uint32_t ta = 0, uq = 0;
         bool ok = true;
         for (long long u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-            UnitInfo ui = unit_info(args, u);
+            UnitInfo ui = unit_info<MODE>(args, u);
             if (ui.j0 >= ui.j1) continue;
             const int qb = uq & 1;
             // queries [qlo, qhi) of this block belong to this warp
@@ -240,8 +294,14 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
             // the unit's head weights are in w_s[qb] once q_full[qb] completed
             if (!mbar_wait(&q_full[qb], (uq >> 1) & 1)) { ok = false; break; }
             const float* wsm = w_s + qb * IDX_NMAX + qlo * H;
-            const long long row0 = (long long)ui.b * args.Lq + ui.i0 + qlo - args.row_base;
+            const long long row0 = ui.row0 + qlo;
             const int t0 = args.q_offset + ui.i0 + qlo;
+            uint32_t thrk[QH];
+            if (MODE == IDX_CAND) {
+#pragma unroll
+                for (int q = 0; q < QH; ++q)
+                    thrk[q] = q < qhi - qlo ? __ldg(args.thr + row0 + q) : 0xFFFFFFFFu;
+            }
             for (int j = ui.j0; j < ui.j1; ++j, ++ta) {
                 const int ab = ta & 1;
                 if (!mbar_wait(&acc_full[ab], (ta >> 1) & 1)) { ok = false; break; }
@@ -278,9 +338,29 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 }
                 tc_fence_before();
                 mbar_arrive(&acc_empty[ab]);
-                const int s = j * IDX_BM + wq * 32 + lane;
-                if (s < args.Lk) {
-                    float* dst = args.scores + row0 * args.ld + s;
+                const int s = j * kstride * IDX_BM + wq * 32 + lane;      // key position
+                if (MODE == IDX_CAND) {
+#pragma unroll
+                    for (int q = 0; q < QH; ++q) {
+                        if (q < qhi - qlo) {                              // warp-uniform
+                            const uint32_t key = score_key(acc[q]);
+                            const bool sel = s <= t0 + q && key >= thrk[q];
+                            const unsigned bal = __ballot_sync(0xffffffffu, sel);
+                            if (bal) {
+                                unsigned base = 0;
+                                if (lane == 0) base = atomicAdd(args.cnt + row0 + q, (unsigned)__popc(bal));
+                                base = __shfl_sync(0xffffffffu, base, 0);
+                                const unsigned slot = base + __popc(bal & lt);
+                                if (sel && slot < (unsigned)args.cap)
+                                    args.cand[(row0 + q) * args.cap + slot] =
+                                        ((unsigned long long)key << 32) | (uint32_t)(~(uint32_t)s);
+                            }
+                        }
+                    }
+                } else if (s < args.Lk) {
+                    const long long col = MODE == IDX_SAMPLE ? (long long)j * IDX_BM + wq * 32 + lane
+                                                             : (long long)s;
+                    float* dst = args.scores + row0 * args.ld + col;
 #pragma unroll
                     for (int q = 0; q < QH; ++q) {
                         if (q < qhi - qlo) {

@@ -125,14 +125,21 @@ class GpuBackend:
         d, L, torch = self.dims, self.layers[l], self.torch
         p = min(int(n_rows), d.Lq)
         i0 = d.Lq - p
-        q_idx = L["q_idx"][:, i0:].contiguous()
-        w = L["w"][:, i0:].contiguous()
-        sc = self.ic.indexer_scores(q_idx, L["k_idx"], w, d.q_offset + i0, stream=self.stream)
-        pidx = self.ic.topk_select(sc, d.k, d.q_offset + i0, stream=self.stream)
-        cached = self.idx_cache[:, i0:].contiguous()
-        counts = self.ic.index_overlap(pidx, cached, d.Lk, stream=self.stream)
+        # The slices are copied and the counts read back on the backend's
+        # stream, so they are ordered after the layers already enqueued there
+        # (the copy of the cache waits for the last F layer's top-k, the read
+        # waits for the overlap kernel).
+        st = self.stream if self.stream is not None else torch.cuda.current_stream()
+        with torch.cuda.stream(st):
+            q_idx = L["q_idx"][:, i0:].contiguous()
+            w = L["w"][:, i0:].contiguous()
+            sc = self.ic.indexer_scores(q_idx, L["k_idx"], w, d.q_offset + i0, stream=st)
+            pidx = self.ic.topk_select(sc, d.k, d.q_offset + i0, stream=st)
+            cached = self.idx_cache[:, i0:].contiguous()
+            counts = self.ic.index_overlap(pidx, cached, d.Lk, stream=st)
+            host = counts.cpu()                     # on st: waits for the overlap kernel
         t = np.tile(np.arange(i0, d.Lq) + d.q_offset, d.B)
-        return counts.cpu().numpy(), t                                  # host sync
+        return host.numpy(), t                                          # host sync
 
     def outputs(self):
         return self.outs

@@ -35,7 +35,8 @@ EXPORTS = ("ic_status_string", "ic_last_error_message", "ic_get_last_device_erro
            "ic_layer_stack_forward", "ic_layer_stack_forward_events", "ic_selftest_wait_timeout",
            "ic_sparse_attn_no_alloc", "ic_kernel_launch_count", "ic_sparse_attn_unique",
            "ic_sparse_attn_unique_workspace_bytes", "ic_index_overlap",
-           "ic_layer_stack_dense_rows")
+           "ic_layer_stack_dense_rows", "ic_layer_stack_forward_opts",
+           "ic_layer_stack_fused_fallback_blocks")
 
 MARKS_PER_LAYER = 5        # IC_MARKS_PER_LAYER
 
@@ -57,6 +58,12 @@ class ICLayer(ctypes.Structure):
     _fields_ = [("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
                 ("q_idx", ctypes.c_void_p), ("k_idx", ctypes.c_void_p), ("w", ctypes.c_void_p),
                 ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p), ("idx_dump", ctypes.c_void_p)]
+
+
+class ICStackOptions(ctypes.Structure):
+    """ic_stack_options: fused_topk -1 (library's choice), 0 (store the scores,
+    then top-k) or 1 (fused indexer -> top-k); z the threshold margin."""
+    _fields_ = [("fused_topk", ctypes.c_int), ("z", ctypes.c_float)]
 
 
 class ICDims(ctypes.Structure):
@@ -103,6 +110,14 @@ _lib.ic_index_overlap.restype = _I
 _lib.ic_index_overlap.argtypes = [_P, _P, ctypes.c_longlong, _I, _I, _P, _P]
 _lib.ic_kernel_launch_count.restype = ctypes.c_ulonglong
 _lib.ic_kernel_launch_count.argtypes = []
+_lib.ic_layer_stack_forward_opts.restype = _I
+_lib.ic_layer_stack_forward_opts.argtypes = [ctypes.c_char_p, _I, ctypes.POINTER(ICLayer),
+                                             ctypes.POINTER(ICDims), ctypes.POINTER(ICStackOptions),
+                                             _P, _P, _Z, _P, _P]
+_lib.ic_layer_stack_fused_fallback_blocks.restype = _I
+_lib.ic_layer_stack_fused_fallback_blocks.argtypes = [ctypes.POINTER(ICDims),
+                                                      ctypes.POINTER(ICStackOptions), _P, _Z, _P,
+                                                      ctypes.POINTER(ctypes.c_int)]
 _lib.ic_layer_stack_forward.restype = _I
 _lib.ic_layer_stack_forward.argtypes = [ctypes.c_char_p, _I, ctypes.POINTER(ICLayer),
                                         ctypes.POINTER(ICDims), _P, _P, _Z, _P]
@@ -336,13 +351,17 @@ class LayerStack:
     """Holds the C layer table for repeated ic_layer_stack_forward calls.
 
     layers: per layer a dict with 'q','k','v' (and 'q_idx','k_idx','w' for F
-    layers) CUDA tensors; outputs are allocated once here.
+    layers) CUDA tensors; outputs are allocated once here.  fused_topk / z
+    are the ic_stack_options fields (None: the library's defaults).
     """
 
     def __init__(self, pattern: str, layers: Sequence[dict], dims: ICDims, *, want_lse=False,
-                 dump_idx=False, ws_bytes: Optional[int] = None, rows_per_chunk: int = 0):
+                 dump_idx=False, ws_bytes: Optional[int] = None, rows_per_chunk: int = 0,
+                 fused_topk: Optional[int] = None, z: float = 0.0):
         self.pattern = pattern
         self.dims = dims
+        self.opts = None if fused_topk is None and not z else ICStackOptions(
+            -1 if fused_topk is None else int(fused_topk), float(z))
         n = len(layers)
         d = dims
         for i, L in enumerate(layers):
@@ -383,7 +402,15 @@ class LayerStack:
     def forward(self, stream=None, events=None):
         """Runs the stack; `events` (a ctypes array of MARKS_PER_LAYER*n_layers
         cudaEvent_t handles, or None) selects ic_layer_stack_forward_events."""
-        if events is None:
+        if self.opts is not None:
+            if events is not None and len(events) < MARKS_PER_LAYER * len(self.layers):
+                raise ValueError(f"events holds {len(events)} handles, the stack records "
+                                 f"{MARKS_PER_LAYER * len(self.layers)}")
+            rc = _lib.ic_layer_stack_forward_opts(
+                self._pattern_b, len(self.layers), self.table, ctypes.byref(self.dims),
+                ctypes.byref(self.opts), _ptr(self.idx_cache), _ptr(self.ws), self.ws.numel(),
+                _stream(stream), None if events is None else ctypes.cast(events, ctypes.c_void_p))
+        elif events is None:
             rc = _lib.ic_layer_stack_forward(self._pattern_b, len(self.layers), self.table,
                                              ctypes.byref(self.dims), _ptr(self.idx_cache),
                                              _ptr(self.ws), self.ws.numel(), _stream(stream))
@@ -397,6 +424,16 @@ class LayerStack:
                 ctypes.cast(events, ctypes.c_void_p))
         _check(rc, "ic_layer_stack_forward")
         return self.outs
+
+    def fused_fallback_blocks(self, stream=None) -> int:
+        """Query blocks of the last F layer's last chunk that the fused top-k
+        re-ran on the plain path (synchronises the stream)."""
+        out = ctypes.c_int(0)
+        rc = _lib.ic_layer_stack_fused_fallback_blocks(
+            ctypes.byref(self.dims), None if self.opts is None else ctypes.byref(self.opts),
+            _ptr(self.ws), self.ws.numel(), _stream(stream), ctypes.byref(out))
+        _check(rc, "ic_layer_stack_fused_fallback_blocks")
+        return int(out.value)
 
 
 def layer_stack_forward(pattern: str, layers: Sequence[dict], dims: ICDims, **kw):

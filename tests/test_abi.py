@@ -338,3 +338,49 @@ def test_binding_rejects_inconsistent_shapes_before_the_library(ic):
         ic.LayerStack("F", [dict(full, q=torch.zeros(1, 8, 8, 128, dtype=bf))], dims)
     with pytest.raises(ValueError, match="CUDA"):             # S layers need no indexer inputs
         ic.LayerStack("FS", [full, {"q": q, "k": kv, "v": kv}], dims)
+
+
+def _opts_call(ic, dims, fused, z=0.0, pattern="FS"):
+    n = len(pattern)
+    table = (ic.ICLayer * n)()
+    for i in range(n):
+        table[i] = ic.ICLayer(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, 0x7000, None, None)
+    opts = ic.ICStackOptions(fused, z)
+    return ic.lib().ic_layer_stack_forward_opts(pattern.encode(), n, table, ctypes.byref(dims),
+                                                ctypes.byref(opts), 0x8000, 0x9000, 1 << 20,
+                                                None, None)
+
+
+def test_stack_options_are_checked_before_launch(ic):
+    before = ic.kernel_launch_count()
+    d = _dims(ic)
+    assert _opts_call(ic, d, 2) == 1                      # fused_topk outside {-1, 0, 1}
+    assert _opts_call(ic, d, -2) == 1
+    assert _opts_call(ic, d, 1, z=float("nan")) == 1
+    assert _opts_call(ic, d, 1, pattern="SF") == 3        # leading S still found first
+    big_k = _dims(ic, Lq=8192, Lk=8192, k=4097)
+    assert _opts_call(ic, big_k, 1) == 2                  # the fused top-k needs k <= 4096
+    long = _dims(ic, Lq=64, Lk=262145, q_offset=262081)
+    assert _opts_call(ic, long, 1) == 2                   # ... and Lk <= 262144
+    assert ic.kernel_launch_count() == before
+
+
+def test_fused_fallback_query_rejects_unfused_dims(ic):
+    d = _dims(ic)
+    out = ctypes.c_int(-1)
+    off = ic.ICStackOptions(0, 0.0)
+    rc = ic.lib().ic_layer_stack_fused_fallback_blocks(ctypes.byref(d), ctypes.byref(off), 0x9000,
+                                                       1 << 20, None, ctypes.byref(out))
+    assert rc == 1 and out.value == -1
+    assert ic.lib().ic_layer_stack_fused_fallback_blocks(ctypes.byref(d), None, None, 0, None,
+                                                         ctypes.byref(out)) == 1
+
+
+def test_workspace_holds_the_fused_chunk(ic):
+    """At 64K the workspace of one chunk of all rows holds the fused path's
+    candidate lists (3k per row, 8 bytes each) and sampled scores."""
+    d = _dims(ic, Lq=65536, Lk=65536, H_I=64, d_I=128, Hq=16, d=128, k=2048)
+    full = ic.layer_stack_workspace_bytes(d, 8)
+    assert full >= 65536 * 3 * 2048 * 8
+    # a chunk of 4 query blocks still holds a fused chunk
+    assert ic.layer_stack_workspace_bytes(d, 8, rows_per_chunk=16) >= 16 * 3 * 2048 * 8

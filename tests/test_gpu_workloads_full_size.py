@@ -17,6 +17,10 @@ Every row of every layer is checked on the device:
 
 A bounded sample of rows is checked against the oracle:
 
+* the index rows of every F layer are bit-exact with the oracle's top-k of
+  the GPU's own indexer scores of those rows (at 64K and 128K the stack
+  fuses the top-k into the indexer and never stores the score matrix; the
+  rows' scores come from ic_indexer_scores on the rows alone);
 * top-k set overlap >= 0.99 against the oracle's own scores;
 * attention within the tolerance against the oracle's attention over the
   GPU's own index rows.  At 64K a row rarely has exactly the oracle's set,
@@ -63,6 +67,20 @@ def bench_rows_per_chunk(wl) -> int:
     return max(1, min(wl.B * wl.Lq, (16 * 2 ** 30) // (4 * wl.Lk)))
 
 
+def topk_of_gpu_rows(ic, wl, L, rows):
+    """The oracle's top-k of the GPU indexer's scores of flattened rows
+    `rows`, each scored alone (a one-row call at its own position; a row's
+    scores do not depend on the rows sharing its query block)."""
+    out = []
+    for r in rows:
+        b, i = divmod(int(r), wl.Lq)
+        sc = ic.indexer_scores(L["q_idx"][b:b + 1, i:i + 1].contiguous(), L["k_idx"][b:b + 1],
+                               L["w"][b:b + 1, i:i + 1].contiguous(), wl.q_offset + i)
+        out.append(sc.reshape(1, wl.Lk).cpu().numpy())
+    tpos = oracle.row_positions(wl.B, wl.Lq, wl.q_offset, rows)
+    return oracle.topk_sort(np.concatenate(out), tpos, wl.k)
+
+
 def check_sampled(ic, wl, layers, ref_layers, ref_wl, rows, ref_rows, sync):
     """Runs the stack on `layers` (device tensors) and checks it as the
     module docstring says.  The oracle runs on `ref_layers` (CPU tensors of
@@ -83,6 +101,10 @@ def check_sampled(ic, wl, layers, ref_layers, ref_wl, rows, ref_rows, sync):
     _, ref_idx, _ = oracle.layer_stack(ref_wl.pattern, ref_layers, ref_wl.k, ref_wl.q_offset,
                                        rows=ref_rows)
     sel = torch.as_tensor(np.asarray(rows, dtype=np.int64), device=st.dumps[0].device)
+    for l, c in enumerate(wl.pattern):
+        if c in "F1":
+            want = topk_of_gpu_rows(ic, wl, layers[l], rows)
+            assert np.array_equal(st.dumps[l].reshape(-1, wl.k)[sel].cpu().numpy(), want), l
     for l in range(wl.n_layers):
         gidx = st.dumps[l].reshape(-1, wl.k)[sel].cpu().numpy()
         ov = [len(set(a[a >= 0].tolist()) & set(b[b >= 0].tolist())) / max(int((b >= 0).sum()), 1)
@@ -116,8 +138,9 @@ def test_decode_32k_stack_full_size_sampled_rows(ic):
 
 
 def test_sweep_128k_layer_full_size_chunked_scores(ic):
-    """One F layer at L = 131072: its scores exceed one 16 GiB workspace
-    chunk, so the indexer and top-k run over 4 chunks of 32768 rows."""
+    """One F layer at L = 131072 with the workspace bench.py gives it (16 GiB
+    of scores: 4 chunks of 32768 rows on the plain path; the fused top-k,
+    which the stack takes here, fits its candidate lists in fewer)."""
     wl = synth.WORKLOADS["sweep_128k"]
     assert bench_rows_per_chunk(wl) == 32768
     layers = synth.make_layers(wl, device="cuda")

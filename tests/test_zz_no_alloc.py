@@ -57,11 +57,14 @@ def test_no_alloc_matches_workspace_entry_point_twice(ic):
         assert (lse - ref_lse).abs().max().item() <= LSE_ATOL
 
 
-def test_no_alloc_runs_calls_of_many_rows(ic):
-    # many rows: the slot split (and the scratch it uses) shrinks, results
-    # still equal the workspace entry point's
-    wl = synth.custom(B=300, Lq=1, Lk=600, q_offset=599, H_I=4, d_I=64, k=256, Hq=16, d=128,
+@pytest.mark.parametrize("B", [100, 300])
+def test_no_alloc_runs_calls_of_many_rows(ic, B):
+    # 100 rows still split their slots (2 splits: 100 x 2 x 16 x 129 x 4 bytes
+    # of partials in the scratch); 300 rows, at least two per SM, run one split
+    # each and leave the scratch unused.  Both equal the workspace entry point.
+    wl = synth.custom(B=B, Lq=1, Lk=600, q_offset=599, H_I=4, d_I=64, k=256, Hq=16, d=128,
                       cfg_id=33)
+    assert (ic.sparse_attn_workspace_bytes(B, 1, 16, 128, 256) > 0) == (B == 100)
     L = synth.make_layers(wl)[0]
     sc = oracle.indexer_scores(L["q_idx"], L["k_idx"], L["w"], wl.q_offset).astype(np.float32)
     idx = oracle.topk_sort(sc, oracle.row_positions(wl.B, 1, wl.q_offset), wl.k)
