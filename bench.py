@@ -93,6 +93,10 @@ def work_per_layer(wl, lq_d: int = 0):
     w["indexer_bytes"] = (rows * wl.H_I * wl.d_I * 2 + rows * wl.H_I * 4 + B * Lk * wl.d_I * 2
                           + 4 * sum_vis)
     w["topk_bytes"] = 4 * sum_vis + 4.0 * rows * k
+    # fused indexer -> top-k: the F layer's inputs read once and its index
+    # rows written; no score is stored
+    w["fused_bytes"] = (rows * wl.H_I * wl.d_I * 2 + rows * wl.H_I * 4 + B * Lk * wl.d_I * 2
+                        + 4.0 * rows * k)
     qbd = 128 // wl.Hq if lq_d else 0
     # dense-masked rows: useful flops are those of the selected positions;
     # the kernel executes whole 64-key tiles of 128 rows up to each block's last t
@@ -519,8 +523,12 @@ def kernel_times(wl, pattern, marks, steps: int, npl: int, w):
     return {k: v for k, v in ki.items() if v}
 
 
-def kernel_breakdown(ki, w, steps: int, ms_per_step: float, peaks, sm_mhz: float, n_sms: int):
-    """Per-kernel rates and shares of the step from kernel_times() output."""
+def kernel_breakdown(ki, w, steps: int, ms_per_step: float, peaks, sm_mhz: float, n_sms: int,
+                     fused: bool = False):
+    """Per-kernel rates and shares of the step from kernel_times() output.
+    `fused`: the stack fused the top-k into the indexer (the indexer group
+    then covers the sampled pass, the thresholds and the candidate pass, and
+    the top-k group the exact selection and the fallback rounds)."""
     kernels, per_step = {}, {}
     for name, vals in ki.items():
         avg = float(np.mean(vals))
@@ -529,11 +537,18 @@ def kernel_breakdown(ki, w, steps: int, ms_per_step: float, peaks, sm_mhz: float
         ent = {"launches_per_step": len(vals) // steps, "ms_per_launch": avg,
                "share": per_step[name] / ms_per_step}
         if name == "indexer":
+            if fused:
+                ent["covers"] = ("fused indexer: sampled key tiles + per-row thresholds + the "
+                                 "candidate pass (no score stored); tflops counts the flops of "
+                                 "every visible score once")
             ent["tflops"] = w["indexer_flops"] / sec / 1e12
             ent["frac_of_bf16_peak"] = ent["tflops"] / peaks["bf16_tflops"]
             if peaks.get("bf16_tflops_sustained"):
                 ent["frac_of_bf16_sustained"] = ent["tflops"] / peaks["bf16_tflops_sustained"]
             ent["gbs"] = w["indexer_bytes"] / sec / 1e9
+        elif name == "topk" and fused:
+            ent["covers"] = ("exact selection over the candidate lists (also writes the selection "
+                             "bitmask of dense-masked rows) + the fallback rounds")
         elif name == "topk":
             ent["covers"] = "top-k select (also writes the selection bitmask of dense-masked rows)"
             ent["gbs"] = w["topk_bytes"] / sec / 1e9
@@ -587,6 +602,9 @@ def roofline_of(kernels, w, peaks, clk, workload: str):
                 "frac_of_burst": kd["tflops"] / peaks["bf16_tflops"],
                 "algorithmic_per_launch": w["indexer_flops"],
                 "note": "achieved = 2*H_I*d_I flops per (query, visible key) / event time"}
+    elif dom == "topk" and "gbs" not in kd:
+        roof = {"kernel": "fused_select", "bound": "latency", "achieved": None, "peak": None,
+                "unit": None, "frac": None}
     elif dom == "topk":
         roof = {"kernel": "topk_select", "bound": "hbm", "achieved": kd["gbs"],
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": kd["gbs"] / peaks["hbm_gbs"],
@@ -620,6 +638,16 @@ def default_rows_per_chunk(wl) -> int:
     return max(1, min(wl.B * wl.Lq, (16 * 2 ** 30) // (4 * wl.Lk)))
 
 
+def fused_state(ic, stack):
+    """(fused, fallback blocks): whether the stack fused the top-k into the
+    indexer, and how many query blocks of its last F layer's last chunk fell
+    back to the plain path (synchronises)."""
+    try:
+        return True, stack.fused_fallback_blocks()
+    except ic.IndexCacheError:
+        return False, None
+
+
 def stack_point(ic, wl, pattern, layers, stream, flush, peaks, n_sms, clk, budget_ms,
                 rows_per_chunk=0, warmup=1):
     """One supplementary stack measurement: step time, tokens/s, the indexer
@@ -634,10 +662,11 @@ def stack_point(ic, wl, pattern, layers, stream, flush, peaks, n_sms, clk, budge
         raise RuntimeError(f"device error in the {wl.name} {pattern} point")
     w = work_per_layer(wl, lq_d)
     msps = float(np.mean(ms))
+    fused, fallback = fused_state(ic, stack)
     ki = kernel_times(wl, pattern, marks, steps, ic.MARKS_PER_LAYER, w)
     kern, per_step = kernel_breakdown(ki, w, steps, msps, peaks,
-                                      (clk or {}).get("sm_mhz") or 1965.0, n_sms)
-    out = {"pattern": pattern, "steps": steps, "ms_per_step": msps,
+                                      (clk or {}).get("sm_mhz") or 1965.0, n_sms, fused)
+    out = {"pattern": pattern, "steps": steps, "ms_per_step": msps, "fused_topk": fused,
            "tokens_per_s": wl.B * wl.Lq / (msps * 1e-3),
            "indexer_share": (per_step.get("indexer", 0) + per_step.get("topk", 0)) / msps}
     if "indexer" in kern:
@@ -751,6 +780,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-all-f", action="store_true")
+    ap.add_argument("--no-fused-compare", action="store_true",
+                    help="skip timing the plain (unfused) top-k path beside the fused one")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the supplementary points (16-layer sweep, decode_32k)")
     ap.add_argument("--sweep", default="4,16,64,128",
@@ -844,9 +875,11 @@ def main():
     ms_per_step, tokens, value = aggregate_over_ranks(local_ms, float(wl.B * wl.Lq), pg, dev)
 
     w = work_per_layer(wl, lq_d)
+    fused, fallback = fused_state(ic, stack)
     ki = kernel_times(wl, pattern, marks, args.steps, npl, w)
     sm_mhz = (clk or {}).get("sm_mhz") or 1965.0
-    kernels, per_step = kernel_breakdown(ki, w, args.steps, ms_per_step, peaks, sm_mhz, n_sms)
+    kernels, per_step = kernel_breakdown(ki, w, args.steps, ms_per_step, peaks, sm_mhz, n_sms,
+                                         fused)
     roof = roofline_of(kernels, w, peaks, clk, wl.name)
     del marks
 
@@ -860,6 +893,32 @@ def main():
             "wall_s_timed": wall}
     if clk is not None:
         line["clocks"] = clk
+
+    # ---- the fused indexer -> top-k against the plain path (scores stored per chunk)
+    if fused:
+        f_ms = float(np.mean(ki["indexer"])) + float(np.mean(ki["topk"]))
+        ent = {"ms_per_f_layer": f_ms,
+               "bytes_per_f_layer": w["fused_bytes"],
+               "gbs": w["fused_bytes"] / (f_ms * 1e-3) / 1e9,
+               "note": ("indexer + top-k of one F layer: inputs read once and index rows "
+                        "written, no score stored; bound by the tensor cores, not by these bytes"),
+               "fallback_blocks_last_f_layer": fallback}
+        ent["frac_of_hbm"] = ent["gbs"] / peaks["hbm_gbs"]
+        line["fused_topk"] = ent
+    if fused and not args.no_fused_compare:
+        ent = line["fused_topk"]
+        f_ms = ent["ms_per_f_layer"]
+        plain = ic.LayerStack(pattern, layers, dims, rows_per_chunk=rpc, fused_topk=0)
+        ms_p, marks_p = time_stack(ic, plain, stream, flush, max(3, args.steps // 4), 1)
+        ki_p = kernel_times(wl, pattern, marks_p, len(ms_p), npl, w)
+        ent["plain_ms_per_f_layer"] = (float(np.mean(ki_p["indexer"]))
+                                       + float(np.mean(ki_p["topk"])))
+        ent["plain_ms_per_step"] = float(np.mean(ms_p))
+        ent["speedup_of_fusion_per_f_layer"] = ent["plain_ms_per_f_layer"] / f_ms
+        line["fused_topk"] = ent
+        del plain, marks_p
+        if ic.get_last_device_error() != 0:
+            raise RuntimeError("device error in the plain-path leg")
 
     # ---- the same stack with every layer Full, for the F/S speed-up
     if need_all:

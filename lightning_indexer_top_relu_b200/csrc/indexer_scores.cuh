@@ -19,8 +19,9 @@
 //               weights w (bulk copy), once per work unit, double-buffered;
 //               k_I tiles (A operand) through a 3-stage ring
 //   warp 1      TMEM allocator + single-thread MMA issuer
-//   warps 2..9  epilogue: tcgen05.ld -> ReLU -> w-weighted head sum -> causal
-//               mask -> output.  Warp w reads TMEM lane quarter w % 4 and the
+//   warps 2..9  epilogue: tcgen05.ld -> ReLU -> w-weighted head sum (with
+//               16+ heads, two packed f32x2 partial sums per query: four
+//               independent FMA chains) -> causal mask -> output.  Warp w reads TMEM lane quarter w % 4 and the
 //               half of the block's queries given by (w-2) / 4, so two warps
 //               share each SM sub-partition.  Two TMEM accumulators
 //               (2 x 256 columns) let the epilogue of tile j overlap the MMA
@@ -306,9 +307,18 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 const int ab = ta & 1;
                 if (!mbar_wait(&acc_full[ab], (ta >> 1) & 1)) { ok = false; break; }
                 tc_fence_after();
-                float acc[QH];
+                // H >= 16: two packed (f32x2) partial sums per query, over heads
+                // 4i+{0,1} and 4i+{2,3} -- four independent FMA chains instead
+                // of one.  H <= 8 (short chains, many queries per warp): one
+                // scalar sum per query.
+                constexpr bool PACKED = H >= 16;
+                constexpr int QP = PACKED ? QH : 1;
+                float2 acc2[QP][2];
+                float accs[PACKED ? 1 : QH];
 #pragma unroll
-                for (int q = 0; q < QH; ++q) acc[q] = 0.0f;
+                for (int q = 0; q < QP; ++q) acc2[q][0] = acc2[q][1] = make_float2(0.0f, 0.0f);
+#pragma unroll
+                for (int q = 0; q < (PACKED ? 1 : QH); ++q) accs[q] = 0.0f;
                 const uint32_t taddr =
                     tmem_base + lane_base + (uint32_t)(ab * IDX_NMAX + qlo * H);
                 // 64 columns per batch: two 32-column TMEM loads, one wait, reduce.
@@ -325,16 +335,35 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
                         for (int jj = 0; jj < 64; jj += 4) {
                             const int c = bt * 64 + jj;
                             if (c < ncol) {
+                                // columns c..c+3 are four heads of one query (H % 4 == 0)
+                                const int q = c / H;
                                 const float4 wv = *reinterpret_cast<const float4*>(wsm + c);
-                                const float wj[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-                                for (int e = 0; e < 4; ++e) {
-                                    const int q = (bt * 64 + jj + e) / H;
-                                    acc[q] = fmaf(wj[e], fmaxf(__uint_as_float(v[jj + e]), 0.0f), acc[q]);
+                                const float2 r01 = make_float2(fmaxf(__uint_as_float(v[jj]), 0.0f),
+                                                               fmaxf(__uint_as_float(v[jj + 1]), 0.0f));
+                                const float2 r23 = make_float2(fmaxf(__uint_as_float(v[jj + 2]), 0.0f),
+                                                               fmaxf(__uint_as_float(v[jj + 3]), 0.0f));
+                                if constexpr (PACKED) {
+                                    acc2[q % QP][0] = __ffma2_rn(make_float2(wv.x, wv.y), r01, acc2[q % QP][0]);
+                                    acc2[q % QP][1] = __ffma2_rn(make_float2(wv.z, wv.w), r23, acc2[q % QP][1]);
+                                } else {
+                                    float& a = accs[q];
+                                    a = fmaf(wv.x, r01.x, a);
+                                    a = fmaf(wv.y, r01.y, a);
+                                    a = fmaf(wv.z, r23.x, a);
+                                    a = fmaf(wv.w, r23.y, a);
                                 }
                             }
                         }
                     }
+                }
+                float acc[QH];
+#pragma unroll
+                for (int q = 0; q < QH; ++q) {
+                    if constexpr (PACKED)
+                        acc[q] = (acc2[q % QP][0].x + acc2[q % QP][0].y) +
+                                 (acc2[q % QP][1].x + acc2[q % QP][1].y);
+                    else
+                        acc[q] = accs[q % (PACKED ? 1 : QH)];
                 }
                 tc_fence_before();
                 mbar_arrive(&acc_empty[ab]);

@@ -17,6 +17,8 @@ Workloads (named by what they are):
   cache (q_offset = 32767), 16 layers (FSSS)x4, indexer 64 x 128, k=2048.
 * ``sweep_<L>``     B=1, one layer, L in {4096, 16384, 65536, 131072},
   indexer 64 x 128, k=2048.
+* ``layer_32k``     B=1, one F layer at L=32768 with the sweep's shapes (the
+  smallest prefill whose late rows gather K/V rows; used for kernel profiles).
 
 Correlated layers: the pages report that adjacent layers share 70-100% of
 their top-k selections (IndexCache technical summary, Probleemstelling; kualia
@@ -84,6 +86,9 @@ WORKLOADS: Dict[str, Workload] = {
 for _L in (4096, 16384, 65536, 131072):
     WORKLOADS[f"sweep_{_L // 1024}k"] = _prefill(f"sweep_{_L // 1024}k", _L, 1, 64, 128, 2048, 16,
                                                  128, "F", 5)
+# A single F layer at L=32768 (shapes of the sweep): the smallest prefill in
+# which rows t >= 8k = 16384 gather their K/V rows, for kernel profiles.
+WORKLOADS["layer_32k"] = _prefill("layer_32k", 32768, 1, 64, 128, 2048, 16, 128, "F", 6)
 
 
 def custom(name: str = "custom", *, B=1, Lq, Lk=None, n_layers=1, H_I=4, d_I=64, k=64, Hq=8,

@@ -118,7 +118,7 @@ def test_every_row_falls_back_when_all_scores_tie(ic):
     """w = 0: every score is 0, so every row with more than 3k visible
     positions has all of them as candidates, overflows its list and falls
     back; every row's index row is the closed form [0 .. min(k, t+1) - 1]."""
-    wl = synth.Workload("w_zero", 1, 4096, 4096, 0, 32, 128, 256, 16, 128, "FS", 0, 52, True)
+    wl = synth.Workload("w_zero", 1, 4096, 4096, 2, 32, 128, 256, 16, 128, "FS", 0, 52, True)
     cpu = synth.make_layers(wl)
     cpu[0]["w"] = torch.zeros_like(cpu[0]["w"])
     layers = [{n: t.cuda() for n, t in L.items()} for L in cpu]
@@ -137,7 +137,7 @@ def test_tiny_margin_mixes_fallback_and_fused_rows(ic):
     """z = 0.001 puts the threshold near the sample quantile itself, so about
     half the long rows find fewer than k candidates: their blocks fall back,
     the others are selected from candidates; all rows stay exact."""
-    wl = synth.Workload("z_tiny", 1, 6144, 6144, 0, 64, 128, 256, 16, 128, "FS", 0, 53, True)
+    wl = synth.Workload("z_tiny", 1, 6144, 6144, 2, 64, 128, 256, 16, 128, "FS", 0, 53, True)
     layers = [{n: t.cuda() for n, t in L.items()} for L in synth.make_layers(wl)]
     st = _stack(ic, wl, layers, 1, z=0.001)
     QB = 256 // wl.H_I
@@ -153,7 +153,7 @@ def test_chunked_workspace_with_fallback_rounds(ic, rows_per_chunk):
     several chunks, each with its own thresholds, candidates and 8 fallback
     rounds over a buffer of an eighth of its blocks; a tiny margin makes
     blocks of every chunk fall back."""
-    wl = synth.Workload("chunks", 1, 5000, 5000, 0, 32, 128, 128, 16, 128, "FS", 0, 54, True)
+    wl = synth.Workload("chunks", 1, 5000, 5000, 2, 32, 128, 128, 16, 128, "FS", 0, 54, True)
     layers = [{n: t.cuda() for n, t in L.items()} for L in synth.make_layers(wl)]
     st = _stack(ic, wl, layers, 1, z=0.001, rows_per_chunk=rows_per_chunk)
     want = _expected(ic, wl, layers[0])
@@ -167,7 +167,7 @@ def test_indexer_rows_do_not_depend_on_their_query_block(ic):
     (the full-size tests take expected index rows from row slices of the
     indexer): rows [i0, i0 + n) scored with q_offset = i0 equal those rows
     of the full call."""
-    wl = synth.Workload("slices", 1, 2000, 2000, 0, 64, 128, 128, 16, 128, "F", 0, 55, True)
+    wl = synth.Workload("slices", 1, 2000, 2000, 1, 64, 128, 128, 16, 128, "F", 0, 55, True)
     L = {n: t.cuda() for n, t in synth.make_layers(wl)[0].items()}
     full = ic.indexer_scores(L["q_idx"], L["k_idx"], L["w"], 0)
     for i0, n in ((0, 5), (3, 7), (1001, 999), (1998, 2), (500, 1)):

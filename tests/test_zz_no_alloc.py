@@ -59,8 +59,8 @@ def test_no_alloc_matches_workspace_entry_point_twice(ic):
 
 @pytest.mark.parametrize("B", [100, 300])
 def test_no_alloc_runs_calls_of_many_rows(ic, B):
-    # 100 rows still split their slots (2 splits: 100 x 2 x 16 x 129 x 4 bytes
-    # of partials in the scratch); 300 rows, at least two per SM, run one split
+    # 100 rows still split their slots (their partials go through the
+    # scratch); 300 rows fill the CTAs the GPU holds at once, run one split
     # each and leave the scratch unused.  Both equal the workspace entry point.
     wl = synth.custom(B=B, Lq=1, Lk=600, q_offset=599, H_I=4, d_I=64, k=256, Hq=16, d=128,
                       cfg_id=33)
