@@ -87,7 +87,7 @@ def work_per_layer(wl, lq_d: int = 0):
     sel_row = np.minimum(vis, k)
     sum_vis = B * vis.sum()                       # sum over rows of visible positions
     rows = B * Lq
-    w = {}
+    w = {"rows": rows}
     w["indexer_flops"] = 2.0 * wl.H_I * wl.d_I * sum_vis
     # q_I + w read once, k_I once per batch element, causal scores written
     w["indexer_bytes"] = (rows * wl.H_I * wl.d_I * 2 + rows * wl.H_I * 4 + B * Lk * wl.d_I * 2
@@ -122,33 +122,58 @@ def work_per_layer(wl, lq_d: int = 0):
 
 # ---------------------------------------------------------------- ncu traffic
 
-_KERNEL_SRC = {"sparse_attn": ("sparse_attn_kernel", "sparse_attn.cuh"),
-               "dense_attn": ("dense_attn_kernel", "dense_attn.cuh"),
-               "indexer_scores": ("indexer_scores_kernel", "indexer_scores.cuh"),
-               "topk_select": ("topk_select_kernel", "topk_select.cuh")}
+_KERNEL_SRC = {"sparse_attn": ("sparse_attn_kernel", ("sparse_attn.cuh",)),
+               "dense_attn": ("dense_attn_kernel", ("dense_attn.cuh",)),
+               "indexer_scores": ("indexer_scores_kernel", ("indexer_scores.cuh",)),
+               "topk_select": ("topk_select_kernel", ("topk_select.cuh",)),
+               "fused_select": ("fused_select_kernel", ("fused_topk.cuh",))}
 
 
-def profile_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from the committed ncu summary of this kernel and
-    workload, or None when there is none or the kernel source changed since
-    the counters were taken (the summary records a hash of the source)."""
+def _read_profile(path, srcs):
+    """(dram bytes per launch, units per launch or None) of a committed ncu
+    summary, or None when the kernel's sources changed since the capture
+    (the summary records a hash of them)."""
     import hashlib
-    name, src = _KERNEL_SRC[kernel]
-    path = os.path.join(ROOT, "profiles", f"{name}_{workload}.md")
-    if not os.path.exists(path):
-        return None
     h = hashlib.sha256()
-    for f in (src, "common.cuh"):
+    for f in tuple(srcs) + ("common.cuh",):
         with open(os.path.join(ROOT, "lightning_indexer_top_relu_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
-    want, traffic = None, None
+    want = traffic = units = None
     with open(path) as fh:
         for line in fh:
             if line.startswith("source_hash:"):
                 want = line.split(":", 1)[1].strip()
             elif line.startswith("dram_bytes_per_launch:"):
-                traffic = int(line.split(":", 1)[1].strip())
-    return traffic if want == h.hexdigest()[:16] else None
+                try:
+                    traffic = int(line.split(":", 1)[1].strip())
+                except ValueError:
+                    traffic = None
+            elif line.startswith("units_per_launch:"):
+                units = float(line.split(":", 1)[1].strip())
+    if want != h.hexdigest()[:16] or traffic is None:
+        return None
+    return traffic, units
+
+
+def profile_traffic(kernel: str, workload: str, units: float = 0.0):
+    """DRAM bytes per launch of `kernel` from the committed ncu summaries:
+    the summary of this workload when there is one; otherwise a summary of a
+    smaller case of the same kernel that records its units per launch (query
+    rows), scaled by units / its units -- the full-size workloads are too
+    large for a full ncu capture.  Returns (bytes or None, where from)."""
+    import glob
+    name, srcs = _KERNEL_SRC[kernel]
+    path = os.path.join(ROOT, "profiles", f"{name}_{workload}.md")
+    if os.path.exists(path):
+        got = _read_profile(path, srcs)
+        return (got[0], os.path.basename(path)) if got else (None, None)
+    if units > 0:
+        for path in sorted(glob.glob(os.path.join(ROOT, "profiles", f"{name}_*.md"))):
+            got = _read_profile(path, srcs)
+            if got and got[1]:
+                return int(got[0] * units / got[1]), (f"{os.path.basename(path)} scaled by "
+                                                      f"{units:g} / {got[1]:g} rows")
+    return None, None
 
 
 # ---------------------------------------------------------------- clocks
@@ -629,7 +654,13 @@ def roofline_of(kernels, w, peaks, clk, workload: str):
                 "note": ("achieved counts the logical K/V gather bytes; when a layer's K/V stay "
                          "L2-resident, DRAM traffic (`traffic`) is far below them")}
     roof["peak_source"] = peaks["source"]
-    roof["traffic"] = profile_traffic(roof["kernel"], workload)
+    units = {"indexer_scores": w.get("rows", 0), "sparse_attn": w.get("gather_rows", 0),
+             "dense_attn": w.get("dense_rows", 0), "topk_select": w.get("rows", 0),
+             "fused_select": w.get("rows", 0)}.get(roof["kernel"], 0)
+    roof["traffic"], src = (profile_traffic(roof["kernel"], workload, units)
+                            if roof["kernel"] in _KERNEL_SRC else (None, None))
+    if src:
+        roof["traffic_from"] = src
     return roof
 
 
@@ -724,12 +755,16 @@ def decode_point(ic, dev, stream, flush, peaks, n_sms, clk):
 
 
 def e2e_leg(ic, stack, layers, pattern, stream, steps: int, pg, dev, tokens: float):
-    """The same stack end to end through the public call with host buffers:
-    every step copies that step's inputs (every layer's q/K/V and the F
+    """The same stack end to end through the public call with host buffers.
+    Every step copies that step's inputs (every layer's q/K/V and the F
     layers' q_I/k_I/w) from pinned host memory to the device, runs the stack,
-    and copies every layer's output back to pinned host memory, all inside
-    the timed region.  The host copies are made once from the device-drawn
-    inputs (drawing several GB on the host would take minutes)."""
+    and copies every layer's output back to pinned host memory; all of it is
+    inside the timed region.  Steps are pipelined the way a serving loop
+    would run them: two device copies of the inputs and outputs alternate, the
+    host-to-device copies of step s+1 run on one copy stream and the
+    device-to-host copies of step s-1 on another while step s computes.  The
+    host copies are made once from the device-drawn inputs (drawing several
+    GB on the host would take minutes)."""
     used = [{k: v for k, v in L.items() if k in ("q", "k", "v") or pattern[i] in "F1"}
             for i, L in enumerate(layers)]
     pinned = []
@@ -744,29 +779,69 @@ def e2e_leg(ic, stack, layers, pattern, stream, steps: int, pg, dev, tokens: flo
     h2d = sum(v.numel() * v.element_size() for L in pinned for v in L.values())
     d2h = sum(o.numel() * o.element_size() for o in stack.outs)
 
-    def e2e_step():
-        for i, L in enumerate(pinned):
-            for k, v in L.items():
-                layers[i][k].copy_(v, non_blocking=True)
-        stack.forward(stream)
-        for o, h in zip(stack.outs, outs_host):
-            h.copy_(o, non_blocking=True)
+    # a second device copy of the inputs, and a second stack (its own outputs,
+    # the first stack's workspace: both run on the compute stream, in order)
+    layers2 = [{k: torch.empty_like(v) for k, v in L.items()} for L in layers]
+    stack2 = ic.LayerStack(pattern, layers2, stack.dims, ws_bytes=16,
+                           fused_topk=None if stack.opts is None else stack.opts.fused_topk,
+                           z=0.0 if stack.opts is None else stack.opts.z)
+    stack2.ws = stack.ws
+    sets = [(layers, stack), (layers2, stack2)]
+    up, down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    uploaded = [torch.cuda.Event() for _ in sets]
+    computed = [torch.cuda.Event() for _ in sets]
+    fetched = [torch.cuda.Event() for _ in sets]
 
-    e2e_step()
+    def upload(b):
+        # set b's inputs are free once its last stack run is done
+        up.wait_event(computed[b])
+        with torch.cuda.stream(up):
+            for i, L in enumerate(pinned):
+                for k, v in L.items():
+                    sets[b][0][i][k].copy_(v, non_blocking=True)
+        uploaded[b].record(up)
+
+    def run(b):
+        stream.wait_event(uploaded[b])
+        stream.wait_event(fetched[b])          # set b's outputs were read back
+        sets[b][1].forward(stream)
+        computed[b].record(stream)
+        down.wait_event(computed[b])
+        with torch.cuda.stream(down):
+            for o, h in zip(sets[b][1].outs, outs_host):
+                h.copy_(o, non_blocking=True)
+        fetched[b].record(down)
+
+    for b in range(2):                        # untimed warm-up of both sets
+        computed[b].record(stream)
+        fetched[b].record(down)
+    for b in range(2):
+        upload(b)
+        run(b)
     torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if pg is not None:
         pg.barrier()
-    a.record(stream)
-    for _ in range(steps):
-        e2e_step()
-    b.record(stream)
     torch.cuda.synchronize()
-    e_ms, _, e_val = aggregate_over_ranks(a.elapsed_time(b) / steps, tokens, pg, dev)
-    del pinned, outs_host
+    t0.record(up)
+    upload(0)
+    for s in range(steps):
+        b = s % 2
+        if s + 1 < steps:
+            upload(1 - b)                     # next step's inputs while this one computes
+        run(b)
+    end = torch.cuda.Event(enable_timing=True)
+    end.record(down)
+    up.wait_event(end)
+    t1.record(up)
+    torch.cuda.synchronize()
+    e_ms, _, e_val = aggregate_over_ranks(t0.elapsed_time(t1) / steps, tokens, pg, dev)
+    del pinned, outs_host, layers2, stack2
     return {"value": e_val, "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "ms_per_step": e_ms, "steps": steps,
-            "note": "pinned host buffers; copies and the stack on one stream, in order"}
+            "note": ("pinned host buffers; per step the inputs are copied in and every output "
+                     "copied out; copies of neighbouring steps overlap the stack on two copy "
+                     "streams (two device sets of inputs and outputs alternate)")}
 
 
 def main():
@@ -780,6 +855,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-all-f", action="store_true")
+    ap.add_argument("--fused-topk", type=int, default=-1, choices=[-1, 0, 1],
+                    help="F layers: -1 the library's choice, 0 scores stored then top-k, "
+                         "1 fused indexer -> top-k")
     ap.add_argument("--no-fused-compare", action="store_true",
                     help="skip timing the plain (unfused) top-k path beside the fused one")
     ap.add_argument("--no-extras", action="store_true",
@@ -830,7 +908,8 @@ def main():
     torch.cuda.synchronize()
     dims = ic.make_dims(wl.B, wl.Lq, wl.Lk, wl.q_offset, wl.H_I, wl.d_I, wl.Hq, wl.d, wl.k)
     rpc = args.rows_per_chunk if args.rows_per_chunk > 0 else default_rows_per_chunk(wl)
-    stack = ic.LayerStack(pattern, layers, dims, rows_per_chunk=rpc)
+    fmode = None if args.fused_topk < 0 else args.fused_topk
+    stack = ic.LayerStack(pattern, layers, dims, rows_per_chunk=rpc, fused_topk=fmode)
     lq_d = ic.layer_stack_dense_rows(dims, stack.ws.numel())
     stream = torch.cuda.current_stream()
     n = wl.n_layers
@@ -922,7 +1001,7 @@ def main():
 
     # ---- the same stack with every layer Full, for the F/S speed-up
     if need_all:
-        stack_f = ic.LayerStack("F" * n, layers, dims, rows_per_chunk=rpc)
+        stack_f = ic.LayerStack("F" * n, layers, dims, rows_per_chunk=rpc, fused_topk=fmode)
         k_f = max(3, args.steps // 2)
         ms_f, marks_f = time_stack(ic, stack_f, stream, flush, k_f, 2)
         msf = float(np.mean(ms_f))

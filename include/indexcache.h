@@ -147,10 +147,10 @@ size_t ic_sparse_attn_workspace_bytes(int B, int Lq, int Hq, int d, int k_slots)
  * partial results in a fixed 4 MiB array inside the library instead of a
  * workspace; every GPU that loads the library holds that array until the
  * process exits.
- *   - Rows split their slots only while rows x splits stays within three
- *     CTAs per SM, so with the supported Hq <= 16 and d <= 128 the partials
- *     take at most 3 x SMs x 16 x 129 x 4 bytes (3.7 MB on a 148-SM B200) and
- *     the preferred split always fits.  On a GPU with more SMs the call would run
+ *   - Rows split their slots only while rows x splits stays within two CTAs
+ *     per SM, so with the supported Hq <= 16 and d <= 128 the partials take
+ *     at most 2 x SMs x 16 x 129 x 4 bytes (2.4 MB on a 148-SM B200) and the
+ *     preferred split always fits.  On a GPU with more SMs the call would run
  *     with fewer splits (one split needs no scratch); results are the same.
  *   - The first call on a device looks up the array's device address (once per
  *     device, with that device current); make that first call before any

@@ -20,7 +20,6 @@
 #include "common.cuh"
 #include "dense_attn.cuh"
 #include "fused_topk.cuh"
-#include "gather_attn.cuh"
 #include "index_overlap.cuh"
 #include "indexer_scores.cuh"
 #include "sparse_attn.cuh"
@@ -307,19 +306,11 @@ int launch_topk(const float* scores, long long ld, long long row_base, long long
 
 // ---------------------------------------------------------------- sparse attention
 
-// Gather rows into tensor-core fragments in registers (gather_attn_kernel)
-// rather than through cp.async into shared memory (sparse_attn_kernel).
-constexpr bool GATHER_IN_REGISTERS = true;
-
 int attn_splits(long long n_rows, int k_slots, int sms) {
-    // rows x splits CTAs fill the CTAs per SM that fit, in one wave; each
-    // split keeps at least a few slot groups per warp (pair) for its pipeline
-    const long long per_sm = GATHER_IN_REGISTERS ? 3 : 2;
-    const long long grain = GATHER_IN_REGISTERS ? 4LL * ic::GA_PAIRS * ic::GA_GROUP
-                                                : (long long)ic::SA_WARPS * ic::SA_BLOCK;
-    if (n_rows >= per_sm * sms) return 1;
-    long long s = (per_sm * sms) / n_rows;
-    s = std::min<long long>(s, (k_slots + grain - 1) / grain);
+    // rows x splits CTAs fill the 2 CTAs per SM that fit, in one wave
+    if (n_rows >= 2LL * sms) return 1;
+    long long s = (2LL * sms) / n_rows;
+    s = std::min<long long>(s, (k_slots + ic::SA_WARPS * ic::SA_BLOCK - 1) / (ic::SA_WARPS * ic::SA_BLOCK));
     s = std::min<long long>(s, 64);
     return (int)std::max<long long>(1, s);
 }
@@ -365,12 +356,7 @@ int launch_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, const i
     a.rows_per_b = rows_per_b;
     a.row_i0 = row_i0;
     dim3 grid((unsigned)n_rows, (unsigned)splits);
-    if (GATHER_IN_REGISTERS) {
-        if (d == 64)
-            ic::gather_attn_kernel<64><<<grid, ic::GA_THREADS, ic::GaSmem<64>::BYTES, st>>>(a);
-        else
-            ic::gather_attn_kernel<128><<<grid, ic::GA_THREADS, ic::GaSmem<128>::BYTES, st>>>(a);
-    } else if (d == 64) {
+    if (d == 64) {
         ic::sparse_attn_kernel<64><<<grid, ic::SA_THREADS, ic::SaSmem<64>::BYTES, st>>>(a);
     } else {
         ic::sparse_attn_kernel<128><<<grid, ic::SA_THREADS, ic::SaSmem<128>::BYTES, st>>>(a);
@@ -727,10 +713,6 @@ int device_setup(int* dev_out, int* sms_out) {
                              cudaFuncAttributeMaxDynamicSharedMemorySize, ic::SaSmem<64>::BYTES);
         cudaFuncSetAttribute(ic::sparse_attn_kernel<128>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, ic::SaSmem<128>::BYTES);
-        cudaFuncSetAttribute(ic::gather_attn_kernel<64>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, ic::GaSmem<64>::BYTES);
-        cudaFuncSetAttribute(ic::gather_attn_kernel<128>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, ic::GaSmem<128>::BYTES);
         e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
         g_sms[dev] = sms;

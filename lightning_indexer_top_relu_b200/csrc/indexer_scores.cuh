@@ -19,9 +19,11 @@
 //               weights w (bulk copy), once per work unit, double-buffered;
 //               k_I tiles (A operand) through a 3-stage ring
 //   warp 1      TMEM allocator + single-thread MMA issuer
-//   warps 2..9  epilogue: tcgen05.ld -> ReLU -> w-weighted head sum (with
-//               16+ heads, two packed f32x2 partial sums per query: four
-//               independent FMA chains) -> causal mask -> output.  Warp w reads TMEM lane quarter w % 4 and the
+//   warps 2..9  epilogue: tcgen05.ld -> ReLU -> w-weighted head sum -> causal
+//               mask -> output.  With 16+ heads the TMEM reads use the
+//               16x256b shape: a thread holds 2 keys x a quarter of the
+//               columns, its quarter of the head weights stays in registers
+//               for the unit, and a quad adds its partial sums by shuffles.  Warp w reads TMEM lane quarter w % 4 and the
 //               half of the block's queries given by (w-2) / 4, so two warps
 //               share each SM sub-partition.  Two TMEM accumulators
 //               (2 x 256 columns) let the epilogue of tile j overlap the MMA
@@ -58,6 +60,30 @@ constexpr int IDX_EPI_WARPS = 8;
 constexpr int IDX_THREADS = 64 + 32 * IDX_EPI_WARPS;
 
 enum : int { IDX_SCORES = 0, IDX_SAMPLE = 1, IDX_CAND = 2 };
+
+// 16 lanes x (16 x 8) 32-bit columns: repetition r covers columns
+// [8r, 8r+8); thread i of the warp gets, in r[4r .. 4r+3], lane (base + i/4)
+// columns 8r + 2(i%4) + {0, 1}, then lane (base + 8 + i/4), same columns.
+__device__ __forceinline__ void tmem_ld_16x256b_x16(uint32_t taddr, uint32_t (&r)[64]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+        "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+        "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]),
+          "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]),
+          "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]),
+          "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]),
+          "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]),
+          "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+        : "r"(taddr));
+}
 
 struct IndexerArgs {
     const float* w;        // [B, Lq, H]
@@ -279,6 +305,7 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
         const int cg = (warp - 2) >> 2;           // which half of the block's queries
         const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
         constexpr int QH = (QBMAX + 1) / 2;       // queries per half at most
+        constexpr bool QUAD = H >= 16;            // 16x256b TMEM reads, weights in registers
         const unsigned lt = (1u << lane) - 1u;
         uint32_t ta = 0, uq = 0;
         bool ok = true;
@@ -296,98 +323,189 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
             if (!mbar_wait(&q_full[qb], (uq >> 1) & 1)) { ok = false; break; }
             const float* wsm = w_s + qb * IDX_NMAX + qlo * H;
             const long long row0 = ui.row0 + qlo;
-            const int t0 = args.q_offset + ui.i0 + qlo;
-            uint32_t thrk[QH];
-            if (MODE == IDX_CAND) {
+            // QUAD: this thread's head weights of the unit, heads 8m + 2(lane%4) + {0,1}
+            float2 wr[QUAD ? QH : 1][QUAD ? H / 8 : 1];
+            if constexpr (QUAD) {
 #pragma unroll
                 for (int q = 0; q < QH; ++q)
+#pragma unroll
+                    for (int m = 0; m < H / 8; ++m)
+                        wr[q][m] = q < qhi - qlo
+                                       ? *reinterpret_cast<const float2*>(wsm + q * H + 8 * m + 2 * (lane & 3))
+                                       : make_float2(0.0f, 0.0f);
+            }
+            const int t0 = args.q_offset + ui.i0 + qlo;
+            uint32_t thrk[QH];
+            // IDX_CAND: a tile's candidates reserve their list slots with one
+            // atomic per query and are stored two tiles later, so the atomics'
+            // round trip (long under contention) overlaps the next two tiles
+            // instead of stalling this one.  Pending sets: 0 older, 1 newer.
+            // With more than 4 queries per warp (8 heads or fewer) the state
+            // would not fit in registers, and each tile stores its own.
+            constexpr bool DEFER = QH <= 4;
+            uint32_t pkey[2][QH];
+            unsigned pbal[2][QH], pbase[2][QH];
+            int ps[2] = {0, 0};
+            auto flush_older = [&]() {
+#pragma unroll
+                for (int q = 0; q < QH; ++q) {
+                    if (q < qhi - qlo && pbal[0][q] != 0u) {              // warp-uniform
+                        const unsigned base = __shfl_sync(0xffffffffu, pbase[0][q], 0);
+                        if ((pbal[0][q] >> lane) & 1u) {
+                            const unsigned slot = base + __popc(pbal[0][q] & lt);
+                            if (slot < (unsigned)args.cap)
+                                args.cand[(row0 + q) * args.cap + slot] =
+                                    ((unsigned long long)pkey[0][q] << 32) |
+                                    (uint32_t)(~(uint32_t)ps[0]);
+                        }
+                    }
+                }
+            };
+            auto shift_pending = [&]() {                                  // newer -> older, newer empty
+#pragma unroll
+                for (int q = 0; q < QH; ++q) {
+                    pkey[0][q] = pkey[1][q];
+                    pbal[0][q] = pbal[1][q];
+                    pbase[0][q] = pbase[1][q];
+                    pbal[1][q] = 0u;
+                }
+                ps[0] = ps[1];
+            };
+            if (MODE == IDX_CAND) {
+#pragma unroll
+                for (int q = 0; q < QH; ++q) {
                     thrk[q] = q < qhi - qlo ? __ldg(args.thr + row0 + q) : 0xFFFFFFFFu;
+#pragma unroll
+                    for (int b = 0; b < 2; ++b) {
+                        pbal[b][q] = 0u;
+                        pbase[b][q] = 0u;
+                        pkey[b][q] = 0u;
+                    }
+                }
             }
             for (int j = ui.j0; j < ui.j1; ++j, ++ta) {
                 const int ab = ta & 1;
                 if (!mbar_wait(&acc_full[ab], (ta >> 1) & 1)) { ok = false; break; }
                 tc_fence_after();
-                // H >= 16: two packed (f32x2) partial sums per query, over heads
-                // 4i+{0,1} and 4i+{2,3} -- four independent FMA chains instead
-                // of one.  H <= 8 (short chains, many queries per warp): one
-                // scalar sum per query.
-                constexpr bool PACKED = H >= 16;
-                constexpr int QP = PACKED ? QH : 1;
-                float2 acc2[QP][2];
-                float accs[PACKED ? 1 : QH];
+                // Head-weighted ReLU sums.
+                //  H >= 16: TMEM is read with the 16x256b shape, so a thread
+                //  holds two keys (rows j and j+8 of each 16-lane half) x two
+                //  columns of every 8-column block and needs only a quarter of
+                //  the head weights, kept in registers for the unit (no
+                //  shared-memory reads per tile).  Each (key, query) sum runs in
+                //  packed f32x2 chains over the thread's heads; the four threads
+                //  of a quad then add their partial sums with two shuffles.
+                //  Afterwards thread (j = lane/4, e = lane%4) holds key
+                //  klane = 16(e/2) + 8(e%2) + j of the warp's 32.
+                //  H <= 8 (many queries per warp): 32x32b loads, one key per
+                //  thread over all heads, weights broadcast from shared memory.
+                float acc[QH];
+                int klane = lane;
+                if constexpr (QUAD) {
+                    float p[2][2][QH];                                    // [lane half][row][query]
 #pragma unroll
-                for (int q = 0; q < QP; ++q) acc2[q][0] = acc2[q][1] = make_float2(0.0f, 0.0f);
+                    for (int lh = 0; lh < 2; ++lh) {
+                        float2 a2[2][QH];
 #pragma unroll
-                for (int q = 0; q < (PACKED ? 1 : QH); ++q) accs[q] = 0.0f;
-                const uint32_t taddr =
-                    tmem_base + lane_base + (uint32_t)(ab * IDX_NMAX + qlo * H);
-                // 64 columns per batch: two 32-column TMEM loads, one wait, reduce.
+                        for (int q = 0; q < QH; ++q) a2[0][q] = a2[1][q] = make_float2(0.0f, 0.0f);
+                        if (qhi > qlo) {                                  // warp-uniform
+                            uint32_t v[64];
+                            tmem_ld_16x256b_x16(tmem_base + ((uint32_t)(wq * 32 + 16 * lh) << 16) +
+                                                    (uint32_t)(ab * IDX_NMAX + qlo * H),
+                                                v);
+                            tmem_ld_wait();
 #pragma unroll
-                for (int bt = 0; bt < (QH * H + 63) / 64; ++bt) {
-                    if (bt * 2 < nchunk) {
-                        uint32_t v[64];
-                        tmem_ld_32x32b_x32(taddr + bt * 64, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-                        if (bt * 2 + 1 < nchunk)
-                            tmem_ld_32x32b_x32(taddr + bt * 64 + 32,
-                                               *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-                        tmem_ld_wait();
+                            for (int r = 0; r < 16; ++r) {
+                                const int q = (8 * r) / H, m = ((8 * r) % H) / 8;
+                                const float2 r0 = make_float2(fmaxf(__uint_as_float(v[4 * r]), 0.0f),
+                                                              fmaxf(__uint_as_float(v[4 * r + 1]), 0.0f));
+                                const float2 r1 = make_float2(fmaxf(__uint_as_float(v[4 * r + 2]), 0.0f),
+                                                              fmaxf(__uint_as_float(v[4 * r + 3]), 0.0f));
+                                a2[0][q] = __ffma2_rn(wr[q][m], r0, a2[0][q]);
+                                a2[1][q] = __ffma2_rn(wr[q][m], r1, a2[1][q]);
+                            }
+                        }
 #pragma unroll
-                        for (int jj = 0; jj < 64; jj += 4) {
-                            const int c = bt * 64 + jj;
-                            if (c < ncol) {
-                                // columns c..c+3 are four heads of one query (H % 4 == 0)
-                                const int q = c / H;
-                                const float4 wv = *reinterpret_cast<const float4*>(wsm + c);
-                                const float2 r01 = make_float2(fmaxf(__uint_as_float(v[jj]), 0.0f),
-                                                               fmaxf(__uint_as_float(v[jj + 1]), 0.0f));
-                                const float2 r23 = make_float2(fmaxf(__uint_as_float(v[jj + 2]), 0.0f),
-                                                               fmaxf(__uint_as_float(v[jj + 3]), 0.0f));
-                                if constexpr (PACKED) {
-                                    acc2[q % QP][0] = __ffma2_rn(make_float2(wv.x, wv.y), r01, acc2[q % QP][0]);
-                                    acc2[q % QP][1] = __ffma2_rn(make_float2(wv.z, wv.w), r23, acc2[q % QP][1]);
-                                } else {
-                                    float& a = accs[q];
-                                    a = fmaf(wv.x, r01.x, a);
-                                    a = fmaf(wv.y, r01.y, a);
-                                    a = fmaf(wv.z, r23.x, a);
-                                    a = fmaf(wv.w, r23.y, a);
+                        for (int q = 0; q < QH; ++q) {
+                            p[lh][0][q] = a2[0][q].x + a2[0][q].y;
+                            p[lh][1][q] = a2[1][q].x + a2[1][q].y;
+                        }
+                    }
+#pragma unroll
+                    for (int lh = 0; lh < 2; ++lh)
+#pragma unroll
+                        for (int rw = 0; rw < 2; ++rw)
+#pragma unroll
+                            for (int q = 0; q < QH; ++q) {
+                                float x = p[lh][rw][q];
+                                x += __shfl_xor_sync(0xffffffffu, x, 1);
+                                x += __shfl_xor_sync(0xffffffffu, x, 2);
+                                p[lh][rw][q] = x;
+                            }
+                    const int e = lane & 3;
+                    klane = 16 * (e >> 1) + 8 * (e & 1) + (lane >> 2);
+#pragma unroll
+                    for (int q = 0; q < QH; ++q)
+                        acc[q] = e == 0 ? p[0][0][q] : e == 1 ? p[0][1][q] : e == 2 ? p[1][0][q] : p[1][1][q];
+                } else {
+                    const uint32_t taddr =
+                        tmem_base + lane_base + (uint32_t)(ab * IDX_NMAX + qlo * H);
+#pragma unroll
+                    for (int q = 0; q < QH; ++q) acc[q] = 0.0f;
+                    // 64 columns per batch: two 32-column TMEM loads, one wait, reduce.
+#pragma unroll
+                    for (int bt = 0; bt < (QH * H + 63) / 64; ++bt) {
+                        if (bt * 2 < nchunk) {
+                            uint32_t v[64];
+                            tmem_ld_32x32b_x32(taddr + bt * 64, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+                            if (bt * 2 + 1 < nchunk)
+                                tmem_ld_32x32b_x32(taddr + bt * 64 + 32,
+                                                   *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int jj = 0; jj < 64; jj += 4) {
+                                const int c = bt * 64 + jj;
+                                if (c < ncol) {
+                                    // columns c..c+3 are four heads of one query (H % 4 == 0)
+                                    const int q = c / H;
+                                    const float4 wv = *reinterpret_cast<const float4*>(wsm + c);
+                                    float& a = acc[q];
+                                    a = fmaf(wv.x, fmaxf(__uint_as_float(v[jj]), 0.0f), a);
+                                    a = fmaf(wv.y, fmaxf(__uint_as_float(v[jj + 1]), 0.0f), a);
+                                    a = fmaf(wv.z, fmaxf(__uint_as_float(v[jj + 2]), 0.0f), a);
+                                    a = fmaf(wv.w, fmaxf(__uint_as_float(v[jj + 3]), 0.0f), a);
                                 }
                             }
                         }
                     }
                 }
-                float acc[QH];
-#pragma unroll
-                for (int q = 0; q < QH; ++q) {
-                    if constexpr (PACKED)
-                        acc[q] = (acc2[q % QP][0].x + acc2[q % QP][0].y) +
-                                 (acc2[q % QP][1].x + acc2[q % QP][1].y);
-                    else
-                        acc[q] = accs[q % (PACKED ? 1 : QH)];
-                }
                 tc_fence_before();
                 mbar_arrive(&acc_empty[ab]);
-                const int s = j * kstride * IDX_BM + wq * 32 + lane;      // key position
+                const int s = j * kstride * IDX_BM + wq * 32 + klane;     // key position
                 if (MODE == IDX_CAND) {
+                    if constexpr (DEFER) {
+                        flush_older();                                    // the tile two back
+                        shift_pending();
+                    }
 #pragma unroll
                     for (int q = 0; q < QH; ++q) {
                         if (q < qhi - qlo) {                              // warp-uniform
                             const uint32_t key = score_key(acc[q]);
                             const bool sel = s <= t0 + q && key >= thrk[q];
                             const unsigned bal = __ballot_sync(0xffffffffu, sel);
-                            if (bal) {
-                                unsigned base = 0;
-                                if (lane == 0) base = atomicAdd(args.cnt + row0 + q, (unsigned)__popc(bal));
-                                base = __shfl_sync(0xffffffffu, base, 0);
-                                const unsigned slot = base + __popc(bal & lt);
-                                if (sel && slot < (unsigned)args.cap)
-                                    args.cand[(row0 + q) * args.cap + slot] =
-                                        ((unsigned long long)key << 32) | (uint32_t)(~(uint32_t)s);
-                            }
+                            pkey[1][q] = key;
+                            pbal[1][q] = bal;
+                            if (lane == 0 && bal != 0u)
+                                pbase[1][q] = atomicAdd(args.cnt + row0 + q, (unsigned)__popc(bal));
                         }
                     }
+                    ps[1] = s;
+                    if constexpr (!DEFER) {                               // store this tile's now
+                        shift_pending();
+                        flush_older();
+                    }
                 } else if (s < args.Lk) {
-                    const long long col = MODE == IDX_SAMPLE ? (long long)j * IDX_BM + wq * 32 + lane
+                    const long long col = MODE == IDX_SAMPLE ? (long long)j * IDX_BM + wq * 32 + klane
                                                              : (long long)s;
                     float* dst = args.scores + row0 * args.ld + col;
 #pragma unroll
@@ -400,6 +518,11 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 }
             }
             if (!ok) break;
+            if (MODE == IDX_CAND && DEFER) {                              // the unit's last two tiles
+                flush_older();
+                shift_pending();
+                flush_older();
+            }
             __syncwarp();
             if (lane == 0) mbar_arrive(&q_empty[qb]);
             ++uq;

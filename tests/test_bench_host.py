@@ -48,10 +48,30 @@ def test_profile_traffic_only_for_matching_source(tmp_path, monkeypatch):
     h = hashlib.sha256(b"kernel v1" + b"common").hexdigest()[:16]
     (prof / "dense_attn_kernel_prefill_8k.md").write_text(
         f"source_hash: {h}\ndram_bytes_per_launch: 12345\n")
-    assert bench.profile_traffic("dense_attn", "prefill_8k") == 12345
-    assert bench.profile_traffic("dense_attn", "prefill_64k") is None      # no capture
+    assert bench.profile_traffic("dense_attn", "prefill_8k") == (12345, "dense_attn_kernel_prefill_8k.md")
+    # no capture of this workload, and the one there is records no units: nothing to scale
+    assert bench.profile_traffic("dense_attn", "prefill_64k", 65536) == (None, None)
     (csrc / "dense_attn.cuh").write_text("kernel v2")                      # source changed
-    assert bench.profile_traffic("dense_attn", "prefill_8k") is None
+    assert bench.profile_traffic("dense_attn", "prefill_8k") == (None, None)
+
+
+def test_profile_traffic_scales_a_smaller_capture_by_its_rows(tmp_path, monkeypatch):
+    prof = tmp_path / "profiles"
+    csrc = tmp_path / "lightning_indexer_top_relu_b200" / "csrc"
+    prof.mkdir()
+    csrc.mkdir(parents=True)
+    (csrc / "sparse_attn.cuh").write_text("s")
+    (csrc / "common.cuh").write_text("c")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    import hashlib
+    h = hashlib.sha256(b"s" + b"c").hexdigest()[:16]
+    (prof / "sparse_attn_kernel_layer_32k.md").write_text(
+        f"source_hash: {h}\ndram_bytes_per_launch: 1000\nunits_per_launch: 16384\n")
+    got, src = bench.profile_traffic("sparse_attn", "prefill_64k", 49152)
+    assert got == 3000 and "sparse_attn_kernel_layer_32k.md" in src and "scaled" in src
+    assert bench.profile_traffic("sparse_attn", "layer_32k", 16384)[0] == 1000
+    (csrc / "sparse_attn.cuh").write_text("s2")                            # source changed
+    assert bench.profile_traffic("sparse_attn", "prefill_64k", 49152) == (None, None)
 
 
 def test_input_bytes_and_device_drawing_threshold():
