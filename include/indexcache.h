@@ -286,16 +286,17 @@ int ic_layer_stack_forward_events(const char *pattern, int n_layers, const ic_la
  *                    gives each row a threshold -- the r-th largest sampled
  *                    score, r = ceil(m p + z sqrt(m p (1 - p))) + 1 for m
  *                    visible samples and p = k / (t + 1) -- then the indexer
- *                    runs again keeping only scores at or above it (at most
- *                    3k per row; rows with at most 3k visible positions keep
- *                    them all), and an exact selection runs on those
- *                    candidates.  A row with fewer than k candidates or more
- *                    than 3k has its query block re-run the way of mode 0, so
- *                    the index rows equal mode 0's bit for bit in every case.
- *                    Needs k <= 4096 and Lk <= 262144 (IC_ERR_UNSUPPORTED
- *                    otherwise);
+ *                    runs again keeping only scores at or above it, in a list
+ *                    of 4k slots per row (rows with at most 2k visible
+ *                    positions keep them all; rows with at most k need no
+ *                    list), and an exact selection runs on those candidates.
+ *                    A row with fewer than k candidates, or whose reserved
+ *                    slots overflow its list, has its query block re-run the
+ *                    way of mode 0, so the index rows equal mode 0's bit for
+ *                    bit in every case.  Needs k <= 4096 and Lk <= 262144
+ *                    (IC_ERR_UNSUPPORTED otherwise);
  *                -1  (default) the library's choice: fused when the longest
- *                    row sees more than 6k positions and there are at least
+ *                    row sees more than 8k positions and there are at least
  *                    1024 query rows, else mode 0.
  *   z           the threshold's margin in binomial standard deviations
  *               (<= 0: 4).  Larger keeps more candidates and falls back less

@@ -121,7 +121,8 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t x, uint32_t* wsum, 
 struct FusedArgs {
     long long row_base, n_rows;   // flattened rows [row_base, row_base + n_rows) of this chunk
     int Lq, Lk, q_offset, k;
-    int cap;                      // candidates kept per row
+    int cap;                      // candidates a row may keep; rows with n <= cap keep all
+    int lstride;                  // list slots per row (cap + room for unused reserved slots)
     int stride;                   // sampled key tiles: m * stride
     int ns;                       // sample tiles per sample row (row stride ns * 128)
     float z;                      // threshold margin, in binomial standard deviations
@@ -131,7 +132,7 @@ struct FusedArgs {
     const float* samp;            // [n_rows, ns * 128] sampled scores (-inf past t)
     uint32_t* thr;                // [n_rows] threshold key
     uint32_t* cnt;                // [n_rows] candidates found
-    const unsigned long long* cand;   // [n_rows, cap]
+    const unsigned long long* cand;   // [n_rows, lstride]
     uint32_t* bflag;              // [n_blocks] block needs the exact fallback
     int* blist;                   // [n_blocks] flagged blocks (global block ids)
     int* list_count;              // number of flagged blocks
@@ -151,12 +152,14 @@ __device__ __forceinline__ int visible_samples(int t, int stride, int ns) {
 }
 
 // Per row: the threshold key, and the row's candidate counter cleared.  Rows
-// with at most `cap` visible positions take key 0 (every visible score is a
-// candidate).  Other rows: with m visible samples and p = k / n, the
-// threshold is the r-th largest sampled key, r = ceil(m p + z sqrt(m p (1-p)))
-// + 1, so the row's share of scores at or above it exceeds p unless the
-// sample is off by about z standard deviations.  Also clears the chunk's
-// block flags and the flagged-block count.
+// with n <= k visible positions keep them all and need no candidate (key
+// 0xFFFFFFFF: no score reaches it); rows with at most cap take key 0 (every
+// visible score is a candidate).  Other rows, with m visible
+// samples and p = k / n, take the r-th largest sampled key,
+// r = ceil(m p + z sqrt(m p (1-p))) + 1, so the row's share of scores at or
+// above it exceeds p unless the sample is off by about z standard
+// deviations.  Also clears the chunk's block flags and the flagged-block
+// count.
 __global__ void __launch_bounds__(FT_THREADS)
 fused_threshold_kernel(const FusedArgs a) {
     __shared__ uint32_t vals[FT_MAX_SAMPLES];
@@ -173,7 +176,7 @@ fused_threshold_kernel(const FusedArgs a) {
         const int n = min(t + 1, a.Lk);
         if (threadIdx.x == 0) a.cnt[rr] = 0u;
         if (n <= a.cap) {
-            if (threadIdx.x == 0) a.thr[rr] = 0u;
+            if (threadIdx.x == 0) a.thr[rr] = n <= a.k ? 0xFFFFFFFFu : 0u;
             continue;
         }
         const int span = a.stride * 128;
@@ -201,8 +204,10 @@ fused_threshold_kernel(const FusedArgs a) {
 }
 
 // Per row: the exact top-k over the row's candidates when there are at least
-// k of them and none was dropped; otherwise the row's query block is flagged
-// (and listed once) for the exact fallback.  The selection is the k largest
+// k of them and none was dropped (the row's reserved slots, counted by the
+// counter, fit in the list); otherwise the row's query block is flagged (and
+// listed once) for the exact fallback.  Reserved slots the indexer left
+// unused hold 0, below every candidate, and are not counted.  The selection is the k largest
 // candidate values (all distinct); it is written in ascending position order
 // through a bitmap of the row's visible positions, which is also the row's
 // selection bitmask when the row attends dense-masked.
@@ -214,8 +219,8 @@ fused_select_kernel(const FusedArgs a) {
     uint32_t* wsum = reinterpret_cast<uint32_t*>(fs_smem + 1040);           // 8
     uint32_t* tot = wsum + FS_THREADS / 32;                                 // 1
     unsigned long long* one = reinterpret_cast<unsigned long long*>(fs_smem + 1088);
-    unsigned long long* vals = reinterpret_cast<unsigned long long*>(fs_smem + 1152);   // cap
-    uint32_t* bm = reinterpret_cast<uint32_t*>(fs_smem + 1152 + (size_t)a.cap * 8);     // words
+    unsigned long long* vals = reinterpret_cast<unsigned long long*>(fs_smem + 1152);   // lstride
+    uint32_t* bm = reinterpret_cast<uint32_t*>(fs_smem + 1152 + (size_t)a.lstride * 8); // words
 
     const int tid = threadIdx.x;
     const long long rr = a.n_rows - 1 - (long long)blockIdx.x;   // longest rows first
@@ -236,7 +241,19 @@ fused_select_kernel(const FusedArgs a) {
         return;
     }
     const uint32_t c = __ldg(a.cnt + rr);
-    if (c < (uint32_t)a.k || c > (uint32_t)a.cap) {
+    uint32_t valid = 0;
+    if (c <= (uint32_t)a.lstride) {                 // uniform
+        const unsigned long long* crow = a.cand + rr * (long long)a.lstride;
+        uint32_t mine = 0;
+        for (uint32_t j = tid; j < c; j += FS_THREADS) {
+            const unsigned long long v = __ldg(crow + j);
+            vals[j] = v;
+            mine += v != 0ull;
+        }
+        block_excl_scan<FS_THREADS>(mine, wsum, tot);
+        valid = *tot;
+    }
+    if (c > (uint32_t)a.lstride || valid < (uint32_t)a.k) {
         if (tid == 0) {
             const long long g = (r / a.Lq) * a.nqb + i / a.QB;
             if (atomicExch(a.bflag + (g - a.g0), 1u) == 0u) {
@@ -246,8 +263,6 @@ fused_select_kernel(const FusedArgs a) {
         }
         return;
     }
-    const unsigned long long* crow = a.cand + rr * (long long)a.cap;
-    for (uint32_t j = tid; j < c; j += FS_THREADS) vals[j] = __ldg(crow + j);
     for (int w = tid; w < nw; w += FS_THREADS) bm[w] = 0u;
     __syncthreads();
     const unsigned long long T =
@@ -280,10 +295,10 @@ fused_select_kernel(const FusedArgs a) {
         for (int w = tid; w < a.W; w += FS_THREADS) mrow[w] = w < nw ? bm[w] : 0u;
 }
 
-// Shared memory of fused_select_kernel for a candidate capacity and a row
+// Shared memory of fused_select_kernel for a list of lstride slots and a row
 // length (bitmap words).
-__host__ __device__ constexpr size_t fused_select_smem(int cap, int Lk) {
-    return 1152 + (size_t)cap * 8 + (size_t)((Lk + 31) / 32) * 4;
+__host__ __device__ constexpr size_t fused_select_smem(int lstride, int Lk) {
+    return 1152 + (size_t)lstride * 8 + (size_t)((Lk + 31) / 32) * 4;
 }
 
 }  // namespace ic

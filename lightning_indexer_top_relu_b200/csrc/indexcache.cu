@@ -183,6 +183,7 @@ struct IdxExtra {
     const int* blk_list = nullptr;        // block list (blocks of [g0, g1) only)
     const int* blk_count = nullptr;
     int list_off = 0, list_len = 0;
+    int tpu = 0;                          // key tiles per work unit (0: sized from the work)
 };
 
 // Scores query blocks [g0, g1) into `scores` (row = flattened row - row of g0),
@@ -219,6 +220,7 @@ int launch_indexer(const uint16_t* q_idx, const uint16_t* k_idx, const float* w,
     }
     int tpu = (int)std::min<long long>(64, std::max<long long>(4, total / (6LL * sms)));
     if (listed) tpu = std::max(4, std::min(tpu, max_nt / 8));
+    if (x.tpu > 0) tpu = x.tpu;
     tpu = std::min(tpu, std::max(1, max_nt));
     const int max_splits = (max_nt + tpu - 1) / tpu;
 
@@ -509,19 +511,22 @@ int attn_step(const ic_dims& D, const ic_layer& L, const int32_t* idx, AttnMode 
 
 // ---------------------------------------------------------------- fused indexer -> top-k
 
-constexpr int FUSED_CAP_FACTOR = 3;     // candidates a row may keep: 3k
+constexpr int FUSED_CAP_FACTOR = 4;     // list slots a row may use: 4k
 constexpr float FUSED_Z = 4.0f;         // threshold margin in binomial standard deviations
 constexpr int FUSED_FB_DIV = 8;         // fallback scores: 1/8 of a chunk's blocks per round
-constexpr int FUSED_MAX_K = 4096;       // candidate list in shared memory: 3k x 8 bytes
+constexpr int FUSED_MAX_K = 4096;       // candidate list in shared memory: 4k x 8 bytes
 constexpr int FUSED_MAX_LK = 262144;    // bitmap of a row's positions in shared memory
 constexpr int FUSED_AUTO_MIN_ROWS = 1024;
 
 // Sizes of the fused path for given dims (ok = false when it cannot run).
+constexpr int FUSED_TPU = 64;           // key tiles per unit of the candidate pass
+
 struct FusedGeom {
     bool ok = false;
     int stride = 1;          // sampled key tiles m * stride
     int ns = 0;              // sampled tiles per row at most (<= 32)
-    int cap = 0;             // candidates kept per row
+    int cap = 0;             // candidates a row may keep (4k); rows with n <= cap keep all
+    int lstride = 0;         // list slots per row: cap + what reserved, unused slots may take
     int n_max = 0;           // longest row's visible positions
 };
 
@@ -533,8 +538,13 @@ FusedGeom fused_geom(const ic_dims& D) {
     f.stride = std::max(1, nt_max / 16);
     f.ns = (nt_max + f.stride - 1) / f.stride;
     f.cap = FUSED_CAP_FACTOR * D.k;
+    // Each writer of a row's list (4 warp lane quarters x the candidate
+    // pass's units of FUSED_TPU key tiles) leaves fewer than 2 reserved ranges
+    // unused.
+    const int splits = (nt_max + FUSED_TPU - 1) / FUSED_TPU;
+    f.lstride = f.cap + 2 * (int)ic::IDX_RES * 4 * splits;
     f.ok = f.ns * ic::IDX_BM <= ic::FT_MAX_SAMPLES &&
-           ic::fused_select_smem(f.cap, D.Lk) <= (size_t)ic::MAX_DYN_SMEM;
+           ic::fused_select_smem(f.lstride, D.Lk) <= (size_t)ic::MAX_DYN_SMEM;
     return f;
 }
 
@@ -561,7 +571,7 @@ FusedLayout fused_layout(const FusedGeom& f, long long blocks, int QB, int Lk) {
     L.fb_blocks = (blocks + FUSED_FB_DIV - 1) / FUSED_FB_DIV;
     size_t o = 0;
     L.samp = o;   o = align256(o + rows * (size_t)f.ns * ic::IDX_BM * 4);
-    L.cand = o;   o = align256(o + rows * (size_t)f.cap * 8);
+    L.cand = o;   o = align256(o + rows * (size_t)f.lstride * 8);
     L.thr = o;    o = align256(o + rows * 4);
     L.cnt = o;    o = align256(o + rows * 4);
     L.flag = o;   o = align256(o + (size_t)blocks * 4);
@@ -606,6 +616,7 @@ int fused_chunk(const ic_dims& D, const ic_layer& Lr, const IndexerGeom& geo, co
     fa.q_offset = D.q_offset;
     fa.k = D.k;
     fa.cap = f.cap;
+    fa.lstride = f.lstride;
     fa.stride = f.stride;
     fa.ns = f.ns;
     fa.z = z;
@@ -640,7 +651,8 @@ int fused_chunk(const ic_dims& D, const ic_layer& Lr, const IndexerGeom& geo, co
     xc.thr = fa.thr;
     xc.cnt = fa.cnt;
     xc.cand = reinterpret_cast<unsigned long long*>(base + lay.cand);
-    xc.cap = f.cap;
+    xc.cap = f.lstride;
+    xc.tpu = FUSED_TPU;
     rc = launch_indexer(Lr.q_idx, Lr.k_idx, Lr.w, D.B, D.Lq, D.Lk, D.H_I, D.d_I, D.q_offset, g0,
                         g1, nullptr, 0, false, sms, st, xc);
     if (rc) return rc;
@@ -649,7 +661,7 @@ int fused_chunk(const ic_dims& D, const ic_layer& Lr, const IndexerGeom& geo, co
         if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
     }
     ic::fused_select_kernel<<<(unsigned)fa.n_rows, ic::FS_THREADS,
-                              ic::fused_select_smem(f.cap, D.Lk), st>>>(fa);
+                              ic::fused_select_smem(f.lstride, D.Lk), st>>>(fa);
     if (launched(cudaGetLastError(), "fused_select launch")) return IC_ERR_CUDA;
     float* fb = reinterpret_cast<float*>(base + lay.fb);
     for (long long off = 0; off < g1 - g0; off += lay.fb_blocks) {
@@ -701,9 +713,7 @@ int device_setup(int* dev_out, int* sms_out) {
         cudaFuncSetAttribute(ic::dense_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              ic::DenseSmem::ALLOC);
         cudaFuncSetAttribute(ic::fused_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)std::min<size_t>(ic::MAX_DYN_SMEM,
-                                                   ic::fused_select_smem(FUSED_CAP_FACTOR * FUSED_MAX_K,
-                                                                         FUSED_MAX_LK)));
+                             ic::MAX_DYN_SMEM);
         cudaFuncSetAttribute(ic::index_overlap_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              2 * (ic::OV_MAX_LK / 32) * 4);
         cudaFuncSetAttribute(ic::index_overlap_warp_kernel,

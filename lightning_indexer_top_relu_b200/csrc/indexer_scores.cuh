@@ -29,7 +29,8 @@
 //               (2 x 256 columns) let the epilogue of tile j overlap the MMA
 //               of tile j+1.
 // A work unit is (query block, run of up to `tpu` key tiles); units are
-// walked longest-causal-row first and dealt round-robin to the CTAs.
+// ordered split-major, longest causal rows first within a split, and dealt
+// round-robin to the CTAs.
 //
 // Epilogue modes (a template parameter; the MMA and the score arithmetic are
 // the same code in every mode, so a score is bit-identical whichever mode
@@ -42,8 +43,10 @@
 //               is at least the row's threshold key: each is appended to the
 //               row's candidate list as (key << 32) | ~s, one 64-bit value
 //               whose unsigned order is (score descending, position
-//               ascending).  The row's counter counts every candidate, also
-//               those past the list's capacity (which are dropped).
+//               ascending).  Warps reserve list slots in ranges of IDX_RES;
+//               the row's counter counts every reserved slot, also those past
+//               the list's capacity (whose candidates are dropped), and
+//               reserved slots left unused hold 0.
 // With a block list (the exact fallback of the fused top-k), the launch's
 // query blocks are taken from a device array whose length is read on the
 // device, and scores go to consecutive buffer rows of those blocks.
@@ -60,6 +63,8 @@ constexpr int IDX_EPI_WARPS = 8;
 constexpr int IDX_THREADS = 64 + 32 * IDX_EPI_WARPS;
 
 enum : int { IDX_SCORES = 0, IDX_SAMPLE = 1, IDX_CAND = 2 };
+constexpr unsigned IDX_RES = 32;              // IDX_CAND: list slots reserved per atomic
+constexpr uint32_t IDX_NONE = 0xFFFFFFFFu;    // IDX_CAND threshold: the row keeps no candidate
 
 // 16 lanes x (16 x 8) 32-bit columns: repetition r covers columns
 // [8r, 8r+8); thread i of the warp gets, in r[4r .. 4r+3], lane (base + i/4)
@@ -136,27 +141,33 @@ struct UnitInfo {
     long long row0;          // output row of the block's first query
 };
 
-// Work units of this launch (in block-list mode the length is read on the device).
-__device__ __forceinline__ long long idx_units(const IndexerArgs& a) {
+// Query blocks of this launch (in block-list mode the length is read on the device).
+__device__ __forceinline__ long long idx_blocks(const IndexerArgs& a) {
     long long nb = (long long)(a.g1 - a.g0);
     if (a.blk_list != nullptr) {
         const long long have = (long long)__ldg(a.blk_count) - a.list_off;
         nb = have < 0 ? 0 : (have < a.list_len ? have : a.list_len);
     }
-    return nb * a.max_splits;
+    return nb;
 }
 
+// Unit u of nb * max_splits, split-major: every block's first run of key
+// tiles (longest rows first), then every block's second run, and so on.
+// Units dealt round-robin to the CTAs then come in windows of similar size;
+// block-major order would give each CTA the same split of every block (with
+// an even grid and two splits, half the CTAs would get only the short
+// remainders).
 template <int MODE>
-__device__ __forceinline__ UnitInfo unit_info(const IndexerArgs& a, long long u) {
+__device__ __forceinline__ UnitInfo unit_info(const IndexerArgs& a, long long u, long long nb) {
     UnitInfo r;
-    const int slot = (int)(u / a.max_splits);
+    const int slot = (int)(u % nb);
     int g;
     if (a.blk_list != nullptr) {
         g = __ldg(a.blk_list + a.list_off + slot);
     } else {
         g = a.g1 - 1 - slot;
     }
-    const int split = (int)(u % a.max_splits);
+    const int split = (int)(u / nb);
     r.b = g / a.nqb;
     r.i0 = (g % a.nqb) * a.QB;
     r.nq = min(a.QB, a.Lq - r.i0);
@@ -196,7 +207,8 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const long long n_units = idx_units(args);
+    const long long n_blocks = idx_blocks(args);
+    const long long n_units = n_blocks * args.max_splits;
     const int kstride = MODE == IDX_SAMPLE ? args.stride : 1;   // key tile = visited index * kstride
 
     if (threadIdx.x == 0) {
@@ -233,7 +245,7 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
             uint32_t uq = 0, ta = 0;
             bool ok = true;
             for (long long u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-                UnitInfo ui = unit_info<MODE>(args, u);
+                UnitInfo ui = unit_info<MODE>(args, u, n_blocks);
                 if (ui.j0 >= ui.j1) continue;
                 const int qb = uq & 1;
                 if (!mbar_wait(&q_empty[qb], ((uq >> 1) & 1) ^ 1)) { ok = false; break; }
@@ -269,7 +281,7 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
             uint32_t uq = 0, ta = 0;
             bool ok = true;
             for (long long u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-                UnitInfo ui = unit_info<MODE>(args, u);
+                UnitInfo ui = unit_info<MODE>(args, u, n_blocks);
                 if (ui.j0 >= ui.j1) continue;
                 const int qb = uq & 1;
                 if (!mbar_wait(&q_full[qb], (uq >> 1) & 1)) { ok = false; break; }
@@ -305,12 +317,12 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
         const int cg = (warp - 2) >> 2;           // which half of the block's queries
         const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
         constexpr int QH = (QBMAX + 1) / 2;       // queries per half at most
-        constexpr bool QUAD = H >= 16;            // 16x256b TMEM reads, weights in registers
+        constexpr bool QUAD = H >= 64;            // 16x256b TMEM reads, weights in registers
         const unsigned lt = (1u << lane) - 1u;
         uint32_t ta = 0, uq = 0;
         bool ok = true;
         for (long long u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-            UnitInfo ui = unit_info<MODE>(args, u);
+            UnitInfo ui = unit_info<MODE>(args, u, n_blocks);
             if (ui.j0 >= ui.j1) continue;
             const int qb = uq & 1;
             // queries [qlo, qhi) of this block belong to this warp
@@ -336,51 +348,29 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
             }
             const int t0 = args.q_offset + ui.i0 + qlo;
             uint32_t thrk[QH];
-            // IDX_CAND: a tile's candidates reserve their list slots with one
-            // atomic per query and are stored two tiles later, so the atomics'
-            // round trip (long under contention) overlaps the next two tiles
-            // instead of stalling this one.  Pending sets: 0 older, 1 newer.
-            // With more than 4 queries per warp (8 heads or fewer) the state
-            // would not fit in registers, and each tile stores its own.
-            constexpr bool DEFER = QH <= 4;
-            uint32_t pkey[2][QH];
-            unsigned pbal[2][QH], pbase[2][QH];
-            int ps[2] = {0, 0};
-            auto flush_older = [&]() {
-#pragma unroll
-                for (int q = 0; q < QH; ++q) {
-                    if (q < qhi - qlo && pbal[0][q] != 0u) {              // warp-uniform
-                        const unsigned base = __shfl_sync(0xffffffffu, pbase[0][q], 0);
-                        if ((pbal[0][q] >> lane) & 1u) {
-                            const unsigned slot = base + __popc(pbal[0][q] & lt);
-                            if (slot < (unsigned)args.cap)
-                                args.cand[(row0 + q) * args.cap + slot] =
-                                    ((unsigned long long)pkey[0][q] << 32) |
-                                    (uint32_t)(~(uint32_t)ps[0]);
-                        }
-                    }
-                }
+            // IDX_CAND: list slots are reserved ahead of need.  Per query the
+            // warp holds a current range of IDX_RES slots [cpos, cend) and the
+            // result (lane 0) of the atomic that reserved the next range,
+            // issued when the current range was taken; a tile waits on an
+            // atomic only when it crosses into a new range.  Slots still
+            // unused when the unit ends are filled with 0, a value no
+            // candidate takes (it would need a NaN key and position
+            // 0xFFFFFFFF); the selection skips them.
+            unsigned cpos[QH], cend[QH], npend[QH];
+            auto reserve_next = [&](int q) {
+                if (lane == 0) npend[q] = atomicAdd(args.cnt + row0 + q, (unsigned)IDX_RES);
             };
-            auto shift_pending = [&]() {                                  // newer -> older, newer empty
-#pragma unroll
-                for (int q = 0; q < QH; ++q) {
-                    pkey[0][q] = pkey[1][q];
-                    pbal[0][q] = pbal[1][q];
-                    pbase[0][q] = pbase[1][q];
-                    pbal[1][q] = 0u;
-                }
-                ps[0] = ps[1];
+            auto pad = [&](int q, unsigned from, unsigned to) {          // sentinel-fill [from, to)
+                for (unsigned x = from + lane; x < to; x += 32)
+                    if (x < (unsigned)args.cap) args.cand[(row0 + q) * args.cap + x] = 0ull;
             };
             if (MODE == IDX_CAND) {
 #pragma unroll
                 for (int q = 0; q < QH; ++q) {
-                    thrk[q] = q < qhi - qlo ? __ldg(args.thr + row0 + q) : 0xFFFFFFFFu;
-#pragma unroll
-                    for (int b = 0; b < 2; ++b) {
-                        pbal[b][q] = 0u;
-                        pbase[b][q] = 0u;
-                        pkey[b][q] = 0u;
-                    }
+                    thrk[q] = q < qhi - qlo ? __ldg(args.thr + row0 + q) : IDX_NONE;
+                    cpos[q] = cend[q] = 0u;
+                    npend[q] = 0u;
+                    if (q < qhi - qlo && thrk[q] != IDX_NONE) reserve_next(q);
                 }
             }
             for (int j = ui.j0; j < ui.j1; ++j, ++ta) {
@@ -483,26 +473,29 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 mbar_arrive(&acc_empty[ab]);
                 const int s = j * kstride * IDX_BM + wq * 32 + klane;     // key position
                 if (MODE == IDX_CAND) {
-                    if constexpr (DEFER) {
-                        flush_older();                                    // the tile two back
-                        shift_pending();
-                    }
 #pragma unroll
                     for (int q = 0; q < QH; ++q) {
-                        if (q < qhi - qlo) {                              // warp-uniform
+                        if (q < qhi - qlo && thrk[q] != IDX_NONE) {       // warp-uniform
                             const uint32_t key = score_key(acc[q]);
                             const bool sel = s <= t0 + q && key >= thrk[q];
                             const unsigned bal = __ballot_sync(0xffffffffu, sel);
-                            pkey[1][q] = key;
-                            pbal[1][q] = bal;
-                            if (lane == 0 && bal != 0u)
-                                pbase[1][q] = atomicAdd(args.cnt + row0 + q, (unsigned)__popc(bal));
+                            if (bal != 0u) {
+                                const unsigned n = __popc(bal), rank = __popc(bal & lt);
+                                const unsigned a = min(n, cend[q] - cpos[q]);
+                                unsigned slot = cpos[q] + rank;
+                                cpos[q] += a;
+                                if (n > a) {                              // into the next range
+                                    const unsigned nb = __shfl_sync(0xffffffffu, npend[q], 0);
+                                    if (rank >= a) slot = nb + (rank - a);
+                                    cpos[q] = nb + (n - a);
+                                    cend[q] = nb + IDX_RES;
+                                    reserve_next(q);
+                                }
+                                if (sel && slot < (unsigned)args.cap)
+                                    args.cand[(row0 + q) * args.cap + slot] =
+                                        ((unsigned long long)key << 32) | (uint32_t)(~(uint32_t)s);
+                            }
                         }
-                    }
-                    ps[1] = s;
-                    if constexpr (!DEFER) {                               // store this tile's now
-                        shift_pending();
-                        flush_older();
                     }
                 } else if (s < args.Lk) {
                     const long long col = MODE == IDX_SAMPLE ? (long long)j * IDX_BM + wq * 32 + klane
@@ -518,10 +511,15 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 }
             }
             if (!ok) break;
-            if (MODE == IDX_CAND && DEFER) {                              // the unit's last two tiles
-                flush_older();
-                shift_pending();
-                flush_older();
+            if (MODE == IDX_CAND) {                                       // unused reserved slots
+#pragma unroll
+                for (int q = 0; q < QH; ++q) {
+                    if (q < qhi - qlo && thrk[q] != IDX_NONE) {
+                        pad(q, cpos[q], cend[q]);
+                        const unsigned nb = __shfl_sync(0xffffffffu, npend[q], 0);
+                        pad(q, nb, nb + IDX_RES);
+                    }
+                }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&q_empty[qb]);

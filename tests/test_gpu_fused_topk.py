@@ -11,8 +11,8 @@ north_star's "top-k bit-exact when run on the same score tensor"), and with
 the unfused stack (index rows and attention outputs identical).
 
 Cases: ragged and multi-tile shapes, B > 1 with a continuation chunk, the
-benchmarked 8K prefill, every row falling back (w = 0: all scores tie at 0,
-the closed form [0 .. k-1]), about half the rows falling back (a tiny
+benchmarked 8K prefill, the long rows falling back (w = 0: all scores tie
+at 0, the closed form [0 .. k-1]), about half the rows falling back (a tiny
 threshold margin), and small workspaces that split the rows into chunks with
 several fallback rounds each.
 """
@@ -114,17 +114,22 @@ def test_fused_8k_prefill_equals_unfused_stack(ic):
     assert np.array_equal(got, want)
 
 
-def test_every_row_falls_back_when_all_scores_tie(ic):
-    """w = 0: every score is 0, so every row with more than 3k visible
-    positions has all of them as candidates, overflows its list and falls
-    back; every row's index row is the closed form [0 .. min(k, t+1) - 1]."""
+def test_long_rows_fall_back_when_all_scores_tie(ic):
+    """w = 0: every score is 0, so every threshold is 0 and every visible
+    position is a candidate.  Rows with up to 4k positions fit their lists and
+    are selected from their candidates; rows with more than 8k overflow (the
+    list holds 4k candidates plus at most 4k reserved-but-unused slots at this
+    size) and fall back; rows in between may do either.  Every index row is
+    the closed form [0 .. min(k, t+1) - 1] (ties go to the lower position)."""
     wl = synth.Workload("w_zero", 1, 4096, 4096, 2, 32, 128, 256, 16, 128, "FS", 0, 52, True)
     cpu = synth.make_layers(wl)
     cpu[0]["w"] = torch.zeros_like(cpu[0]["w"])
     layers = [{n: t.cuda() for n, t in L.items()} for L in cpu]
     st = _stack(ic, wl, layers, 1)
     QB = 256 // wl.H_I
-    assert st.fused_fallback_blocks() == _blocks_with_long_rows(wl, QB, 3 * wl.k)
+    fb = st.fused_fallback_blocks()
+    assert _blocks_with_long_rows(wl, QB, 8 * wl.k) <= fb <= _blocks_with_long_rows(wl, QB, 4 * wl.k)
+    assert fb > 0
     got = st.dumps[0].cpu().numpy().reshape(-1, wl.k)
     t = np.arange(wl.Lq)
     want = np.where(np.arange(wl.k)[None, :] <= t[:, None], np.arange(wl.k)[None, :], -1)
@@ -135,14 +140,15 @@ def test_every_row_falls_back_when_all_scores_tie(ic):
 
 def test_tiny_margin_mixes_fallback_and_fused_rows(ic):
     """z = 0.001 puts the threshold near the sample quantile itself, so about
-    half the long rows find fewer than k candidates: their blocks fall back,
-    the others are selected from candidates; all rows stay exact."""
+    half the rows with sampled thresholds (more than 4k positions) find fewer
+    than k candidates: their blocks fall back, the others are selected from
+    candidates; all rows stay exact."""
     wl = synth.Workload("z_tiny", 1, 6144, 6144, 2, 64, 128, 256, 16, 128, "FS", 0, 53, True)
     layers = [{n: t.cuda() for n, t in L.items()} for L in synth.make_layers(wl)]
     st = _stack(ic, wl, layers, 1, z=0.001)
     QB = 256 // wl.H_I
     fb = st.fused_fallback_blocks()
-    assert 0 < fb < _blocks_with_long_rows(wl, QB, 3 * wl.k)
+    assert 0 < fb < _blocks_with_long_rows(wl, QB, 4 * wl.k)
     want = _expected(ic, wl, layers[0])
     assert np.array_equal(st.dumps[0].cpu().numpy().reshape(-1, wl.k), want)
 
