@@ -735,6 +735,44 @@ def sweep_points(ic, lengths_k, dev, stream, flush, peaks, n_sms, clk):
     return out
 
 
+def graph_point(ic, wl, pattern, layers, flush, steps: int = 20, warmup: int = 3):
+    """The same stack replayed from a CUDA graph (one forward captured after
+    warm-up): the launches of a step are submitted at once, so small steps
+    (decode) lose the gaps between kernel launches.  The library issues no
+    host synchronisation inside a forward, which is what makes it capturable."""
+    dims = ic.make_dims(wl.B, wl.Lq, wl.Lk, wl.q_offset, wl.H_I, wl.d_I, wl.Hq, wl.d, wl.k)
+    stack = ic.LayerStack(pattern, layers, dims, rows_per_chunk=default_rows_per_chunk(wl))
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for _ in range(warmup):
+            stack.forward(side)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        stack.forward()
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    for s in range(steps):
+        flush.fill_(float(s))
+        starts[s].record(st)
+        g.replay()
+        ends[s].record(st)
+    torch.cuda.synchronize()
+    if ic.get_last_device_error() != 0:
+        raise RuntimeError(f"device error in the {wl.name} graph replay")
+    ms = float(np.mean([a.elapsed_time(b) for a, b in zip(starts, ends)]))
+    del g, stack
+    return {"pattern": pattern, "steps": steps, "ms_per_step": ms,
+            "tokens_per_s": wl.B * wl.Lq / (ms * 1e-3), "replay": "cuda graph"}
+
+
 def decode_point(ic, dev, stream, flush, peaks, n_sms, clk):
     """decode_32k: B = 32 sequences, one new query each over a 32768-token
     cache, 16 layers (FSSS)x4 vs all-F; tokens/s = 32 tokens per step."""
@@ -749,6 +787,10 @@ def decode_point(ic, dev, stream, flush, peaks, n_sms, clk):
         pt[key] = stack_point(ic, wl, pat, layers, stream, flush, peaks, n_sms, clk,
                               budget_ms=500.0, warmup=3)
     pt["speedup_of_pattern"] = pt["all_f"]["ms_per_step"] / pt["fsss_x4"]["ms_per_step"]
+    pt["fsss_x4_graph"] = graph_point(ic, wl, wl.pattern, layers, flush)
+    pt["all_f_graph"] = graph_point(ic, wl, "F" * wl.n_layers, layers, flush)
+    pt["speedup_of_pattern_graph"] = (pt["all_f_graph"]["ms_per_step"]
+                                      / pt["fsss_x4_graph"]["ms_per_step"])
     del layers
     torch.cuda.empty_cache()
     return pt
