@@ -124,7 +124,7 @@ def work_per_layer(wl, lq_d: int = 0):
 
 _KERNEL_SRC = {"sparse_attn": ("sparse_attn_kernel", ("sparse_attn.cuh",)),
                "dense_attn": ("dense_attn_kernel", ("dense_attn.cuh",)),
-               "indexer_scores": ("indexer_scores_kernel", ("indexer_scores.cuh",)),
+               "indexer_scores": ("indexer_scores_kernel", ("indexer_scores.cuh", "fused_topk.cuh")),
                "topk_select": ("topk_select_kernel", ("topk_select.cuh",)),
                "fused_select": ("fused_select_kernel", ("fused_topk.cuh",))}
 

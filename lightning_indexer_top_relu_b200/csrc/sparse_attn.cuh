@@ -14,9 +14,11 @@
 // is a full, coalesced 128-byte line pair; rows land XOR-swizzled in shared
 // memory so the ldmatrix reads are bank-conflict free.  S = Q K^T and
 // O += P V run on the tensor cores (m16n8k16, bf16 in, fp32 accumulate); the
-// softmax is online in fp32 (exp2 with the scale pre-multiplied by log2 e)
-// and the O rescale is skipped while the running max does not move.  The
-// warps' partial (max, sum, O) merge through shared memory at the end; with
+// softmax is online in fp32 (exp2, the scale times log2 e folded into the
+// exponent's FMA); the exponent base moves, and O is rescaled, only when a
+// block's maximum passes it by more than 2^8, and a tile with no empty slot
+// skips the masking.  The warps' partial (base, sum, O) merge through shared
+// memory at the end, one weight per (head, warp); with
 // several splits per row each split writes (O / l, log2-sum-exp) to the
 // caller's workspace and a combine kernel merges the splits.
 #pragma once
@@ -43,6 +45,14 @@ constexpr int SA_THREADS = 32 * SA_WARPS;
 constexpr int SA_STAGES = IC_SA_STAGES;
 static_assert(SA_BLOCK == 16 || SA_BLOCK == 32 || SA_BLOCK == 64, "block of 16, 32 or 64 slots");
 constexpr int SA_IDX_TILE = 2048;            // indices staged in shared memory at a time
+constexpr float SA_RESCALE = 8.0f;           // log2 headroom before the exponent base moves
+
+// 2^x on the special-function unit (subnormal results flush to 0).
+__device__ __forceinline__ float sa_ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 struct SparseAttnArgs {
     const __nv_bfloat16* q;    // [B, Lq, Hq, D]
@@ -79,9 +89,11 @@ struct SaSmem {
     static constexpr int OFF_IDX = OFF_KV + SA_WARPS * WARP_KV;
     static constexpr int BYTES = OFF_IDX + SA_IDX_TILE * 4;
     // merge buffers reuse the K/V rings once every warp has finished
-    static constexpr int MERGE_O = OFF_KV;                                  // [4][16][D] f32
-    static constexpr int MERGE_ML = OFF_KV + SA_WARPS * 16 * D * 4;         // [4][16][2] f32
-    static_assert(MERGE_ML + SA_WARPS * 16 * 2 * 4 <= OFF_IDX, "merge buffer overflow");
+    static constexpr int MROW = D + 8;                                      // padded merge rows
+    static constexpr int MERGE_O = OFF_KV;                                  // [4][16][MROW] f32
+    static constexpr int MERGE_ML = OFF_KV + SA_WARPS * 16 * MROW * 4;      // [4][16][2] f32
+    static constexpr int MERGE_W = MERGE_ML + SA_WARPS * 16 * 2 * 4;        // [16][4] + [16] f32
+    static_assert(MERGE_W + (16 * SA_WARPS + 16) * 4 <= OFF_IDX, "merge buffer overflow");
 };
 
 // Byte offset of 16-byte chunk c of row r in a [rows][D] bf16 tile whose
@@ -95,6 +107,9 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool v
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
                  "r"(valid ? 16 : 0)
                  : "memory");
+}
+__device__ __forceinline__ void cp_async16_full(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
@@ -151,6 +166,8 @@ sparse_attn_kernel(const SparseAttnArgs a) {
 
     const __nv_bfloat16* kb = a.k + (long long)b * a.Lk * D;
     const __nv_bfloat16* vb = a.v + (long long)b * a.Lk * D;
+    const __nv_bfloat16* kl = kb + (lane % (D / 8)) * 8;     // this lane's 16-byte chunk
+    const __nv_bfloat16* vl = vb + (lane % (D / 8)) * 8;
     const int32_t* irow = a.idx + row * a.kslots;
     const uint32_t kv_base = sbase + S::OFF_KV + warp * S::WARP_KV;
     int32_t* idx_s = reinterpret_cast<int32_t*>(sa_smem + S::OFF_IDX);
@@ -177,6 +194,8 @@ sparse_attn_kernel(const SparseAttnArgs a) {
         const int tile1 = min(tile0 + SA_IDX_TILE, s1);
         const int ntile = max(tile1 - tile0, 0);
         __syncthreads();                  // previous tile fully consumed
+        const int nfill = (ntile + SA_BLOCK - 1) / SA_BLOCK * SA_BLOCK;   // slots the blocks read
+        int empty = 0;
         for (int i = tid; i < SA_IDX_TILE; i += SA_THREADS) {
             int id = -1;
             if (i < ntile) {
@@ -186,9 +205,12 @@ sparse_attn_kernel(const SparseAttnArgs a) {
                     id = -1;
                 }
             }
+            empty |= (id < 0) & (i < nfill);
             idx_s[i] = id;
         }
-        __syncthreads();
+        // Tiles whose blocks hold no empty slot (every row with at least k
+        // positions) skip the per-slot masking below.
+        const bool masked = __syncthreads_or(empty) != 0;
         if (tile0 == s0) {
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
@@ -200,20 +222,31 @@ sparse_attn_kernel(const SparseAttnArgs a) {
         const int nblk = (ntile + SA_BLOCK - 1) / SA_BLOCK;
         const int niter = nblk > warp ? (nblk - warp + SA_WARPS - 1) / SA_WARPS : 0;
 
-        // Copies block (warp + SA_WARPS * it) of this tile into stage `st`.
+        // Copies block (warp + SA_WARPS * it) of this tile into stage `st`;
+        // empty slots (only in masked tiles) are zero-filled.
         auto issue = [&](int it, int st) {
             const int* ids = idx_s + (warp + SA_WARPS * it) * SA_BLOCK;
             const uint32_t kdst = kv_base + st * S::STAGE;
             const uint32_t vdst = kdst + S::BLK;
             const int c = lane % CPR;
+            if (masked) {
 #pragma unroll
-            for (int i = 0; i < SA_BLOCK / RPI; ++i) {
-                const int r = i * RPI + lane / CPR;
-                const int rid = ids[r];
-                const bool ok = rid >= 0;
-                const long long off = (long long)(ok ? rid : 0) * D + c * 8;
-                cp_async16(kdst + swz<D>(r, c), kb + off, ok);
-                cp_async16(vdst + swz<D>(r, c), vb + off, ok);
+                for (int i = 0; i < SA_BLOCK / RPI; ++i) {
+                    const int r = i * RPI + lane / CPR;
+                    const int rid = ids[r];
+                    const bool ok = rid >= 0;
+                    const long long off = (long long)(ok ? rid : 0) * D + c * 8;
+                    cp_async16(kdst + swz<D>(r, c), kb + off, ok);
+                    cp_async16(vdst + swz<D>(r, c), vb + off, ok);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < SA_BLOCK / RPI; ++i) {
+                    const int r = i * RPI + lane / CPR;
+                    const uint32_t rid = (uint32_t)ids[r];
+                    cp_async16_full(kdst + swz<D>(r, c), kl + (size_t)rid * D);
+                    cp_async16_full(vdst + swz<D>(r, c), vl + (size_t)rid * D);
+                }
             }
         };
 #pragma unroll
@@ -248,45 +281,42 @@ sparse_attn_kernel(const SparseAttnArgs a) {
                     mma_bf16(sc[2 * np + 1], qf[kk], b2, b3);
                 }
             }
-            const int* ids = idx_s + (warp + SA_WARPS * it) * SA_BLOCK;
+            // Raw scores; the scale (times log2 e) is applied inside the
+            // exponent's FMA.  Empty slots score -inf.
+            if (masked) {
+                const int* ids = idx_s + (warp + SA_WARPS * it) * SA_BLOCK;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        if (ids[nt * 8 + (lane & 3) * 2 + e] < 0) sc[nt][e] = sc[nt][2 + e] = -INFINITY;
+                    }
+                }
+            }
             float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const bool valid = ids[nt * 8 + (lane & 3) * 2 + e] >= 0;
-                    sc[nt][e] = valid ? sc[nt][e] * a.scale_log2 : -INFINITY;
-                    sc[nt][2 + e] = valid ? sc[nt][2 + e] * a.scale_log2 : -INFINITY;
-                    mx0 = fmaxf(mx0, sc[nt][e]);
-                    mx1 = fmaxf(mx1, sc[nt][2 + e]);
-                }
+                mx0 = fmaxf(mx0, fmaxf(sc[nt][0], sc[nt][1]));
+                mx1 = fmaxf(mx1, fmaxf(sc[nt][2], sc[nt][3]));
             }
             mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
             mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
             mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
             mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-            const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-            const float base0 = mn0 == -INFINITY ? 0.0f : mn0;
-            const float base1 = mn1 == -INFINITY ? 0.0f : mn1;
-            const float al0 = exp2f(m0 - base0), al1 = exp2f(m1 - base1);
-            m0 = mn0;
-            m1 = mn1;
-            float rs0 = 0.0f, rs1 = 0.0f;
-            uint32_t pa[KS][4];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const float p0 = exp2f(sc[nt][0] - base0);
-                const float p1 = exp2f(sc[nt][1] - base0);
-                const float p2 = exp2f(sc[nt][2] - base1);
-                const float p3 = exp2f(sc[nt][3] - base1);
-                rs0 += p0 + p1;
-                rs1 += p2 + p3;
-                pa[nt >> 1][(nt & 1) * 2 + 0] = pack_bf16(p0, p1);
-                pa[nt >> 1][(nt & 1) * 2 + 1] = pack_bf16(p2, p3);
-            }
-            l0 = l0 * al0 + rs0;
-            l1 = l1 * al1 + rs1;
-            if (__any_sync(0xffffffffu, al0 != 1.0f || al1 != 1.0f)) {
+            mx0 *= a.scale_log2;
+            mx1 *= a.scale_log2;
+            // The exponent base m moves only when the block's maximum passes
+            // it by more than SA_RESCALE (log2 units): below that the
+            // probabilities stay under 2^SA_RESCALE, and O and l, which share
+            // the base, need no rescale.  The final O / l is the same.
+            const bool up0 = mx0 > m0 + SA_RESCALE, up1 = mx1 > m1 + SA_RESCALE;
+            if (__any_sync(0xffffffffu, up0 || up1)) {
+                const float al0 = up0 ? sa_ex2(m0 - mx0) : 1.0f;    // 0 while m was -inf
+                const float al1 = up1 ? sa_ex2(m1 - mx1) : 1.0f;
+                if (up0) m0 = mx0;
+                if (up1) m1 = mx1;
+                l0 *= al0;
+                l1 *= al1;
 #pragma unroll
                 for (int i = 0; i < D / 8; ++i) {
                     o[i][0] *= al0;
@@ -295,6 +325,23 @@ sparse_attn_kernel(const SparseAttnArgs a) {
                     o[i][3] *= al1;
                 }
             }
+            const float nb0 = m0 == -INFINITY ? 0.0f : -m0;
+            const float nb1 = m1 == -INFINITY ? 0.0f : -m1;
+            float rs0 = 0.0f, rs1 = 0.0f;
+            uint32_t pa[KS][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const float p0 = sa_ex2(fmaf(sc[nt][0], a.scale_log2, nb0));
+                const float p1 = sa_ex2(fmaf(sc[nt][1], a.scale_log2, nb0));
+                const float p2 = sa_ex2(fmaf(sc[nt][2], a.scale_log2, nb1));
+                const float p3 = sa_ex2(fmaf(sc[nt][3], a.scale_log2, nb1));
+                rs0 += p0 + p1;
+                rs1 += p2 + p3;
+                pa[nt >> 1][(nt & 1) * 2 + 0] = pack_bf16(p0, p1);
+                pa[nt >> 1][(nt & 1) * 2 + 1] = pack_bf16(p2, p3);
+            }
+            l0 += rs0;
+            l1 += rs1;
 #pragma unroll
             for (int ks = 0; ks < KS; ++ks) {
 #pragma unroll
@@ -323,15 +370,13 @@ sparse_attn_kernel(const SparseAttnArgs a) {
     __syncthreads();       // all warps are past their rings: reuse them for the merge
     float* mo = reinterpret_cast<float*>(sa_smem + S::MERGE_O);
     float* ml = reinterpret_cast<float*>(sa_smem + S::MERGE_ML);
+    float* mw = reinterpret_cast<float*>(sa_smem + S::MERGE_W);
     const int g = lane >> 2, cq = (lane & 3) * 2;
 #pragma unroll
     for (int i = 0; i < D / 8; ++i) {
-        float* r0 = mo + (warp * 16 + g) * D + i * 8 + cq;
-        float* r1 = mo + (warp * 16 + g + 8) * D + i * 8 + cq;
-        r0[0] = o[i][0];
-        r0[1] = o[i][1];
-        r1[0] = o[i][2];
-        r1[1] = o[i][3];
+        // rows padded to D + 8 floats: the quad's float2 stores of 8 rows hit distinct banks
+        *reinterpret_cast<float2*>(mo + (warp * 16 + g) * S::MROW + i * 8 + cq) = make_float2(o[i][0], o[i][1]);
+        *reinterpret_cast<float2*>(mo + (warp * 16 + g + 8) * S::MROW + i * 8 + cq) = make_float2(o[i][2], o[i][3]);
     }
     if ((lane & 3) == 0) {
         ml[(warp * 16 + g) * 2 + 0] = m0;
@@ -340,23 +385,31 @@ sparse_attn_kernel(const SparseAttnArgs a) {
         ml[(warp * 16 + g + 8) * 2 + 1] = l1;
     }
     __syncthreads();
-
-    for (int e = tid; e < a.Hq * D; e += SA_THREADS) {
-        const int h = e / D, dcol = e % D;
+    // Per head: the warps' weights 2^(m_w - M) / L and the log2-sum-exp M + log2 L.
+    if (tid < 16) {
+        const int h = tid;
         float M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < SA_WARPS; ++w) M = fmaxf(M, ml[(w * 16 + h) * 2]);
-        float L = 0.0f, acc = 0.0f;
-        if (M != -INFINITY) {
+        float f[SA_WARPS], L = 0.0f;
 #pragma unroll
-            for (int w = 0; w < SA_WARPS; ++w) {
-                const float f = exp2f(ml[(w * 16 + h) * 2] - M);
-                L += f * ml[(w * 16 + h) * 2 + 1];
-                acc += f * mo[(w * 16 + h) * D + dcol];
-            }
+        for (int w = 0; w < SA_WARPS; ++w) {
+            f[w] = M == -INFINITY ? 0.0f : sa_ex2(ml[(w * 16 + h) * 2] - M);
+            L += f[w] * ml[(w * 16 + h) * 2 + 1];
         }
-        const float val = L > 0.0f ? acc / L : 0.0f;
-        const float lse2 = L > 0.0f ? M + log2f(L) : -INFINITY;
+        const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+#pragma unroll
+        for (int w = 0; w < SA_WARPS; ++w) mw[h * SA_WARPS + w] = f[w] * inv;
+        mw[16 * SA_WARPS + h] = L > 0.0f ? M + log2f(L) : -INFINITY;
+    }
+    __syncthreads();
+
+    for (int e = tid; e < a.Hq * D; e += SA_THREADS) {
+        const int h = e / D, dcol = e % D;
+        float val = 0.0f;
+#pragma unroll
+        for (int w = 0; w < SA_WARPS; ++w) val = fmaf(mw[h * SA_WARPS + w], mo[(w * 16 + h) * S::MROW + dcol], val);
+        const float lse2 = mw[16 * SA_WARPS + h];
         if (a.splits == 1) {
             a.out[(row * a.Hq + h) * D + dcol] = __float2bfloat16_rn(val);
             if (a.lse && dcol == 0) a.lse[row * a.Hq + h] = lse2 * LN2;
