@@ -59,8 +59,19 @@ namespace ic {
 constexpr int IDX_BM = 128;          // keys per tile = TMEM lanes
 constexpr int IDX_NMAX = 256;        // max (query, head) columns per MMA
 constexpr int IDX_STAGES = 3;        // k_I tile ring depth
-constexpr int IDX_EPI_WARPS = 8;
-constexpr int IDX_THREADS = 64 + 32 * IDX_EPI_WARPS;
+#ifndef IC_IDX_EARLY_FREE
+#define IC_IDX_EARLY_FREE 1
+#endif
+// 16x256b epilogue: a tile's TMEM accumulator is released as soon as its
+// last read has landed, before the second lane half's arithmetic.
+constexpr bool IDX_EARLY_FREE = IC_IDX_EARLY_FREE != 0;
+#ifndef IC_IDX_EPI_WIDE
+#define IC_IDX_EPI_WIDE 16
+#endif
+// Epilogue warps: with 64 heads (a block of 4 queries) four warps per TMEM
+// lane quarter, one query each; otherwise two per quarter.
+__host__ __device__ constexpr int idx_epi_warps(int H) { return H == 64 ? IC_IDX_EPI_WIDE : 8; }
+__host__ __device__ constexpr int idx_threads(int H) { return 64 + 32 * idx_epi_warps(H); }
 
 enum : int { IDX_SCORES = 0, IDX_SAMPLE = 1, IDX_CAND = 2 };
 constexpr unsigned IDX_RES = 32;              // IDX_CAND: list slots reserved per atomic
@@ -87,6 +98,21 @@ __device__ __forceinline__ void tmem_ld_16x256b_x16(uint32_t taddr, uint32_t (&r
           "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]),
           "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]),
           "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+        : "r"(taddr));
+}
+
+// The same shape with 8 repetitions (columns [0, 64)).
+__device__ __forceinline__ void tmem_ld_16x256b_x8(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x8.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
         : "r"(taddr));
 }
 
@@ -183,12 +209,14 @@ __device__ __forceinline__ UnitInfo unit_info(const IndexerArgs& a, long long u,
 }
 
 template <int H, int DI, int MODE>
-__global__ void __launch_bounds__(IDX_THREADS, 1)
+__global__ void __launch_bounds__(idx_threads(H), 1)
 indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
                       const __grid_constant__ CUtensorMap tmap_k, const IndexerArgs args) {
     using S = IndexerSmem<DI>;
     constexpr int KBOX = DI / 64;                 // 64-element (128-byte) swizzle boxes along d_I
     constexpr int QBMAX = IDX_NMAX / H;
+    constexpr int EPI = idx_epi_warps(H);
+    constexpr int NG = EPI / 4;                   // epilogue warps per TMEM lane quarter
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align_smem_1024(smem_raw, S::BYTES);
@@ -216,9 +244,9 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
             mbar_init(&q_full[i], 1);
             // freed by the MMA commit of the unit's last tile and by every
             // epilogue warp once it has read the unit's head weights
-            mbar_init(&q_empty[i], 1 + IDX_EPI_WARPS);
+            mbar_init(&q_empty[i], 1 + EPI);
             mbar_init(&acc_full[i], 1);
-            mbar_init(&acc_empty[i], 32 * IDX_EPI_WARPS);
+            mbar_init(&acc_empty[i], 32 * EPI);
         }
         for (int i = 0; i < IDX_STAGES; ++i) {
             mbar_init(&a_full[i], 1);
@@ -312,11 +340,11 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
             }
         }
     } else {
-        // ---------------- epilogue (warps 2..9)
+        // ---------------- epilogue (warps 2 .. 1 + EPI)
         const int wq = warp & 3;                  // TMEM lane quarter this warp may read
-        const int cg = (warp - 2) >> 2;           // which half of the block's queries
+        const int cg = (warp - 2) >> 2;           // which part of the block's queries (of NG)
         const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
-        constexpr int QH = (QBMAX + 1) / 2;       // queries per half at most
+        constexpr int QH = (QBMAX + NG - 1) / NG; // queries per part at most
         constexpr bool QUAD = H >= 64;            // 16x256b TMEM reads, weights in registers
         const unsigned lt = (1u << lane) - 1u;
         uint32_t ta = 0, uq = 0;
@@ -326,9 +354,9 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
             if (ui.j0 >= ui.j1) continue;
             const int qb = uq & 1;
             // queries [qlo, qhi) of this block belong to this warp
-            const int qhalf = (args.QB + 1) / 2;
-            const int qlo = cg * qhalf;
-            const int qhi = min(ui.nq, qlo + qhalf);
+            const int qpart = (args.QB + NG - 1) / NG;
+            const int qlo = cg * qpart;
+            const int qhi = min(ui.nq, qlo + qpart);
             const int ncol = (qhi > qlo ? qhi - qlo : 0) * H;        // multiple of 4
             const int nchunk = (ncol + 31) / 32;
             // the unit's head weights are in w_s[qb] once q_full[qb] completed
@@ -399,13 +427,22 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
 #pragma unroll
                         for (int q = 0; q < QH; ++q) a2[0][q] = a2[1][q] = make_float2(0.0f, 0.0f);
                         if (qhi > qlo) {                                  // warp-uniform
-                            uint32_t v[64];
-                            tmem_ld_16x256b_x16(tmem_base + ((uint32_t)(wq * 32 + 16 * lh) << 16) +
-                                                    (uint32_t)(ab * IDX_NMAX + qlo * H),
-                                                v);
+                            constexpr int REPS = QH * H / 8;              // 8-column repetitions
+                            static_assert(REPS == 8 || REPS == 16, "16x256b reads of 64 or 128 columns");
+                            uint32_t v[4 * REPS];
+                            const uint32_t ta16 = tmem_base + ((uint32_t)(wq * 32 + 16 * lh) << 16) +
+                                                  (uint32_t)(ab * IDX_NMAX + qlo * H);
+                            if constexpr (REPS == 16)
+                                tmem_ld_16x256b_x16(ta16, *reinterpret_cast<uint32_t(*)[64]>(&v[0]));
+                            else
+                                tmem_ld_16x256b_x8(ta16, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
                             tmem_ld_wait();
+                            if (IDX_EARLY_FREE && lh == 1) {          // the tile's TMEM is read
+                                tc_fence_before();
+                                mbar_arrive(&acc_empty[ab]);
+                            }
 #pragma unroll
-                            for (int r = 0; r < 16; ++r) {
+                            for (int r = 0; r < REPS; ++r) {
                                 const int q = (8 * r) / H, m = ((8 * r) % H) / 8;
                                 const float2 r0 = make_float2(fmaxf(__uint_as_float(v[4 * r]), 0.0f),
                                                               fmaxf(__uint_as_float(v[4 * r + 1]), 0.0f));
@@ -414,6 +451,10 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
                                 a2[0][q] = __ffma2_rn(wr[q][m], r0, a2[0][q]);
                                 a2[1][q] = __ffma2_rn(wr[q][m], r1, a2[1][q]);
                             }
+                        }
+                        if (IDX_EARLY_FREE && lh == 1 && qhi <= qlo) {
+                            tc_fence_before();
+                            mbar_arrive(&acc_empty[ab]);
                         }
 #pragma unroll
                         for (int q = 0; q < QH; ++q) {
@@ -469,8 +510,10 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
                         }
                     }
                 }
-                tc_fence_before();
-                mbar_arrive(&acc_empty[ab]);
+                if (!(QUAD && IDX_EARLY_FREE)) {
+                    tc_fence_before();
+                    mbar_arrive(&acc_empty[ab]);
+                }
                 const int s = j * kstride * IDX_BM + wq * 32 + klane;     // key position
                 if (MODE == IDX_CAND) {
 #pragma unroll
