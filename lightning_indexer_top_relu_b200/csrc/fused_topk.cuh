@@ -243,12 +243,29 @@ fused_select_kernel(const FusedArgs a) {
     const uint32_t c = __ldg(a.cnt + rr);
     uint32_t valid = 0;
     if (c <= (uint32_t)a.lstride) {                 // uniform
-        const unsigned long long* crow = a.cand + rr * (long long)a.lstride;
+        // The list in pairs (lstride is even, so a row starts 16-byte
+        // aligned and the pair holding entry c-1 lies inside the row), four
+        // independent 16-byte loads per thread in flight.
+        const ulonglong2* crow = reinterpret_cast<const ulonglong2*>(a.cand + rr * (long long)a.lstride);
+        const uint32_t npair = (c + 1) / 2;
         uint32_t mine = 0;
-        for (uint32_t j = tid; j < c; j += FS_THREADS) {
-            const unsigned long long v = __ldg(crow + j);
-            vals[j] = v;
-            mine += v != 0ull;
+        for (uint32_t p0 = tid; p0 < npair; p0 += 4 * FS_THREADS) {
+            ulonglong2 x[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (p0 + u * FS_THREADS < npair) x[u] = __ldg(crow + p0 + u * FS_THREADS);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const uint32_t pj = p0 + u * FS_THREADS;
+                if (pj < npair) {
+                    vals[2 * pj] = x[u].x;
+                    mine += x[u].x != 0ull;
+                    if (2 * pj + 1 < c) {
+                        vals[2 * pj + 1] = x[u].y;
+                        mine += x[u].y != 0ull;
+                    }
+                }
+            }
         }
         block_excl_scan<FS_THREADS>(mine, wsum, tot);
         valid = *tot;

@@ -148,11 +148,11 @@ cudaError_t launch_indexer_t(int mode, const CUtensorMap& tq, const CUtensorMap&
                              const ic::IndexerArgs& a, int grid, cudaStream_t st) {
     constexpr int SM = ic::IndexerSmem<DI>::ALLOC;
     if (mode == ic::IDX_SAMPLE)
-        ic::indexer_scores_kernel<H, DI, ic::IDX_SAMPLE><<<grid, ic::idx_threads(H), SM, st>>>(tq, tk, a);
+        ic::indexer_scores_kernel<H, DI, ic::IDX_SAMPLE><<<grid, ic::idx_threads(H, ic::IDX_SAMPLE), SM, st>>>(tq, tk, a);
     else if (mode == ic::IDX_CAND)
-        ic::indexer_scores_kernel<H, DI, ic::IDX_CAND><<<grid, ic::idx_threads(H), SM, st>>>(tq, tk, a);
+        ic::indexer_scores_kernel<H, DI, ic::IDX_CAND><<<grid, ic::idx_threads(H, ic::IDX_CAND), SM, st>>>(tq, tk, a);
     else
-        ic::indexer_scores_kernel<H, DI, ic::IDX_SCORES><<<grid, ic::idx_threads(H), SM, st>>>(tq, tk, a);
+        ic::indexer_scores_kernel<H, DI, ic::IDX_SCORES><<<grid, ic::idx_threads(H, ic::IDX_SCORES), SM, st>>>(tq, tk, a);
     return cudaGetLastError();
 }
 

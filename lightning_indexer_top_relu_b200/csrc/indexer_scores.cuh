@@ -59,6 +59,7 @@ namespace ic {
 constexpr int IDX_BM = 128;          // keys per tile = TMEM lanes
 constexpr int IDX_NMAX = 256;        // max (query, head) columns per MMA
 constexpr int IDX_STAGES = 3;        // k_I tile ring depth
+enum : int { IDX_SCORES = 0, IDX_SAMPLE = 1, IDX_CAND = 2 };
 #ifndef IC_IDX_EARLY_FREE
 #define IC_IDX_EARLY_FREE 1
 #endif
@@ -68,12 +69,18 @@ constexpr bool IDX_EARLY_FREE = IC_IDX_EARLY_FREE != 0;
 #ifndef IC_IDX_EPI_WIDE
 #define IC_IDX_EPI_WIDE 16
 #endif
+#ifndef IC_IDX_WIDE32
+#define IC_IDX_WIDE32 1
+#endif
 // Epilogue warps: with 64 heads (a block of 4 queries) four warps per TMEM
-// lane quarter, one query each; otherwise two per quarter.
-__host__ __device__ constexpr int idx_epi_warps(int H) { return H == 64 ? IC_IDX_EPI_WIDE : 8; }
-__host__ __device__ constexpr int idx_threads(int H) { return 64 + 32 * idx_epi_warps(H); }
+// lane quarter, one query each, and likewise with 32 heads (8 queries, two
+// per warp) except in the candidate pass, whose extra state would not fit the
+// registers of 18 warps; otherwise two warps per quarter.
+__host__ __device__ constexpr int idx_epi_warps(int H, int mode) {
+    return (H == 64 || (IC_IDX_WIDE32 && H == 32 && mode != IDX_CAND)) ? IC_IDX_EPI_WIDE : 8;
+}
+__host__ __device__ constexpr int idx_threads(int H, int mode) { return 64 + 32 * idx_epi_warps(H, mode); }
 
-enum : int { IDX_SCORES = 0, IDX_SAMPLE = 1, IDX_CAND = 2 };
 constexpr unsigned IDX_RES = 32;              // IDX_CAND: list slots reserved per atomic
 constexpr uint32_t IDX_NONE = 0xFFFFFFFFu;    // IDX_CAND threshold: the row keeps no candidate
 
@@ -209,13 +216,13 @@ __device__ __forceinline__ UnitInfo unit_info(const IndexerArgs& a, long long u,
 }
 
 template <int H, int DI, int MODE>
-__global__ void __launch_bounds__(idx_threads(H), 1)
+__global__ void __launch_bounds__(idx_threads(H, MODE), 1)
 indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
                       const __grid_constant__ CUtensorMap tmap_k, const IndexerArgs args) {
     using S = IndexerSmem<DI>;
     constexpr int KBOX = DI / 64;                 // 64-element (128-byte) swizzle boxes along d_I
     constexpr int QBMAX = IDX_NMAX / H;
-    constexpr int EPI = idx_epi_warps(H);
+    constexpr int EPI = idx_epi_warps(H, MODE);
     constexpr int NG = EPI / 4;                   // epilogue warps per TMEM lane quarter
 
     extern __shared__ uint8_t smem_raw[];
