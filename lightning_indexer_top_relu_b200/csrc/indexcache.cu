@@ -71,6 +71,8 @@ constexpr int MAX_DEV = 64;
 std::mutex g_mu;
 int g_sms[MAX_DEV];
 bool g_attr_done[MAX_DEV];
+// 8-CTA clusters of the gather kernel fit on the device (checked at setup)
+bool g_attn_cluster[MAX_DEV];
 
 int device_setup(int* dev_out, int* sms_out);
 
@@ -317,6 +319,55 @@ int attn_splits(long long n_rows, int k_slots, int sms) {
     return (int)std::max<long long>(1, s);
 }
 
+// Splits of up to ATTN_CLUSTER_MAX CTAs run as one thread-block cluster per
+// row and merge through distributed shared memory (no workspace, no combine
+// launch); a one-wave split count up to twice that is trimmed to it.
+constexpr int ATTN_CLUSTER_MAX = 8;
+
+template <int D>
+bool attn_cluster_fits() {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1, ATTN_CLUSTER_MAX, 1);
+    cfg.blockDim = dim3(ic::SA_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = ic::SaSmem<D>::BYTES;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 1;
+    at[0].val.clusterDim.y = ATTN_CLUSTER_MAX;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int n = 0;
+    return cudaOccupancyMaxActiveClusters(&n, ic::sparse_attn_kernel<D>, &cfg) == cudaSuccess && n > 0;
+}
+
+bool attn_cluster_available() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEV) return false;
+    return g_attn_cluster[dev];
+}
+
+template <int D>
+cudaError_t launch_attn_kernel(const ic::SparseAttnArgs& a, dim3 grid, bool cluster, cudaStream_t st) {
+    if (!cluster) {
+        ic::sparse_attn_kernel<D><<<grid, ic::SA_THREADS, ic::SaSmem<D>::BYTES, st>>>(a);
+        return cudaGetLastError();
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(ic::SA_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = ic::SaSmem<D>::BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 1;
+    at[0].val.clusterDim.y = grid.y;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, ic::sparse_attn_kernel<D>, a);
+}
+
 size_t attn_ws_bytes(long long n_rows, int splits, int Hq, int d) {
     if (splits <= 1) return 0;
     return (size_t)n_rows * splits * (size_t)Hq * (d + 1) * sizeof(float);
@@ -332,7 +383,9 @@ int launch_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, const i
     const long long n_rows = (long long)B * rows_per_b;
     if (n_rows <= 0) return IC_OK;
     int splits = attn_splits(n_rows, k_slots, sms);
-    while (splits > 1 && (ws == nullptr || attn_ws_bytes(n_rows, splits, Hq, d) > ws_bytes))
+    const bool cluster = splits > 1 && splits <= 2 * ATTN_CLUSTER_MAX && attn_cluster_available();
+    if (cluster) splits = std::min(splits, ATTN_CLUSTER_MAX);
+    while (!cluster && splits > 1 && (ws == nullptr || attn_ws_bytes(n_rows, splits, Hq, d) > ws_bytes))
         splits = splits / 2;
     ic::SparseAttnArgs a;
     a.q = reinterpret_cast<const __nv_bfloat16*>(q);
@@ -341,9 +394,10 @@ int launch_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, const i
     a.idx = idx;
     a.out = reinterpret_cast<__nv_bfloat16*>(out);
     a.lse = lse;
-    a.part_o = splits > 1 ? reinterpret_cast<float*>(ws) : nullptr;
-    a.part_lse = splits > 1 ? reinterpret_cast<float*>(ws) + n_rows * splits * (long long)Hq * d
-                            : nullptr;
+    a.cluster = cluster ? 1 : 0;
+    a.part_o = splits > 1 && !cluster ? reinterpret_cast<float*>(ws) : nullptr;
+    a.part_lse = splits > 1 && !cluster ? reinterpret_cast<float*>(ws) + n_rows * splits * (long long)Hq * d
+                                        : nullptr;
     a.Lq = Lq;
     a.Lk = Lk;
     a.Hq = Hq;
@@ -358,14 +412,10 @@ int launch_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, const i
     a.rows_per_b = rows_per_b;
     a.row_i0 = row_i0;
     dim3 grid((unsigned)n_rows, (unsigned)splits);
-    if (d == 64) {
-        ic::sparse_attn_kernel<64><<<grid, ic::SA_THREADS, ic::SaSmem<64>::BYTES, st>>>(a);
-    } else {
-        ic::sparse_attn_kernel<128><<<grid, ic::SA_THREADS, ic::SaSmem<128>::BYTES, st>>>(a);
-    }
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = d == 64 ? launch_attn_kernel<64>(a, grid, cluster, st)
+                            : launch_attn_kernel<128>(a, grid, cluster, st);
     if (launched(e, "sparse_attn launch")) return IC_ERR_CUDA;
-    if (splits > 1) {
+    if (splits > 1 && !cluster) {
         const dim3 cg((unsigned)n_rows, (unsigned)Hq);
         if (d == 64)
             ic::sparse_attn_combine_kernel<64><<<cg, 64, 0, st>>>(a);
@@ -725,6 +775,8 @@ int device_setup(int* dev_out, int* sms_out) {
                              cudaFuncAttributeMaxDynamicSharedMemorySize, ic::SaSmem<128>::BYTES);
         e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+        g_attn_cluster[dev] = attn_cluster_fits<64>() && attn_cluster_fits<128>();
+        cudaGetLastError();                         // a refused query only disables clusters
         g_sms[dev] = sms;
         g_attr_done[dev] = true;
     }

@@ -82,6 +82,9 @@ __host__ __device__ constexpr int idx_epi_warps(int H, int mode) {
 __host__ __device__ constexpr int idx_threads(int H, int mode) { return 64 + 32 * idx_epi_warps(H, mode); }
 
 constexpr unsigned IDX_RES = 32;              // IDX_CAND: list slots reserved per atomic
+// One ballot takes up to 32 candidates, and what the current range cannot
+// hold goes to the single range reserved ahead: a range holds at least a warp.
+static_assert(IDX_RES >= 32, "a reserved range must hold one ballot's candidates");
 constexpr uint32_t IDX_NONE = 0xFFFFFFFFu;    // IDX_CAND threshold: the row keeps no candidate
 
 // 16 lanes x (16 x 8) 32-bit columns: repetition r covers columns

@@ -18,9 +18,12 @@
 // exponent's FMA); the exponent base moves, and O is rescaled, only when a
 // block's maximum passes it by more than 2^8, and a tile with no empty slot
 // skips the masking.  The warps' partial (base, sum, O) merge through shared
-// memory at the end, one weight per (head, warp); with
-// several splits per row each split writes (O / l, log2-sum-exp) to the
-// caller's workspace and a combine kernel merges the splits.
+// memory at the end, one weight per (head, warp).  With several splits per
+// row (few rows: decode), up to 8 splits run as one thread-block cluster:
+// each keeps its (O / l, log2-sum-exp) in shared memory and, after a cluster
+// barrier, split r merges heads r, r + splits, ... from every split through
+// distributed shared memory.  With more splits each writes its partial to
+// the caller's workspace and a combine kernel merges them.
 #pragma once
 
 #include "common.cuh"
@@ -61,8 +64,9 @@ struct SparseAttnArgs {
     const int32_t* idx;        // [B*Lq, kslots]
     __nv_bfloat16* out;        // [B, Lq, Hq, D]
     float* lse;                // [B, Lq, Hq] or null
-    float* part_o;             // [rows, splits, Hq, D] (splits > 1)
+    float* part_o;             // [rows, splits, Hq, D] (splits > 1, not clustered)
     float* part_lse;           // [rows, splits, Hq]
+    int cluster;               // the row's splits form one thread-block cluster (splits <= 8)
     int Lq, Lk, Hq, kslots, q_offset;
     int splits, slots_per_split;
     int trim;                  // slots past min(k, t+1) are known empty
@@ -93,7 +97,8 @@ struct SaSmem {
     static constexpr int MERGE_O = OFF_KV;                                  // [4][16][MROW] f32
     static constexpr int MERGE_ML = OFF_KV + SA_WARPS * 16 * MROW * 4;      // [4][16][2] f32
     static constexpr int MERGE_W = MERGE_ML + SA_WARPS * 16 * 2 * 4;        // [16][4] + [16] f32
-    static_assert(MERGE_W + (16 * SA_WARPS + 16) * 4 <= OFF_IDX, "merge buffer overflow");
+    static constexpr int FIN = MERGE_W + (16 * SA_WARPS + 16) * 4;          // [16][D] f32 (clustered)
+    static_assert(FIN + 16 * D * 4 <= OFF_IDX, "merge buffer overflow");
 };
 
 // Byte offset of 16-byte chunk c of row r in a [rows][D] bf16 tile whose
@@ -142,6 +147,20 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&p);
+}
+
+// Thread-block cluster primitives: a barrier over the cluster's CTAs
+// (release / acquire, so shared-memory writes before it are visible to the
+// other CTAs after it) and a 32-bit load from another CTA's shared memory.
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t local_addr, uint32_t rank) {
+    uint32_t remote;
+    float v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+    return v;
 }
 
 template <int D>
@@ -413,11 +432,48 @@ sparse_attn_kernel(const SparseAttnArgs a) {
         if (a.splits == 1) {
             a.out[(row * a.Hq + h) * D + dcol] = __float2bfloat16_rn(val);
             if (a.lse && dcol == 0) a.lse[row * a.Hq + h] = lse2 * LN2;
+        } else if (a.cluster) {
+            reinterpret_cast<float*>(sa_smem + S::FIN)[h * D + dcol] = val;
         } else {
             const long long pr = (pidx * a.splits + split) * a.Hq + h;
             a.part_o[pr * D + dcol] = val;
             if (dcol == 0) a.part_lse[pr] = lse2;
         }
+    }
+    if (a.splits > 1 && a.cluster) {
+        // The row's splits are one cluster (rank = split).  Each split's
+        // (O / l, log2-sum-exp) stays in its shared memory; rank r merges
+        // heads r, r + splits, ... from every rank's copy, with the same
+        // weights as the combine kernel.
+        cluster_sync_all();
+        const uint32_t fin_addr = sbase + (uint32_t)S::FIN;
+        const uint32_t lse_addr = sbase + (uint32_t)(S::MERGE_W + 16 * SA_WARPS * 4);
+        for (int h = split; h < a.Hq; h += a.splits) {
+            float lr[8];
+            float M = -INFINITY;
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                lr[r] = r < a.splits ? ld_cluster_f32(lse_addr + (uint32_t)h * 4u, (uint32_t)r) : -INFINITY;
+                M = fmaxf(M, lr[r]);
+            }
+            float W = 0.0f;
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                lr[r] = M == -INFINITY ? 0.0f : sa_ex2(lr[r] - M);
+                W += lr[r];
+            }
+            const float inv = W > 0.0f ? 1.0f / W : 0.0f;
+            for (int dcol = tid; dcol < D; dcol += SA_THREADS) {
+                float acc = 0.0f;
+#pragma unroll
+                for (int r = 0; r < 8; ++r)
+                    if (r < a.splits)
+                        acc = fmaf(lr[r], ld_cluster_f32(fin_addr + (uint32_t)(h * D + dcol) * 4u, (uint32_t)r), acc);
+                a.out[(row * a.Hq + h) * D + dcol] = __float2bfloat16_rn(acc * inv);
+                if (a.lse && dcol == 0) a.lse[row * a.Hq + h] = W > 0.0f ? (M + log2f(W)) * LN2 : -INFINITY;
+            }
+        }
+        cluster_sync_all();            // no CTA leaves while another may read its shared memory
     }
 }
 
