@@ -168,11 +168,18 @@ def profile_traffic(kernel: str, workload: str, units: float = 0.0):
         got = _read_profile(path, srcs)
         return (got[0], os.path.basename(path)) if got else (None, None)
     if units > 0:
+        # the matching capture whose size is nearest (in ratio) to this launch's
+        best = None
         for path in sorted(glob.glob(os.path.join(ROOT, "profiles", f"{name}_*.md"))):
             got = _read_profile(path, srcs)
             if got and got[1]:
-                return int(got[0] * units / got[1]), (f"{os.path.basename(path)} scaled by "
-                                                      f"{units:g} / {got[1]:g} rows")
+                dist = abs(math.log(units / got[1]))
+                if best is None or dist < best[0]:
+                    best = (dist, path, got)
+        if best:
+            _, path, got = best
+            return int(got[0] * units / got[1]), (f"{os.path.basename(path)} scaled by "
+                                                  f"{units:g} / {got[1]:g} rows")
     return None, None
 
 
