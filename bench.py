@@ -713,6 +713,11 @@ def stack_point(ic, wl, pattern, layers, stream, flush, peaks, n_sms, clk, budge
         out["indexer_frac_of_bf16_peak"] = kern["indexer"]["frac_of_bf16_peak"]
     if "topk" in kern:
         out["topk_ms_per_launch"] = kern["topk"]["ms_per_launch"]
+        if "indexer" in kern and kern["topk"]["ms_per_launch"] < 0.01 * kern["indexer"]["ms_per_launch"]:
+            # an F layer run in several workspace chunks interleaves the
+            # indexer and the top-k of each chunk: the layer's one indexer
+            # span then covers both (its rate is a lower bound)
+            out["indexer_span_includes_topk"] = True
     for name in ("attn_dense", "attn_gather"):
         if name in kern:
             out[f"{name}_ms_per_launch"] = kern[name]["ms_per_launch"]

@@ -19,15 +19,18 @@
 //               weights w (bulk copy), once per work unit, double-buffered;
 //               k_I tiles (A operand) through a 3-stage ring
 //   warp 1      TMEM allocator + single-thread MMA issuer
-//   warps 2..9  epilogue: tcgen05.ld -> ReLU -> w-weighted head sum -> causal
-//               mask -> output.  With 16+ heads the TMEM reads use the
-//               16x256b shape: a thread holds 2 keys x a quarter of the
-//               columns, its quarter of the head weights stays in registers
-//               for the unit, and a quad adds its partial sums by shuffles.  Warp w reads TMEM lane quarter w % 4 and the
-//               half of the block's queries given by (w-2) / 4, so two warps
+//   warps 2..   epilogue (16 warps with 64 heads, and with 32 heads outside
+//               the candidate pass; else 8): tcgen05.ld -> ReLU -> w-weighted
+//               head sum -> causal mask -> output.  With 64+ heads the TMEM
+//               reads use the 16x256b shape: a thread holds 2 keys x a
+//               quarter of its columns, its quarter of the head weights stays
+//               in registers for the unit, and a quad adds its partial sums
+//               by shuffles.  Warp w reads TMEM lane quarter w % 4 and the
+//               part (w-2) / 4 of the block's queries, so 4 (or 2) warps
 //               share each SM sub-partition.  Two TMEM accumulators
 //               (2 x 256 columns) let the epilogue of tile j overlap the MMA
-//               of tile j+1.
+//               of tile j+1; with 16x256b reads a tile's accumulator is
+//               released as soon as its last read lands.
 // A work unit is (query block, run of up to `tpu` key tiles); units are
 // ordered split-major, longest causal rows first within a split, and dealt
 // round-robin to the CTAs.
