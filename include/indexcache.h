@@ -124,9 +124,13 @@ int ic_topk_select(const float *scores, int B, int Lq, int Lk, int q_offset, int
  * Slots holding -1 are empty.  A slot outside [0, t] is skipped and flags
  * IC_ERR_INVALID_ARG in the device error word.  A row with no valid slot
  * gives out = 0, lse = -INFINITY.  scale <= 0 selects 1/sqrt(d).
- * ws/ws_bytes: optional device workspace; with at least
- * ic_sparse_attn_workspace_bytes(...) bytes, rows with few of them (decode)
- * split their slots over several CTAs.  ws may be NULL (ws_bytes 0).
+ * ws/ws_bytes: optional device workspace.  When there are few rows (decode)
+ * each row splits its slots over several CTAs.  Up to 8 splits of a row run
+ * as one thread-block cluster and merge through distributed shared memory,
+ * with no workspace.  More splits (fewer than about 19 rows on a 148-SM
+ * B200) need ic_sparse_attn_workspace_bytes(...) bytes for their partials;
+ * with less, fewer splits run and the results are the same.  ws may be NULL
+ * (ws_bytes 0).
  */
 int ic_sparse_attn(const uint16_t *q, const uint16_t *k, const uint16_t *v, const int32_t *idx,
                    int B, int Lq, int Lk, int Hq, int Hkv, int d, int k_slots, int q_offset,
@@ -143,10 +147,11 @@ size_t ic_sparse_attn_workspace_bytes(int B, int Lq, int Hq, int d, int k_slots)
  * GPU memory and hands a plugin only its inputs and outputs, or a decode loop
  * that must not call cudaMalloc (it can synchronise the device and its cost is
  * unpredictable).  Same arguments, semantics and results as ic_sparse_attn.
- * Rows that split their slots over several CTAs (decode) keep the per-split
- * partial results in a fixed 4 MiB array inside the library instead of a
- * workspace; every GPU that loads the library holds that array until the
- * process exits.
+ * Rows that split their slots over more CTAs than one 8-CTA cluster holds
+ * (decode with fewer than about 19 rows) keep the per-split partial results
+ * in a fixed 4 MiB array inside the library instead of a workspace; every
+ * GPU that loads the library holds that array until the process exits.  Up
+ * to 8 splits merge inside their cluster and use no array.
  *   - Rows split their slots only while rows x splits stays within two CTAs
  *     per SM, so with the supported Hq <= 16 and d <= 128 the partials take
  *     at most 2 x SMs x 16 x 129 x 4 bytes (2.4 MB on a 148-SM B200) and the
