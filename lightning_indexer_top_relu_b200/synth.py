@@ -159,7 +159,8 @@ def make_layers(wl: Workload, layers: Optional[List[int]] = None, indexer_for_al
                 d["q_idx"] = t["q_idx"].to(torch.bfloat16)
                 d["k_idx"] = t["k_idx"].to(torch.bfloat16)
                 d["w"] = t["w"].contiguous()
-            out.append(d)
+            # drawn on the host (the fixed-order stream), then placed on `device`
+            out.append({n: v.to(device) for n, v in d.items()})
         return out
 
     dev = device

@@ -264,3 +264,13 @@ def test_default_workload_is_the_64k_prefill():
     src = inspect.getsource(bench.main)
     assert 'default="prefill_64k"' in src
     assert synth.WORKLOADS["prefill_64k"].pattern == "FSSSFSSS"
+
+
+def test_uncorrelated_workloads_are_placed_on_the_requested_device():
+    """The fixed-order draws of the tiny prefill land on the device asked for
+    (the bench asks for the GPU); 'meta' stands in for it on the CPU."""
+    layers = synth.make_layers(synth.WORKLOADS["tiny_prefill"], device="meta")
+    assert len(layers) == 4
+    assert all(t.device.type == "meta" for L in layers for t in L.values())
+    host = synth.make_layers(synth.WORKLOADS["tiny_prefill"])
+    assert all(t.device.type == "cpu" for L in host for t in L.values())

@@ -176,7 +176,10 @@ ATTN_CASES = [
     # B, Lq, Lk, q_offset, Hq, d, k
     (1, 512, 512, 0, 8, 64, 64),
     (2, 300, 300, 0, 16, 128, 100),
-    (4, 1, 3000, 2999, 16, 128, 2048),     # decode: slots split over CTAs + combine
+    (4, 1, 3000, 2999, 16, 128, 2048),     # decode: 32 splits, workspace + combine kernel
+    (40, 1, 3000, 2999, 16, 128, 2048),    # decode: 7 splits, one 7-CTA cluster per row
+    (20, 1, 3000, 2999, 16, 128, 2048),    # decode: 14 splits trimmed to one 8-CTA cluster
+    (37, 1, 5000, 4999, 16, 64, 1024),     # decode, d = 64: 8 splits in a cluster
     (1, 200, 200, 0, 16, 64, 256),         # k > L: padded tails
 ]
 
@@ -194,6 +197,32 @@ def test_sparse_attn_matches_oracle(ic, B, Lq, Lk, q_offset, Hq, d, k):
     got = out.float().cpu().numpy().reshape(B * Lq, Hq, d)
     assert np.abs(got - ref).max() <= ATTN_ATOL
     assert np.abs(lse.cpu().numpy().reshape(B * Lq, Hq) - ref_lse).max() <= LSE_ATOL
+
+
+def test_clustered_decode_splits_without_valid_slots(ic):
+    """Decode rows whose valid slots all sit in the first split: the other
+    splits of the row's cluster hold no slot (log-sum-exp -inf) and the
+    merge through distributed shared memory must weigh them 0; one row has
+    no valid slot at all (out 0, lse -inf)."""
+    B, Lk, Hq, d, k = 40, 3000, 16, 128, 2048
+    wl = synth.custom(B=B, Lq=1, Lk=Lk, q_offset=Lk - 1, H_I=4, d_I=64, k=k, Hq=Hq, d=d, cfg_id=24)
+    lay = synth.make_layers(wl)[0]
+    rng = np.random.default_rng(5)
+    idx = np.full((B, k), -1, dtype=np.int32)
+    for b in range(1, B):
+        n = int(rng.integers(1, 200))
+        idx[b, :n] = rng.choice(Lk, size=n, replace=False)
+    ref, ref_lse = oracle.sparse_attn(lay["q"], lay["k"], lay["v"], idx, Lk - 1)
+    out, lse = ic.sparse_attn(lay["q"].cuda(), lay["k"].cuda(), lay["v"].cuda(),
+                              torch.from_numpy(idx).reshape(B, 1, k).cuda(), Lk - 1)
+    assert ic.get_last_device_error() == 0
+    got = out.float().cpu().numpy().reshape(B, Hq, d)
+    assert np.abs(got - ref).max() <= ATTN_ATOL
+    assert np.all(got[0] == 0.0)
+    g_lse = lse.cpu().numpy().reshape(B, Hq)
+    fin = np.isfinite(ref_lse)
+    assert np.array_equal(np.isfinite(g_lse), fin) and not fin[0].any()
+    assert np.abs(g_lse[fin] - ref_lse[fin]).max() <= LSE_ATOL
 
 
 def test_sparse_attn_with_holes_and_bad_indices(ic):
