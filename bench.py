@@ -530,6 +530,12 @@ def time_stack(ic, stack, stream, flush, steps: int, warmup: int, with_marks: bo
     return [starts[s].elapsed_time(ends[s]) for s in range(steps)], marks
 
 
+def timed_steps_for(step_ms: float, target_ms: float = 2000.0, lo: int = 20, hi: int = 2000) -> int:
+    """Steps of the main timed region: enough for about target_ms (so the
+    clock sampler, one sample per 200 ms, sees the region), within [lo, hi]."""
+    return int(min(hi, max(lo, math.ceil(target_ms / max(step_ms, 1e-3)))))
+
+
 def auto_steps(ic, stack, stream, flush, budget_ms: float, lo: int = 2, hi: int = 10) -> int:
     """Timed steps for a supplementary point: enough to fill about budget_ms
     (one untimed probe step gives the step time), clamped to [lo, hi]."""
@@ -901,7 +907,9 @@ def e2e_leg(ic, stack, layers, pattern, stream, steps: int, pg, dev, tokens: flo
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=0,
+                    help="timed steps (0: enough for a timed region of about 2 s, at least 20; "
+                         "20 for the reference arm and the row-sharded mode)")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="prefill_64k", choices=sorted(synth.WORKLOADS))
@@ -935,6 +943,9 @@ def main():
         wl = dataclasses.replace(wl, n_layers=len(pattern), pattern=pattern)
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    auto = args.steps <= 0
+    if auto and (args.impl == "reference" or args.shard == "rows"):
+        args.steps = 20
     if args.impl == "reference":
         return run_reference(args, wl, pattern)
 
@@ -976,6 +987,14 @@ def main():
     torch.cuda.synchronize()
     if ic.get_last_device_error() != 0:
         raise RuntimeError("device error during warm-up")
+    if auto:
+        # one untimed probe step sizes the timed region (every rank takes the
+        # slowest rank's figure, so all time the same number of steps)
+        probe, _ = time_stack(ic, stack, stream, flush, 1, 0, with_marks=False)
+        pms = torch.tensor([probe[0]], device=dev, dtype=torch.float64)
+        if pg is not None:
+            pg.all_reduce(pms, op=pg.ReduceOp.MAX)
+        args.steps = timed_steps_for(float(pms.item()))
 
     marks = [new_marks(stream, n, npl) for _ in range(args.steps)]
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]

@@ -274,3 +274,10 @@ def test_uncorrelated_workloads_are_placed_on_the_requested_device():
     assert all(t.device.type == "meta" for L in layers for t in L.values())
     host = synth.make_layers(synth.WORKLOADS["tiny_prefill"])
     assert all(t.device.type == "cpu" for L in host for t in L.values())
+
+
+def test_timed_region_is_sized_to_about_two_seconds():
+    assert bench.timed_steps_for(124.0) == 20          # the 64K step: 20 steps, 2.5 s
+    assert bench.timed_steps_for(3.3) == 607           # the 8K step: about 2 s
+    assert bench.timed_steps_for(0.12) == 2000         # capped
+    assert bench.timed_steps_for(0.0) == 2000
