@@ -281,3 +281,23 @@ def test_timed_region_is_sized_to_about_two_seconds():
     assert bench.timed_steps_for(3.3) == 607           # the 8K step: about 2 s
     assert bench.timed_steps_for(0.12) == 2000         # capped
     assert bench.timed_steps_for(0.0) == 2000
+
+
+def test_profile_traffic_scales_from_the_capture_nearest_in_size(tmp_path, monkeypatch):
+    prof = tmp_path / "profiles"
+    csrc = tmp_path / "lightning_indexer_top_relu_b200" / "csrc"
+    prof.mkdir()
+    csrc.mkdir(parents=True)
+    (csrc / "sparse_attn.cuh").write_text("s")
+    (csrc / "common.cuh").write_text("c")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    import hashlib
+    h = hashlib.sha256(b"s" + b"c").hexdigest()[:16]
+    (prof / "sparse_attn_kernel_decode_32k.md").write_text(
+        f"source_hash: {h}\ndram_bytes_per_launch: 32\nunits_per_launch: 32\n")
+    (prof / "sparse_attn_kernel_layer_32k.md").write_text(
+        f"source_hash: {h}\ndram_bytes_per_launch: 1000\nunits_per_launch: 16384\n")
+    got, src = bench.profile_traffic("sparse_attn", "prefill_64k", 49152)
+    assert got == 3000 and src.startswith("sparse_attn_kernel_layer_32k.md")
+    got, src = bench.profile_traffic("sparse_attn", "decode_b64", 64)
+    assert got == 64 and src.startswith("sparse_attn_kernel_decode_32k.md")
