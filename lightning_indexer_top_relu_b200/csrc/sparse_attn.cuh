@@ -6,10 +6,13 @@
 // held in the index cache; all query heads share the one K/V head).
 //
 // One CTA handles one query row (all heads) and one split of its slots.  The
-// CTA first stages up to 2048 of the row's indices in shared memory in one
-// coalesced burst (validating them), so no copy ever waits on an index load.
-// Its 4 warps then work independently on interleaved blocks of 16 slots (warp
-// w takes blocks w, w+4, ...).  Each warp runs its own 3-stage cp.async pipeline: 16
+// CTA stages up to 1024 of the row's indices at a time in shared memory in
+// one coalesced burst (validating them), so no copy ever waits on an index
+// load.  Its 4 warps then work independently on interleaved blocks of 16
+// slots (warp w takes blocks w, w+4, ...).  Three CTAs share an SM (168
+// registers a thread, 72 KB of shared memory each): the kernel is bound by
+// latency, and a third CTA beat a third pipeline stage.  Each warp runs its
+// own 2-stage cp.async pipeline: 16
 // lanes copy one 256-byte K row (or V row) per instruction, so every request
 // is a full, coalesced 128-byte line pair; rows land XOR-swizzled in shared
 // memory so the ldmatrix reads are bank-conflict free.  S = Q K^T and
@@ -37,17 +40,20 @@ namespace ic {
 #define IC_SA_WARPS 4
 #endif
 #ifndef IC_SA_STAGES
-#define IC_SA_STAGES 3
+#define IC_SA_STAGES 2
 #endif
 #ifndef IC_SA_MINB
-#define IC_SA_MINB 2
+#define IC_SA_MINB 3
 #endif
 constexpr int SA_BLOCK = IC_SA_BLOCK;        // slots per warp iteration (16, 32 or 64)
 constexpr int SA_WARPS = IC_SA_WARPS;
 constexpr int SA_THREADS = 32 * SA_WARPS;
 constexpr int SA_STAGES = IC_SA_STAGES;
 static_assert(SA_BLOCK == 16 || SA_BLOCK == 32 || SA_BLOCK == 64, "block of 16, 32 or 64 slots");
-constexpr int SA_IDX_TILE = 2048;            // indices staged in shared memory at a time
+#ifndef IC_SA_IDX_TILE
+#define IC_SA_IDX_TILE 1024
+#endif
+constexpr int SA_IDX_TILE = IC_SA_IDX_TILE;  // indices staged in shared memory at a time
 constexpr float SA_RESCALE = 8.0f;           // log2 headroom before the exponent base moves
 
 // 2^x on the special-function unit (subnormal results flush to 0).
