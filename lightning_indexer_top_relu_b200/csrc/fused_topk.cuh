@@ -207,10 +207,16 @@ fused_threshold_kernel(const FusedArgs a) {
 // k of them and none was dropped (the row's reserved slots, counted by the
 // counter, fit in the list); otherwise the row's query block is flagged (and
 // listed once) for the exact fallback.  Reserved slots the indexer left
-// unused hold 0, below every candidate, and are not counted.  The selection is the k largest
-// candidate values (all distinct); it is written in ascending position order
-// through a bitmap of the row's visible positions, which is also the row's
-// selection bitmask when the row attends dense-masked.
+// unused hold 0 and are not counted.  The selection is the k largest
+// candidate values (key << 32 | ~s, all distinct).  Only the 32-bit score
+// keys stay in shared memory (so four CTAs share an SM): the k-th largest key
+// T is selected on them; every candidate with a larger key is kept, and of
+// those whose key equals T the lowest positions are kept, as many as the top
+// k needs (a second selection over the tied positions, only when ties are
+// cut).  The positions come from a second read of the row's list, which is
+// still in L2, and go through a bitmap of the row's visible positions that
+// yields them in ascending order and is also the row's selection bitmask
+// when the row attends dense-masked.
 __global__ void __launch_bounds__(FS_THREADS)
 fused_select_kernel(const FusedArgs a) {
     extern __shared__ __align__(16) uint8_t fs_smem[];
@@ -218,9 +224,10 @@ fused_select_kernel(const FusedArgs a) {
     int* sc = reinterpret_cast<int*>(fs_smem + 1024);                       // 4
     uint32_t* wsum = reinterpret_cast<uint32_t*>(fs_smem + 1040);           // 8
     uint32_t* tot = wsum + FS_THREADS / 32;                                 // 1
-    unsigned long long* one = reinterpret_cast<unsigned long long*>(fs_smem + 1088);
-    unsigned long long* vals = reinterpret_cast<unsigned long long*>(fs_smem + 1152);   // lstride
-    uint32_t* bm = reinterpret_cast<uint32_t*>(fs_smem + 1152 + (size_t)a.lstride * 8); // words
+    uint32_t* one = reinterpret_cast<uint32_t*>(fs_smem + 1088);
+    uint32_t* nties = reinterpret_cast<uint32_t*>(fs_smem + 1092);
+    uint32_t* keys = reinterpret_cast<uint32_t*>(fs_smem + 1152);                       // lstride
+    uint32_t* bm = reinterpret_cast<uint32_t*>(fs_smem + 1152 + (size_t)a.lstride * 4); // words
 
     const int tid = threadIdx.x;
     const long long rr = a.n_rows - 1 - (long long)blockIdx.x;   // longest rows first
@@ -241,27 +248,28 @@ fused_select_kernel(const FusedArgs a) {
         return;
     }
     const uint32_t c = __ldg(a.cnt + rr);
+    const unsigned long long* crow = a.cand + rr * (long long)a.lstride;
     uint32_t valid = 0;
     if (c <= (uint32_t)a.lstride) {                 // uniform
         // The list in pairs (lstride is even, so a row starts 16-byte
         // aligned and the pair holding entry c-1 lies inside the row), four
         // independent 16-byte loads per thread in flight.
-        const ulonglong2* crow = reinterpret_cast<const ulonglong2*>(a.cand + rr * (long long)a.lstride);
+        const ulonglong2* crow2 = reinterpret_cast<const ulonglong2*>(crow);
         const uint32_t npair = (c + 1) / 2;
         uint32_t mine = 0;
         for (uint32_t p0 = tid; p0 < npair; p0 += 4 * FS_THREADS) {
             ulonglong2 x[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u)
-                if (p0 + u * FS_THREADS < npair) x[u] = __ldg(crow + p0 + u * FS_THREADS);
+                if (p0 + u * FS_THREADS < npair) x[u] = __ldg(crow2 + p0 + u * FS_THREADS);
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const uint32_t pj = p0 + u * FS_THREADS;
                 if (pj < npair) {
-                    vals[2 * pj] = x[u].x;
+                    keys[2 * pj] = (uint32_t)(x[u].x >> 32);
                     mine += x[u].x != 0ull;
                     if (2 * pj + 1 < c) {
-                        vals[2 * pj + 1] = x[u].y;
+                        keys[2 * pj + 1] = (uint32_t)(x[u].y >> 32);
                         mine += x[u].y != 0ull;
                     }
                 }
@@ -281,13 +289,43 @@ fused_select_kernel(const FusedArgs a) {
         return;
     }
     for (int w = tid; w < nw; w += FS_THREADS) bm[w] = 0u;
+    if (tid == 0) *nties = 0u;
     __syncthreads();
-    const unsigned long long T =
-        block_kth_largest<unsigned long long, FS_THREADS>(vals, (int)c, a.k, hist, sc, one);
+    // Padding keys are 0, below every key of a finite score, so with at
+    // least k candidates the k-th largest key T is a candidate's.
+    const uint32_t T = block_kth_largest<uint32_t, FS_THREADS>(keys, (int)c, a.k, hist, sc, one);
+    uint32_t gt = 0, eq = 0;
     for (uint32_t j = tid; j < c; j += FS_THREADS) {
-        const unsigned long long v = vals[j];
-        if (v >= T) {
-            const uint32_t s = ~(uint32_t)v;
+        const uint32_t kk = keys[j];
+        gt += kk > T;
+        eq += kk == T;
+    }
+    block_excl_scan<FS_THREADS>(gt, wsum, tot);
+    const uint32_t n_gt = *tot;
+    __syncthreads();                                   // tot is rewritten below
+    block_excl_scan<FS_THREADS>(eq, wsum, tot);
+    const uint32_t n_eq = *tot;
+    const uint32_t need = (uint32_t)a.k - n_gt;        // candidates with key T that are kept
+    // Every candidate with key T is kept when exactly `need` of them exist
+    // (T > 0: padding cannot share the key).  Otherwise the kept ones are the
+    // `need` lowest positions: the need-th largest ~s among them.
+    const bool all_ties = T != 0u && n_eq == need;     // uniform
+    uint32_t cut = 0u;
+    if (!all_ties) {
+        __syncthreads();                               // keys[] is free: it collects ~s of the ties
+        for (uint32_t j = tid; j < c; j += FS_THREADS) {
+            const unsigned long long v = __ldg(crow + j);
+            if (v != 0ull && (uint32_t)(v >> 32) == T) keys[atomicAdd(nties, 1u)] = (uint32_t)v;
+        }
+        __syncthreads();
+        cut = block_kth_largest<uint32_t, FS_THREADS>(keys, (int)*nties, (int)need, hist, sc, one);
+    }
+    // positions from a second read of the list (in L2 since the first)
+    for (uint32_t j = tid; j < c; j += FS_THREADS) {
+        const unsigned long long v = __ldg(crow + j);
+        const uint32_t kk = (uint32_t)(v >> 32), lo = (uint32_t)v;
+        if (v != 0ull && (kk > T || (kk == T && (all_ties || lo >= cut)))) {
+            const uint32_t s = ~lo;
             atomicOr(&bm[s >> 5], 1u << (s & 31));
         }
     }
@@ -315,7 +353,7 @@ fused_select_kernel(const FusedArgs a) {
 // Shared memory of fused_select_kernel for a list of lstride slots and a row
 // length (bitmap words).
 __host__ __device__ constexpr size_t fused_select_smem(int lstride, int Lk) {
-    return 1152 + (size_t)lstride * 8 + (size_t)((Lk + 31) / 32) * 4;
+    return 1152 + (size_t)lstride * 4 + (size_t)((Lk + 31) / 32) * 4;
 }
 
 }  // namespace ic

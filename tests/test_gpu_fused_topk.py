@@ -95,6 +95,38 @@ def test_fused_rows_equal_topk_of_gpu_scores_and_unfused_stack(ic, case):
         assert torch.equal(fused.outs[l], plain.outs[l])
 
 
+def test_fused_selection_cuts_ties_at_the_kth_score(ic):
+    """300 positions share one (scaled) key vector, so every query scores
+    them equally, and where that score is positive they are a row's top
+    scores: rows that see more of them than k keep only the lowest
+    positions of the tie (the exact selection's tie cut).  Index rows equal
+    the oracle's sort of the GPU's own scores, fused or not."""
+    wl = synth.Workload("tie_cut", 1, 3000, 3000, 2, 8, 64, 128, 8, 64, "FS", 0, 53, True)
+    layers = [{n: t.cuda() for n, t in L.items()} for L in synth.make_layers(wl)]
+    tied = torch.arange(7, 3000, 10, device="cuda")                    # 300 positions
+    kk = layers[0]["k_idx"]
+    kk[0, tied] = (8.0 * kk[0, 7].float()).to(kk.dtype)
+    fused = _stack(ic, wl, layers, 1)
+    plain = _stack(ic, wl, layers, 0)
+    want = _expected(ic, wl, layers[0])
+    got = fused.dumps[0].cpu().numpy().reshape(-1, wl.k)
+    bad = np.nonzero(~np.all(got == want, axis=1))[0]
+    assert bad.size == 0, f"{bad.size} rows differ, first {bad[:5]}"
+    assert torch.equal(fused.dumps[0], plain.dumps[0])
+    # rows late enough hold more than k of the tied positions among their top scores
+    sc = ic.indexer_scores(layers[0]["q_idx"], layers[0]["k_idx"], layers[0]["w"], 0).reshape(-1, 3000)
+    t = 2999
+    row = sc[t, : t + 1].float()
+    top_tie = (row[tied] == row.max()).all().item()
+    cut_rows = int(top_tie)
+    for t in range(2000, 3000, 97):
+        row = sc[t, : t + 1].float()
+        vis = tied[tied <= t]
+        if (row[vis] == row.max()).all() and vis.numel() > wl.k:
+            cut_rows += 1
+    assert cut_rows > 0, "no row's top-k cut the tie; the case does not exercise the cut"
+
+
 def test_fused_8k_prefill_equals_unfused_stack(ic):
     """The benchmarked 8K prefill (8 layers FSSSFSSS, k = 2048), fused and
     unfused: the same index rows in every layer and the same outputs, whose
