@@ -285,7 +285,7 @@ int launch_topk(const float* scores, long long ld, long long row_base, long long
     cudaError_t e;
     if (n_rows < 2LL * sms && n_max > 4096) {
         // few long rows (decode): a 1024-thread CTA per row, one per SM
-        if (n_max <= ic::TK_CACHE_MAX) {
+        if (n_max <= ic::TK_CACHE_MAX_FEW) {
             ic::topk_select_kernel<ic::TK_THREADS_FEW, true>
                 <<<grid, ic::TK_THREADS_FEW, ic::TK_SMEM_FIXED + n_max * 4, st>>>(
                     scores, ld, row_base, n_rows, Lq, Lk, q_offset, k, idx, mask, Lq_d, W, lst);
@@ -756,7 +756,7 @@ int device_setup(int* dev_out, int* sms_out) {
         set_indexer_attr<128, 64>(); set_indexer_attr<128, 128>();
         cudaFuncSetAttribute(ic::topk_select_kernel<ic::TK_THREADS_FEW, true>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             ic::TK_SMEM_FIXED + ic::TK_CACHE_MAX * 4);
+                             ic::TK_SMEM_FIXED + ic::TK_CACHE_MAX_FEW * 4);
         cudaFuncSetAttribute(ic::topk_select_kernel<ic::TK_THREADS, true>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              ic::TK_SMEM_FIXED + ic::TK_CACHE_MAX * 4);

@@ -40,7 +40,10 @@ namespace ic {
 
 // Threads per row.  Rows longer than TK_CACHE_MAX re-read their scores from
 // L2/HBM; measured at L=65536, eight 256-thread CTAs per SM beat 2 x 512 and
-// 1 x 1024 threads (more rows in flight outweigh keeping them in L2).
+// 1 x 1024 threads (more rows in flight outweigh keeping them in L2).  The
+// same holds from 16K positions down: 16K rows took 0.72 ms per layer
+// re-reading (eight CTAs per SM) against 0.90 ms cached (64 KB a CTA, three
+// per SM), while 8K rows are faster cached (0.19 vs 0.21 ms: four per SM).
 constexpr int TK_THREADS = 256;
 constexpr int TK_THREADS_LONG = 256;
 constexpr int TK_THREADS_FEW = 1024;     // fewer rows than 2 x SMs (decode): more threads per row
@@ -48,7 +51,11 @@ constexpr int TK_BINS = 2048;
 constexpr int TK_CAND = 2048;                                     // candidate keys kept in smem
 // hist + candidate keys + candidate warp ids + scratch
 constexpr int TK_SMEM_FIXED = TK_BINS * 4 + TK_CAND * 4 + TK_CAND + 1024;
-constexpr int TK_CACHE_MAX = 45056;                               // longest row kept in smem
+#ifndef IC_TK_CACHE_MAX
+#define IC_TK_CACHE_MAX 8192
+#endif
+constexpr int TK_CACHE_MAX = IC_TK_CACHE_MAX;                     // longest row kept in smem
+constexpr int TK_CACHE_MAX_FEW = 45056;   // the same with few rows (one 1024-thread CTA per SM)
 constexpr int TK_VB = 8;                                          // float4 loads in flight per thread
 
 // Suffix scan of the 2048-bin histogram: finds the bin b whose count makes
