@@ -436,7 +436,10 @@ int launch_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, const i
 // Measured on B200 at k = 2048, Hq = 16: a dense-masked row costs about
 // 8.4 ps per visible position, a gathered row about 149 ns, so the two meet
 // near t = 8.7k.
-constexpr int DENSE_FACTOR = 8;
+#ifndef IC_DENSE_FACTOR
+#define IC_DENSE_FACTOR 8
+#endif
+constexpr int DENSE_FACTOR = IC_DENSE_FACTOR;
 // Keys a dense-masked row may see (bounds the bitmask row: 8 KB of shared
 // memory in the mask build, and the transposed V copy).
 constexpr int DENSE_MAX_KEYS = 65536;
