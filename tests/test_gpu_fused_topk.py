@@ -7,8 +7,8 @@ certify the result fall back to the plain indexer + top-k.  Whatever the
 thresholds do, the index rows must be exactly the top-k of the scores the
 GPU's indexer computes (ic_indexer_scores), so every test compares them bit
 for bit with the oracle's sort-based top-k run on those very scores (the
-north_star's "top-k bit-exact when run on the same score tensor"), and with
-the unfused stack (index rows and attention outputs identical).
+parity rule for the top-k: bit-exact on the same score tensor), and with the
+unfused stack (index rows and attention outputs identical).
 
 Cases: ragged and multi-tile shapes, B > 1 with a continuation chunk, the
 benchmarked 8K prefill, the long rows falling back (w = 0: all scores tie
