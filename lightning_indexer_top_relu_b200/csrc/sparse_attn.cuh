@@ -6,7 +6,7 @@
 // held in the index cache; all query heads share the one K/V head).
 //
 // One CTA handles one query row (all heads) and one split of its slots.  The
-// CTA stages up to 1024 of the row's indices at a time in shared memory in
+// CTA stages up to 2048 of the row's indices at a time in shared memory in
 // one coalesced burst (validating them), so no copy ever waits on an index
 // load.  Its 4 warps then work independently on interleaved blocks of 16
 // slots (warp w takes blocks w, w+4, ...).  Three CTAs share an SM (168
@@ -51,7 +51,7 @@ constexpr int SA_THREADS = 32 * SA_WARPS;
 constexpr int SA_STAGES = IC_SA_STAGES;
 static_assert(SA_BLOCK == 16 || SA_BLOCK == 32 || SA_BLOCK == 64, "block of 16, 32 or 64 slots");
 #ifndef IC_SA_IDX_TILE
-#define IC_SA_IDX_TILE 1024
+#define IC_SA_IDX_TILE 2048
 #endif
 constexpr int SA_IDX_TILE = IC_SA_IDX_TILE;  // indices staged in shared memory at a time
 constexpr float SA_RESCALE = 8.0f;           // log2 headroom before the exponent base moves
@@ -93,8 +93,11 @@ struct SaSmem {
     static constexpr int ROW = D * 2;                          // bytes per K/V/Q row
     static constexpr int BLK = SA_BLOCK * ROW;                 // one block of K (or V) rows
     static constexpr int STAGE = 2 * BLK;                      // K then V
+    // The Q rows are read into registers once, before any ring stage is
+    // written, so they share warp 0's first stage.
     static constexpr int OFF_Q = 0;
-    static constexpr int OFF_KV = 16 * ROW;
+    static constexpr int OFF_KV = 0;
+    static_assert(16 * ROW <= STAGE, "the Q rows fit in one ring stage");
     static constexpr int WARP_KV = SA_STAGES * STAGE;
     static constexpr int OFF_IDX = OFF_KV + SA_WARPS * WARP_KV;
     static constexpr int BYTES = OFF_IDX + SA_IDX_TILE * 4;
@@ -243,6 +246,7 @@ sparse_attn_kernel(const SparseAttnArgs a) {
                 const int c = 2 * kk + (lane >> 4);
                 ldsm_x4(sbase + S::OFF_Q + swz<D>(r, c), qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3]);
             }
+            __syncthreads();              // every warp holds Q before warp 0's ring overwrites it
         }
         const int nblk = (ntile + SA_BLOCK - 1) / SA_BLOCK;
         const int niter = nblk > warp ? (nblk - warp + SA_WARPS - 1) / SA_WARPS : 0;
