@@ -1091,7 +1091,7 @@ def main():
 
     # ---- end to end through the public API with host buffers
     if not args.no_e2e:
-        line["e2e"] = e2e_leg(ic, stack, layers, pattern, stream, max(3, args.steps // 2), pg,
+        line["e2e"] = e2e_leg(ic, stack, layers, pattern, stream, max(3, min(args.steps, 300)), pg,
                               dev, float(wl.B * wl.Lq))
         if ic.get_last_device_error() != 0:
             raise RuntimeError("device error in the end-to-end leg")
