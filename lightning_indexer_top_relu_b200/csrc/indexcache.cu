@@ -222,6 +222,24 @@ int launch_indexer(const uint16_t* q_idx, const uint16_t* k_idx, const float* w,
     }
     int tpu = (int)std::min<long long>(64, std::max<long long>(4, total / (6LL * sms)));
     if (listed) tpu = std::max(4, std::min(tpu, max_nt / 8));
+#ifndef IC_IDX_EVEN_UNITS
+#define IC_IDX_EVEN_UNITS 1
+#endif
+    if (IC_IDX_EVEN_UNITS && !listed && total == blocks * (long long)max_nt && max_nt > 4) {
+        // Every block has the same number of key tiles (decode: one row per
+        // sequence, all at the same position), so every unit costs the same
+        // and the busiest CTA sets the time: take the unit length that
+        // minimises its tiles, counting one tile of overhead per unit.
+        long long best = -1;
+        for (int c = 4; c <= std::min(64, max_nt); ++c) {
+            const long long units = blocks * (long long)((max_nt + c - 1) / c);
+            const long long cost = (units + sms - 1) / sms * (long long)(c + 1);
+            if (best < 0 || cost < best) {
+                best = cost;
+                tpu = c;
+            }
+        }
+    }
     if (x.tpu > 0) tpu = x.tpu;
     tpu = std::min(tpu, std::max(1, max_nt));
     const int max_splits = (max_nt + tpu - 1) / tpu;
