@@ -329,7 +329,8 @@ int launch_topk(const float* scores, long long ld, long long row_base, long long
 // ---------------------------------------------------------------- sparse attention
 
 int attn_splits(long long n_rows, int k_slots, int sms) {
-    // rows x splits CTAs fill the 2 CTAs per SM that fit, in one wave
+    // rows x splits CTAs fill two CTAs per SM in one wave (three fit: the
+    // spare slot absorbs the ragged end of the wave)
     if (n_rows >= 2LL * sms) return 1;
     long long s = (2LL * sms) / n_rows;
     s = std::min<long long>(s, (k_slots + ic::SA_WARPS * ic::SA_BLOCK - 1) / (ic::SA_WARPS * ic::SA_BLOCK));
