@@ -158,9 +158,13 @@ def _read_profile(path, srcs):
 def profile_traffic(kernel: str, workload: str, units: float = 0.0):
     """DRAM bytes per launch of `kernel` from the committed ncu summaries:
     the summary of this workload when there is one; otherwise a summary of a
-    smaller case of the same kernel that records its units per launch (query
-    rows), scaled by units / its units -- the full-size workloads are too
-    large for a full ncu capture.  Returns (bytes or None, where from)."""
+    case of the same kernel and the same kind (decode rows or prefill rows)
+    that records its units per launch (query rows), within 4x of this
+    launch's, scaled by units / its units -- the full-size workloads are too
+    large for a full ncu capture.  Traffic per row differs between regimes
+    (decode rows read K/V from HBM, prefill rows from L2), and so does the
+    share that does not grow with the rows, so nothing further is scaled:
+    (None, None).  Returns (bytes or None, where from)."""
     import glob
     name, srcs = _KERNEL_SRC[kernel]
     path = os.path.join(ROOT, "profiles", f"{name}_{workload}.md")
@@ -169,12 +173,16 @@ def profile_traffic(kernel: str, workload: str, units: float = 0.0):
         return (got[0], os.path.basename(path)) if got else (None, None)
     if units > 0:
         # the matching capture whose size is nearest (in ratio) to this launch's
+        decode = workload.startswith("decode")
         best = None
         for path in sorted(glob.glob(os.path.join(ROOT, "profiles", f"{name}_*.md"))):
+            other = os.path.basename(path)[len(name) + 1:-3]
+            if other.startswith("decode") != decode:
+                continue
             got = _read_profile(path, srcs)
             if got and got[1]:
                 dist = abs(math.log(units / got[1]))
-                if best is None or dist < best[0]:
+                if dist <= math.log(4.0) and (best is None or dist < best[0]):
                     best = (dist, path, got)
         if best:
             _, path, got = best

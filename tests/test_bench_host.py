@@ -301,3 +301,8 @@ def test_profile_traffic_scales_from_the_capture_nearest_in_size(tmp_path, monke
     assert got == 3000 and src.startswith("sparse_attn_kernel_layer_32k.md")
     got, src = bench.profile_traffic("sparse_attn", "decode_b64", 64)
     assert got == 64 and src.startswith("sparse_attn_kernel_decode_32k.md")
+    # another regime (prefill rows from a decode capture) or a size more than
+    # 4x away: no figure
+    assert bench.profile_traffic("sparse_attn", "tiny_prefill", 32) == (None, None)
+    assert bench.profile_traffic("sparse_attn", "prefill_512k", 16384 * 5) == (None, None)
+    assert bench.profile_traffic("sparse_attn", "decode_b512", 512) == (None, None)
