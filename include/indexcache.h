@@ -280,8 +280,8 @@ int ic_layer_stack_forward_events(const char *pattern, int n_layers, const ic_la
 
 /*
  * Options of ic_layer_stack_forward_opts (NULL = all defaults).
- *   fused_topk  how an F layer turns scores into index rows (next step f1;
- *               the kualia.ai review, "The Hidden Quadratic": the indexer's
+ *   fused_topk  how an F layer turns scores into index rows (the kualia.ai
+ *               review, "The Hidden Quadratic": the indexer's
  *               O(L^2) work and its L x L score matrix dominate long
  *               prefills):
  *                 0  store each chunk's causal scores in the workspace, then
@@ -338,7 +338,7 @@ int ic_layer_stack_fused_fallback_blocks(const ic_dims *dims, const ic_stack_opt
                                          int *blocks);
 
 /*
- * Next step f2 -- cross-layer overlap of two layers' index sets (skill page,
+ * Cross-layer overlap of two layers' index sets (skill page,
  * Step 1 "Analyze Index Correlation Across Layers": top-k sets of
  * consecutive layers compared per query position; kualia.ai review: in
  * adjacent layers 70-100% of the k picks coincide).

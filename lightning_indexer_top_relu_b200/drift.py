@@ -1,4 +1,4 @@
-"""Drift-triggered index refresh: a dynamic F/S schedule (next step f3).
+"""Drift-triggered index refresh: a dynamic F/S schedule.
 
 IndexCache fixes the F/S pattern offline.  The kualia.ai review of the paper
 (Conclusion) asks whether sharing should instead be decided at run time:

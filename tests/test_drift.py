@@ -1,4 +1,4 @@
-"""Drift-triggered refresh (next step f3) on CPU: the policy of
+"""Drift-triggered refresh on CPU: the policy of
 DriftRefreshStack driven by an oracle backend.  Its outputs must equal the
 static oracle stack run with the F/S pattern the policy chose, and the policy
 must refresh exactly the layers whose own top-k has drifted from the cache."""

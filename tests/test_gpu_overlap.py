@@ -1,4 +1,4 @@
-"""Next step f2 -- cross-layer index overlap on the GPU against the oracle
+"""Cross-layer index overlap on the GPU against the oracle
 (integer results: bit-exact), through the C ABI."""
 import numpy as np
 import pytest

@@ -1,4 +1,4 @@
-"""Row sharding of the layer stack (next step f4) on CPU: the partition of
+"""Row sharding of the layer stack on CPU: the partition of
 rows / sequences over ranks, and that the pieces reproduce the whole stack
 (query rows are independent given the prefix), checked with the oracle and
 with two gloo ranks.  The GPU side of a shard is an ordinary stack call with
