@@ -89,7 +89,7 @@ int ic_get_last_device_error(ic_stream_t stream);
 int ic_selftest_wait_timeout(int timeout_us, ic_stream_t stream);
 
 /*
- * Step a1 — lightning indexer scores (digest Abstract; review Introduction:
+ * Lightning indexer scores (digest Abstract; review Introduction:
  * one indexer pass rates every earlier token of each query).
  *   q_idx  [B, Lq, H_I, d_I] bf16     k_idx [B, Lk, d_I] bf16
  *   w      [B, Lq, H_I]      fp32     scores [B, Lq, Lk] fp32 (written)
@@ -102,7 +102,7 @@ int ic_indexer_scores(const uint16_t *q_idx, const uint16_t *k_idx, const float 
                       ic_stream_t stream);
 
 /*
- * Step a2 — per-row top-k (digest Abstract: k tokens are kept per query).
+ * Per-row top-k (digest Abstract: k tokens are kept per query).
  *   scores [B, Lq, Lk] fp32 (only s <= t is read)   idx [B, Lq, k] int32 (written)
  * Row (b, i) keeps the min(k, t+1) visible positions first in the order
  * (score descending, position ascending), written in ascending position
@@ -114,7 +114,7 @@ int ic_topk_select(const float *scores, int B, int Lq, int Lk, int q_offset, int
                    int32_t *idx, ic_stream_t stream);
 
 /*
- * Step a4 — sparse attention over the cached positions (digest Abstract:
+ * Sparse attention over the cached positions (digest Abstract:
  * core attention over k tokens; knowledge note: every later layer attends
  * sparsely over the stored set).  MQA: Hkv must be 1.
  *   q [B, Lq, Hq, d] bf16   k, v [B, Lk, Hkv, d] bf16   idx [B, Lq, k] int32
@@ -173,7 +173,7 @@ int ic_sparse_attn_no_alloc(const uint16_t *q, const uint16_t *k, const uint16_t
                             ic_stream_t stream);
 
 /*
- * Step a4 as the layer stack runs it, for index rows that hold every position
+ * The sparse attention step as the layer stack runs it, for index rows that hold every position
  * at most once (top-k output always does).  Same arguments, layout and
  * results as ic_sparse_attn, except that a position repeated within a row
  * counts once here (ic_sparse_attn counts every slot).  Rows whose selection
@@ -235,7 +235,7 @@ size_t ic_layer_stack_workspace_bytes(const ic_dims *dims, int n_layers, long lo
 int ic_layer_stack_dense_rows(const ic_dims *dims, size_t ws_bytes);
 
 /*
- * Steps a1-a5 — the IndexCache layer loop (skill page Step 3; technical
+ * The IndexCache layer loop (skill page Step 3; technical
  * summary, Methodologie; review, "The Redundancy That Was Sitting There": the
  * loop gains one branch per layer).
  * pattern: n_layers characters, 'F' or '1' = Full layer, 'S' or '0' = Shared.

@@ -71,7 +71,7 @@ void or_set_num_threads(int n)
 }
 
 /*
- * Step a1, lightning indexer score (Abstract of the IndexCache digest; the
+ * Lightning indexer score (Abstract of the IndexCache digest; the
  * score form is the standard one stated in the header above).
  *   qI  [B, Lq, H, dI] bf16 bits      kI [B, Lk, dI] bf16 bits
  *   w   [B, Lq, H]     float          out [n_rows, Lk] double
@@ -113,7 +113,7 @@ int or_indexer_scores(const uint16_t *qI, const uint16_t *kI, const float *w,
 }
 
 /* ------------------------------------------------------------------ */
-/* Step a2, per-row top-k.  A row at position t sees n = min(t+1, Lk)   */
+/* Per-row top-k.  A row at position t sees n = min(t+1, Lk)           */
 /* positions.  The selected set is the min(k, n) positions that come    */
 /* first in the order (score descending, position ascending); it is     */
 /* written in ascending position order and padded with -1.              */
@@ -188,7 +188,7 @@ int or_topk_count(const float *scores, const int64_t *tpos, int64_t n_rows, int 
 }
 
 /* ------------------------------------------------------------------ */
-/* Step a4, sparse attention over the cached positions (IndexCache      */
+/* Sparse attention over the cached positions (IndexCache              */
 /* digest, Abstract: core attention over k selected tokens; knowledge   */
 /* note, How It Works: every later layer attends sparsely over the     */
 /* stored set).  MQA: every query head reads the one K/V head.          */

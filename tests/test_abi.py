@@ -217,6 +217,25 @@ def test_unique_attention_rejects_bad_arguments_before_launch(ic):
     assert ic.kernel_launch_count() == before
 
 
+def test_empty_batches_and_rows_are_no_ops(ic):
+    """An empty batch or zero query rows is a valid call: every entry point
+    returns IC_OK and launches nothing (no device is touched, so this runs
+    without a GPU)."""
+    lib = ic.lib()
+    before = ic.kernel_launch_count()
+    for B, Lq, q0 in ((0, 4, 0), (1, 0, 4)):
+        assert lib.ic_indexer_scores(0x1000, 0x1000, 0x2000, B, Lq, 4, 4, 64, q0, 0x3000, None) == 0
+        assert lib.ic_topk_select(0x1000, B, Lq, 4, q0, 2, 0x2000, None) == 0
+        args = (0x1000, 0x1000, 0x1000, 0x1000, B, Lq, 4, 8, 1, 64, 2, q0, 0.0, 0x1000, None)
+        assert lib.ic_sparse_attn(*args, None, 0, None) == 0
+        assert lib.ic_sparse_attn_no_alloc(*args, None) == 0
+        assert lib.ic_sparse_attn_unique(*args, None, 0, None) == 0
+        d = _dims(ic, B=B, Lq=Lq, Lk=4, q_offset=q0, k=2)
+        assert _stack_call(ic, "FS", d) == 0
+    assert lib.ic_index_overlap(0x1000, 0x1000, 0, 8, 16, 0x2000, None) == 0
+    assert ic.kernel_launch_count() == before
+
+
 def test_unique_attention_workspace_query(ic):
     q = ic.sparse_attn_unique_workspace_bytes
     assert q(1, 700, 700, 0, 16, 128, 96) > 700 * 12 * 4        # bitmask + V^T at least

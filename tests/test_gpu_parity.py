@@ -72,7 +72,7 @@ def check_idx_valid(idx: torch.Tensor, q_offset: int, k: int):
     assert torch.all(torch.where(valid[None, :, 1:], d > 0, True))
 
 
-# ------------------------------------------------------------------ a1 indexer
+# ------------------------------------------------------------------ indexer
 
 INDEXER_SHAPES = [
     # B, Lq, Lk, q_offset, H_I, d_I
@@ -112,7 +112,7 @@ def test_indexer_small_integers_are_bit_exact(ic):
     assert np.array_equal(gpu, ref)
 
 
-# ------------------------------------------------------------------ a2 top-k
+# ------------------------------------------------------------------ top-k
 
 def _score_draw(kind, rows, Lk, seed):
     rng = np.random.default_rng(seed)
@@ -164,7 +164,7 @@ def test_topk_on_oracle_indexer_scores(ic):
     assert np.array_equal(gpu.cpu().numpy().reshape(512, wl.k), ref)
 
 
-# ------------------------------------------------------------------ a4 sparse attention
+# ------------------------------------------------------------------ sparse attention
 
 def _oracle_idx(L, k, q_offset):
     B, Lq = L["q_idx"].shape[:2]
@@ -359,7 +359,7 @@ def test_unique_attn_rows_raising_their_max_after_the_first_tile(ic):
     assert np.abs(lse.cpu().numpy().reshape(L, Hq) - ref_lse).max() <= LSE_ATOL
 
 
-# ------------------------------------------------------------------ a3/a5 layer stack
+# ------------------------------------------------------------------ index cache and layer stack
 
 def _run_stack(ic, wl, layers, pattern=None, **kw):
     pattern = pattern or wl.pattern

@@ -23,7 +23,7 @@ GOLDEN = os.path.join(ROOT, "tests", "golden")
 # (name, file, [(original text, replacement), ...]); every original must
 # occur exactly as often as its count in the list says (once by default).
 MUTANTS = [
-    # ---- a1 indexer
+    # ---- indexer
     ("relu_dropped", "oracle.c",
      [("double relu = dot > 0.0 ? dot : 0.0;", "double relu = dot;")]),
     ("relu_after_the_head_weight", "oracle.c",
@@ -44,7 +44,7 @@ MUTANTS = [
     ("indexer_position_without_offset", "oracle.c",
      [("int64_t t = (int64_t)q_offset + i;\n        const uint16_t *q = qI",
        "int64_t t = i;\n        const uint16_t *q = qI")]),
-    # ---- a2 top-k
+    # ---- top-k
     ("ties_to_the_higher_position", "oracle.c",
      [("return (x->s < y->s) ? -1 : (x->s > y->s);", "return (x->s > y->s) ? -1 : (x->s < y->s);"),
       ("(S[s2] == S[s] && s2 < s)", "(S[s2] == S[s] && s2 > s)")]),
@@ -65,7 +65,7 @@ MUTANTS = [
      [("if (x->v > y->v) return -1;\n    if (x->v < y->v) return 1;",
        "if (x->v > y->v) return -1;\n    if (x->v < y->v) return 1;\n"
        "    if (signbit(x->v) != signbit(y->v)) return signbit(x->v) ? 1 : -1;")]),
-    # ---- a4 attention
+    # ---- attention
     ("softmax_scale_missing", "oracle.c",
      [("z[i] = scale * dot;", "z[i] = dot;")]),
     ("softmax_not_normalised", "oracle.c",
@@ -119,7 +119,7 @@ MUTANTS = [
     ("stack_attention_ignores_the_row_sample", "__init__.py",
      [('o, lse = sparse_attn(L["q"], L["k"], L["v"], cached, q_offset, scale, rows)',
        'o, lse = sparse_attn(L["q"], L["k"], L["v"], cached, q_offset, scale)')]),
-    # ---- a3 / a5 layer stack
+    # ---- index cache and layer stack
     ("shared_layers_keep_the_first_full_layer", "__init__.py",
      [("            cached = topk_sort(sc.astype(np.float32), row_positions(B, Lq, q_offset, rows), k)",
        "            cached = cached if cached is not None else topk_sort(\n"

@@ -32,7 +32,7 @@ def _num(x):
     return float(x)
 
 
-# ------------------------------------------------------------------ indexer (a1)
+# ------------------------------------------------------------------ indexer
 
 def test_indexer_hand_worked_example(golden_dir):
     g = _load(golden_dir, "indexer_hand_example.json")
@@ -127,7 +127,7 @@ def test_indexer_row_sampling_matches_full():
     assert np.array_equal(part, full[rows])
 
 
-# ------------------------------------------------------------------ top-k (a2)
+# ------------------------------------------------------------------ top-k
 
 @pytest.mark.parametrize("draw", ["ties", "gauss", "signed_zero"])
 def test_topk_sort_equals_bruteforce_count(draw):
@@ -189,7 +189,7 @@ def test_topk_increasing_scores_closed_form():
         assert idx[t].tolist() == list(range(t - m + 1, t + 1)) + [-1] * (k - m)
 
 
-# ------------------------------------------------------------------ attention (a4)
+# ------------------------------------------------------------------ attention
 
 def test_attention_hand_worked_example(golden_dir):
     g = _load(golden_dir, "attn_hand_example.json")
