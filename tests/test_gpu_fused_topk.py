@@ -11,7 +11,7 @@ parity rule for the top-k: bit-exact on the same score tensor), and with the
 unfused stack (index rows and attention outputs identical).
 
 Cases: ragged and multi-tile shapes, B > 1 with a continuation chunk, the
-benchmarked 8K prefill, the long rows falling back (w = 0: all scores tie
+largest k the fused path takes (4096), the benchmarked 8K prefill, the long rows falling back (w = 0: all scores tie
 at 0, the closed form [0 .. k-1]), about half the rows falling back (a tiny
 threshold margin), and small workspaces that split the rows into chunks with
 several fallback rounds each.
@@ -76,6 +76,9 @@ CASES = [
     ("eight_k_k512", 1, 8192, 8192, 0, 32, 128, 512, 16, 128),
     ("batch2_continuation", 2, 1500, 6000, 4500, 64, 128, 256, 16, 128),
     ("heads128", 1, 3000, 3000, 0, 128, 64, 128, 8, 64),
+    # the largest k the fused path takes (4096): rows t >= 10000 see more
+    # than twice the 4k-entry list, so they run on sampled thresholds
+    ("max_k_continuation", 1, 2000, 12000, 10000, 16, 128, 4096, 8, 64),
 ]
 
 
