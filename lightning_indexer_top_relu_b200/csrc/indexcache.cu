@@ -340,8 +340,13 @@ int attn_splits(long long n_rows, int k_slots, int sms) {
 
 // Splits of up to ATTN_CLUSTER_MAX CTAs run as one thread-block cluster per
 // row and merge through distributed shared memory (no workspace, no combine
-// launch); a one-wave split count up to twice that is trimmed to it.
-constexpr int ATTN_CLUSTER_MAX = 8;
+// launch); a one-wave split count up to 16 is trimmed to it.  Measured on
+// decode rows of 2048 slots: 8 beats 4, 6 and 10.
+#ifndef IC_ATTN_CLUSTER_MAX
+#define IC_ATTN_CLUSTER_MAX 8
+#endif
+constexpr int ATTN_CLUSTER_MAX = IC_ATTN_CLUSTER_MAX;
+static_assert(ATTN_CLUSTER_MAX >= 2 && ATTN_CLUSTER_MAX <= 8, "portable cluster sizes only");
 
 template <int D>
 bool attn_cluster_fits() {
@@ -402,7 +407,7 @@ int launch_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, const i
     const long long n_rows = (long long)B * rows_per_b;
     if (n_rows <= 0) return IC_OK;
     int splits = attn_splits(n_rows, k_slots, sms);
-    const bool cluster = splits > 1 && splits <= 2 * ATTN_CLUSTER_MAX && attn_cluster_available();
+    const bool cluster = splits > 1 && splits <= 16 && attn_cluster_available();
     if (cluster) splits = std::min(splits, ATTN_CLUSTER_MAX);
     while (!cluster && splits > 1 && (ws == nullptr || attn_ws_bytes(n_rows, splits, Hq, d) > ws_bytes))
         splits = splits / 2;
