@@ -58,6 +58,22 @@ constexpr int TK_CACHE_MAX = IC_TK_CACHE_MAX;                     // longest row
 constexpr int TK_CACHE_MAX_FEW = 45056;   // the same with few rows (one 1024-thread CTA per SM)
 constexpr int TK_VB = 8;                                          // float4 loads in flight per thread
 
+// Sum of vals[w] over the warps w < warp (NW <= 32 per-warp totals in shared
+// memory): each warp scans the NW totals with shuffles.
+template <int NW>
+__device__ __forceinline__ uint32_t tk_warps_before(const uint32_t* vals, int warp, int lane) {
+    static_assert(NW >= 1 && NW <= 32, "one warp scans the totals");
+    uint32_t x = lane < NW ? vals[lane] : 0u;
+#pragma unroll
+    for (int o = 1; o < NW; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    // inclusive scan at lane warp - 1 = the exclusive prefix of warp
+    const uint32_t incl = __shfl_sync(0xffffffffu, x, warp > 0 ? warp - 1 : 0);
+    return warp > 0 ? incl : 0u;
+}
+
 // Suffix scan of the 2048-bin histogram: finds the bin b whose count makes
 // the running total (from the top bin down) reach `remaining`.  Writes
 // found[0] = b, found[1] = count of elements in bins above b.  All threads.
@@ -82,9 +98,7 @@ __device__ __forceinline__ void tk_find_bin(const uint32_t* hist, int remaining,
     }
     if (lane == 31) wsum[warp] = x;
     __syncthreads();
-    uint32_t before = 0;
-#pragma unroll
-    for (int w = 0; w < NT / 32; ++w) before += (w < warp) ? wsum[w] : 0u;
+    const uint32_t before = tk_warps_before<NT / 32>(wsum, warp, lane);
     uint32_t above = before + x - mine;
 #pragma unroll
     for (int e = 0; e < PER; ++e) {
@@ -332,12 +346,8 @@ topk_select_kernel(const float* __restrict__ scores, long long ld, long long row
             }
         }
         __syncthreads();
-        unsigned g = 0, e = 0;
-#pragma unroll
-        for (int w = 0; w < NW; ++w) {
-            g += (w < warp) ? wgt[w] : 0u;
-            e += (w < warp) ? weq[w] : 0u;
-        }
+        unsigned g = tk_warps_before<NW>(wgt, warp, lane);
+        unsigned e = tk_warps_before<NW>(weq, warp, lane);
         const unsigned lt = (1u << lane) - 1u;
         for (int gbase = s0; gbase < s1; gbase += 32 * TK_VB) {
             uint32_t kb[TK_VB];
