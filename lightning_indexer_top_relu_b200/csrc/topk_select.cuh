@@ -349,6 +349,32 @@ topk_select_kernel(const float* __restrict__ scores, long long ld, long long row
         unsigned g = tk_warps_before<NW>(wgt, warp, lane);
         unsigned e = tk_warps_before<NW>(weq, warp, lane);
         const unsigned lt = (1u << lane) - 1u;
+        if (tk_warps_before<NW>(weq, NW, lane) == (unsigned)need) {
+            // Every key equal to T is kept (the usual case: T is unique), so
+            // the selection is {key >= T}, exactly k keys: one ballot per 32
+            // positions gives both the output slots and the mask word.
+            unsigned base = g + e;
+            for (int gbase = s0; gbase < s1; gbase += 32 * TK_VB) {
+                uint32_t kb[TK_VB];
+#pragma unroll
+                for (int u = 0; u < TK_VB; ++u) {
+                    const int i = gbase + u * 32 + lane;
+                    kb[u] = i < s1 ? key_at(i) : 0u;
+                }
+#pragma unroll
+                for (int u = 0; u < TK_VB; ++u) {
+                    const int i = gbase + u * 32 + lane;
+                    const unsigned ms = __ballot_sync(0xffffffffu, i < s1 && kb[u] >= T);
+                    if ((ms >> lane) & 1u) out[base + __popc(ms & lt)] = i;
+                    if (mrow != nullptr) {
+                        const int w0 = (gbase + u * 32) >> 5;
+                        if (lane == 0 && gbase + u * 32 < s1 && w0 < W) mrow[w0] = ms;
+                    }
+                    base += __popc(ms);
+                }
+            }
+            continue;
+        }
         for (int gbase = s0; gbase < s1; gbase += 32 * TK_VB) {
             uint32_t kb[TK_VB];
 #pragma unroll
