@@ -1,4 +1,5 @@
-"""The layer stack captured into a CUDA graph and replayed, through the C ABI.
+"""The layer stack captured into a CUDA graph and replayed, and two stacks
+running at once on two streams, through the C ABI.
 
 ic_layer_stack_forward enqueues kernels (and, for decode rows, cluster
 launches) on the caller's stream without any host synchronisation, so a
@@ -81,3 +82,35 @@ def test_graph_replay_equals_eager_run(ic, case):
         assert torch.equal(replayed[1][l], fresh[1][l]), (name, l)
     assert not all(torch.equal(a, b) for a, b in zip(fresh[0], outs))
     del g
+
+
+def test_two_stacks_on_two_streams_run_independently(ic):
+    """The library keeps no state from one call to the next: two stacks over
+    different inputs, enqueued on two streams without synchronising in
+    between (so their kernels may overlap), each give their own sequential
+    results bit for bit."""
+    runs = []
+    for cfg, pattern in ((63, "FSFS"), (64, "FFSS")):
+        wl = synth.custom(B=2, Lq=300, Lk=1300, q_offset=1000, n_layers=4, H_I=32, d_I=128, k=256,
+                          Hq=16, d=128, pattern=pattern, cfg_id=cfg)
+        layers = [{n: t.cuda() for n, t in L.items()} for L in synth.make_layers(wl)]
+        dims = ic.make_dims(wl.B, wl.Lq, wl.Lk, wl.q_offset, wl.H_I, wl.d_I, wl.Hq, wl.d, wl.k)
+        runs.append(ic.LayerStack(pattern, layers, dims, want_lse=True, dump_idx=True))
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    for s in streams:
+        s.wait_stream(torch.cuda.current_stream())     # inputs and workspaces are ready
+    alone = [_eager(ic, st, s) for st, s in zip(runs, streams)]
+    for st in runs:
+        for o in st.outs:
+            o.zero_()
+    torch.cuda.synchronize()
+    for _ in range(3):                       # several overlapping rounds
+        for st, s in zip(runs, streams):
+            with torch.cuda.stream(s):
+                st.forward(s)
+    torch.cuda.synchronize()
+    assert ic.get_last_device_error() == 0
+    for st, (outs, dumps) in zip(runs, alone):
+        for l in range(4):
+            assert torch.equal(st.outs[l], outs[l])
+            assert torch.equal(st.dumps[l], dumps[l])
