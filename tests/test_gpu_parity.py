@@ -13,7 +13,6 @@ Bars (stated for bf16 inputs with fp32 accumulation):
     sets agree, S-layer indices bitwise equal to their F layer's.
 """
 import ctypes
-import math
 
 import numpy as np
 import pytest
