@@ -200,14 +200,18 @@ sparse_attn_kernel(const SparseAttnArgs a) {
     const uint32_t kv_base = sbase + S::OFF_KV + warp * S::WARP_KV;
     int32_t* idx_s = reinterpret_cast<int32_t*>(sa_smem + S::OFF_IDX);
 
-    // Q rows (heads) -> shared memory, rows >= Hq zero.
+    // Q rows (heads) are loaded into registers here and stored to shared
+    // memory (rows >= Hq zero) only after the first index tile's loads are
+    // issued, so the two memory latencies overlap.
+    constexpr int QPT = (16 * CPR + SA_THREADS - 1) / SA_THREADS;   // 16-byte chunks a thread
+    uint4 qv[QPT];
     {
         const uint4* qsrc = reinterpret_cast<const uint4*>(a.q + row * a.Hq * D);
-        for (int p = tid; p < 16 * CPR; p += SA_THREADS) {
-            const int h = p / CPR, c = p % CPR;
-            uint4 val = make_uint4(0, 0, 0, 0);
-            if (h < a.Hq) val = qsrc[h * CPR + c];
-            *reinterpret_cast<uint4*>(sa_smem + S::OFF_Q + swz<D>(h, c)) = val;
+#pragma unroll
+        for (int u = 0; u < QPT; ++u) {
+            const int p = tid + u * SA_THREADS;
+            qv[u] = make_uint4(0, 0, 0, 0);
+            if (p < 16 * CPR && p / CPR < a.Hq) qv[u] = qsrc[p];
         }
     }
 
@@ -235,6 +239,14 @@ sparse_attn_kernel(const SparseAttnArgs a) {
             }
             empty |= (id < 0) & (i < nfill);
             idx_s[i] = id;
+        }
+        if (tile0 == s0) {
+#pragma unroll
+            for (int u = 0; u < QPT; ++u) {
+                const int p = tid + u * SA_THREADS;
+                if (p < 16 * CPR)
+                    *reinterpret_cast<uint4*>(sa_smem + S::OFF_Q + swz<D>(p / CPR, p % CPR)) = qv[u];
+            }
         }
         // Tiles whose blocks hold no empty slot (every row with at least k
         // positions) skip the per-slot masking below.
