@@ -59,9 +59,11 @@ def test_no_alloc_matches_workspace_entry_point_twice(ic):
 
 @pytest.mark.parametrize("B", [100, 300])
 def test_no_alloc_runs_calls_of_many_rows(ic, B):
-    # 100 rows still split their slots (their partials go through the
-    # scratch); 300 rows fill the CTAs the GPU holds at once, run one split
-    # each and leave the scratch unused.  Both equal the workspace entry point.
+    # 100 rows still split their slots, over a thread-block cluster per row
+    # that merges in distributed shared memory (the scratch stays unused; the
+    # workspace query still counts the partials a cluster-less device would
+    # need); 300 rows fill the CTAs the GPU holds at once and run one split
+    # each.  Both equal the workspace entry point.
     wl = synth.custom(B=B, Lq=1, Lk=600, q_offset=599, H_I=4, d_I=64, k=256, Hq=16, d=128,
                       cfg_id=33)
     assert (ic.sparse_attn_workspace_bytes(B, 1, 16, 128, 256) > 0) == (B == 100)
