@@ -403,3 +403,24 @@ def test_workspace_holds_the_fused_chunk(ic):
     assert full >= 65536 * 3 * 2048 * 8
     # a chunk of 4 query blocks still holds a fused chunk
     assert ic.layer_stack_workspace_bytes(d, 8, rows_per_chunk=16) >= 16 * 3 * 2048 * 8
+
+
+def test_binding_fails_loudly_without_the_library(tmp_path):
+    """No CPU fallback: a copy of the package whose library was never built
+    cannot be imported, and neither can the GPU backends that reach the
+    library through it."""
+    import shutil
+    import subprocess
+    import sys
+    pkg = build.PKG
+    dst = tmp_path / os.path.basename(pkg)
+    shutil.copytree(pkg, dst, ignore=shutil.ignore_patterns("*.so", "__pycache__", "csrc"))
+    name = os.path.basename(pkg)
+    env = dict(os.environ, PYTHONPATH=str(tmp_path))
+    for stmt in (f"import {name}.indexcache",
+                 f"from {name}.drift import GpuBackend; GpuBackend([], None)",
+                 f"from {name}.sharding import ShardedStack; ShardedStack('F', [], None, 1, 0)"):
+        r = subprocess.run([sys.executable, "-c", stmt], env=env, cwd=str(tmp_path),
+                           capture_output=True, text=True, timeout=300)
+        assert r.returncode != 0, stmt
+        assert "no CPU fallback" in r.stderr, (stmt, r.stderr[-500:])
