@@ -600,7 +600,7 @@ def kernel_breakdown(ki, w, steps: int, ms_per_step: float, peaks, sm_mhz: float
             ent["gbs"] = w["topk_bytes"] / sec / 1e9
             ent["frac_of_hbm"] = ent["gbs"] / peaks["hbm_gbs"]
         elif name == "attn_dense":
-            ent["covers"] = "V transpose + dense-masked tcgen05 attention, rows t < 8k"
+            ent["covers"] = "V transpose + dense-masked tcgen05 attention, rows t < 6k"
             ent["rows"] = int(w["dense_rows"])
             ent["tflops"] = w["dense_flops"] / sec / 1e12
             ent["frac_of_bf16_peak"] = ent["tflops"] / peaks["bf16_tflops"]
@@ -610,7 +610,7 @@ def kernel_breakdown(ki, w, steps: int, ms_per_step: float, peaks, sm_mhz: float
             ent["exp2_per_s"] = w["dense_exec_exps"] / sec
             ent["frac_of_sfu_peak"] = ent["exp2_per_s"] / sfu_peak
         else:
-            ent["covers"] = "gather attention (+ split combine), rows t >= 8k"
+            ent["covers"] = "gather attention (+ split combine), rows t >= 6k"
             ent["rows"] = int(w["gather_rows"])
             ent["tflops"] = w["gather_flops"] / sec / 1e12
             ent["logical_gbs"] = w["gather_bytes"] / sec / 1e9

@@ -177,7 +177,7 @@ int ic_sparse_attn_no_alloc(const uint16_t *q, const uint16_t *k, const uint16_t
  * at most once (top-k output always does).  Same arguments, layout and
  * results as ic_sparse_attn, except that a position repeated within a row
  * counts once here (ic_sparse_attn counts every slot).  Rows whose selection
- * covers an eighth of their visible positions or more (t < 8k, in whole blocks of
+ * covers a sixth of their visible positions or more (t < 6k, in whole blocks of
  * 128/Hq queries; d = 128 and Hq dividing 128; at most 65536 visible keys)
  * attend tile-dense on the tensor cores under a bitmask of the selection --
  * probability exactly 0 outside it -- when ws holds at least
@@ -227,7 +227,7 @@ size_t ic_layer_stack_workspace_bytes(const ic_dims *dims, int n_layers, long lo
 /*
  * Rows per sequence (the first ones, i < returned value) that
  * ic_layer_stack_forward sends to the dense-masked attention for these dims
- * and a workspace of ws_bytes: rows with t < 8k in whole blocks of 128/Hq
+ * and a workspace of ws_bytes: rows with t < 6k in whole blocks of 128/Hq
  * queries, when d = 128, Hq divides 128, at most 65536 keys are visible and
  * the workspace holds the selection bitmask next to one block of scores and
  * the transposed V.  The other rows gather.  0 for invalid dims.
@@ -268,7 +268,7 @@ int ic_layer_stack_forward(const char *pattern, int n_layers, const ic_layer *la
  *       after indexer + top-k),
  *   j=2 before the attention (after the top-k and, on F layers whose rows
  *       take the dense-masked path, the bitmask build),
- *   j=3 after the dense-masked attention of the rows with t < 8k (the
+ *   j=3 after the dense-masked attention of the rows with t < 6k (the
  *       transposed V copy included; equal to j=2 when no row takes it),
  *   j=4 after the attention.
  * For S layers j=0..2 coincide.  events holds IC_MARKS_PER_LAYER*n_layers

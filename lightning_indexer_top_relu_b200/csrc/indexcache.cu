@@ -458,10 +458,11 @@ int launch_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, const i
 // gather.  Only used inside the layer stack, whose index rows hold distinct
 // positions (a bitmask cannot count a repeated index twice).
 // Measured on B200 at k = 2048, Hq = 16: a dense-masked row costs about
-// 8.4 ps per visible position, a gathered row about 149 ns, so the two meet
-// near t = 8.7k.
+// 9.6 ps per visible position, a gathered row about 103 ns, so the two meet
+// near t = 5.3k; a factor of 6 against 8 took the 64K step from 111.2 to
+// 109.9 ms and a 32K layer from 10.90 to 10.72 ms (same box).
 #ifndef IC_DENSE_FACTOR
-#define IC_DENSE_FACTOR 8
+#define IC_DENSE_FACTOR 6
 #endif
 constexpr int DENSE_FACTOR = IC_DENSE_FACTOR;
 // Keys a dense-masked row may see (bounds the bitmask row: 8 KB of shared
@@ -478,7 +479,7 @@ DenseGeom dense_geom(const ic_dims& D) {
     DenseGeom g;
     if (D.d != 128 || (128 % D.Hq) != 0) return g;
     g.QBD = 128 / D.Hq;
-    long long lim = (long long)DENSE_FACTOR * D.k - D.q_offset;     // rows i with t < 8k
+    long long lim = (long long)DENSE_FACTOR * D.k - D.q_offset;     // rows i with t < 6k
     lim = std::min<long long>(lim, (long long)DENSE_MAX_KEYS - D.q_offset);
     lim = std::min<long long>(lim, D.Lq);
     if (lim < g.QBD) return g;
@@ -547,7 +548,7 @@ int launch_dense_attn(const DenseGeom& g, const ic_dims& D, const ic_layer& L,
     return launched(e, "dense_attn launch");
 }
 
-// How the attention step treats rows with t < 8k.
+// How the attention step treats rows with t < 6k.
 enum AttnMode {
     ATTN_GATHER = 0,        // every row gathers
     ATTN_MASK_READY = 1,    // dense-masked; the workspace already holds the bitmask
@@ -556,7 +557,7 @@ enum AttnMode {
 
 // Attention of one layer over index rows that hold each position at most
 // once.  Dense modes (the caller checked dense_geom(D).on and that ws holds
-// dense_geom(D).total bytes): rows with t < 8k, whole blocks, on the
+// dense_geom(D).total bytes): rows with t < 6k, whole blocks, on the
 // dense-masked kernel -- bitmask at ws, V^T after it, the gathered rows'
 // split partials after both -- and the rest gathered.  `trim` says slots past
 // min(k, t+1) are empty (top-k output); `mid` (may be null) is recorded
@@ -1020,7 +1021,7 @@ size_t ic_sparse_attn_unique_workspace_bytes(int B, int Lq, int Lk, int q_offset
     D.k = k_slots;
     const DenseGeom dg = dense_geom(D);
     if (!dg.on) return ic_sparse_attn_workspace_bytes(B, Lq, Hq, d, k_slots);
-    const int rows_g = Lq - dg.Lq_d;            // rows that still gather (t >= 8k)
+    const int rows_g = Lq - dg.Lq_d;            // rows that still gather (t >= 6k)
     return dg.total + (rows_g > 0 ? ic_sparse_attn_workspace_bytes(B, rows_g, Hq, d, k_slots) : 0);
 }
 
@@ -1114,7 +1115,7 @@ size_t ic_layer_stack_workspace_bytes(const ic_dims* dims, int n_layers, long lo
     (void)n_rows;
     // dense-masked rows: the bitmask (written by the top-k) sits before the
     // score chunk; V^T and the split partials of the rows that still gather
-    // (t >= 8k) reuse the score region
+    // (t >= 6k) reuse the score region
     if (dg.on) {
         const int rows_g = dims->Lq - dg.Lq_d;
         const size_t attn_g =
@@ -1185,7 +1186,7 @@ static int stack_forward(const char* pattern, int n_layers, const ic_layer* laye
         return fail(IC_ERR_WORKSPACE_TOO_SMALL,
                     "workspace of %zu bytes is below one query block of scores (%zu bytes)",
                     ws_bytes, block_bytes);
-    // Rows with t < 8k attend dense-masked when the workspace holds the
+    // Rows with t < 6k attend dense-masked when the workspace holds the
     // bitmask (which the top-k writes, ahead of the score chunk) plus one
     // block of scores, and V^T (which, like the gathered rows' partials,
     // reuses the score region once the layer's top-k is done).  The bitmask

@@ -282,7 +282,7 @@ def sparse_attn_unique_workspace_bytes(B: int, Lq: int, Lk: int, q_offset: int, 
 def sparse_attn_unique(q, k, v, idx, q_offset: int = 0, scale: float = 0.0, out=None, lse=None,
                        want_lse: bool = True, ws=None, stream=None):
     """ic_sparse_attn_unique: the layer stack's attention step for index rows
-    that hold each position at most once (dense-masked rows t < 8k when the
+    that hold each position at most once (dense-masked rows t < 6k when the
     workspace allows, gathered rows otherwise).  ws=None allocates the full
     workspace; pass an empty tensor to force the gather path."""
     B, Lq, Hq, d, Lk, Hkv = _kv_shapes(q, k, v)

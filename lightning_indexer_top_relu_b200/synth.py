@@ -86,8 +86,8 @@ WORKLOADS: Dict[str, Workload] = {
 for _L in (4096, 16384, 65536, 131072):
     WORKLOADS[f"sweep_{_L // 1024}k"] = _prefill(f"sweep_{_L // 1024}k", _L, 1, 64, 128, 2048, 16,
                                                  128, "F", 5)
-# A single F layer at L=32768 (shapes of the sweep): the smallest prefill in
-# which rows t >= 8k = 16384 gather their K/V rows, for kernel profiles.
+# A single F layer at L=32768 (shapes of the sweep), long enough that most of
+# its rows gather their K/V rows (t >= 6k = 12288), for kernel profiles.
 WORKLOADS["layer_32k"] = _prefill("layer_32k", 32768, 1, 64, 128, 2048, 16, 128, "F", 6)
 
 

@@ -147,7 +147,7 @@ def test_index_overlap_rejects_bad_sizes_before_launch(ic):
 
 
 def test_layer_stack_dense_rows(ic):
-    """Rows t < 8k, whole blocks of 128/Hq queries, d = 128, with a workspace
+    """Rows t < 6k, whole blocks of 128/Hq queries, d = 128, with a workspace
     that holds the bitmask, one block of scores and V^T; 0 otherwise."""
     def rows(ws=None, **kw):
         d = dict(B=1, Lq=700, Lk=700, q_offset=0, H_I=32, d_I=128, Hq=16, d=128, k=96)
@@ -157,11 +157,12 @@ def test_layer_stack_dense_rows(ic):
         if ws is None:
             ws = ic.layer_stack_workspace_bytes(dims, 2)
         return ic.layer_stack_dense_rows(dims, ws)
-    assert rows() == 696                       # min(8k, L) = 700 -> 87 blocks of 8
-    assert rows(k=48) == 384                   # 8k = 384
-    assert rows(Hq=8) == 688                   # blocks of 16 queries
+    assert rows() == 576                       # min(6k, L) = 576 -> 72 blocks of 8
+    assert rows(k=48) == 288                   # 6k = 288
+    assert rows(k=128) == 696                  # min(6k, L) = 700 -> 87 blocks of 8
+    assert rows(k=128, Hq=8) == 688            # blocks of 16 queries
     assert rows(d=64, Hq=8) == 0               # the dense kernel needs d = 128
-    assert rows(Lq=1, Lk=32768, q_offset=32767, k=2048) == 0     # decode: t far beyond 8k
+    assert rows(Lq=1, Lk=32768, q_offset=32767, k=2048) == 0     # decode: t far beyond 6k
     assert rows(Lq=300, Lk=1324, q_offset=1024, k=512) == 296    # mid-sequence chunk
     assert rows(ws=1000) == 0                  # workspace too small: every row gathers
     assert rows(d_I=96) == 0                   # invalid dims
@@ -172,7 +173,7 @@ def test_layer_stack_dense_rows(ic):
        k=st.integers(1, 4096), Hq=st.sampled_from([1, 2, 4, 8, 16, 32, 64, 128, 12, 48]),
        d=st.sampled_from([64, 128]), B=st.integers(1, 3), rpc=st.sampled_from([0, 1, 200]))
 def test_layer_stack_dense_rows_rule_and_own_workspace(ic, Lq, q0, extra, k, Hq, d, B, rpc):
-    """The rule as stated (rows t < 8k, at most 65536 visible keys, whole
+    """The rule as stated (rows t < 6k, at most 65536 visible keys, whole
     blocks of 128/Hq queries, d = 128) holds on random shapes, and the size
     the workspace query returns always lets the stack take the dense path,
     whatever the score chunking."""
@@ -183,7 +184,7 @@ def test_layer_stack_dense_rows_rule_and_own_workspace(ic, Lq, q0, extra, k, Hq,
         want = 0
     else:
         qbd = 128 // Hq
-        lim = min(8 * k - q0, 65536 - q0, Lq)
+        lim = min(6 * k - q0, 65536 - q0, Lq)
         want = lim // qbd * qbd if lim >= qbd else 0
     ws = ic.layer_stack_workspace_bytes(dims, 2, rpc)
     assert ws > 0

@@ -133,7 +133,7 @@ def test_fused_selection_cuts_ties_at_the_kth_score(ic):
 def test_fused_8k_prefill_equals_unfused_stack(ic):
     """The benchmarked 8K prefill (8 layers FSSSFSSS, k = 2048), fused and
     unfused: the same index rows in every layer and the same outputs, whose
-    rows t < 16384 attend dense-masked over the bitmask the fused selection
+    rows (all t < 6k = 12288) attend dense-masked over the bitmask the fused selection
     wrote.  Sampled rows also equal the oracle's top-k of the GPU scores."""
     wl = synth.WORKLOADS["prefill_8k"]
     layers = [{n: t.cuda() for n, t in L.items()}

@@ -438,7 +438,7 @@ def test_stack_continuation_chunk_with_dense_rows(ic):
 
 
 def test_stack_timing_marks_are_recorded_in_order(ic):
-    # rows t < 8k take the dense-masked kernel, the rest gather: every mark
+    # rows t < 6k take the dense-masked kernel, the rest gather: every mark
     # of every layer is recorded, in stream order
     wl = synth.custom(Lq=700, n_layers=2, H_I=32, d_I=128, k=96, Hq=16, d=128, pattern="FS",
                       cfg_id=26)
