@@ -261,11 +261,11 @@ def test_sparse_attn_with_holes_and_bad_indices(ic):
 
 
 DENSE_CASES = [
-    # B, Lq, Lk, q_offset, Hq, d, k   (rows t < 8k take the dense-masked kernel)
-    (1, 700, 700, 0, 16, 128, 48),          # 48 dense blocks, 316 gathered rows
-    (1, 700, 700, 0, 16, 128, 96),          # 87 dense blocks, 4 gathered rows split over CTAs
+    # B, Lq, Lk, q_offset, Hq, d, k   (rows t < 6k take the dense-masked kernel)
+    (1, 700, 700, 0, 16, 128, 48),          # 36 dense blocks, 412 gathered rows
+    (1, 700, 700, 0, 16, 128, 96),          # 72 dense blocks, 124 gathered rows split over CTAs
     (2, 1000, 1000, 0, 16, 128, 256),       # all dense, B = 2, ragged last key tile
-    (1, 300, 1324, 1024, 16, 128, 512),     # mid-sequence chunk, 4 gathered tail rows
+    (1, 300, 1324, 1024, 16, 128, 512),     # mid-sequence chunk, 4 gathered tail rows (8 splits)
     (1, 500, 500, 0, 8, 128, 128),          # 16 queries per block
 ]
 
@@ -298,7 +298,7 @@ def test_unique_attn_dense_and_gathered_rows_match_oracle(ic, B, Lq, Lk, q_offse
 def test_unique_attn_dense_rows_with_holes_and_bad_indices(ic):
     """The dense-masked kernel sees the selection only as a bitmask: -1 slots
     anywhere, unsorted rows, and an index beyond t (skipped and reported)."""
-    B, L, Hq, d, k = 1, 160, 16, 128, 40                 # every row t < 8k = 320
+    B, L, Hq, d, k = 1, 160, 16, 128, 40                 # every row t < 6k = 240
     wl = synth.custom(B=B, Lq=L, H_I=4, d_I=64, k=k, Hq=Hq, d=d, cfg_id=28)
     lay = synth.make_layers(wl)[0]
     rng = np.random.default_rng(5)
@@ -346,7 +346,7 @@ def _first_tile_empty_idx(L, k, seed):
 def test_unique_attn_rows_raising_their_max_after_the_first_tile(ic):
     """Rows of one warp raise the running max at different tiles; the O
     rescale in TMEM is warp-collective and must stay correct for all rows."""
-    B, L, Hq, d, k = 1, 256, 16, 128, 40                  # every row t < 8k = 320
+    B, L, Hq, d, k = 1, 256, 16, 128, 40                  # rows t < 6k = 240 dense, 16 gather
     wl = synth.custom(B=B, Lq=L, H_I=4, d_I=64, k=k, Hq=Hq, d=d, cfg_id=30)
     lay = synth.make_layers(wl)[0]
     idx = _first_tile_empty_idx(L, k, 11)

@@ -83,7 +83,7 @@ def test_topk_long_tied_rows_bit_exact(ic, B, Lq, Lk, q_offset, k, draw):
 @pytest.mark.gpu
 def test_stack_with_zero_head_weights_keeps_the_first_positions(ic):
     """w = 0: all scores 0, so every row keeps its first min(k, t+1)
-    positions; rows t < 8k attend dense-masked, the rest gather, both over
+    positions; rows t < 6k attend dense-masked, the rest gather, both over
     those positions, and agree with the oracle's attention on them."""
     wl = synth.custom(Lq=3000, n_layers=2, H_I=32, d_I=128, k=64, Hq=16, d=128, pattern="FS",
                       cfg_id=36)
